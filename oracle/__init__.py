@@ -1,0 +1,130 @@
+"""KDA oracle (test infrastructure only).
+
+A plain fp64 CPU implementation of the fine-grained gated delta rule, written
+in C (``kda_oracle.c``) and called here through ctypes. Only ``tests/``,
+``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline / reference legs
+use it; the product package never imports it, and it never imports the
+product package.
+
+Sources followed: "Decoding Hybrid Attention Architectures" section 3.4 (the
+KDA update and the variant table), section 3.2 (role of beta), section 4 (the
+chunkwise form); "Technical Analysis ... Novel Hybrid Linear Attention"
+sections 2.4 and 3.1-3.2. Every function is pinned by tests/test_oracle.py.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+# Planted-mistake selectors (mirror the enum in kda_oracle.c); 0 = correct.
+MUTATIONS = {
+    "no_decay": 1,
+    "decay_after": 2,
+    "erase_sign": 3,
+    "read_before": 4,
+    "transposed_read": 5,
+    "beta_write_only": 6,
+    "decay_columns": 7,
+    "prefix_decay_k": 8,
+    "strict_tril_o": 9,
+}
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so with gcc (plain C11, -O2, pthreads)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, _SRC,
+                               "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        lib.kda_oracle_recurrent.argtypes = [P] * 8 + [I] * 7
+        lib.kda_oracle_recurrent.restype = I
+        lib.kda_oracle_chunkwise.argtypes = [P] * 8 + [I] * 6 + [P, P, I, I]
+        lib.kda_oracle_chunkwise.restype = I
+        lib.kda_oracle_decode_step.argtypes = [P] * 8 + [I] * 5
+        lib.kda_oracle_decode_step.restype = I
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor -> numpy, no arithmetic
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def recurrent(q, k, v, log_alpha, beta, S0=None, nthreads: int = 0, mutation: str | None = None):
+    """Token-by-token fp64 recurrence. Shapes: q,k,log_alpha [B,T,H,dk];
+    v [B,T,H,dv]; beta [B,T,H]; S0 [B,H,dk,dv] or None. Returns (o, S_T)."""
+    q, k, v, la, beta, S0 = map(_f64, (q, k, v, log_alpha, beta, S0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dk, dv))
+    rc = _load().kda_oracle_recurrent(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0),
+                                      _ptr(o), _ptr(ST), B, T, H, dk, dv, nthreads,
+                                      MUTATIONS[mutation] if mutation else 0)
+    if rc:
+        raise ValueError("kda_oracle_recurrent: bad sizes")
+    return o, ST
+
+
+def chunkwise(q, k, v, log_alpha, beta, S0=None, C: int = 64, nthreads: int = 0,
+              mutation: str | None = None, debug: bool = False):
+    """fp64 chunkwise reformulation. Returns (o, S_T) or, with debug=True,
+    (o, S_T, A, Tinv) where A and Tinv are [B,H,NC,C,C]."""
+    q, k, v, la, beta, S0 = map(_f64, (q, k, v, log_alpha, beta, S0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    NC = (T + C - 1) // C
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dk, dv))
+    A = np.zeros((B, H, NC, C, C)) if debug else None
+    Ti = np.zeros((B, H, NC, C, C)) if debug else None
+    rc = _load().kda_oracle_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0),
+                                      _ptr(o), _ptr(ST), B, T, H, dk, dv, C, _ptr(A), _ptr(Ti),
+                                      nthreads, MUTATIONS[mutation] if mutation else 0)
+    if rc:
+        raise ValueError("kda_oracle_chunkwise: bad sizes")
+    return (o, ST, A, Ti) if debug else (o, ST)
+
+
+def decode_step(q, k, v, log_alpha, beta, S, nthreads: int = 0):
+    """One recurrent step for [N,H,*] inputs and state S [N,H,dk,dv].
+    Returns (o, S_new)."""
+    q, k, v, la, beta, S = map(_f64, (q, k, v, log_alpha, beta, S))
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((N, H, dv))
+    Sn = np.zeros((N, H, dk, dv))
+    rc = _load().kda_oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S),
+                                        _ptr(Sn), _ptr(o), N, H, dk, dv, nthreads)
+    if rc:
+        raise ValueError("kda_oracle_decode_step: bad sizes")
+    return o, Sn

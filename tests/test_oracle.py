@@ -1,0 +1,132 @@
+"""CPU tests: the fp64 oracle against what the pages and mathematics fix.
+
+P1-P5 are closed forms / special cases of the update rule (tests/pins.py).
+P6: the token recurrence and the chunkwise reformulation agree by brute force
+    for many chunk sizes, ragged tails included (two independent formulations).
+P7: state passing: one call over [0,T) equals two calls chained through S_T.
+P8: T chained single-token decode steps equal the prefill recurrence.
+P9: the chunkwise intermediate T is the inverse of (I + A).
+Mutation test: each planted mistake in the oracle makes at least one pin fail.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from tests import pins
+
+TOL = 1e-12
+
+
+def rec(mutation=None):
+    return lambda q, k, v, la, b, S0: oracle.recurrent(q, k, v, la, b, S0, mutation=mutation)
+
+
+def chk(C, mutation=None):
+    return lambda q, k, v, la, b, S0: oracle.chunkwise(q, k, v, la, b, S0, C=C, mutation=mutation)
+
+
+RUNNERS = {"recurrent": rec(), "chunkwise_c1": chk(1), "chunkwise_c4": chk(4), "chunkwise_c16": chk(16),
+           "chunkwise_c64": chk(64)}
+
+
+@pytest.mark.parametrize("runner", list(RUNNERS))
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
+def test_pins(pin, runner):
+    assert pin(RUNNERS[runner]) < TOL
+
+
+@pytest.mark.parametrize("C", [1, 2, 3, 4, 5, 8, 16, 64])
+@pytest.mark.parametrize("T", [1, 7, 33, 64, 100])
+def test_p6_recurrence_equals_chunkwise(C, T):
+    q, k, v, la, beta, S0 = pins.random_inputs(100 + T + 7 * C, T=T, dk=6, dv=5)
+    o1, s1 = oracle.recurrent(q, k, v, la, beta, S0)
+    o2, s2 = oracle.chunkwise(q, k, v, la, beta, S0, C=C)
+    scale = max(1.0, np.abs(o1).max())
+    assert np.abs(o1 - o2).max() / scale < 1e-12
+    assert np.abs(s1 - s2).max() / max(1.0, np.abs(s1).max()) < 1e-12
+
+
+def test_p6_strong_decay_chunkwise():
+    # Per-token decay up to e^-5: inside a 64-token chunk G reaches about -300,
+    # where the printed K/Gamma form would overflow; the oracle's exponent is
+    # always G_r - G_s <= 0.
+    q, k, v, la, beta, S0 = pins.random_inputs(7, T=130, dk=6, dv=4, la_range=(0.5, 5.0))
+    o1, s1 = oracle.recurrent(q, k, v, la, beta, S0)
+    o2, s2 = oracle.chunkwise(q, k, v, la, beta, S0, C=64)
+    assert np.isfinite(o2).all() and np.isfinite(s2).all()
+    assert np.abs(o1 - o2).max() < 1e-12 and np.abs(s1 - s2).max() < 1e-12
+
+
+@pytest.mark.parametrize("T1", [0, 1, 31, 64, 65])
+def test_p7_state_passing(T1):
+    q, k, v, la, beta, S0 = pins.random_inputs(21, T=97, dk=8, dv=8)
+    o, ST = oracle.recurrent(q, k, v, la, beta, S0)
+    oa, Sa = oracle.chunkwise(q[:, :T1], k[:, :T1], v[:, :T1], la[:, :T1], beta[:, :T1], S0, C=16)
+    ob, Sb = oracle.chunkwise(q[:, T1:], k[:, T1:], v[:, T1:], la[:, T1:], beta[:, T1:], Sa, C=16)
+    assert np.abs(np.concatenate([oa, ob], axis=1) - o).max() < 1e-12
+    assert np.abs(Sb - ST).max() < 1e-12
+
+
+def test_p8_decode_chain_equals_recurrence():
+    q, k, v, la, beta, S0 = pins.random_inputs(22, T=40, dk=8, dv=6, B_=3, H_=2)
+    o, ST = oracle.recurrent(q, k, v, la, beta, S0)
+    S = S0
+    for t in range(q.shape[1]):
+        ot, S = oracle.decode_step(q[:, t], k[:, t], v[:, t], la[:, t], beta[:, t], S)
+        assert np.abs(ot - o[:, t]).max() < 1e-12
+    assert np.abs(S - ST).max() < 1e-12
+
+
+@pytest.mark.parametrize("C", [4, 16, 64])
+def test_p9_inverse(C):
+    q, k, v, la, beta, S0 = pins.random_inputs(23, T=100, dk=8, dv=8)
+    _, _, A, Ti = oracle.chunkwise(q, k, v, la, beta, S0, C=C, debug=True)
+    eye = np.eye(C)
+    res = np.einsum("bhnrs,bhnsj->bhnrj", eye + A, Ti) - eye
+    assert np.abs(res).max() < 1e-12
+    # A strictly lower, T unit lower triangular
+    assert np.abs(np.triu(A)).max() == 0.0
+    assert np.allclose(np.diagonal(Ti, axis1=-2, axis2=-1), 1.0)
+
+
+def test_zero_length_and_empty_batch():
+    q, k, v, la, beta, S0 = pins.random_inputs(24, T=5, dk=4, dv=4)
+    o, ST = oracle.recurrent(q[:, :0], k[:, :0], v[:, :0], la[:, :0], beta[:, :0], S0)
+    assert o.shape == (1, 0, 2, 4) and np.array_equal(ST, S0)
+    o, ST = oracle.chunkwise(q[:, :0], k[:, :0], v[:, :0], la[:, :0], beta[:, :0], S0, C=4)
+    assert np.array_equal(ST, S0)
+
+
+RECURRENT_MUTANTS = ["no_decay", "decay_after", "erase_sign", "read_before", "transposed_read",
+                     "beta_write_only", "decay_columns"]
+CHUNKWISE_MUTANTS = ["prefix_decay_k", "strict_tril_o"]
+
+
+@pytest.mark.parametrize("mutant", RECURRENT_MUTANTS + CHUNKWISE_MUTANTS)
+def test_planted_mistake_is_caught(mutant):
+    run = rec(mutant) if mutant in RECURRENT_MUTANTS else chk(4, mutant)
+    errs = {p.__name__: p(run) for p in pins.ALL_PINS}
+    # the chunkwise-only mistakes are also visible to the brute-force pin P6
+    if mutant in CHUNKWISE_MUTANTS:
+        q, k, v, la, beta, S0 = pins.random_inputs(31, T=20, dk=8, dv=8)
+        o1, s1 = oracle.recurrent(q, k, v, la, beta, S0)
+        o2, s2 = run(q, k, v, la, beta, S0)
+        errs["p6"] = max(np.abs(o1 - o2).max(), np.abs(s1 - s2).max())
+    assert max(errs.values()) > 1e-6, errs
+
+
+def test_hand_worked_example():
+    """Two tokens worked by hand from the update rule (tests/golden)."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_worked_t2_d2.json")))
+    q = np.array(g["q"])[None, :, None]
+    k = np.array(g["k"])[None, :, None]
+    v = np.array(g["v"])[None, :, None]
+    la = np.log(np.array(g["alpha"]))[None, :, None]
+    beta = np.array(g["beta"])[None, :, None]
+    S0 = np.array(g["S0"])[None, None]
+    for run in (rec(), chk(1), chk(2), chk(64)):
+        o, ST = run(q, k, v, la, beta, S0)
+        assert np.abs(o[0, :, 0] - np.array(g["o"])).max() < 1e-12
+        assert np.abs(ST[0, 0] - np.array(g["S_T"])).max() < 1e-12
