@@ -1,0 +1,172 @@
+"""KDA (fine-grained gated delta rule) for B200: Python binding of libkda.so.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/kda.h. PyTorch provides device
+memory and the current CUDA stream. There is no CPU fallback: if the library
+cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = ["load", "chunk_fwd", "decode_step", "workspace_size", "workspace_status", "KDAError",
+           "library_path", "STATUS"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA",
+          4: "KDA_ERR_TIMEOUT"}
+_DTYPE = {"f32": 0, "bf16": 1}
+_ALGO = {"auto": 0, "simt": 1, "tc": 2}
+
+
+class KDAError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} -> {STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load(build_if_stale: bool = True):
+    """Load libkda.so (building it in-tree with nvcc if it is missing or older
+    than its sources). Raises if it cannot be built or loaded."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if build_if_stale:
+        from . import build as _build
+        if not _build.up_to_date():
+            _build.build()
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"libkda.so not found at {_LIB_PATH}; run python -m gated_delta_rule_134_b200.build")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.kda_status_string.argtypes = [I]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_chunk_fwd_workspace_size.argtypes = [I] * 8
+    lib.kda_chunk_fwd_workspace_size.restype = Z
+    lib.kda_chunk_fwd.argtypes = [P] * 8 + [I] * 7 + [P, Z, P]
+    lib.kda_chunk_fwd.restype = I
+    lib.kda_chunk_fwd_ex.argtypes = [P] * 8 + [I] * 7 + [P, Z, I, P]
+    lib.kda_chunk_fwd_ex.restype = I
+    lib.kda_workspace_status.argtypes = [P, Z, P]
+    lib.kda_workspace_status.restype = I
+    lib.kda_decode_step.argtypes = [P] * 8 + [I] * 5 + [P]
+    lib.kda_decode_step.restype = I
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise KDAError(fn, code, load().kda_status_string(code).decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_of(t) -> str:
+    import torch
+    if t.dtype == torch.float32:
+        return "f32"
+    if t.dtype == torch.bfloat16:
+        return "bf16"
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, shape, dtype, device):
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor (this library has no CPU path)")
+    if t.device != device or t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)} on {device}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def workspace_size(B, T, H, dk, dv, chunk=64, dtype="bf16", algo="auto") -> int:
+    return int(load().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, _DTYPE[dtype], _ALGO[algo]))
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, chunk: int = 64, algo: str = "auto",
+              output_final_state: bool = True, o=None, S_T=None, workspace=None, stream=None):
+    """kda_chunk_fwd(q, k, v, log_alpha, beta, S0 -> o, S_T) on CUDA tensors.
+
+    q, k, log_alpha: [B,T,H,dk]; v: [B,T,H,dv]; beta: [B,T,H] (all float32 or
+    all bfloat16); S0: [B,H,dk,dv] float32 or None. Returns (o, S_T) with S_T
+    None when output_final_state is False."""
+    import torch
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt, dev = q.dtype, q.device
+    _need(q, "q", (B, T, H, dk), dt, dev)
+    _need(k, "k", (B, T, H, dk), dt, dev)
+    _need(log_alpha, "log_alpha", (B, T, H, dk), dt, dev)
+    _need(v, "v", (B, T, H, dv), dt, dev)
+    _need(beta, "beta", (B, T, H), dt, dev)
+    if S0 is not None:
+        _need(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=dt, device=dev)
+    _need(o, "o", (B, T, H, dv), dt, dev)
+    if output_final_state and S_T is None:
+        S_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", (B, H, dk, dv), torch.float32, dev)
+    dts = _dtype_of(q)
+    ws_bytes = workspace_size(B, T, H, dk, dv, chunk, dts, algo)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = lib.kda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(o),
+                                _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPE[dts], _ptr(workspace), ws_len,
+                                _ALGO[algo], _stream(stream))
+    _check("kda_chunk_fwd_ex", code)
+    return o, S_T
+
+
+def workspace_status(workspace, stream=None) -> int:
+    """Synchronise and return the device-side status word of a workspace."""
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return int(load().kda_workspace_status(_ptr(workspace), ws_len, _stream(stream)))
+
+
+def decode_step(q, k, v, log_alpha, beta, S, *, S_out=None, o=None, stream=None):
+    """kda_decode_step(q, k, v, log_alpha, beta, S -> o, S'): one token per
+    sequence. q, k, log_alpha [N,H,dk]; v [N,H,dv]; beta [N,H]; S [N,H,dk,dv]
+    float32. S_out defaults to S (in-place update). Returns (o, S_out)."""
+    import torch
+    lib = load()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt, dev = q.dtype, q.device
+    _need(q, "q", (N, H, dk), dt, dev)
+    _need(k, "k", (N, H, dk), dt, dev)
+    _need(log_alpha, "log_alpha", (N, H, dk), dt, dev)
+    _need(v, "v", (N, H, dv), dt, dev)
+    _need(beta, "beta", (N, H), dt, dev)
+    _need(S, "S", (N, H, dk, dv), torch.float32, dev)
+    if S_out is None:
+        S_out = S
+    _need(S_out, "S_out", (N, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=dt, device=dev)
+    _need(o, "o", (N, H, dv), dt, dev)
+    code = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(S_out),
+                               _ptr(o), N, H, dk, dv, _DTYPE[_dtype_of(q)], _stream(stream))
+    _check("kda_decode_step", code)
+    return o, S_out

@@ -1,0 +1,112 @@
+// C-ABI layer of libkda.so: argument validation, workspace sizing and
+// dispatch to the kernels. Declarations and contracts are in include/kda.h.
+#include <stdint.h>
+
+#include "kda.h"
+#include "kda_internal.h"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool head_dims_ok(int dk, int dv) { return dk == dv && (dk == 64 || dk == 128); }
+
+kda_status_t check_chunk_args(const kda::ChunkArgs& a, kda_dtype_t dtype) {
+    if (a.B < 0 || a.T < 0 || a.H < 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (!head_dims_ok(a.dk, a.dv)) return KDA_ERR_UNSUPPORTED;
+    if (a.chunk != 16 && a.chunk != 32 && a.chunk != 64) return KDA_ERR_UNSUPPORTED;
+    if ((long long)a.B * a.H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    const bool has_tokens = (long long)a.B * a.T * a.H > 0;
+    if (has_tokens) {
+        const void* req[] = {a.q, a.k, a.v, a.log_alpha, a.beta, a.o};
+        for (const void* p : req)
+            if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    }
+    if (a.S0 && !aligned16(a.S0)) return KDA_ERR_INVALID_ARG;
+    if (a.ST && !aligned16(a.ST)) return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_status_string(kda_status_t s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: null/misaligned pointer, bad size or workspace too small";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: head size, chunk size or algorithm not implemented";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA launch or query failed";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device-side wait expired";
+    }
+    return "KDA: unknown status";
+}
+
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, kda_dtype_t dtype,
+                                    kda_algo_t algo) {
+    kda::ChunkArgs a{};
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
+    if (B < 0 || T < 0 || H < 0 || !head_dims_ok(dk, dv)) return 0;
+    const bool tc = (algo == KDA_ALGO_TC) || (algo == KDA_ALGO_AUTO && kda::chunk_tc_supported(a));
+    return tc ? kda::chunk_tc_workspace_bytes(B, T, H, dk, dv) : 0;
+}
+
+kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                              const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
+                              kda_dtype_t dtype, void* workspace, size_t workspace_bytes, kda_algo_t algo,
+                              void* stream) {
+    kda::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+    kda_status_t st = check_chunk_args(a, dtype);
+    if (st != KDA_OK) return st;
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TC) return KDA_ERR_INVALID_ARG;
+    const bool tc = (algo == KDA_ALGO_TC) || (algo == KDA_ALGO_AUTO && kda::chunk_tc_supported(a));
+    if (tc && !kda::chunk_tc_supported(a)) return KDA_ERR_UNSUPPORTED;
+    if (tc) {
+        const size_t need = kda::chunk_tc_workspace_bytes(B, T, H, dk, dv);
+        if (need > 0 && (workspace == nullptr || workspace_bytes < need ||
+                         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+            return KDA_ERR_INVALID_ARG;
+    }
+    if ((long long)B * H == 0) return KDA_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t err = tc ? kda::launch_chunk_tc(a, s) : kda::launch_chunk_simt(a, s);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                           const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
+                           kda_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    return kda_chunk_fwd_ex(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, dk, dv, chunk, dtype, workspace,
+                            workspace_bytes, KDA_ALGO_AUTO, stream);
+}
+
+kda_status_t kda_workspace_status(const void* workspace, size_t workspace_bytes, void* stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
+    if (workspace == nullptr || workspace_bytes < sizeof(unsigned)) return KDA_OK;
+    unsigned flag = 0;
+    if (cudaMemcpy(&flag, workspace, sizeof(flag), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+    return flag ? KDA_ERR_TIMEOUT : KDA_OK;
+}
+
+kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                             const float* S_in, float* S_out, void* o, int N, int H, int dk, int dv,
+                             kda_dtype_t dtype, void* stream) {
+    if (N < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (!head_dims_ok(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if ((long long)N * H * (dv / 32) > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    if ((long long)N * H == 0) return KDA_OK;
+    const void* req[] = {q, k, v, log_alpha, beta, S_in, S_out, o};
+    for (const void* p : req)
+        if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    const cudaError_t err = kda::launch_decode(q, k, v, log_alpha, beta, S_in, S_out, o, N, H, dk, dv,
+                                               dtype == KDA_BF16, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,31 @@
+// Internal launch interface between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace kda {
+
+struct ChunkArgs {
+    const void *q, *k, *v, *log_alpha, *beta;
+    const float* S0;
+    void* o;
+    float* ST;
+    int B, T, H, dk, dv, chunk;
+    int bf16;
+    void* workspace;
+    size_t workspace_bytes;
+};
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* la, const void* beta,
+                          const float* S_in, float* S_out, void* o, int N, int H, int dk, int dv, int bf16,
+                          cudaStream_t stream);
+
+cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t stream);
+
+// Fused tensor-core prefill (bf16, dk = dv = 128, chunk = 64).
+bool chunk_tc_supported(const ChunkArgs& a);
+size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv);
+cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t stream);
+
+}  // namespace kda

@@ -1,0 +1,134 @@
+/*
+ * kda.h -- C ABI of libkda.so: KDA (fine-grained gated delta rule) chunkwise
+ * prefill and single-token decode on NVIDIA B200 (sm_100a).
+ *
+ * The operation (pages: "Decoding Hybrid Attention Architectures", section
+ * 3.4 and its variant table; "Technical Analysis ... Novel Hybrid Linear
+ * Attention", section 2 item 4), per sequence and head, token by token:
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * with state S in R^{dk x dv} (row i = key channel i), alpha_t = exp(log_alpha_t)
+ * taken elementwise (no activation is applied to log_alpha), and no scaling of q.
+ * The prefill computes this with the chunkwise-parallel form of section 4 of
+ * the first page (intra-chunk lower-triangular products, inter-chunk state
+ * passing, precomputed U and W); the decode step is the update for one token
+ * ("Decoding Hybrid Attention Architectures", sections 1 and 5: constant
+ * state, cost independent of context length).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, row-major and contiguous, with
+ *     the base address aligned to 16 bytes. The caller owns every buffer.
+ *   - dtype selects the element type of q, k, v, log_alpha, beta and o:
+ *     KDA_F32 (float) or KDA_BF16 (__nv_bfloat16). States are always float.
+ *   - Nothing is allocated and nothing is synchronised: all work is enqueued
+ *     on `stream` (a cudaStream_t; NULL = the legacy default stream) and the
+ *     call returns once it is enqueued.
+ *   - Arguments are validated before anything is launched. A call that
+ *     returns anything but KDA_OK has launched nothing and written nothing,
+ *     except KDA_ERR_CUDA, which reports a launch failure.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, workspace too small */
+    KDA_ERR_UNSUPPORTED = 2, /* valid but not implemented (head size, chunk size, dtype) */
+    KDA_ERR_CUDA = 3,        /* a CUDA launch or query failed; see cudaGetLastError */
+    KDA_ERR_TIMEOUT = 4      /* a bounded device-side wait expired (reported by kda_workspace_status) */
+} kda_status_t;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
+
+/* Which prefill kernels to run. AUTO picks the fused tensor-core kernel when
+ * it supports the shape (bf16, dk = dv = 128, chunk = 64) and the SIMT fp32
+ * kernel otherwise. */
+typedef enum { KDA_ALGO_AUTO = 0, KDA_ALGO_SIMT = 1, KDA_ALGO_TC = 2 } kda_algo_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kda_status_string(kda_status_t status);
+
+/*
+ * Bytes of device workspace kda_chunk_fwd_ex needs for this shape and
+ * algorithm (0 on invalid arguments). The workspace is scratch owned by the
+ * caller, at least 256-byte aligned; its contents need not be initialised and
+ * are overwritten by every call. Two calls in flight at once must not share
+ * a workspace.
+ */
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, kda_dtype_t dtype,
+                                    kda_algo_t algo);
+
+/*
+ * Chunkwise prefill: kda_chunk_fwd(q, k, v, log_alpha, beta, S0 -> o, S_T).
+ *
+ *   q, k, log_alpha : [B, T, H, dk]   dtype
+ *   v               : [B, T, H, dv]   dtype
+ *   beta            : [B, T, H]       dtype, the write strength in (0, 1]
+ *   S0              : [B, H, dk, dv]  float, initial state; NULL means zero
+ *   o               : [B, T, H, dv]   dtype, written
+ *   S_T             : [B, H, dk, dv]  float, final state; NULL means not written
+ *                                     (may equal S0: read fully before written)
+ *   chunk           : tokens per chunk, one of 16, 32, 64 (64 is the tuned size)
+ *   dk, dv          : 64 or 128, dk == dv
+ *   T               : any T >= 0; a ragged last chunk is handled exactly
+ *                     (as if padded with k = q = v = 0, beta = 0, log_alpha = 0)
+ *   workspace       : device scratch of at least
+ *                     kda_chunk_fwd_workspace_size(...) bytes (may be NULL when
+ *                     that size is 0)
+ *
+ * Numerics: state and accumulation in fp32. With dtype KDA_F32 and the SIMT
+ * algorithm every product is fp32. The tensor-core algorithm rounds MMA
+ * operands (decay-scaled keys and queries, the UT inverse, W, the state copy
+ * that feeds the next chunk) to bf16 and accumulates in fp32.
+ * Returns KDA_OK once enqueued.
+ */
+kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const void *log_alpha,
+                           const void *beta, const float *S0, void *o, float *S_T, int B, int T, int H,
+                           int dk, int dv, int chunk, kda_dtype_t dtype, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+/* kda_chunk_fwd with an explicit algorithm. KDA_ALGO_TC returns
+ * KDA_ERR_UNSUPPORTED for shapes it does not cover. */
+kda_status_t kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *log_alpha,
+                              const void *beta, const float *S0, void *o, float *S_T, int B, int T, int H,
+                              int dk, int dv, int chunk, kda_dtype_t dtype, void *workspace,
+                              size_t workspace_bytes, kda_algo_t algo, void *stream);
+
+/*
+ * Device-side status left in `workspace` by the last kda_chunk_fwd_ex that
+ * used it: synchronises `stream`, then returns KDA_OK, or KDA_ERR_TIMEOUT if
+ * a bounded wait inside a kernel gave up (that kernel's outputs are then
+ * invalid), or KDA_ERR_CUDA if the stream reported an error.
+ */
+kda_status_t kda_workspace_status(const void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One recurrent decode step: kda_decode_step(q, k, v, log_alpha, beta, S -> o, S').
+ *
+ *   q, k, log_alpha : [N, H, dk]      dtype
+ *   v               : [N, H, dv]      dtype
+ *   beta            : [N, H]          dtype
+ *   S_in            : [N, H, dk, dv]  float
+ *   S_out           : [N, H, dk, dv]  float, may equal S_in (in-place update)
+ *   o               : [N, H, dv]      dtype
+ *   dk, dv          : 64 or 128 (dk == dv)
+ * Per head: S' = Diag(alpha) S; delta = beta (v - S'^T k); S_out = S' + k delta^T;
+ * o = S_out^T q. State arithmetic in fp32.
+ */
+kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const void *log_alpha,
+                             const void *beta, const float *S_in, float *S_out, void *o, int N, int H,
+                             int dk, int dv, kda_dtype_t dtype, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,135 @@
+"""CPU tests of the C-ABI boundary: the library loads, exports every function
+declared in include/kda.h, and rejects bad arguments with a status code before
+touching the GPU. Only argument combinations that fail validation are passed
+here (they return before any CUDA call), so nothing runs on a device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_134_b200 as kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = kda.load()
+    names = declared_functions()
+    assert "kda_chunk_fwd" in names and "kda_decode_step" in names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    lib = kda.load()
+    for code in range(5):
+        s = lib.kda_status_string(code).decode()
+        assert s.startswith(kda.STATUS[code])
+
+
+def _chunk(lib, ptrs, B=1, T=4, H=1, dk=64, dv=64, chunk=64, dtype=1, ws=None, ws_len=0, algo=0):
+    q, k, v, la, beta, S0, o, ST = ptrs
+    return lib.kda_chunk_fwd_ex(q, k, v, la, beta, S0, o, ST, B, T, H, dk, dv, chunk, dtype, ws, ws_len, algo,
+                                None)
+
+
+GOOD = [ctypes.c_void_p(0x1000 * (i + 1)) for i in range(5)] + [None, ctypes.c_void_p(0x7000), None]
+
+
+@pytest.mark.parametrize("which", range(5))
+def test_chunk_rejects_null_input(which):
+    lib = kda.load()
+    ptrs = list(GOOD)
+    ptrs[which] = None
+    assert _chunk(lib, ptrs) == 1
+
+
+def test_chunk_rejects_null_output():
+    lib = kda.load()
+    ptrs = list(GOOD)
+    ptrs[6] = None
+    assert _chunk(lib, ptrs) == 1
+
+
+def test_chunk_rejects_misaligned():
+    lib = kda.load()
+    ptrs = list(GOOD)
+    ptrs[2] = ctypes.c_void_p(0x3008)
+    assert _chunk(lib, ptrs) == 1
+    ptrs = list(GOOD)
+    ptrs[5] = ctypes.c_void_p(0x9004)  # S0
+    assert _chunk(lib, ptrs) == 1
+
+
+@pytest.mark.parametrize("dk,dv", [(32, 32), (64, 128), (96, 96), (256, 256)])
+def test_chunk_rejects_unsupported_head_size(dk, dv):
+    lib = kda.load()
+    assert _chunk(lib, GOOD, dk=dk, dv=dv) == 2
+
+
+@pytest.mark.parametrize("chunk", [0, 8, 48, 128])
+def test_chunk_rejects_unsupported_chunk(chunk):
+    lib = kda.load()
+    assert _chunk(lib, GOOD, chunk=chunk) == 2
+
+
+def test_chunk_rejects_bad_sizes_and_enums():
+    lib = kda.load()
+    assert _chunk(lib, GOOD, B=-1) == 1
+    assert _chunk(lib, GOOD, T=-3) == 1
+    assert _chunk(lib, GOOD, dtype=7) == 1
+    assert _chunk(lib, GOOD, algo=9) == 1
+
+
+def test_tc_path_rejects_shapes_it_does_not_cover():
+    lib = kda.load()
+    assert _chunk(lib, GOOD, dtype=0, dk=128, dv=128, algo=2) == 2   # fp32
+    assert _chunk(lib, GOOD, dtype=1, dk=64, dv=64, algo=2) == 2     # d = 64
+    assert _chunk(lib, GOOD, dtype=1, dk=128, dv=128, chunk=32, algo=2) == 2
+
+
+def test_workspace_size_is_host_only():
+    lib = kda.load()
+    assert lib.kda_chunk_fwd_workspace_size(1, 16, 1, 64, 64, 64, 0, 1) == 0   # SIMT needs none
+    assert lib.kda_chunk_fwd_workspace_size(1, 16, 1, 48, 48, 64, 0, 0) == 0   # invalid -> 0
+
+
+def test_decode_rejects_bad_args():
+    lib = kda.load()
+    p = [ctypes.c_void_p(0x1000 * (i + 1)) for i in range(8)]
+    f = lib.kda_decode_step
+    for i in range(8):
+        pp = list(p)
+        pp[i] = None
+        assert f(*pp, 2, 2, 128, 128, 1, None) == 1
+    pp = list(p)
+    pp[5] = ctypes.c_void_p(0x6004)
+    assert f(*pp, 2, 2, 128, 128, 1, None) == 1
+    assert f(*p, 2, 2, 96, 96, 1, None) == 2
+    assert f(*p, 2, 2, 128, 64, 1, None) == 2
+    assert f(*p, -1, 2, 128, 128, 1, None) == 1
+    assert f(*p, 2, 2, 128, 128, 5, None) == 1
+
+
+def test_binding_has_no_cpu_fallback():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(1, 4, 1, 64)
+    b = torch.zeros(1, 4, 1)
+    v = torch.zeros(1, 4, 1, 64)
+    # CPU tensors are refused before any call into the library: there is no CPU path.
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kda.chunk_fwd(x, x, v, x, b)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kda.decode_step(x[:, 0], x[:, 0], v[:, 0], x[:, 0], b[:, 0], torch.zeros(1, 1, 64, 64))

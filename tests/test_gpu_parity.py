@@ -1,0 +1,229 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs. Error metric: max|x - ref| / max|ref| over the compared
+elements, separately for o and for the final state. Bars: 1e-4 for fp32
+inputs, 2e-2 for bf16 inputs with fp32 state/accumulation.
+
+bf16 workloads hand the oracle the same bf16-rounded values (upcast to fp64),
+so the measured error is the kernels' own.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_134_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def rel_err(x, ref):
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.abs(ref).max()
+    return float(np.abs(x - ref).max() / (den if den > 0 else 1.0))
+
+
+def to_dev(d):
+    return {k: (None if v is None else v.cuda()) for k, v in d.items()}
+
+
+def algos_for(cfg):
+    out = ["simt"]
+    if cfg.dtype == "bf16" and cfg.dk == 128 and cfg.dv == 128 and cfg.C == 64:
+        out.append("tc")
+    return out
+
+
+def small_cfg(dtype, d, C, T, B=2, H=3, la=(0.01, 1.0), s0=0.3, seed=7):
+    return I.PrefillConfig(f"small_{dtype}_{d}_{C}_{T}", B, H, T, d, d, C, dtype, la[0], la[1], s0, seed)
+
+
+def check_prefill(kda, cfg, algo, heads=None):
+    x = I.prefill_inputs(cfg)
+    xd = to_dev(x)
+    o, ST = kda.chunk_fwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["S0"], chunk=cfg.C, algo=algo)
+    torch.cuda.synchronize()
+    if heads is None:
+        ref_o, ref_S = oracle.recurrent(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"])
+        got_o, got_S = o.float().cpu().numpy(), ST.cpu().numpy()
+    else:
+        xs = I.prefill_inputs(cfg, heads=heads)
+        ref_o, ref_S = oracle.recurrent(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["beta"], xs["S0"])
+        oc, Sc = o.float().cpu(), ST.cpu()
+        got_o = np.stack([oc[b, :, h].numpy() for b, h in heads])[:, :, None]
+        got_S = np.stack([Sc[b, h].numpy() for b, h in heads])[:, None]
+    eo, es = rel_err(got_o, ref_o), rel_err(got_S, ref_S)
+    assert np.isfinite(got_o).all() and np.isfinite(got_S).all()
+    assert eo <= TOL[cfg.dtype] and es <= TOL[cfg.dtype], (cfg.name, algo, eo, es)
+    return eo, es
+
+
+# ---------------------------------------------------------------- prefill, small
+
+
+@pytest.mark.parametrize("T", [1, 17, 64, 65, 130, 333])
+@pytest.mark.parametrize("C", [16, 32, 64])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_prefill_small_simt(cuda_lib, dtype, d, C, T):
+    check_prefill(cuda_lib, small_cfg(dtype, d, C, T), "simt")
+
+
+@pytest.mark.parametrize("s0", [0.0, 0.3])
+@pytest.mark.parametrize("T", [1, 17, 63, 64, 65, 130, 333, 1000])
+def test_prefill_small_tc(cuda_lib, T, s0):
+    check_prefill(cuda_lib, small_cfg("bf16", 128, 64, T, s0=s0), "tc")
+
+
+@pytest.mark.parametrize("algo", ["simt", "tc"])
+@pytest.mark.parametrize("la", [(1.0, 8.0), (0.0, 0.0), (0.0, 1e-4)])
+def test_prefill_decay_extremes(cuda_lib, algo, la):
+    # strong decay (exercises the overflow-safe path of the tensor-core kernel),
+    # no decay at all, and nearly none
+    check_prefill(cuda_lib, small_cfg("bf16", 128, 64, 200, la=la), algo)
+
+
+@pytest.mark.parametrize("algo", ["simt", "tc"])
+def test_prefill_many_heads_small(cuda_lib, algo):
+    # more (b, h) pairs than SMs, ragged tail
+    check_prefill(cuda_lib, small_cfg("bf16", 128, 64, 77, B=3, H=70, seed=9), algo)
+
+
+# ---------------------------------------------------------------- prefill, edge cases
+
+
+@pytest.mark.parametrize("algo", ["simt", "tc"])
+def test_prefill_empty_sequence_copies_state(cuda_lib, algo):
+    cfg = small_cfg("bf16", 128, 64, 0)
+    x = to_dev(I.prefill_inputs(cfg))
+    o, ST = cuda_lib.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], algo=algo)
+    torch.cuda.synchronize()
+    assert o.numel() == 0
+    assert torch.equal(ST, x["S0"])
+    o, ST = cuda_lib.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, algo=algo)
+    assert torch.count_nonzero(ST).item() == 0
+
+
+def test_prefill_empty_batch(cuda_lib):
+    z = torch.empty(0, 5, 2, 128, dtype=torch.bfloat16, device="cuda")
+    o, ST = cuda_lib.chunk_fwd(z, z, z, z, torch.empty(0, 5, 2, dtype=torch.bfloat16, device="cuda"))
+    assert o.shape == (0, 5, 2, 128) and ST.shape == (0, 2, 128, 128)
+
+
+@pytest.mark.parametrize("algo", ["simt", "tc"])
+def test_prefill_state_in_place_and_chaining(cuda_lib, algo):
+    cfg = small_cfg("bf16", 128, 64, 300)
+    x = to_dev(I.prefill_inputs(cfg))
+    o_full, S_full = cuda_lib.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], algo=algo)
+    S = x["S0"].clone()
+    outs = []
+    for a, b in [(0, 100), (100, 101), (101, 300)]:
+        sl = {kk: x[kk][:, a:b].contiguous() for kk in ("q", "k", "v", "log_alpha", "beta")}
+        o, _ = cuda_lib.chunk_fwd(sl["q"], sl["k"], sl["v"], sl["log_alpha"], sl["beta"], S, S_T=S, algo=algo)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert rel_err(torch.cat(outs, 1).float().cpu(), o_full.float().cpu()) < 2e-2
+    assert rel_err(S.cpu(), S_full.cpu()) < 2e-2
+
+
+@pytest.mark.parametrize("algo", ["simt", "tc"])
+def test_prefill_deterministic(cuda_lib, algo):
+    cfg = small_cfg("bf16", 128, 64, 257)
+    x = to_dev(I.prefill_inputs(cfg))
+    r1 = cuda_lib.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], algo=algo)
+    r2 = cuda_lib.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], algo=algo)
+    torch.cuda.synchronize()
+    assert torch.equal(r1[0], r2[0]) and torch.equal(r1[1], r2[1])
+
+
+def test_prefill_no_final_state(cuda_lib):
+    cfg = small_cfg("f32", 64, 64, 70)
+    x = to_dev(I.prefill_inputs(cfg))
+    o, ST = cuda_lib.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"],
+                               output_final_state=False)
+    assert ST is None
+    ref, _ = oracle.recurrent(*[I.prefill_inputs(cfg)[kk] for kk in ("q", "k", "v", "log_alpha", "beta", "S0")])
+    assert rel_err(o.cpu().numpy(), ref) < 1e-4
+
+
+# ---------------------------------------------------------------- prefill, full-size workloads
+
+
+def test_prefill_small_f32_full(cuda_lib):
+    check_prefill(cuda_lib, I.SMALL_F32, "auto")
+
+
+@pytest.mark.parametrize("algo", ["auto", "simt"])
+def test_prefill_b2_h16_t4k(cuda_lib, algo):
+    check_prefill(cuda_lib, I.B2_H16_T4K, algo, heads=[(0, 0), (0, 7), (1, 3), (1, 15)])
+
+
+def test_prefill_b4_h32_t8k(cuda_lib):
+    check_prefill(cuda_lib, I.B4_H32_T8K, "auto", heads=[(0, 0), (0, 31), (1, 5), (2, 17), (3, 2), (3, 30)])
+
+
+def test_prefill_b1_h32_t128k(cuda_lib):
+    check_prefill(cuda_lib, I.B1_H32_T128K, "auto", heads=[(0, 0), (0, 13), (0, 31)])
+
+
+# ---------------------------------------------------------------- decode
+
+
+@pytest.mark.parametrize("inplace", [True, False])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_small_chain(cuda_lib, dtype, d, inplace):
+    cfg = I.DecodeConfig("decode_small", 5, 3, d, d, 30, dtype, 0.001, 0.5, 0.1, 3)
+    S_ref = I.decode_state(cfg).double().numpy()
+    S = I.decode_state(cfg).cuda()
+    for step in range(cfg.steps):
+        x = I.decode_step_inputs(cfg, step)
+        xd = to_dev(x)
+        S_out = S if inplace else torch.empty_like(S)
+        o, S_new = cuda_lib.decode_step(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], S, S_out=S_out)
+        o_ref, S_ref = oracle.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S_ref)
+        assert rel_err(o.float().cpu().numpy(), o_ref) <= TOL[dtype]
+        S = S_new
+    torch.cuda.synchronize()
+    assert rel_err(S.cpu().numpy(), S_ref) <= TOL[dtype]
+
+
+def test_decode_full_first_step_all_heads(cuda_lib):
+    cfg = I.DECODE_N256_H32
+    S0 = I.decode_state(cfg)
+    x = I.decode_step_inputs(cfg, 0)
+    xd = to_dev(x)
+    S = S0.cuda()
+    o, S = cuda_lib.decode_step(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], S)
+    o_ref, S_ref = oracle.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S0)
+    assert rel_err(o.float().cpu().numpy(), o_ref) <= TOL["bf16"]
+    assert rel_err(S.cpu().numpy(), S_ref) <= TOL["bf16"]
+
+
+def test_decode_full_1000_steps_sampled_heads(cuda_lib):
+    """All 1000 chained in-place steps on the full [256,32,128,128] state; the
+    oracle follows 64 seeded heads (heads are independent, so this is exact
+    for the sample)."""
+    cfg = I.DECODE_N256_H32
+    rng = np.random.default_rng(1234)
+    idx = rng.choice(cfg.N * cfg.H, size=64, replace=False)
+    heads = [(int(i) // cfg.H, int(i) % cfg.H) for i in idx]
+    nn = torch.tensor([n for n, _ in heads])
+    hh = torch.tensor([h for _, h in heads])
+    S_full = I.decode_state(cfg)
+    S_ref = S_full[nn, hh].double().numpy()[:, None]
+    S = S_full.cuda()
+    del S_full
+    worst = 0.0
+    for step in range(cfg.steps):
+        x = I.decode_step_inputs(cfg, step)
+        xd = to_dev(x)
+        o, S = cuda_lib.decode_step(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], S)
+        xs = {kk: x[kk][nn, hh][:, None] for kk in x}
+        o_ref, S_ref = oracle.decode_step(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["beta"], S_ref)
+        worst = max(worst, rel_err(o[nn.cuda(), hh.cuda()].float().cpu().numpy()[:, None], o_ref))
+    torch.cuda.synchronize()
+    assert worst <= TOL["bf16"]
+    assert rel_err(S[nn.cuda(), hh.cuda()].cpu().numpy()[:, None], S_ref) <= TOL["bf16"]
