@@ -90,11 +90,21 @@ class ClockSampler:
                 "samples": len(self.rows)}
 
 
-def kernel_source_digest():
-    import glob
+# Source files each profiled kernel is built from: a recorded ncu traffic
+# figure is reported only while these files are unchanged.
+KERNEL_SOURCES = {
+    "decode": ["kda_decode.cu", "kda_common.cuh"],
+    "simt": ["kda_chunk_simt.cu", "kda_common.cuh"],
+    "tc": ["kda_chunk_tc.cu", "kda_common.cuh", "kda_sm100.cuh"],
+}
+
+
+def kernel_source_digest(kind: str) -> str:
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "gated_delta_rule_134_b200", "csrc", "*"))):
-        h.update(open(p, "rb").read())
+    for name in KERNEL_SOURCES[kind]:
+        p = os.path.join(ROOT, "gated_delta_rule_134_b200", "csrc", name)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -107,7 +117,7 @@ def recorded_traffic(workload: str, algo: str):
     try:
         d = json.load(open(p))
         e = d.get(f"{workload}/{algo}")
-        if e and e.get("source_digest") == kernel_source_digest():
+        if e and e.get("source_digest") == kernel_source_digest(algo):
             return e.get("dram_bytes_per_launch")
     except Exception:
         return None
@@ -162,6 +172,192 @@ def run_reference(args):
     return 0
 
 
+class Ctx:
+    """Per-process distributed context (one rank per GPU)."""
+
+    def __init__(self):
+        import torch
+        import torch.distributed as dist
+        self.torch, self.dist = torch, dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(self.local)
+        if self.world > 1:
+            import datetime
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        self.dev = torch.device("cuda", self.local)
+        self.stream = torch.cuda.current_stream(self.dev)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max_over_ranks(self, x: float) -> float:
+        if self.world == 1:
+            return x
+        t = self.torch.tensor([x], dtype=self.torch.float64, device=self.dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
+class Prefill:
+    """The B=4, H=32, T=8192 bf16 prefill workload resident on this rank's GPU."""
+
+    def __init__(self, ctx, kda, I, algo):
+        torch = ctx.torch
+        self.kda, self.ctx, self.algo = kda, ctx, algo
+        base = I.B4_H32_T8K
+        self.cfg = cfg = base.replace(seed=base.seed + 1000 * ctx.rank)
+        self.name = base.name
+        self.x = {k: (None if v is None else v.to(ctx.dev)) for k, v in I.prefill_inputs(cfg).items()}
+        B, T, H, dk, dv = cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv
+        self.o = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=ctx.dev)
+        self.ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=ctx.dev)
+        self.ws_bytes = kda.workspace_size(B, T, H, dk, dv, cfg.C, "bf16", algo)
+        self.ws = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=ctx.dev)
+        self.use_tc = algo == "tc" or (algo == "auto" and self.ws_bytes > 0)
+        self.algo_name = "tc" if self.use_tc else "simt"
+        self.launches_per_step = 1
+        self.tokens_per_step = B * T
+
+    def run(self, x=None):
+        x = x or self.x
+        self.kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], chunk=self.cfg.C,
+                           algo=self.algo, o=self.o, S_T=self.ST, workspace=self.ws if self.ws_bytes else None,
+                           stream=self.ctx.stream)
+
+    def algorithmic_bytes(self):
+        cfg = self.cfg
+        state = self.ST.numel() * 4 * (2 if self.x["S0"] is not None else 1)
+        return BYTES_PER_TOKEN_HEAD * cfg.B * cfg.T * cfg.H + state
+
+    def algorithmic_flops(self):
+        cfg = self.cfg
+        return FLOPS_PER_TOKEN_HEAD * cfg.B * cfg.T * cfg.H
+
+
+def time_prefill(args, ctx, pf, peaks, peak_kind):
+    torch = ctx.torch
+    for _ in range(args.warmup):
+        pf.run()
+    torch.cuda.synchronize()
+    ctx.barrier()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
+    with ClockSampler(ctx.local) as clk:
+        for i in range(args.steps):
+            ev[2 * i].record(ctx.stream)
+            pf.run()
+            ev[2 * i + 1].record(ctx.stream)
+        torch.cuda.synchronize()
+    ctx.barrier()
+    total_ms = ctx.max_over_ranks(ev[0].elapsed_time(ev[-1]))
+    per_launch = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps)]
+    avg_launch_ms = ctx.max_over_ranks(sum(per_launch) / len(per_launch))
+    if pf.use_tc and pf.kda.workspace_status(pf.ws, ctx.stream) != 0:
+        raise RuntimeError("device-side timeout reported by the prefill kernel")
+    ms_per_step = total_ms / args.steps
+    alg_bytes = pf.algorithmic_bytes()
+    achieved = alg_bytes / (avg_launch_ms * 1e-3) / 1e9
+    tflops = pf.algorithmic_flops() / (avg_launch_ms * 1e-3) / 1e12
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic(pf.name, pf.algo_name),
+                "peak_source": ("of measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                                else "of fallback"),
+                "kernel": "kda_chunk_tc_kernel" if pf.use_tc else "chunk_simt_kernel",
+                "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": avg_launch_ms,
+                "tensor": {"achieved_tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
+                           "frac": tflops / peaks["bf16_tflops"],
+                           "algorithmic_flops_per_launch": pf.algorithmic_flops()}}
+    return ms_per_step, roofline, clk.summary()
+
+
+def time_e2e(args, ctx, pf):
+    """Same metric through the C ABI with host buffers: every step copies its
+    inputs host->device from pinned memory and reads o and S_T back."""
+    torch = ctx.torch
+    pin = {k: (None if v is None else v.cpu().pin_memory()) for k, v in pf.x.items()}
+    dbuf = {k: (None if v is None else torch.empty_like(v)) for k, v in pf.x.items()}
+    o_host = torch.empty(pf.o.shape, dtype=pf.o.dtype, pin_memory=True)
+    ST_host = torch.empty(pf.ST.shape, dtype=pf.ST.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in pin.values() if v is not None)
+    d2h = o_host.numel() * o_host.element_size() + ST_host.numel() * ST_host.element_size()
+
+    def step():
+        for k in pin:
+            if pin[k] is not None:
+                dbuf[k].copy_(pin[k], non_blocking=True)
+        pf.run(dbuf)
+        o_host.copy_(pf.o, non_blocking=True)
+        ST_host.copy_(pf.ST, non_blocking=True)
+
+    n = max(3, min(args.steps, 10))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    ctx.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(ctx.stream)
+    for _ in range(n):
+        step()
+    e1.record(ctx.stream)
+    torch.cuda.synchronize()
+    ms = ctx.max_over_ranks(e0.elapsed_time(e1) / n)
+    return {"value": ctx.world * pf.tokens_per_step / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n,
+            "path": "pinned host -> device copies, kda_chunk_fwd, device -> pinned host copies of o and S_T"}
+
+
+def time_decode(args, ctx, kda, I, peaks, peak_kind):
+    """N=256 x H=32, d=128 decode: chained in-place steps with fresh inputs
+    each step (pre-generated on the device by torch's seeded generator)."""
+    torch = ctx.torch
+    dcfg = I.DECODE_N256_H32
+    nd = args.decode_steps
+    g = torch.Generator(device=ctx.dev)
+    g.manual_seed(dcfg.seed + 1000 * ctx.rank)
+    S = dcfg.s_std * torch.randn(dcfg.N, dcfg.H, dcfg.dk, dcfg.dv, device=ctx.dev, generator=g)
+
+    def unit(z):
+        return z / z.norm(dim=-1, keepdim=True)
+
+    shp = (nd, dcfg.N, dcfg.H)
+    dq = unit(torch.randn(*shp, dcfg.dk, device=ctx.dev, generator=g)).bfloat16()
+    dk = unit(torch.randn(*shp, dcfg.dk, device=ctx.dev, generator=g)).bfloat16()
+    dv = torch.randn(*shp, dcfg.dv, device=ctx.dev, generator=g).bfloat16()
+    dla = (-(dcfg.la_lo + (dcfg.la_hi - dcfg.la_lo) * torch.rand(*shp, dcfg.dk, device=ctx.dev,
+                                                                   generator=g))).bfloat16()
+    db = torch.sigmoid(torch.randn(*shp, device=ctx.dev, generator=g)).bfloat16()
+    do = torch.empty(dcfg.N, dcfg.H, dcfg.dv, dtype=torch.bfloat16, device=ctx.dev)
+    for i in range(min(3, nd)):
+        kda.decode_step(dq[i], dk[i], dv[i], dla[i], db[i], S, o=do, stream=ctx.stream)
+    torch.cuda.synchronize()
+    ctx.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(ctx.local) as clk:
+        e0.record(ctx.stream)
+        for i in range(nd):
+            kda.decode_step(dq[i], dk[i], dv[i], dla[i], db[i], S, o=do, stream=ctx.stream)
+        e1.record(ctx.stream)
+        torch.cuda.synchronize()
+    ms = ctx.max_over_ranks(e0.elapsed_time(e1))
+    us = ms * 1e3 / nd
+    nbytes = 2 * S.numel() * 4 + (3 * dq[0].numel() + dv[0].numel() + db[0].numel() + do.numel()) * 2
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"workload": dcfg.name, "value": ctx.world * gbs, "unit": "GB/s", "us_per_step": us, "steps": nd,
+            "algorithmic_bytes_per_step": nbytes, "gpu_launches": nd,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "kernel": "decode_step_kernel",
+                         "peak_source": "of measured" if peak_kind == "measured" else "of fallback",
+                         "traffic": recorded_traffic(dcfg.name, "decode")},
+            "clocks": clk.summary(), "inputs": "pre-generated on the device, fresh each step"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -171,185 +367,50 @@ def main():
     ap.add_argument("--algo", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--parts", default="prefill,e2e,decode",
+                    help="comma list of prefill, e2e, decode (profiling runs select one)")
     args = ap.parse_args()
+    args.parts = set(args.parts.split(","))
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
 
-    import torch
-    import torch.distributed as dist
-
     import gated_delta_rule_134_b200 as kda
     from gated_delta_rule_134_b200 import inputs as I
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = torch.device("cuda", local)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
+    ctx = Ctx()
     kda.load()
     peaks, peak_kind = load_peaks()
-    cfg = I.B4_H32_T8K.replace(seed=I.B4_H32_T8K.seed + 1000 * rank)
-    x = {k: (None if v is None else v.to(dev)) for k, v in I.prefill_inputs(cfg).items()}
-    B, T, H, dk, dv = cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv
-    o = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=dev)
-    ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
-    ws_bytes = kda.workspace_size(B, T, H, dk, dv, cfg.C, "bf16", args.algo)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    use_tc = args.algo == "tc" or (args.algo == "auto" and ws_bytes > 0)
-    algo_name = "tc" if use_tc else "simt"
-    launches_per_step = 1
-
-    def step():
-        kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], chunk=cfg.C, algo=args.algo,
-                      o=o, S_T=ST, workspace=ws if ws_bytes else None, stream=stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
-    with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            ev[2 * i].record(stream)
-            step()
-            ev[2 * i + 1].record(stream)
-        torch.cuda.synchronize()
-    barrier()
-    per_launch_ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps)]
-    total_ms = ev[0].elapsed_time(ev[-1])
-    total_ms = max_over_ranks(total_ms)
-    avg_launch_ms = max_over_ranks(sum(per_launch_ms) / len(per_launch_ms))
-    ms_per_step = total_ms / args.steps
-    tokens_per_step = B * T
-    value = world * tokens_per_step / (ms_per_step * 1e-3)
-    if use_tc and kda.workspace_status(ws, stream) != 0:
-        raise RuntimeError("device-side timeout reported by the prefill kernel")
-
-    alg_bytes = BYTES_PER_TOKEN_HEAD * B * T * H + ST.numel() * 4 + (0 if x["S0"] is None else ST.numel() * 4)
-    achieved_gbs = alg_bytes / (avg_launch_ms * 1e-3) / 1e9
-    alg_flops = FLOPS_PER_TOKEN_HEAD * B * T * H
-    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": recorded_traffic(cfg.name.split("_seed")[0],
-                                                                                     algo_name),
-                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                else "fallback",
-                "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": avg_launch_ms,
-                "kernel": "kda_chunk_tc_kernel" if use_tc else "chunk_simt_kernel",
-                "tensor": {"achieved_tflops": alg_flops / (avg_launch_ms * 1e-3) / 1e12,
-                           "peak_tflops": peaks["bf16_tflops"],
-                           "frac": alg_flops / (avg_launch_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}}
-
-    # ---- end to end through the C ABI with host buffers
-    pin = {k: (None if v is None else v.cpu().pin_memory()) for k, v in x.items()}
-    dbuf = {k: (None if v is None else torch.empty_like(v)) for k, v in x.items()}
-    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    ST_host = torch.empty(ST.shape, dtype=ST.dtype, pin_memory=True)
-    h2d = sum(v.numel() * v.element_size() for v in pin.values() if v is not None)
-    d2h = o_host.numel() * o_host.element_size() + ST_host.numel() * 4
-
-    def e2e_step():
-        for k_ in pin:
-            if pin[k_] is not None:
-                dbuf[k_].copy_(pin[k_], non_blocking=True)
-        kda.chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["log_alpha"], dbuf["beta"], dbuf["S0"], chunk=cfg.C,
-                      algo=args.algo, o=o, S_T=ST, workspace=ws if ws_bytes else None, stream=stream)
-        o_host.copy_(o, non_blocking=True)
-        ST_host.copy_(ST, non_blocking=True)
-
-    e2e_steps = max(3, min(args.steps, 10))
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
-    e2e = {"value": world * tokens_per_step / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
-    del pin, dbuf
-
-    # ---- decode step: N=256 sequences x 32 heads, 1000 chained in-place steps
-    dcfg = I.DECODE_N256_H32
-    nd = args.decode_steps
-    g = torch.Generator(device=dev)
-    g.manual_seed(dcfg.seed + 1000 * rank)
-    S = dcfg.s_std * torch.randn(dcfg.N, dcfg.H, dcfg.dk, dcfg.dv, device=dev, generator=g)
-
-    def unit(z):
-        return z / z.norm(dim=-1, keepdim=True)
-
-    shp = (nd, dcfg.N, dcfg.H)
-    dq = unit(torch.randn(*shp, dcfg.dk, device=dev, generator=g)).bfloat16()
-    dk_ = unit(torch.randn(*shp, dcfg.dk, device=dev, generator=g)).bfloat16()
-    dv_ = torch.randn(*shp, dcfg.dv, device=dev, generator=g).bfloat16()
-    dla = (-(dcfg.la_lo + (dcfg.la_hi - dcfg.la_lo) * torch.rand(*shp, dcfg.dk, device=dev, generator=g))).bfloat16()
-    db = torch.sigmoid(torch.randn(*shp, device=dev, generator=g)).bfloat16()
-    do = torch.empty(dcfg.N, dcfg.H, dcfg.dv, dtype=torch.bfloat16, device=dev)
-    for i in range(3):
-        kda.decode_step(dq[i], dk_[i], dv_[i], dla[i], db[i], S, o=do, stream=stream)
-    torch.cuda.synchronize()
-    barrier()
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as dclk:
-        d0.record(stream)
-        for i in range(nd):
-            kda.decode_step(dq[i], dk_[i], dv_[i], dla[i], db[i], S, o=do, stream=stream)
-        d1.record(stream)
-        torch.cuda.synchronize()
-    dec_ms = max_over_ranks(d0.elapsed_time(d1))
-    us_step = dec_ms * 1e3 / nd
-    dec_bytes = 2 * S.numel() * 4 + (dq[0].numel() * 3 + dv_[0].numel() + db[0].numel() + do.numel()) * 2
-    dec_gbs = dec_bytes / (us_step * 1e-6) / 1e9
-    decode = {"workload": dcfg.name, "value": world * dec_gbs, "unit": "GB/s", "us_per_step": us_step,
-              "steps": nd, "algorithmic_bytes_per_step": dec_bytes,
-              "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": dec_gbs / peaks["hbm_gbs"], "kernel": "decode_step_kernel",
-                           "traffic": recorded_traffic(dcfg.name, "decode")},
-              "clocks": dclk.summary(), "inputs": "pre-generated on the device, fresh each step"}
-    del dq, dk_, dv_, dla, db, S
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_heads = max(1, min(os.cpu_count(), cfg.B * cfg.H))
+    line = {"metric": METRIC, "value": None, "unit": "tokens/s", "n_gpus": ctx.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": None, "data": "synthetic", "config": None, "roofline": None,
+            "cpu_baseline": None, "e2e": None, "gpu_launches": None, "clocks": None, "decode": None}
+    if "prefill" in args.parts or "e2e" in args.parts:
+        pf = Prefill(ctx, kda, I, args.algo)
+        line["config"] = {"workload": pf.name, "B": pf.cfg.B, "H": pf.cfg.H, "T": pf.cfg.T, "dk": pf.cfg.dk,
+                          "dv": pf.cfg.dv, "chunk": pf.cfg.C, "algo": pf.algo_name,
+                          "parallelism": f"replicas x{ctx.world}",
+                          "l2": "inputs larger than L2 (1.07 GB read per step, L2 126 MB)"}
+        line["dtype"] = "bf16" if pf.use_tc else "f32"
+        if "prefill" in args.parts:
+            ms, roof, clocks = time_prefill(args, ctx, pf, peaks, peak_kind)
+            line.update(value=ctx.world * pf.tokens_per_step / (ms * 1e-3), ms_per_step=ms, roofline=roof,
+                        clocks=clocks, gpu_launches=pf.launches_per_step * args.steps)
+        if "e2e" in args.parts:
+            line["e2e"] = time_e2e(args, ctx, pf)
+        del pf
+    if "decode" in args.parts:
+        line["decode"] = time_decode(args, ctx, kda, I, peaks, peak_kind)
+    if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count()
+        n_heads = max(1, min(cores, 128))
         dt, tok, used, sample = oracle_sample(I.B4_H32_T8K, n_heads)
-        cpu = {"value": tok / dt, "unit": "tokens/s", "cores": used, "kind": "oracle", "sample": sample,
-               "seconds": dt}
-
-    if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16" if use_tc else "f32", "data": "synthetic",
-                "config": {"workload": I.B4_H32_T8K.name, "B": B, "H": H, "T": T, "dk": dk, "dv": dv,
-                           "chunk": cfg.C, "algo": algo_name, "parallelism": f"replicas x{world}",
-                           "l2": "inputs larger than L2 (1.07 GB read per step)"},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(), "decode": decode}
+        line["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                                "sample": sample, "seconds": dt}
+    if ctx.rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    ctx.close()
     return 0
 
 
