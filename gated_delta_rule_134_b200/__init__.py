@@ -10,7 +10,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["load", "chunk_fwd", "decode_step", "workspace_size", "workspace_status", "KDAError",
+__all__ = ["load", "chunk_fwd", "chunk_fwd_noalloc", "decode_step", "workspace_size", "workspace_status", "KDAError",
            "library_path", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -61,6 +61,8 @@ def load(build_if_stale: bool = True):
     lib.kda_workspace_status.restype = I
     lib.kda_decode_step.argtypes = [P] * 8 + [I] * 5 + [P]
     lib.kda_decode_step.restype = I
+    lib.kda_chunk_fwd_noalloc.argtypes = [P] * 8 + [I] * 7 + [P]
+    lib.kda_chunk_fwd_noalloc.restype = I
     _lib = lib
     return lib
 
@@ -170,3 +172,32 @@ def decode_step(q, k, v, log_alpha, beta, S, *, S_out=None, o=None, stream=None)
                                _ptr(o), N, H, dk, dv, _DTYPE[_dtype_of(q)], _stream(stream))
     _check("kda_decode_step", code)
     return o, S_out
+
+
+def chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0=None, *, o, S_T=None, chunk: int = 64, stream=None):
+    """kda_chunk_fwd_noalloc: the tensor-core prefill without a workspace.
+
+    For callers that must not allocate device memory where they run the
+    prefill: the library keeps the kernel's small scratch in a fixed array of
+    its own, so only inputs and caller-owned outputs (o, and S_T if wanted)
+    are passed. bf16 inputs, dk = dv = 128, chunk = 64. Calls that overlap on
+    the GPU share that array and race. Returns (o, S_T)."""
+    import torch
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt, dev = q.dtype, q.device
+    _need(q, "q", (B, T, H, dk), dt, dev)
+    _need(k, "k", (B, T, H, dk), dt, dev)
+    _need(log_alpha, "log_alpha", (B, T, H, dk), dt, dev)
+    _need(v, "v", (B, T, H, dv), dt, dev)
+    _need(beta, "beta", (B, T, H), dt, dev)
+    _need(o, "o", (B, T, H, dv), dt, dev)
+    if S0 is not None:
+        _need(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    if S_T is not None:
+        _need(S_T, "S_T", (B, H, dk, dv), torch.float32, dev)
+    code = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(o),
+                                     _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPE[_dtype_of(q)], _stream(stream))
+    _check("kda_chunk_fwd_noalloc", code)
+    return o, S_T

@@ -721,3 +721,80 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace kda
+
+// ---------------------------------------------------------------- allocation-free variant
+//
+// kda_chunk_fwd_noalloc runs the same tensor-core prefill as kda_chunk_fwd
+// but keeps the kernel's scratch (its device status word, padded to 256
+// bytes) in a fixed array that lives inside this library, so the caller
+// passes only inputs and outputs. It exists for callers that must not
+// allocate device memory at the point where they run a prefill, for example
+// code running inside a memory allocator's own callbacks, host applications
+// that forbid cudaMalloc on their worker threads, or runtimes that expose
+// only the tensors they already own.
+#include <mutex>
+
+#include "kda.h"
+
+// Scratch of the allocation-free entry point; every GPU that loads this
+// library holds these bytes until the process exits. In host code this name
+// is only a stand-in for the symbol: its device address comes from
+// cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_kda_noalloc_scratch[256];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 128;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_scratch_addr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up on
+// the first call made with that device current.
+cudaError_t noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_scratch_addr[dev] == nullptr) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_kda_noalloc_scratch);
+        if (err != cudaSuccess) return err;
+        g_noalloc_scratch_addr[dev] = p;
+    }
+    *out = g_noalloc_scratch_addr[dev];
+    return cudaSuccess;
+}
+
+bool noalloc_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const void* log_alpha,
+                                              const void* beta, const float* S0, void* o, float* S_T, int B,
+                                              int T, int H, int dk, int dv, int chunk, kda_dtype_t dtype,
+                                              void* stream) {
+    if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if ((long long)B * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    kda::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
+    if (!kda::chunk_tc_supported(a)) return KDA_ERR_UNSUPPORTED;
+    if ((long long)B * T * H > 0) {
+        const void* req[] = {q, k, v, log_alpha, beta, o};
+        for (const void* p : req)
+            if (p == nullptr || !noalloc_aligned16(p)) return KDA_ERR_INVALID_ARG;
+    }
+    if ((S0 && !noalloc_aligned16(S0)) || (S_T && !noalloc_aligned16(S_T))) return KDA_ERR_INVALID_ARG;
+    // The kernel's scratch must fit the fixed array.
+    if (kda::chunk_tc_workspace_bytes(B, T, H, dk, dv) > sizeof(g_kda_noalloc_scratch)) return KDA_ERR_INVALID_ARG;
+    if ((long long)B * H == 0) return KDA_OK;
+    void* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return KDA_ERR_CUDA;
+    a.workspace = scratch;
+    a.workspace_bytes = sizeof(g_kda_noalloc_scratch);
+    // launch_chunk_tc clears the status word before the kernel runs.
+    const cudaError_t err = kda::launch_chunk_tc(a, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}

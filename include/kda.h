@@ -127,6 +127,34 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const 
                              const void *beta, const float *S_in, float *S_out, void *o, int N, int H,
                              int dk, int dv, kda_dtype_t dtype, void *stream);
 
+/*
+ * Allocation-free prefill (no counterpart in the paper; an addition of this
+ * library). Same operation, arguments and numerics as kda_chunk_fwd with the
+ * tensor-core algorithm, minus the workspace: the kernel's scratch (its
+ * 4-byte device status word) lives in a fixed 256-byte array inside libkda.so.
+ * It is meant for callers that must not allocate device memory where they run
+ * a prefill -- code running inside a memory allocator's own callbacks, hosts
+ * that forbid cudaMalloc on their worker threads, runtimes that only expose
+ * the tensors they already own. The call itself allocates nothing.
+ *
+ *   - Supports what the tensor-core path supports: dtype KDA_BF16,
+ *     dk = dv = 128, chunk = 64 (else KDA_ERR_UNSUPPORTED). A shape whose
+ *     scratch would exceed the 256-byte array is refused with
+ *     KDA_ERR_INVALID_ARG (no supported shape needs more than 256 bytes).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before capturing any CUDA graph.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; each call clears the status word before its kernel runs. Calls
+ *     that overlap on the GPU (different streams, no ordering) race on the
+ *     array. A device-side timeout is recorded in the array and is not
+ *     reported back through kda_workspace_status; callers that need that
+ *     report use kda_chunk_fwd with their own workspace.
+ */
+kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *log_alpha,
+                                   const void *beta, const float *S0, void *o, float *S_T, int B, int T,
+                                   int H, int dk, int dv, int chunk, kda_dtype_t dtype, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
