@@ -55,6 +55,7 @@ def check_prefill(kda, cfg, algo, heads=None):
         got_o = np.stack([oc[b, :, h].numpy() for b, h in heads])[:, :, None]
         got_S = np.stack([Sc[b, h].numpy() for b, h in heads])[:, None]
     eo, es = rel_err(got_o, ref_o), rel_err(got_S, ref_S)
+    print(f"PARITY {cfg.name} algo={algo} o={eo:.3e} S_T={es:.3e} bar={TOL[cfg.dtype]:.0e}")
     assert np.isfinite(got_o).all() and np.isfinite(got_S).all()
     assert eo <= TOL[cfg.dtype] and es <= TOL[cfg.dtype], (cfg.name, algo, eo, es)
     return eo, es
