@@ -77,10 +77,10 @@ template <int DVT>
 struct Layout {
     // shared memory, bytes from a 1024-aligned base
     static constexpr uint32_t RAWK = 0;                  // k tile: 2 TMA boxes [64 tok][64 ch], swizzled
-    static constexpr uint32_t RAWQ = RAWK + 16384;       // q tile; then the delta operand (DOP)
-    static constexpr uint32_t DOP = RAWQ;                //   delta bf16, MN-major (K = 64 tokens) x DVT
+    static constexpr uint32_t RAWQ = RAWK + 16384;       // q tile
     static constexpr uint32_t RAWG = RAWQ + 16384;       // log_alpha tile
-    static constexpr uint32_t RAWV = RAWG + 16384;       // v slice: DVT/64 boxes
+    static constexpr uint32_t RAWV = RAWG + 16384;       // v slice: DVT/64 boxes; then the delta operand
+    static constexpr uint32_t DOP = RAWV;                //   delta bf16, MN-major (K = 64 tokens) x DVT
     static constexpr uint32_t LMAT = RAWV + DVT * 128;   // lower-triangular ones, K-major 64 x 64
     static constexpr uint32_t ROWOP = LMAT + 8192;       // [KE|X|-W'; QE|Q~] MN-major 128 x 128
     static constexpr uint32_t COLOP = ROWOP + 32768;     // 2 x (KF|K~) MN-major 64 x 128
@@ -101,13 +101,13 @@ struct Layout {
     static constexpr uint32_t SMEM_BYTES = END + 1024;   // + alignment slack
     static constexpr uint32_t SBO_V = 1024 * (DVT / 64); // K-group stride of the S / delta operands
     static_assert(SOP + 128 * DVT * 2 <= SMALL, "S operand overflows the scratch");
-    static_assert(DOP + 64 * DVT * 2 <= RAWQ + 16384, "delta operand overflows the q tile");
+    static_assert(DOP + 64 * DVT * 2 <= RAWV + DVT * 128, "delta operand overflows the v tile");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     // tensor memory columns
     static constexpr uint32_t S_COL = 0;                 // R (fp32, lane = key channel)
     static constexpr uint32_t D1_COL = DVT;              // 2 x DVT: U / delta / O accumulators
-    static constexpr uint32_t GW_COL = 3 * DVT;          // 64: cumulative gate, then W'^T
-    static constexpr uint32_t AP_COL = 3 * DVT + 64;     // 64: A (lanes 0-63) and P (lanes 64-127)
+    static constexpr uint32_t G_COL = 3 * DVT;           // 64: cumulative gate of the chunk being prepared
+    static constexpr uint32_t APW_COL = 3 * DVT + 64;    // 64: A (lanes 0-63) and P (lanes 64-127), then W'^T
     static constexpr uint32_t TMEM_COLS = 512;
 };
 
@@ -126,6 +126,17 @@ __device__ __forceinline__ uint32_t km_off(int r, int s) {
     return (uint32_t)(r * 128 + ((((s >> 3) ^ (r & 7))) << 4) + ((s & 7) << 1));
 }
 
+// 1/x for normal positive x, accurate to ~2.4e-4 relative (enough for a bf16
+// result): seed 2^-e (2 - f)/2 for x = 2^e (1 + f), obtained by subtracting
+// the bit pattern from 254 << 23 (seed error <= 12.5%), then two Newton steps
+// r <- r (2 - x r), each squaring the relative error. Runs on the FMA pipe.
+__device__ __forceinline__ float recip_bf16(float x) {
+    float r = __int_as_float(0x7F000000 - __float_as_int(x));
+    r = r * fmaf(-x, r, 2.f);
+    r = r * fmaf(-x, r, 2.f);
+    return r;
+}
+
 // fp32 -> tf32 (round to nearest) for the warp-level MMAs of the UT inverse
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
@@ -142,33 +153,23 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
 }
 
 // acc += X Y restricted to columns [8*nt, 8*nt+8) of the 16x16 product; X and
-// Y are 16x16 fp32 tiles (row stride kLDA) in shared memory. Each operand is
-// split into a tf32 high part and a tf32 remainder, and the three products
-// hi*hi + hi*lo + lo*hi keep the result at fp32 accuracy. Fragment mapping of
-// m16n8k8 (g = lane/4, t = lane%4): A (g|g+8, t|t+4), B (t|t+4, g),
-// C (g|g+8, 2t|2t+1).
+// Y are 16x16 fp32 tiles (row stride kLDA) in shared memory, rounded to tf32
+// (the resulting T' is stored as bf16, which dominates its rounding error).
+// Fragment mapping of m16n8k8 (g = lane/4, t = lane%4): A (g|g+8, t|t+4),
+// B (t|t+4, g), C (g|g+8, 2t|2t+1).
 __device__ __forceinline__ void mm16_ntile(float (&acc)[4], const float* X, const float* Y, int nt, int lane) {
     const int g = lane >> 2, t = lane & 3;
+    float part[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
-        const float x[4] = {X[g * kLDA + 8 * ks + t], X[(g + 8) * kLDA + 8 * ks + t], X[g * kLDA + 8 * ks + t + 4],
-                            X[(g + 8) * kLDA + 8 * ks + t + 4]};
-        const float y[2] = {Y[(8 * ks + t) * kLDA + 8 * nt + g], Y[(8 * ks + t + 4) * kLDA + 8 * nt + g]};
-        uint32_t ah[4], al[4], bh[2], bl[2];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            ah[i] = to_tf32(x[i]);
-            al[i] = to_tf32(x[i] - __uint_as_float(ah[i]));
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            bh[i] = to_tf32(y[i]);
-            bl[i] = to_tf32(y[i] - __uint_as_float(bh[i]));
-        }
-        mma_tf32_16x8x8(acc, al, bh);
-        mma_tf32_16x8x8(acc, ah, bl);
-        mma_tf32_16x8x8(acc, ah, bh);
+        const uint32_t a[4] = {to_tf32(X[g * kLDA + 8 * ks + t]), to_tf32(X[(g + 8) * kLDA + 8 * ks + t]),
+                               to_tf32(X[g * kLDA + 8 * ks + t + 4]), to_tf32(X[(g + 8) * kLDA + 8 * ks + t + 4])};
+        const uint32_t bq[2] = {to_tf32(Y[(8 * ks + t) * kLDA + 8 * nt + g]),
+                                to_tf32(Y[(8 * ks + t + 4) * kLDA + 8 * nt + g])};
+        mma_tf32_16x8x8(part[ks], a, bq);  // two independent accumulators
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] += part[0][e] + part[1][e];
 }
 
 __device__ __forceinline__ void nb_sync(int id, int nthreads) {
@@ -270,12 +271,16 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         atomicExch(status, 1u);
         *s_abort = 1;
     };
-    auto wait_all = [&](uint64_t* bar_, int chunk) {  // every thread waits; MMA results then readable
+    // Waits are executed by whole warps; __syncwarp reconverges the lanes
+    // before the warp-collective instructions (tcgen05.ld, bar) that follow.
+    auto wait_all = [&](uint64_t* bar_, int chunk) {  // compute warps; MMA results then readable
         if (!*s_abort && !mbar_wait_bounded(bar_, (uint32_t)chunk & 1u, kWaitBudget)) fail();
+        __syncwarp();
         tc_fence_after();
     };
-    auto wait_one = [&](uint64_t* bar_, int chunk) {  // thread 0 only (before issuing dependent work)
+    auto wait_one = [&](uint64_t* bar_, int chunk) {  // control warp (before issuing dependent work)
         if (!*s_abort && !mbar_wait_bounded(bar_, (uint32_t)chunk & 1u, kWaitBudget)) fail();
+        __syncwarp();
     };
     auto issue_k = [&](int n) {
         mbar_arrive_expect_tx(bar.k, 2 * 8192);
@@ -311,7 +316,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + L::GW_COL, sdesc_sw128(sb + L::RAWG + kk * 2048, 8192, 1024),
+            mma_bf16_ss(tmem + L::G_COL, sdesc_sw128(sb + L::RAWG + kk * 2048, 8192, 1024),
                         sdesc_sw128(sb + L::LMAT + kk * 32, 16, 1024), ID_CS, kk > 0);
         mma_commit(bar.cs);
     };
@@ -321,12 +326,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const uint32_t col = sb + L::COLOP + (m & 1) * 16384;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_bf16_ss(tmem + L::AP_COL, sdesc_sw128(sb + L::ROWOP + kk * 4096, 1024, 2048),
+                mma_bf16_ss(tmem + L::APW_COL, sdesc_sw128(sb + L::ROWOP + kk * 4096, 1024, 2048),
                             sdesc_sw128(col + kk * 2048, 1024, 1024), ID_AP, kk > 0);
         }
         mma_commit(bar.ap);
     };
-    auto mma_uw = [&](int m) {  // U = [T'; 0] V into D1[m%2];  W'^T = KE^T T'^T
+    auto mma_uw = [&](int m) {  // U = [T'; 0] V into D1[m%2];  W'^T = KE^T T'^T (over A/P, already read)
         tc_fence_after();
         const uint32_t d1 = tmem + L::D1_COL + (m & 1) * DVT;
 #pragma unroll
@@ -335,7 +340,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         sdesc_sw128(sb + L::RAWV + kk * 2048, 8192, 1024), ID_U, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + L::GW_COL, sdesc_sw128(sb + L::ROWOP + kk * 32, 16, 2048),
+            mma_bf16_ss(tmem + L::APW_COL, sdesc_sw128(sb + L::ROWOP + kk * 32, 16, 2048),
                         sdesc_sw128(sb + L::TZP + kk * 32, 16, 1024), ID_WT, kk > 0);
         mma_commit(bar.uw);
     };
@@ -372,7 +377,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     auto p2_compute = [&](int m) -> bool {
         const int c = trow, r0 = 32 * hf;
         uint32_t gv[32];
-        tmem_ld32(lane_addr + L::GW_COL + 32 * hf, gv);
+        tmem_ld32(lane_addr + L::G_COL + 32 * hf, gv);
         tmem_ld_wait(gv);
         sEx[hf * 128 + c] = __uint_as_float(gv[31]);  // G_31 (hf = 0) / G_63 (hf = 1)
         tc_fence_before();
@@ -433,7 +438,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             float e0, e1, f0, f1;
             if (!exact) {
                 e0 = __expf(g0 - Gm); e1 = __expf(g1 - Gm);
-                f0 = __expf(Gm - g0); f1 = __expf(Gm - g1);
+                f0 = recip_bf16(e0); f1 = recip_bf16(e1);
             } else {
                 e0 = __expf(g0); e1 = __expf(g1);
                 f0 = __expf(Gl - g0); f1 = __expf(Gl - g1);
@@ -460,7 +465,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     // ---- P4 of chunk m: A (lanes 0-63) -> fp32 scratch; P (lanes 64-127) -> bf16 operand
     auto p4 = [&](int m) {
         uint32_t v[32];
-        tmem_ld32(lane_addr + L::AP_COL + 32 * hf, v);
+        tmem_ld32(lane_addr + L::APW_COL + 32 * hf, v);
         tmem_ld_wait(v);
         if (quad < 2) {
             const int r = trow;
@@ -518,7 +523,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
         }
         nb_sync(NB_SIMT, kCompute);
-        // Blocks below the diagonal on the tensor cores (m16n8k8, 3xTF32): one
+        // Blocks below the diagonal on the tensor cores (m16n8k8, tf32): one
         // warp per (block, 8-column half). N_ak = T_aa A_ak replaces A_ak.
         auto put_t = [&](int a, int bb, int nt, const float (&acc)[4]) {  // T_ab = -acc
             const int g = lane >> 2, t = lane & 3;
@@ -563,7 +568,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     auto p7 = [&]() {
         const int cc = trow;
         uint32_t v[32];
-        tmem_ld32(lane_addr + L::GW_COL + 32 * hf, v);
+        tmem_ld32(lane_addr + L::APW_COL + 32 * hf, v);
         tmem_ld_wait(v);
 #pragma unroll
         for (int jc = 0; jc < 4; ++jc) {
@@ -652,6 +657,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         dst[jc] = w;
                     }
                 }
+                __syncwarp();  // (ragged tail) reconverge before the next tcgen05.ld
             }
         }
     };
@@ -674,53 +680,68 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 issue_g(0);
                 issue_v(0);
             }
+            __syncwarp();
             wait_one(bar.g, 0);
             if (leader) mma_cumsum();
+            __syncwarp();
             wait_one(bar.cs, 0);
             if (leader && NC > 1) issue_g(1);       // log_alpha tile consumed
-            nb_sync(NB_K, kThreads);                 // k, q tiles of chunk 0 read
+            __syncwarp();
+            nb_sync(NB_K, kThreads);                 // gate and k, q tiles of chunk 0 read
             if (leader && NC > 1) {
                 issue_k(1);
                 issue_q(1);
             }
+            __syncwarp();
             nb_sync(NB_S3, kThreads);                // operands of chunk 0 stored
             if (leader) mma_ap(0, *s_exact != 0);
+            __syncwarp();
+            if (NC > 1) {                            // gate of chunk 1, ready long before it is needed
+                wait_one(bar.g, 1);
+                if (leader) mma_cumsum();
+                __syncwarp();
+            }
             nb_sync(NB_P5, kThreads);                // T' of chunk 0 stored
             wait_one(bar.v, 0);
             if (leader) mma_uw(0);
-            wait_one(bar.uw, 0);
-            if (leader && NC > 1) issue_v(1);
+            __syncwarp();
         }
         for (int n = 0; n < NC; ++n) {
             const bool more = n + 1 < NC;
             if (__syncthreads_or(*s_abort)) break;
             nb_sync(NB_S1, kThreads);                // state operand of chunk n stored
-            if (more) {
-                wait_one(bar.g, n + 1);
-                if (leader) mma_cumsum();
-            }
             if (leader) mma_1(n);
+            __syncwarp();
             if (more) {
-                wait_one(bar.cs, n + 1);
-                if (leader && n + 2 < NC) issue_g(n + 2);
-                nb_sync(NB_K, kThreads);             // k, q tiles of chunk n+1 read
-                if (leader && n + 2 < NC) issue_k(n + 2);
+                wait_one(bar.cs, n + 1);             // (issued one iteration earlier)
+                if (leader && n + 2 < NC) issue_g(n + 2);  // log_alpha tile consumed
+                __syncwarp();
+                nb_sync(NB_K, kThreads);             // gate and k, q tiles of chunk n+1 read
+                if (leader && n + 2 < NC) {
+                    issue_k(n + 2);
+                    issue_q(n + 2);
+                }
+                __syncwarp();
             }
             nb_sync(NB_S3, kThreads);                // delta(n) and operands of chunk n+1 stored
             if (leader) {
                 if (more) mma_ap(n + 1, *s_exact != 0);
                 mma_2(n);
             }
+            __syncwarp();
+            if (n + 2 < NC) {                        // gate of chunk n+2 (the gate TMEM columns are free)
+                wait_one(bar.g, n + 2);
+                if (leader) mma_cumsum();
+                __syncwarp();
+            }
+            wait_one(bar.m2, n);
+            if (leader && more) issue_v(n + 1);      // delta operand (on the v tile) consumed
+            __syncwarp();
             if (more) {
                 nb_sync(NB_P5, kThreads);            // T' of chunk n+1 stored
                 wait_one(bar.v, n + 1);
                 if (leader) mma_uw(n + 1);
-            }
-            wait_one(bar.m2, n);
-            if (leader && n + 2 < NC) issue_q(n + 2);  // delta operand (on the q tile) consumed
-            if (more) {
-                wait_one(bar.uw, n + 1);
-                if (leader && n + 2 < NC) issue_v(n + 2);
+                __syncwarp();
             }
         }
         __syncthreads();
@@ -758,6 +779,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             nb_sync(NB_SIMT, kCompute);  // sBeta visible
             const bool exact0 = p2_compute(0);
             if (tid == 0) *s_exact = exact0;
+            __syncwarp();
             nb_sync(NB_SIMT, kCompute);  // (exact path) staged gate values read before the tiles are overwritten
             nb_arrive(NB_K, kThreads);
             p2_store(0);
@@ -786,6 +808,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 nb_sync(NB_SIMT, kCompute);  // sBeta(n+1) visible
                 exact_next = p2_compute(n + 1);
                 if (tid == 0) *s_exact = exact_next;
+                __syncwarp();
                 nb_sync(NB_SIMT, kCompute);  // k, q tiles (and the exact path's staged gate) read
                 nb_arrive(NB_K, kThreads);
             }
