@@ -45,49 +45,86 @@ def load_peaks():
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples the SM clock and the clock-event (throttle) reasons of one GPU
+    while the timed region runs: NVML polled every ~1 ms from a thread
+    (nvidia-smi as a fallback). Only reads state; changes nothing."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40, "sw_power_cap": 0x4}
 
-    def __init__(self, index: int):
-        self.index = index
-        self.rows = []
-        self.proc = None
+    def __init__(self, torch_device_index: int):
+        self.index = torch_device_index
+        self.samples = []
+        self.max_mhz = None
+        self.err = None
+        self._stop = threading.Event()
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(self.index)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _open(self):
+        """NVML handle and maximum clock, opened before the timed region starts."""
+        try:
+            nv, h = self._handle()
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            return lambda: (float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), int(get_reasons(h)))
+        except Exception as e:
+            self.err = repr(e)
+            return None
+
+    def _smi(self):  # no NVML: one nvidia-smi reading
+        try:
+            out = subprocess.run(["nvidia-smi", "-i", str(self.index), "--query-gpu=clocks.sm,clocks.max.sm",
+                                  "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                 timeout=10).stdout.strip().split(",")
+            self.samples.append((float(out[0]), 0))
+            self.max_mhz = float(out[1])
+        except Exception:
+            pass
+
+    def _run(self):
+        try:
+            while True:
+                self.samples.append(self._read())
+                if self._stop.wait(0.001):
+                    break
+        except Exception as e:
+            self.err = repr(e)
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except FileNotFoundError:
-            self.proc = None
+        self._read = self._open()
+        if self._read is None:
+            self._smi()
+            self._t = None
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.rows.append([x.strip() for x in line.split(",")])
-
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if self._t is not None:
+            self._t.join(timeout=5)
 
     def summary(self):
-        if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm = sorted(float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit())
-        mx = max((float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()), default=None)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
-        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(self.rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no clock samples: " + str(self.err)]}
+        sm = sorted(x for x, _ in self.samples)
+        mask = 0
+        for _, r in self.samples:
+            mask |= r
+        reasons = sorted(k for k, bit in self.REASONS.items() if mask & bit)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "source": "nvml" if self.err is None else "nvidia-smi"}
 
 
 # Source files each profiled kernel is built from: a recorded ncu traffic
@@ -208,12 +245,12 @@ class Ctx:
 class Prefill:
     """The B=4, H=32, T=8192 bf16 prefill workload resident on this rank's GPU."""
 
-    def __init__(self, ctx, kda, I, algo):
+    def __init__(self, ctx, kda, I, algo, profile_T=None):
         torch = ctx.torch
         self.kda, self.ctx, self.algo = kda, ctx, algo
         base = I.B4_H32_T8K
-        self.cfg = cfg = base.replace(seed=base.seed + 1000 * ctx.rank)
-        self.name = base.name
+        self.cfg = cfg = base.replace(seed=base.seed + 1000 * ctx.rank, T=profile_T or base.T)
+        self.name = base.name if not profile_T else f"{base.name}_profile_T{profile_T}"
         self.x = {k: (None if v is None else v.to(ctx.dev)) for k, v in I.prefill_inputs(cfg).items()}
         B, T, H, dk, dv = cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv
         self.o = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=ctx.dev)
@@ -367,6 +404,8 @@ def main():
     ap.add_argument("--algo", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-T", type=int, default=None,
+                    help="shorter sequence for profiler captures (the printed line is then not a bench value)")
     ap.add_argument("--parts", default="prefill,e2e,decode",
                     help="comma list of prefill, e2e, decode (profiling runs select one)")
     args = ap.parse_args()
@@ -387,7 +426,7 @@ def main():
             "vs_baseline": None, "dtype": None, "data": "synthetic", "config": None, "roofline": None,
             "cpu_baseline": None, "e2e": None, "gpu_launches": None, "clocks": None, "decode": None}
     if "prefill" in args.parts or "e2e" in args.parts:
-        pf = Prefill(ctx, kda, I, args.algo)
+        pf = Prefill(ctx, kda, I, args.algo, args.profile_T)
         line["config"] = {"workload": pf.name, "B": pf.cfg.B, "H": pf.cfg.H, "T": pf.cfg.T, "dk": pf.cfg.dk,
                           "dv": pf.cfg.dv, "chunk": pf.cfg.C, "algo": pf.algo_name,
                           "parallelism": f"replicas x{ctx.world}",

@@ -18,10 +18,12 @@
 // and E_r = e^{G_r - G_m}, F_r = e^{G_m - G_r} (per channel):
 //   e^{G_r - G_s} = E_r F_s,  k e^G = (k E) e^{G_m},  k e^{G_last-G} = (k F) e^{G_last-G_m}.
 // So three bf16 tiles, KE = k E, QE = q E and KF = k F, feed every MMA:
+//   G = [L; L] g            -> gate prefix sums (L: lower-triangular ones)
 //   [KE; QE] KF^T           -> A and P (one M=128 MMA)
-//   W' = T' KE              -> W = W' Diag(e^{G_m})
+//   [T'; 0] [v | KE]        -> [U; 0] and W' = T' KE, W = W' Diag(e^{G_m})
 //   D1 += [-W'; QE] (e^{G_m} S)   -> rows 0-63: U - W S = delta, rows 64-127: (q e^G) S
 //   R  = e^{G_m} S + KF^T delta   -> S_next = Diag(e^{G_last-G_m}) R
+//   D1 += [* ; P] delta     -> rows 64-127: O (rows 0-63, already read, take junk)
 // The tensor memory therefore holds R, and the next chunk rescales it per
 // channel while it copies the state into the bf16 MMA operand. Each factor is
 // a single exponential, finite as long as |G_r - G_m| <= 80 and G_m >= -80;
@@ -31,22 +33,27 @@
 // produce the same quantities.
 //
 // Schedule. One CTA owns one (batch, head) and a DVT-wide slice of value
-// channels; its state stays in tensor memory for the whole sequence. Chunk n's
-// state-dependent MMAs overlap the state-independent preparation of chunk n+1
-// on the same warps:
-//   S1(n)  state -> bf16 operand            | cumsum MMA(n+1) issued, then MMA1(n)
-//   P2(n+1) gate, guard, KE/QE/KF in regs   | while MMA1(n) runs
-//   S3(n)  delta -> bf16; P2(n+1) stores    | then AP(n+1), MMA2(n) issued
-//   P4/P5(n+1) A, P readout; (I+A)^{-1}     | while MMA2(n) runs
-//   U(n+1), W'(n+1) issued; S5(n) O out; P7(n+1) -W' stored
-// The cumulative gate itself is an MMA with a lower-triangular ones matrix.
+// channels; its state stays in tensor memory for the whole sequence. Three
+// warp roles run concurrently and hand work over through mbarriers:
+//   prep  (warps 0-7)  per chunk m, ahead of the state: gate prefix sums from
+//                      tensor memory, guard, KE/QE/KF (in place over the raw
+//                      k/q tiles), A and P readout, (I + A)^{-1} -> T', -W'.
+//   chain (warps 8-11) per chunk n, the state-dependent part: state -> bf16
+//                      operand, MMA1 (two halves of the key channels, so one
+//                      16 KB operand buffer serves both), delta -> bf16,
+//                      MMA2, O -> global. Warp 8 issues these MMAs.
+//   control (warp 12)  every TMA load and the state-independent MMAs (prefix
+//                      sums, A/P, U/W), in the order their inputs appear.
+// k/q tiles and the operand tiles built from them are double-buffered by
+// chunk parity, so the prep of chunk n+1 overlaps the state chain of chunk n.
 // (I + A)^{-1}: 16x16 diagonal blocks by forward substitution (four threads per
 // column), N = T_diag A_offdiag, then the blocks below the diagonal level by
 // level, T_ab = -sum_k N_ak T_kb; T' = T Diag(beta) is written as bf16 by the
 // thread that finalises each entry.
 //
 // Every wait on an mbarrier is bounded; on expiry the kernel records status 1
-// in the caller's workspace word, stops, frees its tensor memory and returns.
+// in the caller's workspace word and stops waiting (later waits are skipped,
+// so every role reaches the end), frees its tensor memory and returns.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_sm100.cuh"
@@ -57,16 +64,19 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kCompute = 256;             // 8 compute warps
-constexpr int kCtrlWarp = kCompute / 32;  // warp 8 issues TMA loads and MMAs
-constexpr int kThreads = kCompute + 32;
+constexpr int kPrep = 256;                    // warps 0-7
+constexpr int kChainWarp0 = kPrep / 32;       // warps 8-11
+constexpr int kCtrlWarp = kChainWarp0 + 4;    // warp 12
+constexpr int kThreads = 32 * (kCtrlWarp + 1);
 // named barriers (0 is __syncthreads)
-constexpr int NB_SIMT = 1;  // compute warps only
-constexpr int NB_OR = 2;    // compute warps only, OR-reduction
-constexpr int NB_S1 = 3;    // compute -> control: state operand ready
-constexpr int NB_K = 4;     // compute -> control: k, q tiles consumed
-constexpr int NB_S3 = 5;    // compute -> control: delta / next-chunk operands ready
-constexpr int NB_P5 = 6;    // compute -> control: T' ready
+constexpr int NB_PREP = 1;  // prep warps
+constexpr int NB_OR = 2;    // prep warps, OR-reduction
+constexpr int NB_P2 = 3;    // prep -> control: operand tiles stored, prefix sums read (AP, next prefix sums)
+constexpr int NB_P5 = 4;    // prep -> control: T' stored (U, W)
+constexpr int NB_CHA = 5;   // chain warps 8-9
+constexpr int NB_CHB = 6;   // chain warps 10-11 -> warp 8: second half of the state operand stored
+constexpr int NB_CHC = 7;   // chain warps 10-11
+constexpr int NB_CH = 8;    // all chain warps
 constexpr int kC = 64;    // chunk
 constexpr int kD = 128;   // dk = dv
 constexpr int kLDA = 68;  // fp32 row stride of the A / T scratch (bank spread)
@@ -76,49 +86,64 @@ constexpr long long kWaitBudget = 1ll << 31;  // SM cycles (~1 s)
 template <int DVT>
 struct Layout {
     // shared memory, bytes from a 1024-aligned base
-    static constexpr uint32_t RAWK = 0;                  // k tile: 2 TMA boxes [64 tok][64 ch], swizzled
-    static constexpr uint32_t RAWQ = RAWK + 16384;       // q tile
-    static constexpr uint32_t RAWG = RAWQ + 16384;       // log_alpha tile
-    static constexpr uint32_t RAWV = RAWG + 16384;       // v slice: DVT/64 boxes; then the delta operand
-    static constexpr uint32_t DOP = RAWV;                //   delta bf16, MN-major (K = 64 tokens) x DVT
-    static constexpr uint32_t LMAT = RAWV + DVT * 128;   // lower-triangular ones, K-major 64 x 64
-    static constexpr uint32_t ROWOP = LMAT + 8192;       // [KE|X|-W'; QE|Q~] MN-major 128 x 128
-    static constexpr uint32_t COLOP = ROWOP + 32768;     // 2 x (KF|K~) MN-major 64 x 128
-    static constexpr uint32_t TZP = COLOP + 32768;       // T' | Z | P0 | Z | P1 (8 KB each), K-major
-    static constexpr uint32_t SCR = TZP + 40960;         // A, T fp32 [64][68] (also the S operand)
+    static constexpr uint32_t ROWOP = 0;            // 2 x 32 KB, K-major: per 64-channel box x (x * 16 KB)
+                                                    //   rows 0-63: k -> KE -> -W', rows 64-127: q -> QE
+    static constexpr uint32_t COLOP = 65536;        // 2 x 16 KB: log_alpha tile, then KF (box x at x * 8 KB)
+    static constexpr uint32_t RAWV = 98304;         // v slice: DVT/64 boxes of [64 tok][64 ch]
+    static constexpr uint32_t LMAT = 114688;        // [L; L] K-major 128 x 64
+    static constexpr uint32_t TZP = 131072;         // [T'; 0] K-major 128 x 64
+    static constexpr uint32_t SP = TZP + 16384;     // 2 x P, K-major 64 x 64 bf16 (8 KB each)
+    static constexpr uint32_t SCR = SP + 16384;     // A, T fp32 [64][kLDA] (exact path: G fp32 [64][128])
     static constexpr uint32_t SA = SCR;
     static constexpr uint32_t ST = SCR + 64 * kLDA * 4;
-    static constexpr uint32_t SOP = SCR;                 //   S bf16, MN-major (K = dk) x DVT
-    static constexpr uint32_t SMALL = SCR + 2 * 64 * kLDA * 4;
-    static constexpr uint32_t SBETA = SMALL;             // 64 f32
-    static constexpr uint32_t SOPS = SBETA + 256;        // 128 f32: operand scale per channel
-    static constexpr uint32_t STMS = SOPS + 512;         // 128 f32: tensor-memory scale per channel
-    static constexpr uint32_t SEK = STMS + 512;          // 128 f32: e^{G_last - G_m} of the last prepared chunk
-    static constexpr uint32_t SEX = SEK + 512;           // 2 x 128 f32: G_m, G_last exchange
-    static constexpr uint32_t BARS = SEX + 1024;         // 9 mbarriers
-    static constexpr uint32_t MISC = BARS + 72;          // tmem base, abort flag
+    static constexpr uint32_t SOP = SCR + 2 * 64 * kLDA * 4;  // S half (64 channels) x DVT, bf16 MN-major
+    static constexpr uint32_t DOP = SOP;                      //   then delta (64 tokens) x DVT
+    static constexpr uint32_t SMALL = SOP + 64 * DVT * 2;
+    static constexpr uint32_t SBETA = SMALL;        // 64 f32
+    static constexpr uint32_t SOPS = SBETA + 256;   // 2 x 128 f32: operand scale per channel (by chunk parity)
+    static constexpr uint32_t STMS = SOPS + 1024;   // 2 x 128 f32: tensor-memory scale per channel
+    static constexpr uint32_t SEK = STMS + 1024;    // 128 f32: e^{G_last - G_m} of the last prepared chunk
+    static constexpr uint32_t SGM = SEK + 512;      // 128 f32: G_m of the chunk being prepared
+    static constexpr uint32_t SGL = SGM + 512;      // 128 f32: G_last
+    static constexpr uint32_t BARS = SGL + 512;     // 20 mbarriers
+    static constexpr uint32_t MISC = BARS + 160;    // tmem base, abort flag, guard verdicts
     static constexpr uint32_t END = MISC + 16;
     static constexpr uint32_t SMEM_BYTES = END + 1024;   // + alignment slack
     static constexpr uint32_t SBO_V = 1024 * (DVT / 64); // K-group stride of the S / delta operands
-    static_assert(SOP + 128 * DVT * 2 <= SMALL, "S operand overflows the scratch");
-    static_assert(DOP + 64 * DVT * 2 <= RAWV + DVT * 128, "delta operand overflows the v tile");
+    static_assert(SOP % 1024 == 0, "operand alignment");
+    static_assert(64 * 128 * 4 <= 2 * 64 * kLDA * 4, "exact-path gate staging overflows the scratch");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     // tensor memory columns
-    static constexpr uint32_t S_COL = 0;                 // R (fp32, lane = key channel)
-    static constexpr uint32_t D1_COL = DVT;              // 2 x DVT: U / delta / O accumulators
-    static constexpr uint32_t G_COL = 3 * DVT;           // 64: cumulative gate of the chunk being prepared
-    static constexpr uint32_t APW_COL = 3 * DVT + 64;    // 64: A (lanes 0-63) and P (lanes 64-127), then W'^T
+    static constexpr uint32_t S_COL = 0;     // R (fp32, lane = key channel)
+    static constexpr uint32_t D1_COL = 128;  // [U; 0] -> [delta; O] (lane = token row)
+    static constexpr uint32_t APW_COL = 256; // [A; P] (64 cols), then [W'; 0] (128 cols)
+    static constexpr uint32_t GC_COL = 384;  // [G; G] (lane = token, col = channel)
     static constexpr uint32_t TMEM_COLS = 512;
 };
 
-__device__ __forceinline__ float ld_bf16(const uint8_t* base, uint32_t off) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
-}
+// mbarrier slots
+enum : int {
+    BAR_KQ = 0,      // 2: k/q tiles landed (by chunk parity)
+    BAR_G = 2,       // 2: log_alpha tile landed
+    BAR_V = 4,       // v tile landed
+    BAR_CS = 5,      // prefix-sum MMA done
+    BAR_AP = 6,      // A/P MMA done
+    BAR_UW = 7,      // U/W MMA done
+    BAR_M1A = 8,     // MMA1, first half, done
+    BAR_M1 = 9,      // MMA1 done
+    BAR_M2 = 10,     // MMA2 done
+    BAR_M1B = 11,    // 2: MMA1 of the chunk of this parity done (row operand free)
+    BAR_M2B = 13,    // 2: MMA2 of the chunk of this parity done (KF, P free)
+    BAR_D1 = 15,     // delta and O read out of tensor memory (D1 free)
+    BAR_SC = 16,     // 2: per-channel scales of the chunk of this parity stored
+    BAR_RR = 18,     // 2: row operand [-W'; QE] of the chunk of this parity stored
+    NUM_BARS = 20
+};
 
-// offset of element (token r, channel c) in a [64 tok][128 ch] tile stored as
-// two TMA boxes of [64][64] with the 128-byte swizzle
-__device__ __forceinline__ uint32_t raw_off(int r, int c) {
-    return (uint32_t)((c >> 6) * 8192 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
+// offset of element (row R, channel c) of a row-operand buffer (K-major, two
+// 64-channel boxes of 128 rows, 128-byte swizzle)
+__device__ __forceinline__ uint32_t rop_off(int R, int c) {
+    return (uint32_t)((c >> 6) * 16384 + R * 128 + ((((c & 63) >> 3) ^ (R & 7)) << 4) + ((c & 7) << 1));
 }
 
 // byte offset of element (row r, col s) of a K-major swizzled 64-wide tile
@@ -191,10 +216,6 @@ __device__ __forceinline__ bool nb_or(int id, int nthreads, bool pred) {
     return r != 0;
 }
 
-struct Bars {
-    uint64_t *k, *q, *g, *v, *cs, *ap, *uw, *m1, *m2;
-};
-
 template <int DVT>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
@@ -203,7 +224,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     float* ST, int Tlen, int H, unsigned* status) {
     using L = Layout<DVT>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base (the 128-byte swizzle repeats every 1024 bytes);
+    // offsetting the array itself keeps the pointer in the shared window, so
+    // accesses through it compile to shared-memory instructions
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(sm);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -212,27 +236,24 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const int b = bh / H, h = bh % H;
     const int j0 = (blockIdx.x % nslices) * DVT;
     const int NC = (Tlen + kC - 1) / kC;
-    // thread <-> tensor-memory lane: warp w reads lanes 32*(w%4).. and column half w/4
-    const int quad = warp & 3, hf = warp >> 2;
-    const int trow = 32 * quad + lane;
-    constexpr int NJ = DVT / 2;
+    const int quad = warp & 3;  // tensor-memory lane quadrant this warp may access
 
     float* sBeta = reinterpret_cast<float*>(sm + L::SBETA);
     float* sOpS = reinterpret_cast<float*>(sm + L::SOPS);
     float* sTmS = reinterpret_cast<float*>(sm + L::STMS);
     float* sEK = reinterpret_cast<float*>(sm + L::SEK);
-    float* sEx = reinterpret_cast<float*>(sm + L::SEX);
+    float* sGm = reinterpret_cast<float*>(sm + L::SGM);
+    float* sGl = reinterpret_cast<float*>(sm + L::SGL);
     float* sA = reinterpret_cast<float*>(sm + L::SA);
     float* sT = reinterpret_cast<float*>(sm + L::ST);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BARS);
-    const Bars bar{bars, bars + 1, bars + 2, bars + 3, bars + 4, bars + 5, bars + 6, bars + 7, bars + 8};
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
-    volatile int* s_exact = reinterpret_cast<volatile int*>(sm + L::MISC + 8);  // guard verdict of the chunk being prepared
+    volatile int* s_exact = reinterpret_cast<volatile int*>(sm + L::MISC + 8);  // 2: guard verdict by parity
 
     // ---------------------------------------------------------------- setup
     if (tid == 0) {
-        for (int i = 0; i < 9; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < NUM_BARS; ++i) mbar_init(bars + i, 1);
         *s_abort = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_k);
@@ -244,19 +265,18 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         tmem_alloc(s_tmem, L::TMEM_COLS);
         tmem_relinquish();
     }
-    {
-        // T' (upper part stays zero), both zero blocks; L = lower-triangular ones
-        uint4* z = reinterpret_cast<uint4*>(sm + L::TZP);
-        for (int i = tid; i < 40960 / 16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
-        for (int e = tid; e < 64 * 8; e += kThreads) {
-            const int r = e >> 3, ch = e & 7;
+    {   // constants: [L; L] (row R: ones in columns 0..R%64) and [T'; 0], whose
+        // blocks above the diagonal and zero half are never written again
+        for (int i = tid; i < 128 * 8; i += kThreads) {
+            const int R = i >> 3, j = i & 7, r = R & 63;
             uint32_t w[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int s = 8 * ch + 2 * u;
-                w[u] = (s <= r ? 0x3F80u : 0u) | ((s + 1 <= r) ? 0x3F800000u : 0u);
+                const int s = 8 * j + 2 * u;
+                w[u] = pack_bf16x2(s <= r ? 1.f : 0.f, s + 1 <= r ? 1.f : 0.f);
             }
-            *reinterpret_cast<uint4*>(sm + L::LMAT + r * 128 + ((ch ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            st_shared_v4(sb + L::LMAT + R * 128 + ((j ^ (R & 7)) << 4), w[0], w[1], w[2], w[3]);
+            st_shared_v4(sb + L::TZP + R * 128 + (j << 4), 0u, 0u, 0u, 0u);
         }
         for (int c = tid; c < kD; c += kThreads) sEK[c] = 1.f;
     }
@@ -271,490 +291,128 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         atomicExch(status, 1u);
         *s_abort = 1;
     };
-    // Waits are executed by whole warps; __syncwarp reconverges the lanes
-    // before the warp-collective instructions (tcgen05.ld, bar) that follow.
-    auto wait_all = [&](uint64_t* bar_, int chunk) {  // compute warps; MMA results then readable
-        if (!*s_abort && !mbar_wait_bounded(bar_, (uint32_t)chunk & 1u, kWaitBudget)) fail();
+    // Bounded wait by one thread; after a timeout every later wait is skipped.
+    auto wait1 = [&](int slot, uint32_t parity) {
+        if (!*s_abort && !mbar_wait_bounded(bars + slot, parity & 1u, kWaitBudget)) fail();
+    };
+    // Bounded wait by a whole warp, then reconverge; MMA results readable after.
+    auto waitw = [&](int slot, uint32_t parity) {
+        wait1(slot, parity);
         __syncwarp();
         tc_fence_after();
     };
-    auto wait_one = [&](uint64_t* bar_, int chunk) {  // control warp (before issuing dependent work)
-        if (!*s_abort && !mbar_wait_bounded(bar_, (uint32_t)chunk & 1u, kWaitBudget)) fail();
-        __syncwarp();
-    };
-    auto issue_k = [&](int n) {
-        mbar_arrive_expect_tx(bar.k, 2 * 8192);
-        for (int x = 0; x < 2; ++x) tma_load_4d(sm + L::RAWK + x * 8192, &tm_k, bar.k, 64 * x, h, n * kC, b);
-    };
-    auto issue_q = [&](int n) {
-        mbar_arrive_expect_tx(bar.q, 2 * 8192);
-        for (int x = 0; x < 2; ++x) tma_load_4d(sm + L::RAWQ + x * 8192, &tm_q, bar.q, 64 * x, h, n * kC, b);
-    };
-    auto issue_g = [&](int n) {
-        mbar_arrive_expect_tx(bar.g, 2 * 8192);
-        for (int x = 0; x < 2; ++x) tma_load_4d(sm + L::RAWG + x * 8192, &tm_g, bar.g, 64 * x, h, n * kC, b);
-    };
-    auto issue_v = [&](int n) {
-        mbar_arrive_expect_tx(bar.v, (DVT / 64) * 8192);
-        for (int x = 0; x < DVT / 64; ++x)
-            tma_load_4d(sm + L::RAWV + x * 8192, &tm_v, bar.v, j0 + 64 * x, h, n * kC, b);
-    };
-    auto load_beta = [&](int n) -> float {
-        const int t = n * kC + tid;
-        return (tid < kC && n < NC && t < Tlen) ? __bfloat162float(beta[((size_t)b * Tlen + t) * H + h]) : 0.f;
-    };
+    auto rowop = [&](int par) -> uint32_t { return sb + L::ROWOP + (uint32_t)par * 32768; };
+    auto colop = [&](int par) -> uint32_t { return sb + L::COLOP + (uint32_t)par * 16384; };
 
-    constexpr uint32_t ID_CS = idesc_bf16(128, 64, 1, 0);
-    constexpr uint32_t ID_AP = idesc_bf16(128, 64, 1, 1);
+    constexpr uint32_t ID_CS = idesc_bf16(128, 128, 0, 1);
+    constexpr uint32_t ID_AP = idesc_bf16(128, 64, 0, 0);
     constexpr uint32_t ID_U = idesc_bf16(128, DVT, 0, 1);
-    constexpr uint32_t ID_WT = idesc_bf16(128, 64, 0, 0);
-    constexpr uint32_t ID_M1 = idesc_bf16(128, DVT, 1, 1);
-    constexpr uint32_t ID_M2 = idesc_bf16(128, DVT, 0, 1);
-
-    // ---- MMA issue helpers (thread 0)
-    auto mma_cumsum = [&]() {  // G^T[c][r] = sum_s la[s][c] * L[r][s]
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + L::G_COL, sdesc_sw128(sb + L::RAWG + kk * 2048, 8192, 1024),
-                        sdesc_sw128(sb + L::LMAT + kk * 32, 16, 1024), ID_CS, kk > 0);
-        mma_commit(bar.cs);
-    };
-    auto mma_ap = [&](int m, bool exact) {  // [KE; QE] KF^T
-        tc_fence_after();
-        if (!exact) {
-            const uint32_t col = sb + L::COLOP + (m & 1) * 16384;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_bf16_ss(tmem + L::APW_COL, sdesc_sw128(sb + L::ROWOP + kk * 4096, 1024, 2048),
-                            sdesc_sw128(col + kk * 2048, 1024, 1024), ID_AP, kk > 0);
-        }
-        mma_commit(bar.ap);
-    };
-    auto mma_uw = [&](int m) {  // U = [T'; 0] V into D1[m%2];  W'^T = KE^T T'^T (over A/P, already read)
-        tc_fence_after();
-        const uint32_t d1 = tmem + L::D1_COL + (m & 1) * DVT;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(d1, sdesc_sw128(sb + L::TZP + kk * 32, 16, 1024),
-                        sdesc_sw128(sb + L::RAWV + kk * 2048, 8192, 1024), ID_U, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + L::APW_COL, sdesc_sw128(sb + L::ROWOP + kk * 32, 16, 2048),
-                        sdesc_sw128(sb + L::TZP + kk * 32, 16, 1024), ID_WT, kk > 0);
-        mma_commit(bar.uw);
-    };
-    auto mma_1 = [&](int n) {  // D1[n%2] += [-W'; QE] (scaled S)
-        tc_fence_after();
-        const uint32_t d1 = tmem + L::D1_COL + (n & 1) * DVT;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ss(d1, sdesc_sw128(sb + L::ROWOP + kk * 4096, 1024, 2048),
-                        sdesc_sw128(sb + L::SOP + kk * 2 * L::SBO_V, 1024, L::SBO_V), ID_M1, 1);
-        mma_commit(bar.m1);
-    };
-    auto mma_2 = [&](int n) {  // R += KF^T delta ; D1[n%2] += [0; P] delta
-        tc_fence_after();
-        const uint32_t d1 = tmem + L::D1_COL + (n & 1) * DVT;
-        const uint32_t col = sb + L::COLOP + (n & 1) * 16384;
-        const uint32_t zp = sb + L::TZP + 8192 + (n & 1) * 16384;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + L::S_COL, sdesc_sw128(col + kk * 32, 16, 1024),
-                        sdesc_sw128(sb + L::DOP + kk * 2 * L::SBO_V, 1024, L::SBO_V), ID_M2, 1);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(d1, sdesc_sw128(zp + kk * 32, 16, 1024),
-                        sdesc_sw128(sb + L::DOP + kk * 2 * L::SBO_V, 1024, L::SBO_V), ID_M2, 1);
-        mma_commit(bar.m2);
-    };
-
-    // ---- P2 of chunk m (after its cumulative gate is in TMEM and its k, q tiles are in smem):
-    // thread <-> (channel c = trow, token half hf). Computes the three operand
-    // tiles into registers and the per-channel scales; returns the block-wide
-    // guard verdict. In the exact case it also builds A and P.
-    uint32_t opk[16], opq[16], opf[16];  // packed bf16 pairs along tokens
-    auto p2_compute = [&](int m) -> bool {
-        const int c = trow, r0 = 32 * hf;
-        uint32_t gv[32];
-        tmem_ld32(lane_addr + L::G_COL + 32 * hf, gv);
-        tmem_ld_wait(gv);
-        sEx[hf * 128 + c] = __uint_as_float(gv[31]);  // G_31 (hf = 0) / G_63 (hf = 1)
-        tc_fence_before();
-        nb_sync(NB_SIMT, kCompute);
-        const float Gm = sEx[c], Gl = sEx[128 + c];
-        float dev = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) dev = fmaxf(dev, fabsf(__uint_as_float(gv[i]) - Gm));
-        const bool bad = !(dev <= kGuard) || !(Gm >= -kGuard);
-        const bool exact = nb_or(NB_OR, kCompute, bad);
-        if (hf == 0) {
-            const float ek_prev = sEK[c];
-            if (!exact) {
-                const float s = __expf(Gm) * ek_prev;
-                sOpS[c] = s;
-                sTmS[c] = s;
-                sEK[c] = __expf(Gl - Gm);
-            } else {
-                sOpS[c] = ek_prev;
-                sTmS[c] = __expf(Gl) * ek_prev;
-                sEK[c] = 1.f;
-            }
-        }
-        if (exact) {
-            // exact A and P with per-pair exponentials; G staged as fp32 in the
-            // row-operand tile (free once MMA1 of the previous chunk completed)
-            if (m > 0) wait_all(bar.m1, m - 1);
-            float* sG = reinterpret_cast<float*>(sm + L::ROWOP);  // [64][128]
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sG[(r0 + i) * 128 + c] = __uint_as_float(gv[i]);
-            for (int i = tid; i < 64 * kLDA; i += kCompute) sA[i] = 0.f;
-            uint4* pz = reinterpret_cast<uint4*>(sm + L::TZP + 16384 + (m & 1) * 16384);
-            for (int i = tid; i < 8192 / 16; i += kCompute) pz[i] = make_uint4(0, 0, 0, 0);
-            nb_sync(NB_SIMT, kCompute);
-            uint8_t* pb = sm + L::TZP + 16384 + (m & 1) * 16384;
-            for (int p = tid; p < kC * (kC + 1) / 2; p += kCompute) {
-                int r = (int)((sqrtf(8.f * (float)p + 1.f) - 1.f) * 0.5f);
-                while ((r + 1) * (r + 2) / 2 <= p) ++r;
-                while (r * (r + 1) / 2 > p) --r;
-                const int s = p - r * (r + 1) / 2;
-                float a = 0.f, pp = 0.f;
-                for (int i = 0; i < kD; ++i) {
-                    const int cc = (i + p) & (kD - 1);
-                    const float ks = ld_bf16(sm + L::RAWK, raw_off(s, cc)) * __expf(sG[r * 128 + cc] - sG[s * 128 + cc]);
-                    a = fmaf(ld_bf16(sm + L::RAWK, raw_off(r, cc)), ks, a);
-                    pp = fmaf(ld_bf16(sm + L::RAWQ, raw_off(r, cc)), ks, pp);
-                }
-                if (s < r) sA[r * kLDA + s] = sBeta[r] * a;
-                *reinterpret_cast<__nv_bfloat16*>(pb + km_off(r, s)) = __float2bfloat16_rn(pp);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-            const int r = r0 + i;
-            const float k0 = ld_bf16(sm + L::RAWK, raw_off(r, c)), k1 = ld_bf16(sm + L::RAWK, raw_off(r + 1, c));
-            const float q0 = ld_bf16(sm + L::RAWQ, raw_off(r, c)), q1 = ld_bf16(sm + L::RAWQ, raw_off(r + 1, c));
-            const float g0 = __uint_as_float(gv[i]), g1 = __uint_as_float(gv[i + 1]);
-            float e0, e1, f0, f1;
-            if (!exact) {
-                e0 = __expf(g0 - Gm); e1 = __expf(g1 - Gm);
-                f0 = recip_bf16(e0); f1 = recip_bf16(e1);
-            } else {
-                e0 = __expf(g0); e1 = __expf(g1);
-                f0 = __expf(Gl - g0); f1 = __expf(Gl - g1);
-            }
-            opk[i / 2] = pack_bf16x2(k0 * e0, k1 * e1);
-            opq[i / 2] = pack_bf16x2(q0 * e0, q1 * e1);
-            opf[i / 2] = pack_bf16x2(k0 * f0, k1 * f1);
-        }
-        return exact;
-    };
-    auto p2_store = [&](int m) {
-        const int c = trow;
-        const uint32_t col = sb + L::COLOP + (m & 1) * 16384;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t chunk = (uint32_t)((4 * hf + j) ^ (c & 7)) << 4;
-            const uint32_t mn = (uint32_t)(c >> 3) * 2048 + (uint32_t)(c & 7) * 128 + chunk;
-            st_shared_v4(sb + L::ROWOP + mn, opk[4 * j], opk[4 * j + 1], opk[4 * j + 2], opk[4 * j + 3]);
-            st_shared_v4(sb + L::ROWOP + mn + 1024, opq[4 * j], opq[4 * j + 1], opq[4 * j + 2], opq[4 * j + 3]);
-            st_shared_v4(col + (uint32_t)(c >> 3) * 1024 + (uint32_t)(c & 7) * 128 + chunk, opf[4 * j], opf[4 * j + 1],
-                         opf[4 * j + 2], opf[4 * j + 3]);
-        }
-    };
-    // ---- P4 of chunk m: A (lanes 0-63) -> fp32 scratch; P (lanes 64-127) -> bf16 operand
-    auto p4 = [&](int m) {
-        uint32_t v[32];
-        tmem_ld32(lane_addr + L::APW_COL + 32 * hf, v);
-        tmem_ld_wait(v);
-        if (quad < 2) {
-            const int r = trow;
-            const float br = sBeta[r];
-            float* dst = sA + r * kLDA + 32 * hf;
-#pragma unroll
-            for (int u = 0; u < 32; u += 4) {
-                float4 f;
-                f.x = (32 * hf + u + 0 < r) ? br * __uint_as_float(v[u + 0]) : 0.f;
-                f.y = (32 * hf + u + 1 < r) ? br * __uint_as_float(v[u + 1]) : 0.f;
-                f.z = (32 * hf + u + 2 < r) ? br * __uint_as_float(v[u + 2]) : 0.f;
-                f.w = (32 * hf + u + 3 < r) ? br * __uint_as_float(v[u + 3]) : 0.f;
-                *reinterpret_cast<float4*>(dst + u) = f;
-            }
-        } else {
-            const int r = trow - 64;
-            const uint32_t pbase = sb + L::TZP + 16384 + (m & 1) * 16384;
-#pragma unroll
-            for (int jc = 0; jc < 4; ++jc) {
-                uint32_t w[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int s = 32 * hf + 8 * jc + 2 * u;
-                    const float p0 = (s <= r) ? __uint_as_float(v[8 * jc + 2 * u]) : 0.f;
-                    const float p1 = (s + 1 <= r) ? __uint_as_float(v[8 * jc + 2 * u + 1]) : 0.f;
-                    w[u] = pack_bf16x2(p0, p1);
-                }
-                st_shared_v4(pbase + r * 128 + ((((4 * hf + jc) ^ (r & 7))) << 4), w[0], w[1], w[2], w[3]);
-            }
-        }
-    };
-    // ---- P5: T = (I + A)^{-1}, written as T' = T Diag(beta) in bf16
-    auto store_tprime = [&](int r, int s, float t) {
-        *reinterpret_cast<__nv_bfloat16*>(sm + L::TZP + km_off(r, s)) = __float2bfloat16_rn(t * sBeta[s]);
-    };
-    auto p5 = [&]() {
-        {   // diagonal 16x16 blocks: four threads per column, rows q, q+4, q+8, q+12
-            const int a = tid >> 6, jc = (tid >> 2) & 15, q = tid & 3;
-            const float* Ab = sA + (16 * a) * kLDA + 16 * a;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f}, colv[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const float mine = (r == jc) ? 1.f : ((r > jc) ? -acc[r >> 2] : 0.f);
-                const float t = __shfl_sync(0xffffffffu, mine, (lane & ~3) | (r & 3));
-                if (q == (r & 3)) colv[r >> 2] = t;
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    if (q + 4 * i > r) acc[i] = fmaf(Ab[(q + 4 * i) * kLDA + r], t, acc[i]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = 16 * a + q + 4 * i, s = 16 * a + jc;
-                sT[r * kLDA + s] = colv[i];
-                store_tprime(r, s, colv[i]);
-            }
-        }
-        nb_sync(NB_SIMT, kCompute);
-        // Blocks below the diagonal on the tensor cores (m16n8k8, tf32): one
-        // warp per (block, 8-column half). N_ak = T_aa A_ak replaces A_ak.
-        auto put_t = [&](int a, int bb, int nt, const float (&acc)[4]) {  // T_ab = -acc
-            const int g = lane >> 2, t = lane & 3;
-            const int s = 16 * bb + 8 * nt + 2 * t;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int r = 16 * a + g + 8 * hh;
-                const float v0 = -acc[2 * hh], v1 = -acc[2 * hh + 1];
-                *reinterpret_cast<float2*>(sT + r * kLDA + s) = make_float2(v0, v1);
-                *reinterpret_cast<uint32_t*>(sm + L::TZP + km_off(r, s)) =
-                    pack_bf16x2(v0 * sBeta[s], v1 * sBeta[s + 1]);
-            }
-        };
-        for (int task = warp; task < 12; task += kCompute / 32) {
-            const int blk = task >> 1, nt = task & 1;
-            const int a = (blk == 0) ? 1 : (blk <= 2 ? 2 : 3);
-            const int k = (blk == 0) ? 0 : (blk == 1 ? 0 : (blk == 2 ? 1 : blk - 3));
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            mm16_ntile(acc, sT + (16 * a) * kLDA + 16 * a, sA + (16 * a) * kLDA + 16 * k, nt, lane);
-            __syncwarp();
-            const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                *reinterpret_cast<float2*>(sA + (16 * a + g + 8 * hh) * kLDA + 16 * k + 8 * nt + 2 * t) =
-                    make_float2(acc[2 * hh], acc[2 * hh + 1]);
-        }
-        nb_sync(NB_SIMT, kCompute);
-        // level d: T_ab = -sum_{k=b}^{a-1} N_ak T_kb, a - b = d
-#pragma unroll 1
-        for (int d = 1; d < 4; ++d) {
-            if (warp < 2 * (4 - d)) {
-                const int bb = warp >> 1, nt = warp & 1, a = bb + d;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int kb = bb; kb < a; ++kb)
-                    mm16_ntile(acc, sA + (16 * a) * kLDA + 16 * kb, sT + (16 * kb) * kLDA + 16 * bb, nt, lane);
-                put_t(a, bb, nt, acc);
-            }
-            nb_sync(NB_SIMT, kCompute);
-        }
-    };
-    // ---- P7 of chunk m: -W' (W'^T in TMEM, lane c, columns r) -> rows 0-63 of the row operand
-    auto p7 = [&]() {
-        const int cc = trow;
-        uint32_t v[32];
-        tmem_ld32(lane_addr + L::APW_COL + 32 * hf, v);
-        tmem_ld_wait(v);
-#pragma unroll
-        for (int jc = 0; jc < 4; ++jc) {
-            uint32_t w[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                w[u] = pack_bf16x2(-__uint_as_float(v[8 * jc + 2 * u]), -__uint_as_float(v[8 * jc + 2 * u + 1]));
-            const uint32_t off = (uint32_t)(cc >> 3) * 2048 + (uint32_t)(cc & 7) * 128 +
-                                 ((uint32_t)((4 * hf + jc) ^ (cc & 7)) << 4);
-            st_shared_v4(sb + L::ROWOP + off, w[0], w[1], w[2], w[3]);
-        }
-    };
-    // ---- S1 of chunk n: R -> bf16 operand (times the operand scale); R *= tensor-memory scale
-    auto s1 = [&]() {
-        const int cc = trow;
-        const float os = sOpS[cc], ts = sTmS[cc];
-#pragma unroll
-        for (int gq = 0; gq < NJ / 32; ++gq) {
-            const int jb = hf * NJ + 32 * gq;
-            uint32_t v[32];
-            tmem_ld32(lane_addr + L::S_COL + jb, v);
-            tmem_ld_wait(v);
-#pragma unroll
-            for (int jc = 0; jc < 4; ++jc) {
-                uint32_t w[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]) * os, __uint_as_float(v[8 * jc + 2 * u + 1]) * os);
-                const int j = jb + 8 * jc;
-                const uint32_t off = (uint32_t)(cc >> 3) * L::SBO_V + (uint32_t)(j >> 6) * 1024 +
-                                     (uint32_t)(cc & 7) * 128 + ((uint32_t)(((j & 63) >> 3) ^ (cc & 7)) << 4);
-                st_shared_v4(sb + L::SOP + off, w[0], w[1], w[2], w[3]);
-            }
-#pragma unroll
-            for (int u = 0; u < 32; ++u) v[u] = __float_as_uint(__uint_as_float(v[u]) * ts);
-            tmem_st32(lane_addr + L::S_COL + jb, v);
-        }
-        tmem_st_wait();
-    };
-    // ---- S3 of chunk n: delta (D1 lanes 0-63) -> bf16 operand, MN-major (K = token)
-    auto s3 = [&](int n) {
-        if (quad < 2) {
-            const int r = trow;
-            const uint32_t d1 = L::D1_COL + (n & 1) * DVT;
-#pragma unroll
-            for (int gq = 0; gq < NJ / 32; ++gq) {
-                const int jb = hf * NJ + 32 * gq;
-                uint32_t v[32];
-                tmem_ld32(lane_addr + d1 + jb, v);
-                tmem_ld_wait(v);
-#pragma unroll
-                for (int jc = 0; jc < 4; ++jc) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]), __uint_as_float(v[8 * jc + 2 * u + 1]));
-                    const int j = jb + 8 * jc;
-                    const uint32_t off = (uint32_t)(r >> 3) * L::SBO_V + (uint32_t)(j >> 6) * 1024 +
-                                         (uint32_t)(r & 7) * 128 + ((uint32_t)(((j & 63) >> 3) ^ (r & 7)) << 4);
-                    st_shared_v4(sb + L::DOP + off, w[0], w[1], w[2], w[3]);
-                }
-            }
-        }
-    };
-    // ---- S5 of chunk n: O (D1 lanes 64-127) -> global bf16
-    auto s5 = [&](int n) {
-        if (quad >= 2) {
-            const int r = trow - 64;
-            const int t0 = n * kC;
-            const uint32_t d1 = L::D1_COL + (n & 1) * DVT;
-#pragma unroll
-            for (int gq = 0; gq < NJ / 32; ++gq) {
-                const int jb = hf * NJ + 32 * gq;
-                uint32_t v[32];
-                tmem_ld32(lane_addr + d1 + jb, v);
-                tmem_ld_wait(v);
-                if (t0 + r < Tlen) {
-                    uint4* dst = reinterpret_cast<uint4*>(o + (((size_t)b * Tlen + t0 + r) * H + h) * kD + j0 + jb);
-#pragma unroll
-                    for (int jc = 0; jc < 4; ++jc) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(v[8 * jc + 0]), __uint_as_float(v[8 * jc + 1]));
-                        w.y = pack_bf16x2(__uint_as_float(v[8 * jc + 2]), __uint_as_float(v[8 * jc + 3]));
-                        w.z = pack_bf16x2(__uint_as_float(v[8 * jc + 4]), __uint_as_float(v[8 * jc + 5]));
-                        w.w = pack_bf16x2(__uint_as_float(v[8 * jc + 6]), __uint_as_float(v[8 * jc + 7]));
-                        dst[jc] = w;
-                    }
-                }
-                __syncwarp();  // (ragged tail) reconverge before the next tcgen05.ld
-            }
-        }
-    };
-    // compute warps: operands written -> visible to the control warp's next MMA
-    auto signal = [&](int id) {
-        fence_proxy_async_smem();
-        tc_fence_before();
-        nb_arrive(id, kThreads);
-    };
+    constexpr uint32_t ID_W = idesc_bf16(128, 128, 0, 1);
+    constexpr uint32_t ID_M1 = idesc_bf16(128, DVT, 0, 1);
+    constexpr uint32_t ID_M2S = idesc_bf16(128, DVT, 1, 1);
+    constexpr uint32_t ID_M2P = idesc_bf16(128, DVT, 0, 1);
 
     if (warp == kCtrlWarp) {
         // ============================================================ control warp
-        // Issues every TMA load and MMA (lane 0), in the order the compute
-        // warps signal that operands are ready. Never blocks the compute warps.
         const bool leader = lane == 0;
-        if (NC > 0) {
-            if (leader) {
-                issue_k(0);
-                issue_q(0);
-                issue_g(0);
-                issue_v(0);
+        auto issue_kq = [&](int m) {
+            const int par = m & 1;
+            uint8_t* dst = sm + L::ROWOP + par * 32768;
+            mbar_arrive_expect_tx(bars + BAR_KQ + par, 4 * 8192);
+            for (int x = 0; x < 2; ++x) {
+                tma_load_4d(dst + x * 16384, &tm_k, bars + BAR_KQ + par, 64 * x, h, m * kC, b);
+                tma_load_4d(dst + x * 16384 + 8192, &tm_q, bars + BAR_KQ + par, 64 * x, h, m * kC, b);
             }
-            __syncwarp();
-            wait_one(bar.g, 0);
-            if (leader) mma_cumsum();
-            __syncwarp();
-            wait_one(bar.cs, 0);
-            if (leader && NC > 1) issue_g(1);       // log_alpha tile consumed
-            __syncwarp();
-            nb_sync(NB_K, kThreads);                 // gate and k, q tiles of chunk 0 read
-            if (leader && NC > 1) {
-                issue_k(1);
-                issue_q(1);
-            }
-            __syncwarp();
-            nb_sync(NB_S3, kThreads);                // operands of chunk 0 stored
-            if (leader) mma_ap(0, *s_exact != 0);
-            __syncwarp();
-            if (NC > 1) {                            // gate of chunk 1, ready long before it is needed
-                wait_one(bar.g, 1);
-                if (leader) mma_cumsum();
-                __syncwarp();
-            }
-            nb_sync(NB_P5, kThreads);                // T' of chunk 0 stored
-            wait_one(bar.v, 0);
-            if (leader) mma_uw(0);
-            __syncwarp();
-        }
-        for (int n = 0; n < NC; ++n) {
-            const bool more = n + 1 < NC;
-            if (__syncthreads_or(*s_abort)) break;
-            nb_sync(NB_S1, kThreads);                // state operand of chunk n stored
-            if (leader) mma_1(n);
-            __syncwarp();
-            if (more) {
-                wait_one(bar.cs, n + 1);             // (issued one iteration earlier)
-                if (leader && n + 2 < NC) issue_g(n + 2);  // log_alpha tile consumed
-                __syncwarp();
-                nb_sync(NB_K, kThreads);             // gate and k, q tiles of chunk n+1 read
-                if (leader && n + 2 < NC) {
-                    issue_k(n + 2);
-                    issue_q(n + 2);
-                }
-                __syncwarp();
-            }
-            nb_sync(NB_S3, kThreads);                // delta(n) and operands of chunk n+1 stored
-            if (leader) {
-                if (more) mma_ap(n + 1, *s_exact != 0);
-                mma_2(n);
-            }
-            __syncwarp();
-            if (n + 2 < NC) {                        // gate of chunk n+2 (the gate TMEM columns are free)
-                wait_one(bar.g, n + 2);
-                if (leader) mma_cumsum();
-                __syncwarp();
-            }
-            wait_one(bar.m2, n);
-            if (leader && more) issue_v(n + 1);      // delta operand (on the v tile) consumed
-            __syncwarp();
-            if (more) {
-                nb_sync(NB_P5, kThreads);            // T' of chunk n+1 stored
-                wait_one(bar.v, n + 1);
-                if (leader) mma_uw(n + 1);
-                __syncwarp();
-            }
-        }
-        __syncthreads();
-    } else {
-        // ============================================================ compute warps
-        {   // initial state into TMEM (fp32, lane = key channel)
-            const int c = trow;
+        };
+        auto issue_g = [&](int m) {
+            const int par = m & 1;
+            uint8_t* dst = sm + L::COLOP + par * 16384;
+            mbar_arrive_expect_tx(bars + BAR_G + par, 2 * 8192);
+            for (int x = 0; x < 2; ++x) tma_load_4d(dst + x * 8192, &tm_g, bars + BAR_G + par, 64 * x, h, m * kC, b);
+        };
+        auto issue_v = [&](int m) {
+            mbar_arrive_expect_tx(bars + BAR_V, (DVT / 64) * 8192);
+            for (int x = 0; x < DVT / 64; ++x)
+                tma_load_4d(sm + L::RAWV + x * 8192, &tm_v, bars + BAR_V, j0 + 64 * x, h, m * kC, b);
+        };
+        auto mma_cs = [&](int m) {  // [G; G] = [L; L] g
+            tc_fence_after();
 #pragma unroll
-            for (int gq = 0; gq < NJ / 32; ++gq) {
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tmem + L::GC_COL, sdesc_sw128(sb + L::LMAT + kk * 32, 16, 1024),
+                            sdesc_sw128(colop(m & 1) + kk * 2048, 8192, 1024), ID_CS, kk > 0);
+            mma_commit(bars + BAR_CS);
+        };
+        if (leader) {
+            issue_kq(0);
+            issue_g(0);
+            issue_v(0);
+            if (NC > 1) {
+                issue_kq(1);
+                issue_g(1);
+            }
+            wait1(BAR_G, 0);
+            mma_cs(0);
+        }
+        __syncwarp();
+        for (int m = 0; m < NC; ++m) {
+            const int par = m & 1;
+            const bool more = m + 1 < NC;
+            nb_sync(NB_P2, kPrep + 32);  // operand tiles of chunk m stored, prefix sums read
+            if (leader) {
+                tc_fence_after();
+                if (!s_exact[par]) {  // [KE; QE] KF^T -> [A; P]
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ss(tmem + L::APW_COL,
+                                    sdesc_sw128(rowop(par) + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                    sdesc_sw128(colop(par) + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), ID_AP,
+                                    kk > 0);
+                }
+                mma_commit(bars + BAR_AP);
+                if (m >= 1 && more) {
+                    // the buffers of parity m+1 were last read by the MMAs of chunk m-1
+                    wait1(BAR_M1B + (par ^ 1), (uint32_t)((m - 1) >> 1));
+                    issue_kq(m + 1);
+                    wait1(BAR_M2B + (par ^ 1), (uint32_t)((m - 1) >> 1));
+                    issue_g(m + 1);
+                }
+            }
+            __syncwarp();
+            nb_sync(NB_P5, kPrep + 32);  // T' of chunk m stored
+            if (leader) {
+                wait1(BAR_V, (uint32_t)m);
+                if (m >= 1) wait1(BAR_D1, (uint32_t)(m - 1));
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // [U; 0] = [T'; 0] v
+                    mma_bf16_ss(tmem + L::D1_COL, sdesc_sw128(sb + L::TZP + kk * 32, 16, 1024),
+                                sdesc_sw128(sb + L::RAWV + kk * 2048, 8192, 1024), ID_U, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // [W'; 0] = [T'; 0] KE
+                    mma_bf16_ss(tmem + L::APW_COL, sdesc_sw128(sb + L::TZP + kk * 32, 16, 1024),
+                                sdesc_sw128(rowop(par) + kk * 2048, 16384, 1024), ID_W, kk > 0);
+                mma_commit(bars + BAR_UW);
+                if (more) {
+                    wait1(BAR_G + (par ^ 1), (uint32_t)((m + 1) >> 1));
+                    mma_cs(m + 1);
+                    wait1(BAR_UW, (uint32_t)m);  // v tile consumed
+                    issue_v(m + 1);
+                }
+            }
+            __syncwarp();
+        }
+    } else if (warp >= kChainWarp0) {
+        // ============================================================ chain warps
+        // lane row = 32 * quad + lane: a key channel of the state, a token row of D1
+        const int row = 32 * quad + lane;
+        const bool issuer = (quad == 0) && (lane == 0);
+        {   // initial state into TMEM (fp32, lane = key channel)
+#pragma unroll
+            for (int gq = 0; gq < DVT / 32; ++gq) {
                 uint32_t r[32];
-                const int jb = hf * NJ + 32 * gq;
                 if (S0) {
-                    const float4* src = reinterpret_cast<const float4*>(S0 + ((size_t)bh * kD + c) * kD + j0 + jb);
+                    const float4* src = reinterpret_cast<const float4*>(S0 + ((size_t)bh * kD + row) * kD + j0 + 32 * gq);
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const float4 v = src[u];
@@ -765,90 +423,471 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll
                     for (int u = 0; u < 32; ++u) r[u] = 0u;
                 }
-                tmem_st32(lane_addr + L::S_COL + jb, r);
+                tmem_st32(lane_addr + L::S_COL + 32 * gq, r);
             }
             tmem_st_wait();
-        }
-        float beta_next = 0.f;
-        if (NC > 0) {
-            if (tid < kC) sBeta[tid] = load_beta(0);
-            beta_next = load_beta(1);
-            wait_all(bar.cs, 0);
-            wait_all(bar.k, 0);
-            wait_all(bar.q, 0);
-            nb_sync(NB_SIMT, kCompute);  // sBeta visible
-            const bool exact0 = p2_compute(0);
-            if (tid == 0) *s_exact = exact0;
-            __syncwarp();
-            nb_sync(NB_SIMT, kCompute);  // (exact path) staged gate values read before the tiles are overwritten
-            nb_arrive(NB_K, kThreads);
-            p2_store(0);
-            signal(NB_S3);
-            wait_all(bar.ap, 0);
-            if (!exact0) p4(0);
-            nb_sync(NB_SIMT, kCompute);
-            p5();
-            signal(NB_P5);
-            wait_all(bar.uw, 0);
-            p7();
-        }
-        for (int n = 0; n < NC; ++n) {
-            const bool more = n + 1 < NC;
             tc_fence_before();
-            if (__syncthreads_or(*s_abort)) break;
-            s1();
-            signal(NB_S1);
-            bool exact_next = false;
-            if (more) {
-                if (tid < kC) sBeta[tid] = beta_next;
-                beta_next = load_beta(n + 2);
-                wait_all(bar.cs, n + 1);
-                wait_all(bar.k, n + 1);
-                wait_all(bar.q, n + 1);
-                nb_sync(NB_SIMT, kCompute);  // sBeta(n+1) visible
-                exact_next = p2_compute(n + 1);
-                if (tid == 0) *s_exact = exact_next;
+            nb_sync(NB_CH, 128);
+            tc_fence_after();
+        }
+        // state rows -> bf16 operand (times the operand scale), R *= tensor-memory scale
+        auto s1 = [&](int par) {
+            const float os = sOpS[par * 128 + row], ts = sTmS[par * 128 + row];
+            const int i = row & 63;
+#pragma unroll
+            for (int gq = 0; gq < DVT / 32; ++gq) {
+                uint32_t v[32];
+                tmem_ld32(lane_addr + L::S_COL + 32 * gq, v);
+                tmem_ld_wait(v);
+#pragma unroll
+                for (int jc = 0; jc < 4; ++jc) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]) * os,
+                                           __uint_as_float(v[8 * jc + 2 * u + 1]) * os);
+                    const int j = 32 * gq + 8 * jc;
+                    const uint32_t off = (uint32_t)(i >> 3) * L::SBO_V + (uint32_t)(j >> 6) * 1024 +
+                                         (uint32_t)(i & 7) * 128 + ((uint32_t)(((j & 63) >> 3) ^ (i & 7)) << 4);
+                    st_shared_v4(sb + L::SOP + off, w[0], w[1], w[2], w[3]);
+                }
+#pragma unroll
+                for (int u = 0; u < 32; ++u) v[u] = __float_as_uint(__uint_as_float(v[u]) * ts);
+                tmem_st32(lane_addr + L::S_COL + 32 * gq, v);
+            }
+            tmem_st_wait();
+        };
+        for (int n = 0; n < NC; ++n) {
+            const int par = n & 1;
+            const uint32_t ph = (uint32_t)(n >> 1);
+            if (quad < 2) {
+                if (n > 0) waitw(BAR_M2, (uint32_t)(n - 1));  // state update of the previous chunk done
+                waitw(BAR_SC + par, ph);
+                s1(par);  // key channels 0-63
+                fence_proxy_async_smem();
+                tc_fence_before();
+                nb_sync(NB_CHA, 64);
+                if (quad == 0) {
+                    if (issuer) {
+                        wait1(BAR_RR + par, ph);  // row operand of chunk n stored
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16_ss(tmem + L::D1_COL, sdesc_sw128(rowop(par) + kk * 32, 16, 1024),
+                                        sdesc_sw128(sb + L::SOP + kk * 2 * L::SBO_V, 1024, L::SBO_V), ID_M1, 1);
+                        mma_commit(bars + BAR_M1A);
+                    }
+                    __syncwarp();
+                    nb_sync(NB_CHB, 96);  // key channels 64-127 stored
+                    if (issuer) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16_ss(tmem + L::D1_COL, sdesc_sw128(rowop(par) + 16384 + kk * 32, 16, 1024),
+                                        sdesc_sw128(sb + L::SOP + kk * 2 * L::SBO_V, 1024, L::SBO_V), ID_M1, 1);
+                        mma_commit(bars + BAR_M1);
+                        mma_commit(bars + BAR_M1B + par);
+                    }
+                    __syncwarp();
+                }
+                waitw(BAR_M1, (uint32_t)n);
+                {   // delta (D1 rows 0-63) -> bf16 operand over the state operand
+                    const int r = row;
+#pragma unroll
+                    for (int gq = 0; gq < DVT / 32; ++gq) {
+                        uint32_t v[32];
+                        tmem_ld32(lane_addr + L::D1_COL + 32 * gq, v);
+                        tmem_ld_wait(v);
+#pragma unroll
+                        for (int jc = 0; jc < 4; ++jc) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]),
+                                                   __uint_as_float(v[8 * jc + 2 * u + 1]));
+                            const int j = 32 * gq + 8 * jc;
+                            const uint32_t off = (uint32_t)(r >> 3) * L::SBO_V + (uint32_t)(j >> 6) * 1024 +
+                                                 (uint32_t)(r & 7) * 128 +
+                                                 ((uint32_t)(((j & 63) >> 3) ^ (r & 7)) << 4);
+                            st_shared_v4(sb + L::DOP + off, w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                nb_sync(NB_CHA, 64);
+                if (issuer) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)  // R += KF^T delta
+                        mma_bf16_ss(tmem + L::S_COL, sdesc_sw128(colop(par) + kk * 2048, 8192, 1024),
+                                    sdesc_sw128(sb + L::DOP + kk * 2 * L::SBO_V, 1024, L::SBO_V), ID_M2S, 1);
+                    const uint32_t yp = sb + L::SP + (uint32_t)par * 8192 - 8192;  // [Y; P], Y = the 8 KB before P
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)  // D1 rows 64-127 += P delta
+                        mma_bf16_ss(tmem + L::D1_COL, sdesc_sw128(yp + kk * 32, 16, 1024),
+                                    sdesc_sw128(sb + L::DOP + kk * 2 * L::SBO_V, 1024, L::SBO_V), ID_M2P, 1);
+                    mma_commit(bars + BAR_M2);
+                    mma_commit(bars + BAR_M2B + par);
+                }
                 __syncwarp();
-                nb_sync(NB_SIMT, kCompute);  // k, q tiles (and the exact path's staged gate) read
-                nb_arrive(NB_K, kThreads);
-            }
-            wait_all(bar.m1, n);
-            s3(n);
-            if (more) p2_store(n + 1);
-            signal(NB_S3);
-            if (more) {
-                wait_all(bar.ap, n + 1);
-                if (!exact_next) p4(n + 1);
-                nb_sync(NB_SIMT, kCompute);
-                p5();
-                signal(NB_P5);
-            }
-            wait_all(bar.m2, n);
-            s5(n);
-            if (more) {
-                wait_all(bar.uw, n + 1);
-                p7();
+            } else {
+                waitw(BAR_SC + par, ph);
+                waitw(BAR_M1A, (uint32_t)n);  // first half of the state operand consumed
+                s1(par);                      // key channels 64-127
+                fence_proxy_async_smem();
+                tc_fence_before();
+                nb_arrive(NB_CHB, 96);
+                waitw(BAR_M2, (uint32_t)n);
+                {   // O (D1 rows 64-127) -> global bf16
+                    const int r = row - 64;
+                    const int t0 = n * kC;
+#pragma unroll
+                    for (int gq = 0; gq < DVT / 32; ++gq) {
+                        uint32_t v[32];
+                        tmem_ld32(lane_addr + L::D1_COL + 32 * gq, v);
+                        tmem_ld_wait(v);
+                        if (t0 + r < Tlen) {
+                            uint4* dst = reinterpret_cast<uint4*>(o + (((size_t)b * Tlen + t0 + r) * H + h) * kD + j0 +
+                                                                  32 * gq);
+#pragma unroll
+                            for (int jc = 0; jc < 4; ++jc) {
+                                uint4 w;
+                                w.x = pack_bf16x2(__uint_as_float(v[8 * jc + 0]), __uint_as_float(v[8 * jc + 1]));
+                                w.y = pack_bf16x2(__uint_as_float(v[8 * jc + 2]), __uint_as_float(v[8 * jc + 3]));
+                                w.z = pack_bf16x2(__uint_as_float(v[8 * jc + 4]), __uint_as_float(v[8 * jc + 5]));
+                                w.w = pack_bf16x2(__uint_as_float(v[8 * jc + 6]), __uint_as_float(v[8 * jc + 7]));
+                                dst[jc] = w;
+                            }
+                        }
+                        __syncwarp();  // (ragged tail) reconverge before the next tcgen05.ld
+                    }
+                }
+                tc_fence_before();
+                nb_sync(NB_CHC, 64);
+                if (quad == 2 && lane == 0) mbar_arrive(bars + BAR_D1);
+                __syncwarp();
             }
         }
         // ------------------------------------------------------------ final state S = e^{G_last - G_m} R
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+        if (quad < 2) waitw(BAR_M2, (uint32_t)(NC - 1));
         if (ST && !*s_abort) {
-            const int c = trow;
-            const float ek = sEK[c];
+            const float ek = sEK[row];
 #pragma unroll
-            for (int gq = 0; gq < NJ / 32; ++gq) {
-                const int jb = hf * NJ + 32 * gq;
+            for (int gq = 0; gq < DVT / 32; ++gq) {
                 uint32_t v[32];
-                tmem_ld32(lane_addr + L::S_COL + jb, v);
+                tmem_ld32(lane_addr + L::S_COL + 32 * gq, v);
                 tmem_ld_wait(v);
-                float4* dst = reinterpret_cast<float4*>(ST + ((size_t)bh * kD + c) * kD + j0 + jb);
+                float4* dst = reinterpret_cast<float4*>(ST + ((size_t)bh * kD + row) * kD + j0 + 32 * gq);
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
                     dst[u] = make_float4(__uint_as_float(v[4 * u]) * ek, __uint_as_float(v[4 * u + 1]) * ek,
                                          __uint_as_float(v[4 * u + 2]) * ek, __uint_as_float(v[4 * u + 3]) * ek);
             }
+        }
+    } else {
+        // ============================================================ prep warps
+        const int hf = warp >> 2;
+        const int tok = 32 * (quad & 1) + lane;  // P2: token of this thread
+        const int cb = 2 * (quad >> 1) + hf;     // P2: 32-channel block of this thread
+        auto load_beta = [&](int m) -> float {
+            const int t = m * kC + tid;
+            return (tid < kC && m < NC && t < Tlen) ? __bfloat162float(beta[((size_t)b * Tlen + t) * H + h]) : 0.f;
+        };
+
+        // ---- P2 of chunk m: prefix sums from TMEM, guard, per-channel scales;
+        // KE/QE over the raw k/q rows, KF over the log_alpha tile. Exact path:
+        // A -> sA, P -> sP from per-pair exponentials.
+        auto p2 = [&](int m) -> bool {
+            const int par = m & 1;
+            uint32_t gr[32];
+            tmem_ld32(lane_addr + L::GC_COL + 32 * cb, gr);
+            tmem_ld_wait(gr);
+            if (tok == 31 || tok == 63) {
+                float* dst = (tok == 31 ? sGm : sGl) + 32 * cb;
+#pragma unroll
+                for (int u = 0; u < 32; u += 4)
+                    *reinterpret_cast<float4*>(dst + u) = make_float4(
+                        __uint_as_float(gr[u]), __uint_as_float(gr[u + 1]), __uint_as_float(gr[u + 2]),
+                        __uint_as_float(gr[u + 3]));
+            }
+            nb_sync(NB_PREP, kPrep);
+            float gm[32];
+            bool bad = false;
+#pragma unroll
+            for (int u = 0; u < 32; u += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(sGm + 32 * cb + u);
+                gm[u] = x.x; gm[u + 1] = x.y; gm[u + 2] = x.z; gm[u + 3] = x.w;
+            }
+#pragma unroll
+            for (int u = 0; u < 32; ++u)
+                bad |= !(fabsf(__uint_as_float(gr[u]) - gm[u]) <= kGuard) || !(gm[u] >= -kGuard);
+            const bool exact = nb_or(NB_OR, kPrep, bad);
+            if (tid < kD) {
+                const int c = tid;
+                const float g_m = sGm[c], g_l = sGl[c], ek_prev = sEK[c];
+                if (!exact) {
+                    const float s = __expf(g_m) * ek_prev;
+                    sOpS[par * 128 + c] = s;
+                    sTmS[par * 128 + c] = s;
+                    sEK[c] = __expf(g_l - g_m);
+                } else {
+                    sOpS[par * 128 + c] = ek_prev;
+                    sTmS[par * 128 + c] = __expf(g_l) * ek_prev;
+                    sEK[c] = 1.f;
+                }
+            }
+            const uint32_t rop = rowop(par);
+            if (exact) {
+                // gate as fp32 [64][128] in the A/T scratch (free until P4)
+                float* sG = reinterpret_cast<float*>(sm + L::SCR);
+#pragma unroll
+                for (int u = 0; u < 32; u += 4)
+                    *reinterpret_cast<float4*>(sG + tok * 128 + 32 * cb + u) = make_float4(
+                        __uint_as_float(gr[u]), __uint_as_float(gr[u + 1]), __uint_as_float(gr[u + 2]),
+                        __uint_as_float(gr[u + 3]));
+                nb_sync(NB_PREP, kPrep);
+                const uint8_t* rk = sm + L::ROWOP + par * 32768;
+                float av[9], pv[9];
+#pragma unroll
+                for (int i = 0; i < 9; ++i) {
+                    av[i] = 0.f;
+                    pv[i] = 0.f;
+                    const int p = tid + kPrep * i;
+                    if (p < kC * (kC + 1) / 2) {
+                        int r = (int)((sqrtf(8.f * (float)p + 1.f) - 1.f) * 0.5f);
+                        while ((r + 1) * (r + 2) / 2 <= p) ++r;
+                        while (r * (r + 1) / 2 > p) --r;
+                        const int s = p - r * (r + 1) / 2;
+                        float a = 0.f, pp = 0.f;
+                        for (int i2 = 0; i2 < kD; ++i2) {
+                            const int cc = (i2 + p) & (kD - 1);
+                            const float ks = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(s, cc))) *
+                                             __expf(sG[r * 128 + cc] - sG[s * 128 + cc]);
+                            a = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(r, cc))), ks, a);
+                            pp = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(64 + r, cc))),
+                                      ks, pp);
+                        }
+                        av[i] = (s < r) ? sBeta[r] * a : 0.f;
+                        pv[i] = pp;
+                    }
+                }
+                nb_sync(NB_PREP, kPrep);  // gate staging read
+                for (int i = tid; i < 64 * kLDA; i += kPrep) sA[i] = 0.f;
+                for (int i = tid; i < 8192 / 16; i += kPrep)
+                    st_shared_v4(sb + L::SP + par * 8192 + 16 * i, 0u, 0u, 0u, 0u);
+                nb_sync(NB_PREP, kPrep);
+#pragma unroll
+                for (int i = 0; i < 9; ++i) {
+                    const int p = tid + kPrep * i;
+                    if (p < kC * (kC + 1) / 2) {
+                        int r = (int)((sqrtf(8.f * (float)p + 1.f) - 1.f) * 0.5f);
+                        while ((r + 1) * (r + 2) / 2 <= p) ++r;
+                        while (r * (r + 1) / 2 > p) --r;
+                        const int s = p - r * (r + 1) / 2;
+                        sA[r * kLDA + s] = av[i];
+                        *reinterpret_cast<__nv_bfloat16*>(sm + L::SP + par * 8192 + km_off(r, s)) =
+                            __float2bfloat16_rn(pv[i]);
+                    }
+                }
+            }
+            // operand tiles, in place: 4 chunks of 8 channels of this thread's row
+#pragma unroll
+            for (int u4 = 0; u4 < 4; ++u4) {
+                const int c0 = 32 * cb + 8 * u4;
+                const uint32_t ko = rop_off(tok, c0);
+                const uint32_t fo = (uint32_t)((c0 >> 6) * 8192 + tok * 128 + ((((c0 & 63) >> 3) ^ (tok & 7)) << 4));
+                const uint4 kv = ld_shared_v4(rop + ko);
+                const uint4 qv = ld_shared_v4(rop + ko + 8192);
+                const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w}, qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                uint32_t ke[4], qe[4], kf[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = 8 * u4 + 2 * u;
+                    const float g0 = __uint_as_float(gr[e]), g1 = __uint_as_float(gr[e + 1]);
+                    float e0, e1, f0, f1;
+                    if (!exact) {
+                        e0 = __expf(g0 - gm[e]);
+                        e1 = __expf(g1 - gm[e + 1]);
+                        f0 = recip_bf16(e0);
+                        f1 = recip_bf16(e1);
+                    } else {
+                        const float l0 = sGl[c0 + 2 * u], l1 = sGl[c0 + 2 * u + 1];
+                        e0 = __expf(g0);
+                        e1 = __expf(g1);
+                        f0 = __expf(l0 - g0);
+                        f1 = __expf(l1 - g1);
+                    }
+                    const float k0 = bf16_lo(kw[u]), k1 = bf16_hi(kw[u]);
+                    const float q0 = bf16_lo(qw[u]), q1 = bf16_hi(qw[u]);
+                    ke[u] = pack_bf16x2(k0 * e0, k1 * e1);
+                    qe[u] = pack_bf16x2(q0 * e0, q1 * e1);
+                    kf[u] = pack_bf16x2(k0 * f0, k1 * f1);
+                }
+                st_shared_v4(rop + ko, ke[0], ke[1], ke[2], ke[3]);
+                st_shared_v4(rop + ko + 8192, qe[0], qe[1], qe[2], qe[3]);
+                st_shared_v4(colop(par) + fo, kf[0], kf[1], kf[2], kf[3]);
+            }
+            return exact;
+        };
+        // ---- P4: A (APW lanes 0-63) -> fp32 scratch (beta_r, strictly lower);
+        // P (lanes 64-127) -> bf16 K-major tile of this parity (lower incl.)
+        auto p4 = [&](int par) {
+            uint32_t v[32];
+            tmem_ld32(lane_addr + L::APW_COL + 32 * hf, v);
+            tmem_ld_wait(v);
+            if (quad < 2) {
+                const int r = 32 * quad + lane;
+                const float br = sBeta[r];
+                float* dst = sA + r * kLDA + 32 * hf;
+#pragma unroll
+                for (int u = 0; u < 32; u += 4) {
+                    float4 f;
+                    f.x = (32 * hf + u + 0 < r) ? br * __uint_as_float(v[u + 0]) : 0.f;
+                    f.y = (32 * hf + u + 1 < r) ? br * __uint_as_float(v[u + 1]) : 0.f;
+                    f.z = (32 * hf + u + 2 < r) ? br * __uint_as_float(v[u + 2]) : 0.f;
+                    f.w = (32 * hf + u + 3 < r) ? br * __uint_as_float(v[u + 3]) : 0.f;
+                    *reinterpret_cast<float4*>(dst + u) = f;
+                }
+            } else {
+                const int r = 32 * (quad - 2) + lane;
+#pragma unroll
+                for (int jc = 0; jc < 4; ++jc) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int s = 32 * hf + 8 * jc + 2 * u;
+                        const float p0 = (s <= r) ? __uint_as_float(v[8 * jc + 2 * u]) : 0.f;
+                        const float p1 = (s + 1 <= r) ? __uint_as_float(v[8 * jc + 2 * u + 1]) : 0.f;
+                        w[u] = pack_bf16x2(p0, p1);
+                    }
+                    st_shared_v4(sb + L::SP + par * 8192 + r * 128 + (((4 * hf + jc) ^ (r & 7)) << 4), w[0], w[1],
+                                 w[2], w[3]);
+                }
+            }
+        };
+        // ---- P5: T = (I + A)^{-1} -> T' = T Diag(beta), bf16, rows 0-63 of [T'; 0]
+        auto store_tprime = [&](int r, int s, float t) {
+            *reinterpret_cast<__nv_bfloat16*>(sm + L::TZP + km_off(r, s)) = __float2bfloat16_rn(t * sBeta[s]);
+        };
+        auto p5 = [&]() {
+            {   // diagonal 16x16 blocks: four threads per column, rows q, q+4, q+8, q+12
+                const int a = tid >> 6, jc = (tid >> 2) & 15, q = tid & 3;
+                const float* Ab = sA + (16 * a) * kLDA + 16 * a;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f}, colv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    const float mine = (r == jc) ? 1.f : ((r > jc) ? -acc[r >> 2] : 0.f);
+                    const float t = __shfl_sync(0xffffffffu, mine, (lane & ~3) | (r & 3));
+                    if (q == (r & 3)) colv[r >> 2] = t;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (q + 4 * i > r) acc[i] = fmaf(Ab[(q + 4 * i) * kLDA + r], t, acc[i]);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = 16 * a + q + 4 * i, s = 16 * a + jc;
+                    sT[r * kLDA + s] = colv[i];
+                    store_tprime(r, s, colv[i]);
+                }
+            }
+            nb_sync(NB_PREP, kPrep);
+            // Blocks below the diagonal on the tensor cores (m16n8k8, tf32): one
+            // warp per (block, 8-column half). N_ak = T_aa A_ak replaces A_ak.
+            auto put_t = [&](int a, int bb, int nt, const float (&acc)[4]) {  // T_ab = -acc
+                const int g = lane >> 2, t = lane & 3;
+                const int s = 16 * bb + 8 * nt + 2 * t;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int r = 16 * a + g + 8 * hh;
+                    const float v0 = -acc[2 * hh], v1 = -acc[2 * hh + 1];
+                    *reinterpret_cast<float2*>(sT + r * kLDA + s) = make_float2(v0, v1);
+                    *reinterpret_cast<uint32_t*>(sm + L::TZP + km_off(r, s)) =
+                        pack_bf16x2(v0 * sBeta[s], v1 * sBeta[s + 1]);
+                }
+            };
+            for (int task = warp; task < 12; task += kPrep / 32) {
+                const int blk = task >> 1, nt = task & 1;
+                const int a = (blk == 0) ? 1 : (blk <= 2 ? 2 : 3);
+                const int k = (blk == 0) ? 0 : (blk == 1 ? 0 : (blk == 2 ? 1 : blk - 3));
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                mm16_ntile(acc, sT + (16 * a) * kLDA + 16 * a, sA + (16 * a) * kLDA + 16 * k, nt, lane);
+                __syncwarp();
+                const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    *reinterpret_cast<float2*>(sA + (16 * a + g + 8 * hh) * kLDA + 16 * k + 8 * nt + 2 * t) =
+                        make_float2(acc[2 * hh], acc[2 * hh + 1]);
+            }
+            nb_sync(NB_PREP, kPrep);
+            // level d: T_ab = -sum_{k=b}^{a-1} N_ak T_kb, a - b = d
+#pragma unroll 1
+            for (int d = 1; d < 4; ++d) {
+                if (warp < 2 * (4 - d)) {
+                    const int bb = warp >> 1, nt = warp & 1, a = bb + d;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int kb = bb; kb < a; ++kb)
+                        mm16_ntile(acc, sA + (16 * a) * kLDA + 16 * kb, sT + (16 * kb) * kLDA + 16 * bb, nt, lane);
+                    put_t(a, bb, nt, acc);
+                }
+                if (d < 3) nb_sync(NB_PREP, kPrep);
+            }
+        };
+        // ---- P7: [W'; 0] (APW lanes 0-63) -> -W' over the KE rows
+        auto p7 = [&](int par) {
+            if (quad < 2) {
+                const int r = 32 * quad + lane;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_addr + L::APW_COL + 64 * hf + 32 * hh, v);
+                    tmem_ld_wait(v);
+#pragma unroll
+                    for (int jc = 0; jc < 4; ++jc) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            w[u] = pack_bf16x2(-__uint_as_float(v[8 * jc + 2 * u]),
+                                               -__uint_as_float(v[8 * jc + 2 * u + 1]));
+                        st_shared_v4(rowop(par) + hf * 16384 + r * 128 + (((4 * hh + jc) ^ (r & 7)) << 4), w[0],
+                                     w[1], w[2], w[3]);
+                    }
+                }
+            }
+        };
+
+        float beta_next = load_beta(0);
+        for (int m = 0; m < NC; ++m) {
+            const int par = m & 1;
+            const uint32_t ph = (uint32_t)(m >> 1);
+            if (tid < kC) sBeta[tid] = beta_next;
+            beta_next = load_beta(m + 1);
+            waitw(BAR_CS, (uint32_t)m);
+            waitw(BAR_KQ + par, ph);
+            if (m >= 2) waitw(BAR_M2B + par, ph - 1);  // P (and KF) of chunk m-2 consumed
+            nb_sync(NB_PREP, kPrep);                    // beta of chunk m visible
+            const bool exact = p2(m);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            nb_sync(NB_PREP, kPrep);
+            if (tid == 0) {
+                s_exact[par] = exact;
+                mbar_arrive(bars + BAR_SC + par);
+            }
+            nb_arrive(NB_P2, kPrep + 32);
+            waitw(BAR_AP, (uint32_t)m);
+            if (!exact) p4(par);
+            nb_sync(NB_PREP, kPrep);
+            p5();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            nb_arrive(NB_P5, kPrep + 32);
+            waitw(BAR_UW, (uint32_t)m);
+            p7(par);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            nb_sync(NB_PREP, kPrep);
+            if (tid == 0) mbar_arrive(bars + BAR_RR + par);
         }
     }
     tc_fence_before();
