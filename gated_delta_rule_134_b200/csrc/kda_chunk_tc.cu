@@ -311,6 +311,18 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     constexpr uint32_t ID_M1 = idesc_bf16(128, DVT, 0, 1);
     constexpr uint32_t ID_M2S = idesc_bf16(128, DVT, 1, 1);
     constexpr uint32_t ID_M2P = idesc_bf16(128, DVT, 0, 1);
+    // Shared-memory descriptors, built once: the address field holds addr >> 4,
+    // so an offset of x bytes inside a tile is a plain add of x >> 4.
+    auto dadd = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+    const uint64_t dLMAT = sdesc_sw128(sb + L::LMAT, 16, 1024);          // K-major A
+    const uint64_t dTZP = sdesc_sw128(sb + L::TZP, 16, 1024);            // K-major A
+    const uint64_t dROWK = sdesc_sw128(sb + L::ROWOP, 16, 1024);         // row operand as K-major A
+    const uint64_t dROWN = sdesc_sw128(sb + L::ROWOP, 16384, 1024);      // its KE rows as MN-major B
+    const uint64_t dCOLK = sdesc_sw128(sb + L::COLOP, 16, 1024);         // KF as K-major B
+    const uint64_t dCOLN = sdesc_sw128(sb + L::COLOP, 8192, 1024);       // g as MN-major B, KF^T as MN-major A
+    const uint64_t dV = sdesc_sw128(sb + L::RAWV, 8192, 1024);           // MN-major B
+    const uint64_t dSOP = sdesc_sw128(sb + L::SOP, 1024, L::SBO_V);      // MN-major B (S, then delta)
+    const uint64_t dYP = sdesc_sw128(sb + L::SP - 8192, 16, 1024);       // [Y; P] as K-major A
 
     if (warp == kCtrlWarp) {
         // ============================================================ control warp
@@ -339,8 +351,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + L::GC_COL, sdesc_sw128(sb + L::LMAT + kk * 32, 16, 1024),
-                            sdesc_sw128(colop(m & 1) + kk * 2048, 8192, 1024), ID_CS, kk > 0);
+                mma_bf16_ss(tmem + L::GC_COL, dadd(dLMAT, kk * 32), dadd(dCOLN, (m & 1) * 16384 + kk * 2048), ID_CS,
+                            kk > 0);
             mma_commit(bars + BAR_CS);
         };
         if (leader) {
@@ -358,24 +370,28 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         for (int m = 0; m < NC; ++m) {
             const int par = m & 1;
             const bool more = m + 1 < NC;
+            if (leader && m >= 1 && more) {
+                // the buffers of parity m+1 were last read by the MMAs of chunk m-1;
+                // reload them while the prep warps still work on chunk m
+                wait1(BAR_M1B + (par ^ 1), (uint32_t)((m - 1) >> 1));
+                issue_kq(m + 1);
+                wait1(BAR_M2B + (par ^ 1), (uint32_t)((m - 1) >> 1));
+                issue_g(m + 1);
+            }
+            __syncwarp();
             nb_sync(NB_P2, kPrep + 32);  // operand tiles of chunk m stored, prefix sums read
             if (leader) {
                 tc_fence_after();
                 if (!s_exact[par]) {  // [KE; QE] KF^T -> [A; P]
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ss(tmem + L::APW_COL,
-                                    sdesc_sw128(rowop(par) + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                    sdesc_sw128(colop(par) + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), ID_AP,
-                                    kk > 0);
+                        mma_bf16_ss(tmem + L::APW_COL, dadd(dROWK, par * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32),
+                                    dadd(dCOLK, par * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32), ID_AP, kk > 0);
                 }
                 mma_commit(bars + BAR_AP);
-                if (m >= 1 && more) {
-                    // the buffers of parity m+1 were last read by the MMAs of chunk m-1
-                    wait1(BAR_M1B + (par ^ 1), (uint32_t)((m - 1) >> 1));
-                    issue_kq(m + 1);
-                    wait1(BAR_M2B + (par ^ 1), (uint32_t)((m - 1) >> 1));
-                    issue_g(m + 1);
+                if (more) {  // prefix sums of chunk m+1, ready before the prep warps need them
+                    wait1(BAR_G + (par ^ 1), (uint32_t)((m + 1) >> 1));
+                    mma_cs(m + 1);
                 }
             }
             __syncwarp();
@@ -386,16 +402,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)  // [U; 0] = [T'; 0] v
-                    mma_bf16_ss(tmem + L::D1_COL, sdesc_sw128(sb + L::TZP + kk * 32, 16, 1024),
-                                sdesc_sw128(sb + L::RAWV + kk * 2048, 8192, 1024), ID_U, kk > 0);
+                    mma_bf16_ss(tmem + L::D1_COL, dadd(dTZP, kk * 32), dadd(dV, kk * 2048), ID_U, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)  // [W'; 0] = [T'; 0] KE
-                    mma_bf16_ss(tmem + L::APW_COL, sdesc_sw128(sb + L::TZP + kk * 32, 16, 1024),
-                                sdesc_sw128(rowop(par) + kk * 2048, 16384, 1024), ID_W, kk > 0);
+                    mma_bf16_ss(tmem + L::APW_COL, dadd(dTZP, kk * 32), dadd(dROWN, par * 32768 + kk * 2048), ID_W,
+                                kk > 0);
                 mma_commit(bars + BAR_UW);
                 if (more) {
-                    wait1(BAR_G + (par ^ 1), (uint32_t)((m + 1) >> 1));
-                    mma_cs(m + 1);
                     wait1(BAR_UW, (uint32_t)m);  // v tile consumed
                     issue_v(m + 1);
                 }
@@ -434,7 +447,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         auto s1 = [&](int par) {
             const float os = sOpS[par * 128 + row], ts = sTmS[par * 128 + row];
             const int i = row & 63;
-#pragma unroll
+#pragma unroll 1
             for (int gq = 0; gq < DVT / 32; ++gq) {
                 uint32_t v[32];
                 tmem_ld32(lane_addr + L::S_COL + 32 * gq, v);
@@ -473,8 +486,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16_ss(tmem + L::D1_COL, sdesc_sw128(rowop(par) + kk * 32, 16, 1024),
-                                        sdesc_sw128(sb + L::SOP + kk * 2 * L::SBO_V, 1024, L::SBO_V), ID_M1, 1);
+                            mma_bf16_ss(tmem + L::D1_COL, dadd(dROWK, par * 32768 + kk * 32),
+                                        dadd(dSOP, kk * 2 * L::SBO_V), ID_M1, 1);
                         mma_commit(bars + BAR_M1A);
                     }
                     __syncwarp();
@@ -483,8 +496,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16_ss(tmem + L::D1_COL, sdesc_sw128(rowop(par) + 16384 + kk * 32, 16, 1024),
-                                        sdesc_sw128(sb + L::SOP + kk * 2 * L::SBO_V, 1024, L::SBO_V), ID_M1, 1);
+                            mma_bf16_ss(tmem + L::D1_COL, dadd(dROWK, par * 32768 + 16384 + kk * 32),
+                                        dadd(dSOP, kk * 2 * L::SBO_V), ID_M1, 1);
                         mma_commit(bars + BAR_M1);
                         mma_commit(bars + BAR_M1B + par);
                     }
@@ -493,7 +506,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 waitw(BAR_M1, (uint32_t)n);
                 {   // delta (D1 rows 0-63) -> bf16 operand over the state operand
                     const int r = row;
-#pragma unroll
+#pragma unroll 1
                     for (int gq = 0; gq < DVT / 32; ++gq) {
                         uint32_t v[32];
                         tmem_ld32(lane_addr + L::D1_COL + 32 * gq, v);
@@ -520,13 +533,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // R += KF^T delta
-                        mma_bf16_ss(tmem + L::S_COL, sdesc_sw128(colop(par) + kk * 2048, 8192, 1024),
-                                    sdesc_sw128(sb + L::DOP + kk * 2 * L::SBO_V, 1024, L::SBO_V), ID_M2S, 1);
-                    const uint32_t yp = sb + L::SP + (uint32_t)par * 8192 - 8192;  // [Y; P], Y = the 8 KB before P
+                        mma_bf16_ss(tmem + L::S_COL, dadd(dCOLN, par * 16384 + kk * 2048), dadd(dSOP, kk * 2 * L::SBO_V),
+                                    ID_M2S, 1);
+                    // [Y; P]: Y, the 8 KB before P, only feeds D1 rows 0-63, already read out
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // D1 rows 64-127 += P delta
-                        mma_bf16_ss(tmem + L::D1_COL, sdesc_sw128(yp + kk * 32, 16, 1024),
-                                    sdesc_sw128(sb + L::DOP + kk * 2 * L::SBO_V, 1024, L::SBO_V), ID_M2P, 1);
+                        mma_bf16_ss(tmem + L::D1_COL, dadd(dYP, par * 8192 + kk * 32), dadd(dSOP, kk * 2 * L::SBO_V),
+                                    ID_M2P, 1);
                     mma_commit(bars + BAR_M2);
                     mma_commit(bars + BAR_M2B + par);
                 }
@@ -542,7 +555,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 {   // O (D1 rows 64-127) -> global bf16
                     const int r = row - 64;
                     const int t0 = n * kC;
-#pragma unroll
+#pragma unroll 1
                     for (int gq = 0; gq < DVT / 32; ++gq) {
                         uint32_t v[32];
                         tmem_ld32(lane_addr + L::D1_COL + 32 * gq, v);
@@ -571,7 +584,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
         // ------------------------------------------------------------ final state S = e^{G_last - G_m} R
         if (quad < 2) waitw(BAR_M2, (uint32_t)(NC - 1));
-        if (ST && !*s_abort) {
+        // one decision per warp: the tensor-memory loads below are warp-collective
+        if (__shfl_sync(0xffffffffu, (ST && !*s_abort) ? 1 : 0, 0)) {
             const float ek = sEK[row];
 #pragma unroll
             for (int gq = 0; gq < DVT / 32; ++gq) {
@@ -600,28 +614,43 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         // A -> sA, P -> sP from per-pair exponentials.
         auto p2 = [&](int m) -> bool {
             const int par = m & 1;
-            uint32_t gr[32];
-            tmem_ld32(lane_addr + L::GC_COL + 32 * cb, gr);
-            tmem_ld_wait(gr);
-            if (tok == 31 || tok == 63) {
+            const uint32_t gaddr = lane_addr + L::GC_COL + 32 * cb;  // this thread's 32 channels of G
+            // Rolled loops over groups of 8 channels keep the loop bodies
+            // small: every chunk streams this code again, and what is not
+            // in the instruction cache stalls the warp.
+            {   // G_m, G_last of this thread's channels (tcgen05.ld is warp-collective:
+                // every lane loads, the lanes of tokens 31 and 63 store)
                 float* dst = (tok == 31 ? sGm : sGl) + 32 * cb;
-#pragma unroll
-                for (int u = 0; u < 32; u += 4)
-                    *reinterpret_cast<float4*>(dst + u) = make_float4(
-                        __uint_as_float(gr[u]), __uint_as_float(gr[u + 1]), __uint_as_float(gr[u + 2]),
-                        __uint_as_float(gr[u + 3]));
+#pragma unroll 1
+                for (int u4 = 0; u4 < 4; ++u4) {
+                    uint32_t g8[8];
+                    tmem_ld8(gaddr + 8 * u4, g8);
+                    tmem_ld_wait(g8);
+                    if (tok == 31 || tok == 63) {
+                        *reinterpret_cast<float4*>(dst + 8 * u4) =
+                            make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]), __uint_as_float(g8[2]),
+                                        __uint_as_float(g8[3]));
+                        *reinterpret_cast<float4*>(dst + 8 * u4 + 4) =
+                            make_float4(__uint_as_float(g8[4]), __uint_as_float(g8[5]), __uint_as_float(g8[6]),
+                                        __uint_as_float(g8[7]));
+                    }
+                    __syncwarp();
+                }
             }
             nb_sync(NB_PREP, kPrep);
-            float gm[32];
             bool bad = false;
+#pragma unroll 1
+            for (int u4 = 0; u4 < 4; ++u4) {
+                uint32_t g8[8];
+                tmem_ld8(gaddr + 8 * u4, g8);
+                tmem_ld_wait(g8);
+                const float4 ma = *reinterpret_cast<const float4*>(sGm + 32 * cb + 8 * u4);
+                const float4 mb = *reinterpret_cast<const float4*>(sGm + 32 * cb + 8 * u4 + 4);
+                const float gm8[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
 #pragma unroll
-            for (int u = 0; u < 32; u += 4) {
-                const float4 x = *reinterpret_cast<const float4*>(sGm + 32 * cb + u);
-                gm[u] = x.x; gm[u + 1] = x.y; gm[u + 2] = x.z; gm[u + 3] = x.w;
+                for (int e = 0; e < 8; ++e)
+                    bad |= !(fabsf(__uint_as_float(g8[e]) - gm8[e]) <= kGuard) || !(gm8[e] >= -kGuard);
             }
-#pragma unroll
-            for (int u = 0; u < 32; ++u)
-                bad |= !(fabsf(__uint_as_float(gr[u]) - gm[u]) <= kGuard) || !(gm[u] >= -kGuard);
             const bool exact = nb_or(NB_OR, kPrep, bad);
             if (tid < kD) {
                 const int c = tid;
@@ -641,11 +670,17 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             if (exact) {
                 // gate as fp32 [64][128] in the A/T scratch (free until P4)
                 float* sG = reinterpret_cast<float*>(sm + L::SCR);
-#pragma unroll
-                for (int u = 0; u < 32; u += 4)
-                    *reinterpret_cast<float4*>(sG + tok * 128 + 32 * cb + u) = make_float4(
-                        __uint_as_float(gr[u]), __uint_as_float(gr[u + 1]), __uint_as_float(gr[u + 2]),
-                        __uint_as_float(gr[u + 3]));
+#pragma unroll 1
+                for (int u4 = 0; u4 < 4; ++u4) {
+                    uint32_t g8[8];
+                    tmem_ld8(gaddr + 8 * u4, g8);
+                    tmem_ld_wait(g8);
+                    float* dst = sG + tok * 128 + 32 * cb + 8 * u4;
+                    *reinterpret_cast<float4*>(dst) = make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]),
+                                                                  __uint_as_float(g8[2]), __uint_as_float(g8[3]));
+                    *reinterpret_cast<float4*>(dst + 4) = make_float4(__uint_as_float(g8[4]), __uint_as_float(g8[5]),
+                                                                      __uint_as_float(g8[6]), __uint_as_float(g8[7]));
+                }
                 nb_sync(NB_PREP, kPrep);
                 const uint8_t* rk = sm + L::ROWOP + par * 32768;
                 float av[9], pv[9];
@@ -691,38 +726,44 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     }
                 }
             }
-            // operand tiles, in place: 4 chunks of 8 channels of this thread's row
-#pragma unroll
+            // operand tiles, in place: 4 groups of 8 channels of this thread's row
+#pragma unroll 1
             for (int u4 = 0; u4 < 4; ++u4) {
                 const int c0 = 32 * cb + 8 * u4;
+                uint32_t g8[8];
+                tmem_ld8(gaddr + 8 * u4, g8);
                 const uint32_t ko = rop_off(tok, c0);
                 const uint32_t fo = (uint32_t)((c0 >> 6) * 8192 + tok * 128 + ((((c0 & 63) >> 3) ^ (tok & 7)) << 4));
                 const uint4 kv = ld_shared_v4(rop + ko);
                 const uint4 qv = ld_shared_v4(rop + ko + 8192);
+                const float4 ra = *reinterpret_cast<const float4*>((exact ? sGl : sGm) + c0);
+                const float4 rb = *reinterpret_cast<const float4*>((exact ? sGl : sGm) + c0 + 4);
+                const float ref8[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+                tmem_ld_wait(g8);
                 const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w}, qw[4] = {qv.x, qv.y, qv.z, qv.w};
                 uint32_t ke[4], qe[4], kf[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int e = 8 * u4 + 2 * u;
-                    const float g0 = __uint_as_float(gr[e]), g1 = __uint_as_float(gr[e + 1]);
+                    const float g0 = __uint_as_float(g8[2 * u]), g1 = __uint_as_float(g8[2 * u + 1]);
                     float e0, e1, f0, f1;
-                    if (!exact) {
-                        e0 = __expf(g0 - gm[e]);
-                        e1 = __expf(g1 - gm[e + 1]);
+                    if (!exact) {  // E = e^{G - G_m}, F = 1/E
+                        e0 = __expf(g0 - ref8[2 * u]);
+                        e1 = __expf(g1 - ref8[2 * u + 1]);
                         f0 = recip_bf16(e0);
                         f1 = recip_bf16(e1);
-                    } else {
-                        const float l0 = sGl[c0 + 2 * u], l1 = sGl[c0 + 2 * u + 1];
+                    } else {       // e^G and e^{G_last - G}
                         e0 = __expf(g0);
                         e1 = __expf(g1);
-                        f0 = __expf(l0 - g0);
-                        f1 = __expf(l1 - g1);
+                        f0 = __expf(ref8[2 * u] - g0);
+                        f1 = __expf(ref8[2 * u + 1] - g1);
                     }
-                    const float k0 = bf16_lo(kw[u]), k1 = bf16_hi(kw[u]);
-                    const float q0 = bf16_lo(qw[u]), q1 = bf16_hi(qw[u]);
-                    ke[u] = pack_bf16x2(k0 * e0, k1 * e1);
-                    qe[u] = pack_bf16x2(q0 * e0, q1 * e1);
-                    kf[u] = pack_bf16x2(k0 * f0, k1 * f1);
+                    // packed bf16 products: the factor pairs are rounded to bf16
+                    // first, the products once more (both well inside the bf16
+                    // rounding of the MMA operands)
+                    const uint32_t ep = pack_bf16x2(e0, e1), fp = pack_bf16x2(f0, f1);
+                    ke[u] = hmul2_bf16(kw[u], ep);
+                    qe[u] = hmul2_bf16(qw[u], ep);
+                    kf[u] = hmul2_bf16(kw[u], fp);
                 }
                 st_shared_v4(rop + ko, ke[0], ke[1], ke[2], ke[3]);
                 st_shared_v4(rop + ko + 8192, qe[0], qe[1], qe[2], qe[3]);
@@ -837,7 +878,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         auto p7 = [&](int par) {
             if (quad < 2) {
                 const int r = 32 * quad + lane;
-#pragma unroll
+#pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t v[32];
                     tmem_ld32(lane_addr + L::APW_COL + 64 * hf + 32 * hh, v);
