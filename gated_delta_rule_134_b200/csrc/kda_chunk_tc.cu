@@ -35,21 +35,26 @@
 // Schedule. One CTA owns one (batch, head) and a DVT-wide slice of value
 // channels; its state stays in tensor memory for the whole sequence. Three
 // warp roles run concurrently and hand work over through mbarriers:
-//   prep  (warps 0-7)  per chunk m, ahead of the state: gate prefix sums from
-//                      tensor memory, guard, KE/QE/KF (in place over the raw
-//                      k/q tiles), A and P readout, (I + A)^{-1} -> T', -W'.
+//   prep  (warps 0-7)  per chunk m: A/P readout, (I + A)^{-1} -> T'; then the
+//                      operand tiles of chunk m+1 (prefix sums out of tensor
+//                      memory, guard, KE/QE in place over the raw k/q rows, KF
+//                      over the log_alpha tile), which covers the U/W MMAs of
+//                      chunk m; then -W' of chunk m over its KE rows.
 //   chain (warps 8-11) per chunk n, the state-dependent part: state -> bf16
 //                      operand, MMA1 (two halves of the key channels, so one
 //                      16 KB operand buffer serves both), delta -> bf16,
 //                      MMA2, O -> global. Warp 8 issues these MMAs.
-//   control (warp 12)  every TMA load and the state-independent MMAs (prefix
-//                      sums, A/P, U/W), in the order their inputs appear.
+//   control (warp 12)  every TMA load (plus an L2 prefetch of the next
+//                      chunk's tiles) and the state-independent MMAs, issued
+//                      from a polling loop in the order their inputs appear.
 // k/q tiles and the operand tiles built from them are double-buffered by
-// chunk parity, so the prep of chunk n+1 overlaps the state chain of chunk n.
+// chunk parity, the per-channel scales by chunk mod 4. A/P land in the
+// prefix-sum columns once those are read, so the A/P MMA of chunk m+1 runs
+// while the prep warps finish chunk m.
 // (I + A)^{-1}: 16x16 diagonal blocks by forward substitution (four threads per
-// column), N = T_diag A_offdiag, then the blocks below the diagonal level by
-// level, T_ab = -sum_k N_ak T_kb; T' = T Diag(beta) is written as bf16 by the
-// thread that finalises each entry.
+// column), then one column chain per warp, T_ab = -T_aa sum_k A_ak T_kb, on
+// m16n8k8 tf32 MMAs; T' = T Diag(beta) is written as bf16 by the thread that
+// finalises each entry.
 //
 // Every wait on an mbarrier is bounded; on expiry the kernel records status 1
 // in the caller's workspace word and stops waiting (later waits are skipped,
@@ -64,15 +69,13 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kPrep = 256;                    // warps 0-7
-constexpr int kChainWarp0 = kPrep / 32;       // warps 8-11
-constexpr int kCtrlWarp = kChainWarp0 + 4;    // warp 12
+constexpr int kPrep = 256;                    // warps 0-7: operand tiles, A/P readout, UT inverse, -W'
+constexpr int kChainWarp0 = kPrep / 32;       // warps 8-11: state chain
+constexpr int kCtrlWarp = kChainWarp0 + 4;    // warp 12: loads and state-independent MMAs
 constexpr int kThreads = 32 * (kCtrlWarp + 1);
 // named barriers (0 is __syncthreads)
 constexpr int NB_PREP = 1;  // prep warps
 constexpr int NB_OR = 2;    // prep warps, OR-reduction
-constexpr int NB_P2 = 3;    // prep -> control: operand tiles stored, prefix sums read (AP, next prefix sums)
-constexpr int NB_P5 = 4;    // prep -> control: T' stored (U, W)
 constexpr int NB_CHA = 5;   // chain warps 8-9
 constexpr int NB_CHB = 6;   // chain warps 10-11 -> warp 8: second half of the state operand stored
 constexpr int NB_CHC = 7;   // chain warps 10-11
@@ -99,14 +102,14 @@ struct Layout {
     static constexpr uint32_t SOP = SCR + 2 * 64 * kLDA * 4;  // S half (64 channels) x DVT, bf16 MN-major
     static constexpr uint32_t DOP = SOP;                      //   then delta (64 tokens) x DVT
     static constexpr uint32_t SMALL = SOP + 64 * DVT * 2;
-    static constexpr uint32_t SBETA = SMALL;        // 64 f32
-    static constexpr uint32_t SOPS = SBETA + 256;   // 2 x 128 f32: operand scale per channel (by chunk parity)
-    static constexpr uint32_t STMS = SOPS + 1024;   // 2 x 128 f32: tensor-memory scale per channel
-    static constexpr uint32_t SEK = STMS + 1024;    // 128 f32: e^{G_last - G_m} of the last prepared chunk
+    static constexpr uint32_t SBETA = SMALL;        // 64 f32: beta of the chunk the prep warps work on
+    static constexpr uint32_t SOPS = SBETA + 256;   // 4 x 128 f32: operand scale per channel (by chunk mod 4)
+    static constexpr uint32_t STMS = SOPS + 2048;   // 4 x 128 f32: tensor-memory scale per channel
+    static constexpr uint32_t SEK = STMS + 2048;    // 128 f32: e^{G_last - G_m} of the last prepared chunk
     static constexpr uint32_t SGM = SEK + 512;      // 128 f32: G_m of the chunk being prepared
     static constexpr uint32_t SGL = SGM + 512;      // 128 f32: G_last
-    static constexpr uint32_t BARS = SGL + 512;     // 20 mbarriers
-    static constexpr uint32_t MISC = BARS + 160;    // tmem base, abort flag, guard verdicts
+    static constexpr uint32_t BARS = SGL + 512;     // mbarriers
+    static constexpr uint32_t MISC = BARS + 256;    // tmem base, abort flag, guard verdicts
     static constexpr uint32_t END = MISC + 16;
     static constexpr uint32_t SMEM_BYTES = END + 1024;   // + alignment slack
     static constexpr uint32_t SBO_V = 1024 * (DVT / 64); // K-group stride of the S / delta operands
@@ -116,8 +119,8 @@ struct Layout {
     // tensor memory columns
     static constexpr uint32_t S_COL = 0;     // R (fp32, lane = key channel)
     static constexpr uint32_t D1_COL = 128;  // [U; 0] -> [delta; O] (lane = token row)
-    static constexpr uint32_t APW_COL = 256; // [A; P] (64 cols), then [W'; 0] (128 cols)
-    static constexpr uint32_t GC_COL = 384;  // [G; G] (lane = token, col = channel)
+    static constexpr uint32_t W_COL = 256;   // [W'; 0]
+    static constexpr uint32_t GC_COL = 384;  // [G; G] (lane = token, col = channel), then [A; P] (64 cols)
     static constexpr uint32_t TMEM_COLS = 512;
 };
 
@@ -135,9 +138,12 @@ enum : int {
     BAR_M1B = 11,    // 2: MMA1 of the chunk of this parity done (row operand free)
     BAR_M2B = 13,    // 2: MMA2 of the chunk of this parity done (KF, P free)
     BAR_D1 = 15,     // delta and O read out of tensor memory (D1 free)
-    BAR_SC = 16,     // 2: per-channel scales of the chunk of this parity stored
-    BAR_RR = 18,     // 2: row operand [-W'; QE] of the chunk of this parity stored
-    NUM_BARS = 20
+    BAR_SC = 16,     // 4: per-channel scales of the chunk (mod 4) stored
+    BAR_RR = 20,     // 2: row operand [-W'; QE] of the chunk of this parity stored
+    BAR_P2 = 22,     // operand tiles of a chunk stored, its prefix sums read
+    BAR_P4 = 23,     // A/P of a chunk read out (tensor-memory columns free)
+    BAR_P5 = 24,     // T' of a chunk stored, A/T scratch free
+    NUM_BARS = 25
 };
 
 // offset of element (row R, channel c) of a row-operand buffer (K-major, two
@@ -151,14 +157,11 @@ __device__ __forceinline__ uint32_t km_off(int r, int s) {
     return (uint32_t)(r * 128 + ((((s >> 3) ^ (r & 7))) << 4) + ((s & 7) << 1));
 }
 
-// 1/x for normal positive x, accurate to ~2.4e-4 relative (enough for a bf16
-// result): seed 2^-e (2 - f)/2 for x = 2^e (1 + f), obtained by subtracting
-// the bit pattern from 254 << 23 (seed error <= 12.5%), then two Newton steps
-// r <- r (2 - x r), each squaring the relative error. Runs on the FMA pipe.
-__device__ __forceinline__ float recip_bf16(float x) {
-    float r = __int_as_float(0x7F000000 - __float_as_int(x));
-    r = r * fmaf(-x, r, 2.f);
-    r = r * fmaf(-x, r, 2.f);
+// 1/x by the hardware reciprocal approximation (one MUFU operation; the
+// FMA pipe stays free for the products around it)
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
     return r;
 }
 
@@ -326,36 +329,42 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
     if (warp == kCtrlWarp) {
         // ============================================================ control warp
-        const bool leader = lane == 0;
-        auto issue_kq = [&](int m) {
-            const int par = m & 1;
-            uint8_t* dst = sm + L::ROWOP + par * 32768;
-            mbar_arrive_expect_tx(bars + BAR_KQ + par, 4 * 8192);
-            for (int x = 0; x < 2; ++x) {
-                tma_load_4d(dst + x * 16384, &tm_k, bars + BAR_KQ + par, 64 * x, h, m * kC, b);
-                tma_load_4d(dst + x * 16384 + 8192, &tm_q, bars + BAR_KQ + par, 64 * x, h, m * kC, b);
-            }
-        };
-        auto issue_g = [&](int m) {
-            const int par = m & 1;
-            uint8_t* dst = sm + L::COLOP + par * 16384;
-            mbar_arrive_expect_tx(bars + BAR_G + par, 2 * 8192);
-            for (int x = 0; x < 2; ++x) tma_load_4d(dst + x * 8192, &tm_g, bars + BAR_G + par, 64 * x, h, m * kC, b);
-        };
-        auto issue_v = [&](int m) {
-            mbar_arrive_expect_tx(bars + BAR_V, (DVT / 64) * 8192);
-            for (int x = 0; x < DVT / 64; ++x)
-                tma_load_4d(sm + L::RAWV + x * 8192, &tm_v, bars + BAR_V, j0 + 64 * x, h, m * kC, b);
-        };
-        auto mma_cs = [&](int m) {  // [G; G] = [L; L] g
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + L::GC_COL, dadd(dLMAT, kk * 32), dadd(dCOLN, (m & 1) * 16384 + kk * 2048), ID_CS,
-                            kk > 0);
-            mma_commit(bars + BAR_CS);
-        };
-        if (leader) {
+        // One thread issues every TMA load and the state-independent MMAs. Their
+        // inputs come from three roles in an order that varies from chunk to
+        // chunk, so it polls the hand-over barriers and issues whatever is
+        // ready; each kind of work goes out in chunk order.
+        if (lane == 0) {
+            auto issue_kq = [&](int m) {
+                const int par = m & 1;
+                uint8_t* dst = sm + L::ROWOP + par * 32768;
+                mbar_arrive_expect_tx(bars + BAR_KQ + par, 4 * 8192);
+                for (int x = 0; x < 2; ++x) {
+                    tma_load_4d(dst + x * 16384, &tm_k, bars + BAR_KQ + par, 64 * x, h, m * kC, b);
+                    tma_load_4d(dst + x * 16384 + 8192, &tm_q, bars + BAR_KQ + par, 64 * x, h, m * kC, b);
+                }
+                if (m + 1 < NC) {  // the next chunk's tiles into L2: their loads wait for a free buffer
+                    for (int x = 0; x < 2; ++x) {
+                        tma_prefetch_l2_4d(&tm_k, 64 * x, h, (m + 1) * kC, b);
+                        tma_prefetch_l2_4d(&tm_q, 64 * x, h, (m + 1) * kC, b);
+                    }
+                }
+            };
+            auto issue_g = [&](int m) {
+                const int par = m & 1;
+                uint8_t* dst = sm + L::COLOP + par * 16384;
+                mbar_arrive_expect_tx(bars + BAR_G + par, 2 * 8192);
+                for (int x = 0; x < 2; ++x)
+                    tma_load_4d(dst + x * 8192, &tm_g, bars + BAR_G + par, 64 * x, h, m * kC, b);
+                if (m + 1 < NC)
+                    for (int x = 0; x < 2; ++x) tma_prefetch_l2_4d(&tm_g, 64 * x, h, (m + 1) * kC, b);
+            };
+            auto issue_v = [&](int m) {
+                mbar_arrive_expect_tx(bars + BAR_V, (DVT / 64) * 8192);
+                for (int x = 0; x < DVT / 64; ++x)
+                    tma_load_4d(sm + L::RAWV + x * 8192, &tm_v, bars + BAR_V, j0 + 64 * x, h, m * kC, b);
+                if (m + 1 < NC)
+                    for (int x = 0; x < DVT / 64; ++x) tma_prefetch_l2_4d(&tm_v, j0 + 64 * x, h, (m + 1) * kC, b);
+            };
             issue_kq(0);
             issue_g(0);
             issue_v(0);
@@ -363,65 +372,84 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 issue_kq(1);
                 issue_g(1);
             }
-            wait1(BAR_G, 0);
-            mma_cs(0);
+            // next chunk for each kind of work
+            int ncs = 0, nap = 0, nuw = 0, nv = 1, nkq = 2, ng = 2;
+            long long idle_since = clock64();
+            while ((ncs < NC || nap < NC || nuw < NC || nv < NC || nkq < NC || ng < NC) && !*s_abort) {
+                bool prog = false;
+                // [G; G] = [L; L] g: the tile landed and the previous chunk's A/P were read out
+                if (ncs < NC && mbar_test(bars + BAR_G + (ncs & 1), (uint32_t)(ncs >> 1)) &&
+                    (ncs == 0 || mbar_test(bars + BAR_P4, (uint32_t)(ncs - 1)))) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + L::GC_COL, dadd(dLMAT, kk * 32),
+                                    dadd(dCOLN, (ncs & 1) * 16384 + kk * 2048), ID_CS, kk > 0);
+                    mma_commit(bars + BAR_CS);
+                    ++ncs;
+                    prog = true;
+                }
+                // [A; P] = [KE; QE] KF^T over the prefix-sum columns, once the operand tiles are stored
+                if (nap < ncs && mbar_test(bars + BAR_P2, (uint32_t)nap)) {
+                    const int par = nap & 1;
+                    tc_fence_after();
+                    if (!s_exact[par]) {
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_bf16_ss(tmem + L::GC_COL,
+                                        dadd(dROWK, par * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32),
+                                        dadd(dCOLK, par * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32), ID_AP, kk > 0);
+                    }
+                    mma_commit(bars + BAR_AP);
+                    ++nap;
+                    prog = true;
+                }
+                // [U; 0] = [T'; 0] v and [W'; 0] = [T'; 0] KE: T' stored, v landed, D1 read out
+                if (nuw < nap && mbar_test(bars + BAR_P5, (uint32_t)nuw) && mbar_test(bars + BAR_V, (uint32_t)nuw) &&
+                    (nuw == 0 || mbar_test(bars + BAR_D1, (uint32_t)(nuw - 1)))) {
+                    const int par = nuw & 1;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + L::D1_COL, dadd(dTZP, kk * 32), dadd(dV, kk * 2048), ID_U, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + L::W_COL, dadd(dTZP, kk * 32), dadd(dROWN, par * 32768 + kk * 2048), ID_W,
+                                    kk > 0);
+                    mma_commit(bars + BAR_UW);
+                    ++nuw;
+                    prog = true;
+                }
+                // loads into buffers freed by completed MMAs
+                if (nv < NC && nv <= nuw && mbar_test(bars + BAR_UW, (uint32_t)(nv - 1))) {
+                    issue_v(nv++);
+                    prog = true;
+                }
+                if (nkq < NC && mbar_test(bars + BAR_M1B + (nkq & 1), (uint32_t)((nkq - 2) >> 1))) {
+                    issue_kq(nkq++);
+                    prog = true;
+                }
+                if (ng < NC && mbar_test(bars + BAR_M2B + (ng & 1), (uint32_t)((ng - 2) >> 1))) {
+                    issue_g(ng++);
+                    prog = true;
+                }
+                if (prog) {
+                    idle_since = clock64();
+                } else if (clock64() - idle_since > kWaitBudget) {
+                    fail();
+                } else {
+                    __nanosleep(32);
+                }
+            }
         }
         __syncwarp();
-        for (int m = 0; m < NC; ++m) {
-            const int par = m & 1;
-            const bool more = m + 1 < NC;
-            if (leader && m >= 1 && more) {
-                // the buffers of parity m+1 were last read by the MMAs of chunk m-1;
-                // reload them while the prep warps still work on chunk m
-                wait1(BAR_M1B + (par ^ 1), (uint32_t)((m - 1) >> 1));
-                issue_kq(m + 1);
-                wait1(BAR_M2B + (par ^ 1), (uint32_t)((m - 1) >> 1));
-                issue_g(m + 1);
-            }
-            __syncwarp();
-            nb_sync(NB_P2, kPrep + 32);  // operand tiles of chunk m stored, prefix sums read
-            if (leader) {
-                tc_fence_after();
-                if (!s_exact[par]) {  // [KE; QE] KF^T -> [A; P]
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ss(tmem + L::APW_COL, dadd(dROWK, par * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32),
-                                    dadd(dCOLK, par * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32), ID_AP, kk > 0);
-                }
-                mma_commit(bars + BAR_AP);
-                if (more) {  // prefix sums of chunk m+1, ready before the prep warps need them
-                    wait1(BAR_G + (par ^ 1), (uint32_t)((m + 1) >> 1));
-                    mma_cs(m + 1);
-                }
-            }
-            __syncwarp();
-            nb_sync(NB_P5, kPrep + 32);  // T' of chunk m stored
-            if (leader) {
-                wait1(BAR_V, (uint32_t)m);
-                if (m >= 1) wait1(BAR_D1, (uint32_t)(m - 1));
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // [U; 0] = [T'; 0] v
-                    mma_bf16_ss(tmem + L::D1_COL, dadd(dTZP, kk * 32), dadd(dV, kk * 2048), ID_U, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // [W'; 0] = [T'; 0] KE
-                    mma_bf16_ss(tmem + L::APW_COL, dadd(dTZP, kk * 32), dadd(dROWN, par * 32768 + kk * 2048), ID_W,
-                                kk > 0);
-                mma_commit(bars + BAR_UW);
-                if (more) {
-                    wait1(BAR_UW, (uint32_t)m);  // v tile consumed
-                    issue_v(m + 1);
-                }
-            }
-            __syncwarp();
-        }
-    } else if (warp >= kChainWarp0) {
+    } else if (warp >= kChainWarp0 && warp < kCtrlWarp) {
         // ============================================================ chain warps
         // lane row = 32 * quad + lane: a key channel of the state, a token row of D1
         const int row = 32 * quad + lane;
         const bool issuer = (quad == 0) && (lane == 0);
         {   // initial state into TMEM (fp32, lane = key channel)
-#pragma unroll
+#pragma unroll 1
             for (int gq = 0; gq < DVT / 32; ++gq) {
                 uint32_t r[32];
                 if (S0) {
@@ -444,8 +472,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             tc_fence_after();
         }
         // state rows -> bf16 operand (times the operand scale), R *= tensor-memory scale
-        auto s1 = [&](int par) {
-            const float os = sOpS[par * 128 + row], ts = sTmS[par * 128 + row];
+        auto s1 = [&](int slot) {
+            const float os = sOpS[slot * 128 + row], ts = sTmS[slot * 128 + row];
             const int i = row & 63;
 #pragma unroll 1
             for (int gq = 0; gq < DVT / 32; ++gq) {
@@ -475,8 +503,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const uint32_t ph = (uint32_t)(n >> 1);
             if (quad < 2) {
                 if (n > 0) waitw(BAR_M2, (uint32_t)(n - 1));  // state update of the previous chunk done
-                waitw(BAR_SC + par, ph);
-                s1(par);  // key channels 0-63
+                waitw(BAR_SC + (n & 3), (uint32_t)(n >> 2));
+                s1(n & 3);  // key channels 0-63
                 fence_proxy_async_smem();
                 tc_fence_before();
                 nb_sync(NB_CHA, 64);
@@ -545,9 +573,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
                 __syncwarp();
             } else {
-                waitw(BAR_SC + par, ph);
+                waitw(BAR_SC + (n & 3), (uint32_t)(n >> 2));
                 waitw(BAR_M1A, (uint32_t)n);  // first half of the state operand consumed
-                s1(par);                      // key channels 64-127
+                s1(n & 3);                      // key channels 64-127
                 fence_proxy_async_smem();
                 tc_fence_before();
                 nb_arrive(NB_CHB, 96);
@@ -587,7 +615,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         // one decision per warp: the tensor-memory loads below are warp-collective
         if (__shfl_sync(0xffffffffu, (ST && !*s_abort) ? 1 : 0, 0)) {
             const float ek = sEK[row];
-#pragma unroll
+#pragma unroll 1
             for (int gq = 0; gq < DVT / 32; ++gq) {
                 uint32_t v[32];
                 tmem_ld32(lane_addr + L::S_COL + 32 * gq, v);
@@ -599,8 +627,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                                          __uint_as_float(v[4 * u + 2]) * ek, __uint_as_float(v[4 * u + 3]) * ek);
             }
         }
-    } else {
+    } else if (warp < kChainWarp0) {
         // ============================================================ prep warps
+        // Per chunk m: A/P readout and (I + A)^{-1} -> T'; then the operand
+        // tiles of chunk m+1 (which covers the U/W round trip of chunk m);
+        // then -W' over the KE rows of chunk m (the A/P MMA of chunk m+1 runs
+        // meanwhile).
         const int hf = warp >> 2;
         const int tok = 32 * (quad & 1) + lane;  // P2: token of this thread
         const int cb = 2 * (quad >> 1) + hf;     // P2: 32-channel block of this thread
@@ -608,12 +640,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const int t = m * kC + tid;
             return (tid < kC && m < NC && t < Tlen) ? __bfloat162float(beta[((size_t)b * Tlen + t) * H + h]) : 0.f;
         };
-
-        // ---- P2 of chunk m: prefix sums from TMEM, guard, per-channel scales;
-        // KE/QE over the raw k/q rows, KF over the log_alpha tile. Exact path:
-        // A -> sA, P -> sP from per-pair exponentials.
         auto p2 = [&](int m) -> bool {
-            const int par = m & 1;
+            const int par = m & 1, slot = m & 3;
             const uint32_t gaddr = lane_addr + L::GC_COL + 32 * cb;  // this thread's 32 channels of G
             // Rolled loops over groups of 8 channels keep the loop bodies
             // small: every chunk streams this code again, and what is not
@@ -657,18 +685,20 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 const float g_m = sGm[c], g_l = sGl[c], ek_prev = sEK[c];
                 if (!exact) {
                     const float s = __expf(g_m) * ek_prev;
-                    sOpS[par * 128 + c] = s;
-                    sTmS[par * 128 + c] = s;
+                    sOpS[slot * 128 + c] = s;
+                    sTmS[slot * 128 + c] = s;
                     sEK[c] = __expf(g_l - g_m);
                 } else {
-                    sOpS[par * 128 + c] = ek_prev;
-                    sTmS[par * 128 + c] = __expf(g_l) * ek_prev;
+                    sOpS[slot * 128 + c] = ek_prev;
+                    sTmS[slot * 128 + c] = __expf(g_l) * ek_prev;
                     sEK[c] = 1.f;
                 }
             }
             const uint32_t rop = rowop(par);
             if (exact) {
-                // gate as fp32 [64][128] in the A/T scratch (free until P4)
+                // gate as fp32 [64][128] in the A/T scratch (free: the inverse of the
+                // previous chunk is done); P of chunk m-2 must be consumed first
+                if (m >= 2) waitw(BAR_M2B + par, (uint32_t)((m >> 1) - 1));
                 float* sG = reinterpret_cast<float*>(sm + L::SCR);
 #pragma unroll 1
                 for (int u4 = 0; u4 < 4; ++u4) {
@@ -703,7 +733,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                             pp = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(64 + r, cc))),
                                       ks, pp);
                         }
-                        av[i] = (s < r) ? sBeta[r] * a : 0.f;
+                        const int tr = m * kC + r;  // beta of chunk m (the scratch holds the previous chunk's)
+                        const float br = tr < Tlen ? __bfloat162float(beta[((size_t)b * Tlen + tr) * H + h]) : 0.f;
+                        av[i] = (s < r) ? br * a : 0.f;
                         pv[i] = pp;
                     }
                 }
@@ -749,8 +781,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     if (!exact) {  // E = e^{G - G_m}, F = 1/E
                         e0 = __expf(g0 - ref8[2 * u]);
                         e1 = __expf(g1 - ref8[2 * u + 1]);
-                        f0 = recip_bf16(e0);
-                        f1 = recip_bf16(e1);
+                        f0 = rcp_approx(e0);
+                        f1 = rcp_approx(e1);
                     } else {       // e^G and e^{G_last - G}
                         e0 = __expf(g0);
                         e1 = __expf(g1);
@@ -771,11 +803,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
             return exact;
         };
-        // ---- P4: A (APW lanes 0-63) -> fp32 scratch (beta_r, strictly lower);
+        // ---- P4: A (lanes 0-63 of the prefix-sum columns) -> fp32 scratch (beta_r, strictly lower);
         // P (lanes 64-127) -> bf16 K-major tile of this parity (lower incl.)
         auto p4 = [&](int par) {
             uint32_t v[32];
-            tmem_ld32(lane_addr + L::APW_COL + 32 * hf, v);
+            tmem_ld32(lane_addr + L::GC_COL + 32 * hf, v);
             tmem_ld_wait(v);
             if (quad < 2) {
                 const int r = 32 * quad + lane;
@@ -833,55 +865,49 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
             }
             nb_sync(NB_PREP, kPrep);
-            // Blocks below the diagonal on the tensor cores (m16n8k8, tf32): one
-            // warp per (block, 8-column half). N_ak = T_aa A_ak replaces A_ak.
-            auto put_t = [&](int a, int bb, int nt, const float (&acc)[4]) {  // T_ab = -acc
+            // Blocks below the diagonal, one column chain per warp (block column
+            // bb, 8-column half nt), on the tensor cores (m16n8k8, tf32). For
+            // a = bb+1..3: X = sum_{k=bb}^{a-1} A_ak T_kb, then T_ab = -T_aa X.
+            // Every operand is either a diagonal block or a block this warp
+            // wrote before, so the chain needs no block-wide barrier.
+            {
+                const int bb = warp >> 1, nt = warp & 1;
                 const int g = lane >> 2, t = lane & 3;
-                const int s = 16 * bb + 8 * nt + 2 * t;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int r = 16 * a + g + 8 * hh;
-                    const float v0 = -acc[2 * hh], v1 = -acc[2 * hh + 1];
-                    *reinterpret_cast<float2*>(sT + r * kLDA + s) = make_float2(v0, v1);
-                    *reinterpret_cast<uint32_t*>(sm + L::TZP + km_off(r, s)) =
-                        pack_bf16x2(v0 * sBeta[s], v1 * sBeta[s + 1]);
-                }
-            };
-            for (int task = warp; task < 12; task += kPrep / 32) {
-                const int blk = task >> 1, nt = task & 1;
-                const int a = (blk == 0) ? 1 : (blk <= 2 ? 2 : 3);
-                const int k = (blk == 0) ? 0 : (blk == 1 ? 0 : (blk == 2 ? 1 : blk - 3));
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                mm16_ntile(acc, sT + (16 * a) * kLDA + 16 * a, sA + (16 * a) * kLDA + 16 * k, nt, lane);
-                __syncwarp();
-                const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-                    *reinterpret_cast<float2*>(sA + (16 * a + g + 8 * hh) * kLDA + 16 * k + 8 * nt + 2 * t) =
-                        make_float2(acc[2 * hh], acc[2 * hh + 1]);
-            }
-            nb_sync(NB_PREP, kPrep);
-            // level d: T_ab = -sum_{k=b}^{a-1} N_ak T_kb, a - b = d
+                const int s0 = 16 * bb + 8 * nt + 2 * t;
 #pragma unroll 1
-            for (int d = 1; d < 4; ++d) {
-                if (warp < 2 * (4 - d)) {
-                    const int bb = warp >> 1, nt = warp & 1, a = bb + d;
+                for (int a = bb + 1; a < 4; ++a) {
                     float acc[4] = {0.f, 0.f, 0.f, 0.f};
                     for (int kb = bb; kb < a; ++kb)
                         mm16_ntile(acc, sA + (16 * a) * kLDA + 16 * kb, sT + (16 * kb) * kLDA + 16 * bb, nt, lane);
-                    put_t(a, bb, nt, acc);
+                    float* xb = sT + (16 * a) * kLDA + 16 * bb;  // X staged where T_ab goes
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                        *reinterpret_cast<float2*>(xb + (g + 8 * hh) * kLDA + 8 * nt + 2 * t) =
+                            make_float2(acc[2 * hh], acc[2 * hh + 1]);
+                    __syncwarp();
+                    float tx[4] = {0.f, 0.f, 0.f, 0.f};
+                    mm16_ntile(tx, sT + (16 * a) * kLDA + 16 * a, xb, nt, lane);
+                    __syncwarp();  // X read before T_ab overwrites it
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int r = 16 * a + g + 8 * hh;
+                        const float v0 = -tx[2 * hh], v1 = -tx[2 * hh + 1];
+                        *reinterpret_cast<float2*>(sT + r * kLDA + s0) = make_float2(v0, v1);
+                        *reinterpret_cast<uint32_t*>(sm + L::TZP + km_off(r, s0)) =
+                            pack_bf16x2(v0 * sBeta[s0], v1 * sBeta[s0 + 1]);
+                    }
+                    __syncwarp();
                 }
-                if (d < 3) nb_sync(NB_PREP, kPrep);
             }
         };
-        // ---- P7: [W'; 0] (APW lanes 0-63) -> -W' over the KE rows
+        // ---- P7: [W'; 0] (lanes 0-63) -> -W' over the KE rows
         auto p7 = [&](int par) {
             if (quad < 2) {
                 const int r = 32 * quad + lane;
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t v[32];
-                    tmem_ld32(lane_addr + L::APW_COL + 64 * hf + 32 * hh, v);
+                    tmem_ld32(lane_addr + L::W_COL + 64 * hf + 32 * hh, v);
                     tmem_ld_wait(v);
 #pragma unroll
                     for (int jc = 0; jc < 4; ++jc) {
@@ -897,38 +923,55 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
         };
 
-        float beta_next = load_beta(0);
-        for (int m = 0; m < NC; ++m) {
-            const int par = m & 1;
-            const uint32_t ph = (uint32_t)(m >> 1);
-            if (tid < kC) sBeta[tid] = beta_next;
-            beta_next = load_beta(m + 1);
-            waitw(BAR_CS, (uint32_t)m);
-            waitw(BAR_KQ + par, ph);
-            if (m >= 2) waitw(BAR_M2B + par, ph - 1);  // P (and KF) of chunk m-2 consumed
-            nb_sync(NB_PREP, kPrep);                    // beta of chunk m visible
-            const bool exact = p2(m);
+
+        auto p2_signal = [&](int m, bool exact) {
             fence_proxy_async_smem();
             tc_fence_before();
             nb_sync(NB_PREP, kPrep);
             if (tid == 0) {
-                s_exact[par] = exact;
-                mbar_arrive(bars + BAR_SC + par);
+                s_exact[m & 1] = exact;
+                mbar_arrive(bars + BAR_SC + (m & 3));
+                mbar_arrive(bars + BAR_P2);
             }
-            nb_arrive(NB_P2, kPrep + 32);
+            __syncwarp();
+        };
+        waitw(BAR_CS, 0u);
+        waitw(BAR_KQ, 0u);
+        nb_sync(NB_PREP, kPrep);
+        bool exact_cur = p2(0);
+        p2_signal(0, exact_cur);
+        float beta_next = load_beta(0);
+        for (int m = 0; m < NC; ++m) {
+            const int par = m & 1;
+            if (tid < kC) sBeta[tid] = beta_next;
+            beta_next = load_beta(m + 1);
             waitw(BAR_AP, (uint32_t)m);
-            if (!exact) p4(par);
+            if (!exact_cur && m >= 2) waitw(BAR_M2B + par, (uint32_t)((m >> 1) - 1));  // P of chunk m-2 consumed
+            nb_sync(NB_PREP, kPrep);  // beta of chunk m visible
+            if (!exact_cur) p4(par);
+            fence_proxy_async_smem();
+            tc_fence_before();
             nb_sync(NB_PREP, kPrep);
+            if (tid == 0) mbar_arrive(bars + BAR_P4);  // prefix-sum columns free
             p5();
             fence_proxy_async_smem();
             tc_fence_before();
-            nb_arrive(NB_P5, kPrep + 32);
+            nb_sync(NB_PREP, kPrep);
+            if (tid == 0) mbar_arrive(bars + BAR_P5);  // T' stored
+            bool exact_next = false;
+            if (m + 1 < NC) {
+                waitw(BAR_CS, (uint32_t)(m + 1));
+                waitw(BAR_KQ + (par ^ 1), (uint32_t)((m + 1) >> 1));
+                exact_next = p2(m + 1);
+                p2_signal(m + 1, exact_next);
+            }
             waitw(BAR_UW, (uint32_t)m);
             p7(par);
             fence_proxy_async_smem();
             tc_fence_before();
             nb_sync(NB_PREP, kPrep);
             if (tid == 0) mbar_arrive(bars + BAR_RR + par);
+            exact_cur = exact_next;
         }
     }
     tc_fence_before();
@@ -938,6 +981,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         tmem_dealloc(tmem, L::TMEM_COLS);
     }
 }
+
 
 // ---------------------------------------------------------------- host side
 
