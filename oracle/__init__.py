@@ -7,8 +7,9 @@ use it; the product package never imports it, and it never imports the
 product package.
 
 Sources followed: "Decoding Hybrid Attention Architectures" section 3.4 (the
-KDA update and the variant table), section 3.2 (role of beta), section 4 (the
-chunkwise form); "Technical Analysis ... Novel Hybrid Linear Attention"
+KDA update and the variant table: the erase / gate switches select the delta
+rule, the scalar gated delta rule and the additive-write family), section 3.2
+(role of beta), section 4 (the chunkwise form); "Technical Analysis ... Novel Hybrid Linear Attention"
 sections 2.4 and 3.1-3.2. Every function is pinned by tests/test_oracle.py.
 """
 from __future__ import annotations
@@ -34,7 +35,13 @@ MUTATIONS = {
     "decay_columns": 7,
     "prefix_decay_k": 8,
     "strict_tril_o": 9,
+    "erase_always": 10,
+    "scalar_gate_twice": 11,
 }
+
+# Variant switches (see kda_oracle.c): erase 1 = delta-rule family, 0 = additive
+# write; gate 0 = per-channel log_alpha [.., dk], 1 = one per token and head, 2 = none.
+GATES = {"channel": 0, "scalar": 1, "none": 2}
 
 
 def build(force: bool = False) -> str:
@@ -63,6 +70,12 @@ def _load():
         lib.kda_oracle_chunkwise.restype = I
         lib.kda_oracle_decode_step.argtypes = [P] * 8 + [I] * 5
         lib.kda_oracle_decode_step.restype = I
+        lib.kda_oracle_recurrent_v.argtypes = [P] * 8 + [I] * 9
+        lib.kda_oracle_recurrent_v.restype = I
+        lib.kda_oracle_chunkwise_v.argtypes = [P] * 8 + [I] * 6 + [P, P, I, I, I, I]
+        lib.kda_oracle_chunkwise_v.restype = I
+        lib.kda_oracle_decode_step_v.argtypes = [P] * 8 + [I] * 7
+        lib.kda_oracle_decode_step_v.restype = I
         _lib = lib
     return _lib
 
@@ -79,24 +92,31 @@ def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
-def recurrent(q, k, v, log_alpha, beta, S0=None, nthreads: int = 0, mutation: str | None = None):
-    """Token-by-token fp64 recurrence. Shapes: q,k,log_alpha [B,T,H,dk];
-    v [B,T,H,dv]; beta [B,T,H]; S0 [B,H,dk,dv] or None. Returns (o, S_T)."""
+def _gate(gate):
+    return GATES[gate] if isinstance(gate, str) else int(gate)
+
+
+def recurrent(q, k, v, log_alpha, beta, S0=None, nthreads: int = 0, mutation: str | None = None,
+              erase: bool = True, gate="channel"):
+    """Token-by-token fp64 recurrence. Shapes: q,k [B,T,H,dk]; log_alpha
+    [B,T,H,dk] (gate "channel"), [B,T,H] (gate "scalar") or None (gate
+    "none"); v [B,T,H,dv]; beta [B,T,H]; S0 [B,H,dk,dv] or None. erase=False
+    selects the additive-write family. Returns (o, S_T)."""
     q, k, v, la, beta, S0 = map(_f64, (q, k, v, log_alpha, beta, S0))
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     o = np.zeros((B, T, H, dv))
     ST = np.zeros((B, H, dk, dv))
-    rc = _load().kda_oracle_recurrent(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0),
-                                      _ptr(o), _ptr(ST), B, T, H, dk, dv, nthreads,
-                                      MUTATIONS[mutation] if mutation else 0)
+    rc = _load().kda_oracle_recurrent_v(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0),
+                                        _ptr(o), _ptr(ST), B, T, H, dk, dv, int(bool(erase)), _gate(gate),
+                                        nthreads, MUTATIONS[mutation] if mutation else 0)
     if rc:
-        raise ValueError("kda_oracle_recurrent: bad sizes")
+        raise ValueError("kda_oracle_recurrent_v: bad sizes or switches")
     return o, ST
 
 
 def chunkwise(q, k, v, log_alpha, beta, S0=None, C: int = 64, nthreads: int = 0,
-              mutation: str | None = None, debug: bool = False):
+              mutation: str | None = None, debug: bool = False, erase: bool = True, gate="channel"):
     """fp64 chunkwise reformulation. Returns (o, S_T) or, with debug=True,
     (o, S_T, A, Tinv) where A and Tinv are [B,H,NC,C,C]."""
     q, k, v, la, beta, S0 = map(_f64, (q, k, v, log_alpha, beta, S0))
@@ -107,24 +127,26 @@ def chunkwise(q, k, v, log_alpha, beta, S0=None, C: int = 64, nthreads: int = 0,
     ST = np.zeros((B, H, dk, dv))
     A = np.zeros((B, H, NC, C, C)) if debug else None
     Ti = np.zeros((B, H, NC, C, C)) if debug else None
-    rc = _load().kda_oracle_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0),
-                                      _ptr(o), _ptr(ST), B, T, H, dk, dv, C, _ptr(A), _ptr(Ti),
-                                      nthreads, MUTATIONS[mutation] if mutation else 0)
+    rc = _load().kda_oracle_chunkwise_v(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0),
+                                        _ptr(o), _ptr(ST), B, T, H, dk, dv, C, _ptr(A), _ptr(Ti),
+                                        int(bool(erase)), _gate(gate), nthreads,
+                                        MUTATIONS[mutation] if mutation else 0)
     if rc:
-        raise ValueError("kda_oracle_chunkwise: bad sizes")
+        raise ValueError("kda_oracle_chunkwise_v: bad sizes or switches")
     return (o, ST, A, Ti) if debug else (o, ST)
 
 
-def decode_step(q, k, v, log_alpha, beta, S, nthreads: int = 0):
-    """One recurrent step for [N,H,*] inputs and state S [N,H,dk,dv].
-    Returns (o, S_new)."""
+def decode_step(q, k, v, log_alpha, beta, S, nthreads: int = 0, erase: bool = True, gate="channel"):
+    """One recurrent step for [N,H,*] inputs and state S [N,H,dk,dv]
+    (log_alpha [N,H,dk], [N,H] or None by gate). Returns (o, S_new)."""
     q, k, v, la, beta, S = map(_f64, (q, k, v, log_alpha, beta, S))
     N, H, dk = q.shape
     dv = v.shape[-1]
     o = np.zeros((N, H, dv))
     Sn = np.zeros((N, H, dk, dv))
-    rc = _load().kda_oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S),
-                                        _ptr(Sn), _ptr(o), N, H, dk, dv, nthreads)
+    rc = _load().kda_oracle_decode_step_v(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S),
+                                          _ptr(Sn), _ptr(o), N, H, dk, dv, int(bool(erase)), _gate(gate),
+                                          nthreads)
     if rc:
-        raise ValueError("kda_oracle_decode_step: bad sizes")
+        raise ValueError("kda_oracle_decode_step_v: bad sizes or switches")
     return o, Sn

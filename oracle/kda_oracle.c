@@ -24,6 +24,19 @@
  *   beta            : [B, T, H]          S0, ST : [B, H, dk, dv]
  * alpha = exp(log_alpha); no activation, no q scaling.
  *
+ * Variants (same pages, section 3.4 variant table and sections 3.1-3.3, plus
+ * the per-dimension gated linear attention named beside it). Two switches:
+ *   erase = 1: delta-rule family, S_t = (I - b k k^T) Diag(a_t) S_{t-1} + b k v^T
+ *   erase = 0: linear-attention family, S_t = Diag(a_t) S_{t-1} + b k v^T
+ *              (no erase term; b = 1 gives the pages' plain write k v^T)
+ *   gate  = 0: a_t = exp(log_alpha) per key channel, log_alpha [B, T, H, dk]
+ *   gate  = 1: one decay per token and head, log_alpha [B, T, H] (scalar gated
+ *              delta rule: the scalar commutes with the erase term)
+ *   gate  = 2: no decay (a_t = 1); log_alpha is not read (may be NULL)
+ * So (erase, gate) = (1, 0) is KDA, (1, 1) the scalar gated delta rule, (1, 2)
+ * the delta rule, (0, 0) per-dimension gated linear attention, (0, 2) with
+ * beta = 1 pure linear attention.
+ *
  * Pins: every function here is checked by tests/test_oracle.py against
  * closed forms (identity, linear attention with orthogonal keys, pure decay),
  * the exact-retrieval invariant, an independent scalar-gate recurrence,
@@ -49,6 +62,8 @@ enum {
     MUT_DECAY_COLUMNS = 7,   /* decay scales value channels (needs dk == dv)  */
     MUT_PREFIX_DECAY_K = 8,  /* chunkwise: prefix decay on K in state update  */
     MUT_STRICT_TRIL_O = 9,   /* chunkwise: strict instead of inclusive mask   */
+    MUT_ERASE_ALWAYS = 10,   /* erase = 0 still applies the erase term        */
+    MUT_SCALAR_GATE_TWICE = 11, /* gate = 1 applies the scalar decay twice    */
 };
 
 typedef struct {
@@ -56,6 +71,7 @@ typedef struct {
     double *o, *ST;
     double *dbg_A, *dbg_T; /* chunkwise only: [B,H,NC,C,C] or NULL */
     int B, T, H, dk, dv, C, mutation;
+    int erase, gate; /* variant switches, see the header */
     int next_head; /* shared work counter */
     pthread_mutex_t lock;
 } job_t;
@@ -67,12 +83,23 @@ static int take_head(job_t *J) {
     return h;
 }
 
+/* log a_t for key channel c of token t (see the gate switch). */
+static double log_decay(const job_t *J, int b, int t, int h, int c) {
+    if (J->gate == 2) return 0.0;
+    if (J->gate == 1) {
+        const double g = J->la[((long)b * J->T + t) * J->H + h];
+        return (J->mutation == MUT_SCALAR_GATE_TWICE) ? 2.0 * g : g;
+    }
+    return J->la[(((long)b * J->T + t) * J->H + h) * J->dk + c];
+}
+
 /* Token-by-token recurrence for one (b, h). */
 static void recurrent_head(job_t *J, int b, int h) {
     const int T = J->T, H = J->H, dk = J->dk, dv = J->dv, mut = J->mutation;
     double *S = (double *)malloc(sizeof(double) * dk * dv);
     double *u = (double *)malloc(sizeof(double) * dv);
     double *w = (double *)malloc(sizeof(double) * dv);
+    double *lat = (double *)malloc(sizeof(double) * (dk > dv ? dk : dv));
     const long sbase = ((long)b * H + h) * dk * dv;
     if (J->S0) memcpy(S, J->S0 + sbase, sizeof(double) * dk * dv);
     else memset(S, 0, sizeof(double) * dk * dv);
@@ -80,7 +107,8 @@ static void recurrent_head(job_t *J, int b, int h) {
     for (int t = 0; t < T; ++t) {
         const long tk = (((long)b * T + t) * H + h) * dk;
         const long tv = (((long)b * T + t) * H + h) * dv;
-        const double *qt = J->q + tk, *kt = J->k + tk, *lat = J->la + tk;
+        const double *qt = J->q + tk, *kt = J->k + tk;
+        for (int i = 0; i < dk; ++i) lat[i] = log_decay(J, b, t, h, i);
         const double *vt = J->v + tv;
         const double bt = J->beta[((long)b * T + t) * H + h];
         double *ot = J->o + tv;
@@ -108,9 +136,10 @@ static void recurrent_head(job_t *J, int b, int h) {
             for (int i = 0; i < dk; ++i) acc += S[i * dv + j] * kt[i];
             u[j] = acc;
         }
-        /* (I - b k k^T) S + b k v^T  ==  S + k (b (v - u))^T */
+        /* (I - b k k^T) S + b k v^T  ==  S + k (b (v - u))^T;  no erase: S + k (b v)^T */
         for (int j = 0; j < dv; ++j) {
-            if (mut == MUT_ERASE_SIGN) w[j] = bt * (vt[j] + u[j]);
+            if (!J->erase && mut != MUT_ERASE_ALWAYS) w[j] = bt * vt[j];
+            else if (mut == MUT_ERASE_SIGN) w[j] = bt * (vt[j] + u[j]);
             else if (mut == MUT_BETA_WRITE_ONLY) w[j] = bt * vt[j] - u[j];
             else w[j] = bt * (vt[j] - u[j]);
         }
@@ -141,6 +170,7 @@ static void recurrent_head(job_t *J, int b, int h) {
     free(S);
     free(u);
     free(w);
+    free(lat);
 }
 
 /*
@@ -158,6 +188,7 @@ static void recurrent_head(job_t *J, int b, int h) {
  */
 static void chunkwise_head(job_t *J, int b, int h) {
     const int T = J->T, H = J->H, dk = J->dk, dv = J->dv, C = J->C, mut = J->mutation;
+    const int erase = J->erase || mut == MUT_ERASE_ALWAYS;
     const int NC = (T + C - 1) / C;
     double *S = (double *)malloc(sizeof(double) * dk * dv);
     double *G = (double *)malloc(sizeof(double) * C * dk);
@@ -184,7 +215,7 @@ static void chunkwise_head(job_t *J, int b, int h) {
         for (int c = 0; c < dk; ++c) {
             double acc = 0.0;
             for (int r = 0; r < n; ++r) {
-                acc += J->la[IDXK(t0 + r) + c];
+                acc += log_decay(J, b, t0 + r, h, c);
                 G[r * dk + c] = acc;
             }
         }
@@ -202,7 +233,8 @@ static void chunkwise_head(job_t *J, int b, int h) {
                         p += qr[c] * ks[c] * e;
                     }
                 }
-                A[r * C + s] = (s < r) ? BETA(t0 + r) * a : 0.0;
+                /* no erase: the chunk's tokens do not correct one another */
+                A[r * C + s] = (s < r && erase) ? BETA(t0 + r) * a : 0.0;
                 P[r * C + s] = incl ? p : 0.0;
             }
         }
@@ -241,11 +273,12 @@ static void chunkwise_head(job_t *J, int b, int h) {
                 U[r * dv + j] = acc;
             }
         }
-        /* D = U - W S */
+        /* D = U - W S  (no erase: W S is not subtracted, D = beta V) */
         for (int r = 0; r < n; ++r)
             for (int j = 0; j < dv; ++j) {
                 double acc = U[r * dv + j];
-                for (int c = 0; c < dk; ++c) acc -= W[r * dk + c] * S[c * dv + j];
+                if (erase)
+                    for (int c = 0; c < dk; ++c) acc -= W[r * dk + c] * S[c * dv + j];
                 D[r * dv + j] = acc;
             }
         /* O = (Q * exp(G)) S + P D */
@@ -317,40 +350,70 @@ static int run(job_t *J, int chunkwise, int nthreads) {
     return 0;
 }
 
-/* Token-by-token fp64 recurrence over all (b, h). S0 may be NULL (zero
- * state); ST may be NULL. nthreads <= 0 uses every online core. Returns 0 on
- * success, 1 on bad sizes. */
-int kda_oracle_recurrent(const double *q, const double *k, const double *v, const double *log_alpha,
-                         const double *beta, const double *S0, double *o, double *ST,
-                         int B, int T, int H, int dk, int dv, int nthreads, int mutation) {
+/* Token-by-token fp64 recurrence over all (b, h), variant (erase, gate). S0
+ * may be NULL (zero state); ST may be NULL. nthreads <= 0 uses every online
+ * core. Returns 0 on success, 1 on bad sizes or switches. */
+int kda_oracle_recurrent_v(const double *q, const double *k, const double *v, const double *log_alpha,
+                           const double *beta, const double *S0, double *o, double *ST,
+                           int B, int T, int H, int dk, int dv, int erase, int gate, int nthreads,
+                           int mutation) {
     job_t J;
     memset(&J, 0, sizeof(J));
+    if ((erase != 0 && erase != 1) || gate < 0 || gate > 2 || (gate != 2 && !log_alpha)) return 1;
     J.q = q; J.k = k; J.v = v; J.la = log_alpha; J.beta = beta; J.S0 = S0; J.o = o; J.ST = ST;
     J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv; J.mutation = mutation;
+    J.erase = erase; J.gate = gate;
     return run(&J, 0, nthreads);
 }
 
+/* The KDA recurrence (erase = 1, per-channel gate). */
+int kda_oracle_recurrent(const double *q, const double *k, const double *v, const double *log_alpha,
+                         const double *beta, const double *S0, double *o, double *ST,
+                         int B, int T, int H, int dk, int dv, int nthreads, int mutation) {
+    return kda_oracle_recurrent_v(q, k, v, log_alpha, beta, S0, o, ST, B, T, H, dk, dv, 1, 0, nthreads,
+                                  mutation);
+}
+
 /* fp64 chunkwise reformulation with chunk size C (any C >= 1; the last chunk
- * may be shorter). dbg_A / dbg_T, if non-NULL, receive the per-chunk A and
- * (I+A)^{-1} as [B, H, ceil(T/C), C, C] (padding rows/cols: 0 for A, identity
- * for T). */
+ * may be shorter), variant (erase, gate). dbg_A / dbg_T, if non-NULL, receive
+ * the per-chunk A and (I+A)^{-1} as [B, H, ceil(T/C), C, C] (padding
+ * rows/cols: 0 for A, identity for T). */
+int kda_oracle_chunkwise_v(const double *q, const double *k, const double *v, const double *log_alpha,
+                           const double *beta, const double *S0, double *o, double *ST,
+                           int B, int T, int H, int dk, int dv, int C, double *dbg_A, double *dbg_T,
+                           int erase, int gate, int nthreads, int mutation) {
+    job_t J;
+    memset(&J, 0, sizeof(J));
+    if ((erase != 0 && erase != 1) || gate < 0 || gate > 2 || (gate != 2 && !log_alpha)) return 1;
+    J.q = q; J.k = k; J.v = v; J.la = log_alpha; J.beta = beta; J.S0 = S0; J.o = o; J.ST = ST;
+    J.dbg_A = dbg_A; J.dbg_T = dbg_T;
+    J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv; J.C = C; J.mutation = mutation;
+    J.erase = erase; J.gate = gate;
+    return run(&J, 1, nthreads);
+}
+
+/* The KDA chunkwise form (erase = 1, per-channel gate). */
 int kda_oracle_chunkwise(const double *q, const double *k, const double *v, const double *log_alpha,
                          const double *beta, const double *S0, double *o, double *ST,
                          int B, int T, int H, int dk, int dv, int C, double *dbg_A, double *dbg_T,
                          int nthreads, int mutation) {
-    job_t J;
-    memset(&J, 0, sizeof(J));
-    J.q = q; J.k = k; J.v = v; J.la = log_alpha; J.beta = beta; J.S0 = S0; J.o = o; J.ST = ST;
-    J.dbg_A = dbg_A; J.dbg_T = dbg_T;
-    J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv; J.C = C; J.mutation = mutation;
-    return run(&J, 1, nthreads);
+    return kda_oracle_chunkwise_v(q, k, v, log_alpha, beta, S0, o, ST, B, T, H, dk, dv, C, dbg_A, dbg_T, 1, 0,
+                                  nthreads, mutation);
 }
 
 /* One recurrent decode step for N sequences x H heads: the recurrence with
- * T = 1. Layouts: q, k, log_alpha [N, H, dk]; v, o [N, H, dv]; beta [N, H];
+ * T = 1, variant (erase, gate). Layouts: q, k [N, H, dk]; log_alpha [N, H, dk]
+ * (gate 0), [N, H] (gate 1) or unused (gate 2); v, o [N, H, dv]; beta [N, H];
  * S_in, S_out [N, H, dk, dv] (S_out may equal S_in). */
+int kda_oracle_decode_step_v(const double *q, const double *k, const double *v, const double *log_alpha,
+                             const double *beta, const double *S_in, double *S_out, double *o,
+                             int N, int H, int dk, int dv, int erase, int gate, int nthreads) {
+    return kda_oracle_recurrent_v(q, k, v, log_alpha, beta, S_in, o, S_out, N, 1, H, dk, dv, erase, gate,
+                                  nthreads, 0);
+}
+
 int kda_oracle_decode_step(const double *q, const double *k, const double *v, const double *log_alpha,
                            const double *beta, const double *S_in, double *S_out, double *o,
                            int N, int H, int dk, int dv, int nthreads) {
-    return kda_oracle_recurrent(q, k, v, log_alpha, beta, S_in, o, S_out, N, 1, H, dk, dv, nthreads, 0);
+    return kda_oracle_decode_step_v(q, k, v, log_alpha, beta, S_in, S_out, o, N, H, dk, dv, 1, 0, nthreads);
 }

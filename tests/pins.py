@@ -118,3 +118,87 @@ def p5_scalar_gate(run, seed=15, T=24, dk=8, dv=8):
 
 
 ALL_PINS = [p1_identity, p2_linear_attention, p3_pure_decay, p4_retrieval, p5_scalar_gate]
+
+
+# ---------------------------------------------------------------- variants
+# Each variant pin takes `run(q, k, v, log_alpha, beta, S0, erase=..., gate=...)`
+# and compares with the rule as the pages state it, written out independently.
+
+
+def p10_delta_rule(run, seed=20, T=24, dk=8, dv=8):
+    """Section 3.2 (delta rule, no gate): S_t = (I - b_t k_t k_t^T) S_{t-1}
+    + b_t k_t v_t^T, with explicit matrices."""
+    q, k, v, _, beta, S0 = random_inputs(seed, T, dk, dv)
+    o, ST = run(q, k, v, None, beta, S0, erase=True, gate="none")
+    err = 0.0
+    I = np.eye(dk)
+    for b in range(q.shape[0]):
+        for h in range(q.shape[2]):
+            S = S0[b, h].copy()
+            for t in range(T):
+                kt, bt = k[b, t, h], beta[b, t, h]
+                S = (I - bt * np.outer(kt, kt)) @ S + bt * np.outer(kt, v[b, t, h])
+                err = max(err, np.abs(o[b, t, h] - S.T @ q[b, t, h]).max())
+            err = max(err, np.abs(ST[b, h] - S).max())
+    return err
+
+
+def p11_scalar_gated_delta(run, seed=21, T=24, dk=8, dv=8):
+    """Section 3.3 / variant table (scalar gated delta, one gate per token and
+    head): S_t = a_t (I - b_t k_t k_t^T) S_{t-1} + b_t k_t v_t^T, the scalar
+    applied outside the erase as printed, with explicit matrices."""
+    q, k, v, la, beta, S0 = random_inputs(seed, T, dk, dv)
+    g = la[..., 0]                                  # [B,T,H]
+    o, ST = run(q, k, v, g, beta, S0, erase=True, gate="scalar")
+    err = 0.0
+    I = np.eye(dk)
+    for b in range(q.shape[0]):
+        for h in range(q.shape[2]):
+            S = S0[b, h].copy()
+            for t in range(T):
+                kt, bt = k[b, t, h], beta[b, t, h]
+                S = np.exp(g[b, t, h]) * (I - bt * np.outer(kt, kt)) @ S + bt * np.outer(kt, v[b, t, h])
+                err = max(err, np.abs(o[b, t, h] - S.T @ q[b, t, h]).max())
+            err = max(err, np.abs(ST[b, h] - S).max())
+    return err
+
+
+def p12_gated_linear_attention(run, seed=22, T=24, dk=8, dv=8):
+    """Per-dimension gated linear attention (named beside the variant table):
+    S_t = Diag(a_t) S_{t-1} + b_t k_t v_t^T, so in closed form
+    S_t = Diag(e^{G_t}) S_0 + sum_{s<=t} b_s Diag(e^{G_t - G_s}) k_s v_s^T with
+    G_t = sum_{u<=t} log a_u, and o_t = S_t^T q_t."""
+    q, k, v, la, beta, S0 = random_inputs(seed, T, dk, dv)
+    o, ST = run(q, k, v, la, beta, S0, erase=False, gate="channel")
+    G = np.cumsum(la, axis=1)                       # [B,T,H,dk]
+    err = 0.0
+    for b in range(q.shape[0]):
+        for h in range(q.shape[2]):
+            for t in range(T):
+                S = np.exp(G[b, t, h])[:, None] * S0[b, h]
+                for s_ in range(t + 1):
+                    S = S + beta[b, s_, h] * np.outer(np.exp(G[b, t, h] - G[b, s_, h]) * k[b, s_, h], v[b, s_, h])
+                err = max(err, np.abs(o[b, t, h] - S.T @ q[b, t, h]).max())
+                if t == T - 1:
+                    err = max(err, np.abs(ST[b, h] - S).max())
+    return err
+
+
+def p13_plain_linear_attention(run, seed=23, T=24, dk=8, dv=8):
+    """Section 3.1: S_t = S_{t-1} + k_t v_t^T (no erase, no gate, b = 1):
+    o_t = S_0^T q_t + sum_{s<=t} (q_t . k_s) v_s and S_T = S_0 + sum_s k_s v_s^T,
+    for any keys (not only orthogonal ones)."""
+    q, k, v, _, beta, S0 = random_inputs(seed, T, dk, dv)
+    beta[:] = 1.0
+    o, ST = run(q, k, v, None, beta, S0, erase=False, gate="none")
+    err = 0.0
+    for b in range(q.shape[0]):
+        for h in range(q.shape[2]):
+            for t in range(T):
+                o_ref = S0[b, h].T @ q[b, t, h] + sum((q[b, t, h] @ k[b, s_, h]) * v[b, s_, h] for s_ in range(t + 1))
+                err = max(err, np.abs(o[b, t, h] - o_ref).max())
+            err = max(err, np.abs(ST[b, h] - (S0[b, h] + k[b, :, h].T @ v[b, :, h])).max())
+    return err
+
+
+VARIANT_PINS = [p10_delta_rule, p11_scalar_gated_delta, p12_gated_linear_attention, p13_plain_linear_attention]

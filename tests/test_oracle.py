@@ -6,6 +6,8 @@ P6: the token recurrence and the chunkwise reformulation agree by brute force
 P7: state passing: one call over [0,T) equals two calls chained through S_T.
 P8: T chained single-token decode steps equal the prefill recurrence.
 P9: the chunkwise intermediate T is the inverse of (I + A).
+P10-P13: the variants (delta rule, scalar gated delta rule, gated linear
+    attention, plain linear attention) against their rules written out.
 Mutation test: each planted mistake in the oracle makes at least one pin fail.
 """
 import numpy as np
@@ -130,3 +132,68 @@ def test_hand_worked_example():
         o, ST = run(q, k, v, la, beta, S0)
         assert np.abs(o[0, :, 0] - np.array(g["o"])).max() < 1e-12
         assert np.abs(ST[0, 0] - np.array(g["S_T"])).max() < 1e-12
+
+
+# ---------------------------------------------------------------- variants
+
+
+def vrec(mutation=None):
+    return lambda q, k, v, la, b, S0, erase, gate: oracle.recurrent(q, k, v, la, b, S0, mutation=mutation,
+                                                                   erase=erase, gate=gate)
+
+
+def vchk(C, mutation=None):
+    return lambda q, k, v, la, b, S0, erase, gate: oracle.chunkwise(q, k, v, la, b, S0, C=C, mutation=mutation,
+                                                                   erase=erase, gate=gate)
+
+
+VRUNNERS = {"recurrent": vrec(), "chunkwise_c1": vchk(1), "chunkwise_c5": vchk(5), "chunkwise_c16": vchk(16)}
+
+
+@pytest.mark.parametrize("runner", list(VRUNNERS))
+@pytest.mark.parametrize("pin", pins.VARIANT_PINS, ids=lambda p: p.__name__)
+def test_variant_pins(pin, runner):
+    assert pin(VRUNNERS[runner]) < TOL
+
+
+@pytest.mark.parametrize("erase,gate", [(True, "scalar"), (True, "none"), (False, "channel"), (False, "scalar"),
+                                        (False, "none")])
+@pytest.mark.parametrize("C,T", [(1, 9), (4, 33), (16, 16), (64, 100)])
+def test_variant_recurrence_equals_chunkwise(erase, gate, C, T):
+    q, k, v, la, beta, S0 = pins.random_inputs(300 + T + C, T=T, dk=6, dv=5)
+    g = {"channel": la, "scalar": la[..., 0], "none": None}[gate]
+    o1, s1 = oracle.recurrent(q, k, v, g, beta, S0, erase=erase, gate=gate)
+    o2, s2 = oracle.chunkwise(q, k, v, g, beta, S0, C=C, erase=erase, gate=gate)
+    assert np.abs(o1 - o2).max() / max(1.0, np.abs(o1).max()) < 1e-12
+    assert np.abs(s1 - s2).max() / max(1.0, np.abs(s1).max()) < 1e-12
+
+
+@pytest.mark.parametrize("erase,gate", [(True, "scalar"), (False, "channel"), (False, "none")])
+def test_variant_decode_chaining(erase, gate):
+    """T single-token steps of the variant equal its prefill recurrence."""
+    q, k, v, la, beta, S0 = pins.random_inputs(400, T=12, dk=6, dv=5)
+    g = {"channel": la, "scalar": la[..., 0], "none": None}[gate]
+    o_ref, S_ref = oracle.recurrent(q, k, v, g, beta, S0, erase=erase, gate=gate)
+    S = S0
+    for t in range(q.shape[1]):
+        gt = None if g is None else g[:, t]
+        o, S = oracle.decode_step(q[:, t], k[:, t], v[:, t], gt, beta[:, t], S, erase=erase, gate=gate)
+        assert np.abs(o - o_ref[:, t]).max() < 1e-12
+    assert np.abs(S - S_ref).max() < 1e-12
+
+
+@pytest.mark.parametrize("mutation,pin", [("erase_always", pins.p12_gated_linear_attention),
+                                          ("erase_always", pins.p13_plain_linear_attention),
+                                          ("scalar_gate_twice", pins.p11_scalar_gated_delta)])
+@pytest.mark.parametrize("runner", ["recurrent", "chunkwise"])
+def test_variant_mutations_caught(mutation, pin, runner):
+    run = vrec(mutation) if runner == "recurrent" else vchk(8, mutation)
+    assert pin(run) > 1e-6
+
+
+def test_variant_bad_switches():
+    q, k, v, la, beta, S0 = pins.random_inputs(1, T=4, dk=4, dv=4)
+    with pytest.raises(ValueError):
+        oracle.recurrent(q, k, v, None, beta, S0, gate="channel")  # a gate needs log_alpha
+    with pytest.raises(ValueError):
+        oracle.chunkwise(q, k, v, la, beta, S0, C=4, gate=3)
