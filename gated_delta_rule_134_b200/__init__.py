@@ -20,6 +20,9 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
           4: "KDA_ERR_TIMEOUT"}
 _DTYPE = {"f32": 0, "bf16": 1}
 _ALGO = {"auto": 0, "simt": 1, "tc": 2}
+# Variant switches (include/kda.h): gate "channel" = log_alpha [.., dk], "scalar" =
+# one per token and head, "none" = no decay (log_alpha may be None).
+GATES = {"channel": 0, "scalar": 1, "none": 2}
 
 
 class KDAError(RuntimeError):
@@ -63,6 +66,10 @@ def load(build_if_stale: bool = True):
     lib.kda_decode_step.restype = I
     lib.kda_chunk_fwd_noalloc.argtypes = [P] * 8 + [I] * 7 + [P]
     lib.kda_chunk_fwd_noalloc.restype = I
+    lib.kda_chunk_fwd_v.argtypes = [P] * 8 + [I] * 9 + [P, Z, I, P]
+    lib.kda_chunk_fwd_v.restype = I
+    lib.kda_decode_step_v.argtypes = [P] * 8 + [I] * 7 + [P]
+    lib.kda_decode_step_v.restype = I
     _lib = lib
     return lib
 
@@ -103,13 +110,22 @@ def workspace_size(B, T, H, dk, dv, chunk=64, dtype="bf16", algo="auto") -> int:
     return int(load().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, _DTYPE[dtype], _ALGO[algo]))
 
 
+def _gate_shape(gate, lead, dk):
+    if gate not in GATES:
+        raise ValueError(f"gate must be one of {sorted(GATES)}")
+    return None if gate == "none" else (tuple(lead) + (dk,) if gate == "channel" else tuple(lead))
+
+
 def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, chunk: int = 64, algo: str = "auto",
-              output_final_state: bool = True, o=None, S_T=None, workspace=None, stream=None):
+              output_final_state: bool = True, o=None, S_T=None, workspace=None, stream=None,
+              erase: bool = True, gate: str = "channel"):
     """kda_chunk_fwd(q, k, v, log_alpha, beta, S0 -> o, S_T) on CUDA tensors.
 
-    q, k, log_alpha: [B,T,H,dk]; v: [B,T,H,dv]; beta: [B,T,H] (all float32 or
-    all bfloat16); S0: [B,H,dk,dv] float32 or None. Returns (o, S_T) with S_T
-    None when output_final_state is False."""
+    q, k: [B,T,H,dk]; v: [B,T,H,dv]; beta: [B,T,H]; log_alpha: [B,T,H,dk]
+    (gate "channel"), [B,T,H] (gate "scalar") or None (gate "none"), all
+    float32 or all bfloat16; S0: [B,H,dk,dv] float32 or None. erase=False
+    selects the additive-write variants (kda_chunk_fwd_v). Returns (o, S_T)
+    with S_T None when output_final_state is False."""
     import torch
     lib = load()
     B, T, H, dk = q.shape
@@ -117,7 +133,9 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, chunk: int = 64, algo: str =
     dt, dev = q.dtype, q.device
     _need(q, "q", (B, T, H, dk), dt, dev)
     _need(k, "k", (B, T, H, dk), dt, dev)
-    _need(log_alpha, "log_alpha", (B, T, H, dk), dt, dev)
+    gshape = _gate_shape(gate, (B, T, H), dk)
+    if gshape is not None:
+        _need(log_alpha, "log_alpha", gshape, dt, dev)
     _need(v, "v", (B, T, H, dv), dt, dev)
     _need(beta, "beta", (B, T, H), dt, dev)
     if S0 is not None:
@@ -134,10 +152,11 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, chunk: int = 64, algo: str =
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    code = lib.kda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(o),
-                                _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPE[dts], _ptr(workspace), ws_len,
-                                _ALGO[algo], _stream(stream))
-    _check("kda_chunk_fwd_ex", code)
+    la = log_alpha if gshape is not None else None
+    code = lib.kda_chunk_fwd_v(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0), _ptr(o),
+                               _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPE[dts], int(bool(erase)), GATES[gate],
+                               _ptr(workspace), ws_len, _ALGO[algo], _stream(stream))
+    _check("kda_chunk_fwd_v", code)
     return o, S_T
 
 
@@ -147,10 +166,12 @@ def workspace_status(workspace, stream=None) -> int:
     return int(load().kda_workspace_status(_ptr(workspace), ws_len, _stream(stream)))
 
 
-def decode_step(q, k, v, log_alpha, beta, S, *, S_out=None, o=None, stream=None):
+def decode_step(q, k, v, log_alpha, beta, S, *, S_out=None, o=None, stream=None, erase: bool = True,
+                gate: str = "channel"):
     """kda_decode_step(q, k, v, log_alpha, beta, S -> o, S'): one token per
-    sequence. q, k, log_alpha [N,H,dk]; v [N,H,dv]; beta [N,H]; S [N,H,dk,dv]
-    float32. S_out defaults to S (in-place update). Returns (o, S_out)."""
+    sequence. q, k [N,H,dk]; log_alpha [N,H,dk] / [N,H] / None by gate; v
+    [N,H,dv]; beta [N,H]; S [N,H,dk,dv] float32. S_out defaults to S
+    (in-place update). Returns (o, S_out)."""
     import torch
     lib = load()
     N, H, dk = q.shape
@@ -158,7 +179,9 @@ def decode_step(q, k, v, log_alpha, beta, S, *, S_out=None, o=None, stream=None)
     dt, dev = q.dtype, q.device
     _need(q, "q", (N, H, dk), dt, dev)
     _need(k, "k", (N, H, dk), dt, dev)
-    _need(log_alpha, "log_alpha", (N, H, dk), dt, dev)
+    gshape = _gate_shape(gate, (N, H), dk)
+    if gshape is not None:
+        _need(log_alpha, "log_alpha", gshape, dt, dev)
     _need(v, "v", (N, H, dv), dt, dev)
     _need(beta, "beta", (N, H), dt, dev)
     _need(S, "S", (N, H, dk, dv), torch.float32, dev)
@@ -168,9 +191,11 @@ def decode_step(q, k, v, log_alpha, beta, S, *, S_out=None, o=None, stream=None)
     if o is None:
         o = torch.empty(N, H, dv, dtype=dt, device=dev)
     _need(o, "o", (N, H, dv), dt, dev)
-    code = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(S_out),
-                               _ptr(o), N, H, dk, dv, _DTYPE[_dtype_of(q)], _stream(stream))
-    _check("kda_decode_step", code)
+    la = log_alpha if gshape is not None else None
+    code = lib.kda_decode_step_v(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S), _ptr(S_out),
+                                 _ptr(o), N, H, dk, dv, _DTYPE[_dtype_of(q)], int(bool(erase)), GATES[gate],
+                                 _stream(stream))
+    _check("kda_decode_step_v", code)
     return o, S_out
 
 

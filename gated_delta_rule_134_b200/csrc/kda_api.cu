@@ -17,11 +17,15 @@ kda_status_t check_chunk_args(const kda::ChunkArgs& a, kda_dtype_t dtype) {
     if (!head_dims_ok(a.dk, a.dv)) return KDA_ERR_UNSUPPORTED;
     if (a.chunk != 16 && a.chunk != 32 && a.chunk != 64) return KDA_ERR_UNSUPPORTED;
     if ((long long)a.B * a.H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    if (a.erase != 0 && a.erase != 1) return KDA_ERR_INVALID_ARG;
+    if (a.gate < KDA_GATE_CHANNEL || a.gate > KDA_GATE_NONE) return KDA_ERR_INVALID_ARG;
     const bool has_tokens = (long long)a.B * a.T * a.H > 0;
     if (has_tokens) {
-        const void* req[] = {a.q, a.k, a.v, a.log_alpha, a.beta, a.o};
+        const void* req[] = {a.q, a.k, a.v, a.beta, a.o};
         for (const void* p : req)
             if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+        if (a.gate != KDA_GATE_NONE && (a.log_alpha == nullptr || !aligned16(a.log_alpha)))
+            return KDA_ERR_INVALID_ARG;
     }
     if (a.S0 && !aligned16(a.S0)) return KDA_ERR_INVALID_ARG;
     if (a.ST && !aligned16(a.ST)) return KDA_ERR_INVALID_ARG;
@@ -52,13 +56,14 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chu
     return tc ? kda::chunk_tc_workspace_bytes(B, T, H, dk, dv) : 0;
 }
 
-kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
-                              const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
-                              kda_dtype_t dtype, void* workspace, size_t workspace_bytes, kda_algo_t algo,
-                              void* stream) {
+kda_status_t kda_chunk_fwd_v(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                             const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
+                             kda_dtype_t dtype, int erase, kda_gate_t gate, void* workspace, size_t workspace_bytes,
+                             kda_algo_t algo, void* stream) {
     kda::ChunkArgs a;
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
+    a.erase = erase; a.gate = (int)gate;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
     kda_status_t st = check_chunk_args(a, dtype);
     if (st != KDA_OK) return st;
@@ -77,6 +82,14 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                              const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
+                              kda_dtype_t dtype, void* workspace, size_t workspace_bytes, kda_algo_t algo,
+                              void* stream) {
+    return kda_chunk_fwd_v(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, dk, dv, chunk, dtype, 1, KDA_GATE_CHANNEL,
+                           workspace, workspace_bytes, algo, stream);
+}
+
 kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                            const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
                            kda_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream) {
@@ -93,20 +106,30 @@ kda_status_t kda_workspace_status(const void* workspace, size_t workspace_bytes,
     return flag ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 
-kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
-                             const float* S_in, float* S_out, void* o, int N, int H, int dk, int dv,
-                             kda_dtype_t dtype, void* stream) {
+kda_status_t kda_decode_step_v(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                               const float* S_in, float* S_out, void* o, int N, int H, int dk, int dv,
+                               kda_dtype_t dtype, int erase, kda_gate_t gate, void* stream) {
     if (N < 0 || H < 0) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (erase != 0 && erase != 1) return KDA_ERR_INVALID_ARG;
+    if (gate < KDA_GATE_CHANNEL || gate > KDA_GATE_NONE) return KDA_ERR_INVALID_ARG;
     if (!head_dims_ok(dk, dv)) return KDA_ERR_UNSUPPORTED;
     if ((long long)N * H * (dv / 32) > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
     if ((long long)N * H == 0) return KDA_OK;
-    const void* req[] = {q, k, v, log_alpha, beta, S_in, S_out, o};
+    const void* req[] = {q, k, v, beta, S_in, S_out, o};
     for (const void* p : req)
         if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (gate != KDA_GATE_NONE && (log_alpha == nullptr || !aligned16(log_alpha))) return KDA_ERR_INVALID_ARG;
     const cudaError_t err = kda::launch_decode(q, k, v, log_alpha, beta, S_in, S_out, o, N, H, dk, dv,
-                                               dtype == KDA_BF16, static_cast<cudaStream_t>(stream));
+                                               dtype == KDA_BF16, erase, (int)gate, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                             const float* S_in, float* S_out, void* o, int N, int H, int dk, int dv,
+                             kda_dtype_t dtype, void* stream) {
+    return kda_decode_step_v(q, k, v, log_alpha, beta, S_in, S_out, o, N, H, dk, dv, dtype, 1, KDA_GATE_CHANNEL,
+                             stream);
 }
 
 }  // extern "C"

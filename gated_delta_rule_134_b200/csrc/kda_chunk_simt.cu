@@ -18,6 +18,9 @@
 //   S <- Diag(e^{G_last}) S + (k e^{G_last - G})^T D
 // One CTA owns one (batch, head) and a 32-wide slice of the value channels;
 // the slice's state stays in shared memory across all chunks.
+// Variants (variant table of section 3.4): the gate switch selects a
+// per-channel, per-token-scalar or absent log_alpha; without the erase term
+// (additive write) A = 0 and W = 0, so T = I and D = beta v.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -35,7 +38,7 @@ template <typename T, int DK, int C>
 __global__ void __launch_bounds__(kSimtThreads)
 chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const T* __restrict__ log_alpha, const T* __restrict__ beta, const float* S0,
-                  T* __restrict__ o, float* ST, int Tlen, int H, int dv) {
+                  T* __restrict__ o, float* ST, int Tlen, int H, int dv, int erase, int gate) {
     constexpr int NT = kSimtThreads, DVT = kSimtDVT;
     extern __shared__ float smem[];
     float* sQ = smem;             // q, then q e^G
@@ -69,10 +72,11 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             const int r = e / DK, c = e % DK;
             float qv = 0.f, kv = 0.f, lv = 0.f;
             if (r < len) {
-                const size_t off = (((size_t)b * Tlen + t0 + r) * H + h) * DK + c;
+                const size_t tok = ((size_t)b * Tlen + t0 + r) * H + h;
+                const size_t off = tok * DK + c;
                 qv = to_f32(q[off]);
                 kv = to_f32(k[off]);
-                lv = to_f32(log_alpha[off]);
+                lv = gate == 0 ? to_f32(log_alpha[off]) : (gate == 1 ? to_f32(log_alpha[tok]) : 0.f);
             }
             sQ[e] = qv;
             sK[e] = kv;
@@ -111,7 +115,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
                 a = fmaf(sK[r * DK + c], ks, a);
                 pp = fmaf(sQ[r * DK + c], ks, pp);
             }
-            sA[r * C + s] = (s < r) ? sB[r] * a : 0.f;
+            sA[r * C + s] = (s < r && erase) ? sB[r] * a : 0.f;
             sP[r * C + s] = pp;
             if (s < r) {
                 sA[s * C + r] = 0.f;
@@ -137,7 +141,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         for (int e = tid; e < C * DK; e += NT) {
             const int r = e / DK, c = e % DK;
             const float g = sG[e], eg = expf(g), kv = sK[e];
-            sX[e] = sB[r] * kv * eg;
+            sX[e] = erase ? sB[r] * kv * eg : 0.f;  // W = 0 without the erase term
             sQ[e] *= eg;
             sK[e] = kv * expf(sG[(C - 1) * DK + c] - g);
         }
@@ -202,7 +206,8 @@ static cudaError_t launch_simt_t(const ChunkArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     dim3 grid((unsigned)(a.B * a.H), (unsigned)(a.dv / kSimtDVT));
     kern<<<grid, kSimtThreads, smem, stream>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, (const T*)a.log_alpha,
-                                               (const T*)a.beta, a.S0, (T*)a.o, a.ST, a.T, a.H, a.dv);
+                                               (const T*)a.beta, a.S0, (T*)a.o, a.ST, a.T, a.H, a.dv, a.erase,
+                                               a.gate);
     return cudaGetLastError();
 }
 

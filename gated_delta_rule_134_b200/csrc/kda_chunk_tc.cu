@@ -59,6 +59,8 @@
 // Every wait on an mbarrier is bounded; on expiry the kernel records status 1
 // in the caller's workspace word and stops waiting (later waits are skipped,
 // so every role reaches the end), frees its tensor memory and returns.
+#include <type_traits>
+
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_sm100.cuh"
@@ -108,7 +110,8 @@ struct Layout {
     static constexpr uint32_t SEK = STMS + 2048;    // 128 f32: e^{G_last - G_m} of the last prepared chunk
     static constexpr uint32_t SGM = SEK + 512;      // 128 f32: G_m of the chunk being prepared
     static constexpr uint32_t SGL = SGM + 512;      // 128 f32: G_last
-    static constexpr uint32_t BARS = SGL + 512;     // mbarriers
+    static constexpr uint32_t SGS = SGL + 512;      // 64 f32: prefix sums of a per-token gate
+    static constexpr uint32_t BARS = SGS + 256;     // mbarriers
     static constexpr uint32_t MISC = BARS + 256;    // tmem base, abort flag, guard verdicts
     static constexpr uint32_t END = MISC + 16;
     static constexpr uint32_t SMEM_BYTES = END + 1024;   // + alignment slack
@@ -219,12 +222,16 @@ __device__ __forceinline__ bool nb_or(int id, int nthreads, bool pred) {
     return r != 0;
 }
 
-template <int DVT>
+// ERASE: 1 delta-rule family, 0 additive write. GATE: 0 per-channel log_alpha,
+// 1 one per token and head, 2 none. Compile-time, so each variant is its own
+// kernel and the KDA instance carries no variant branches.
+template <int DVT, int ERASE, int GATE>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
                     const __nv_bfloat16* __restrict__ beta, const float* S0, __nv_bfloat16* __restrict__ o,
-                    float* ST, int Tlen, int H, unsigned* status) {
+                    float* ST, int Tlen, int H, unsigned* status, const __nv_bfloat16* __restrict__ gate_tok) {
+    constexpr int erase = ERASE, gate = GATE;
     using L = Layout<DVT>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base (the 128-byte swizzle repeats every 1024 bytes);
@@ -365,24 +372,26 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 if (m + 1 < NC)
                     for (int x = 0; x < DVT / 64; ++x) tma_prefetch_l2_4d(&tm_v, j0 + 64 * x, h, (m + 1) * kC, b);
             };
+            // a per-token gate or none: no log_alpha tile and no prefix-sum MMA
+            // (the prefix-sum barrier still completes, with an empty commit)
             issue_kq(0);
-            issue_g(0);
+            if (gate == 0) issue_g(0);
             issue_v(0);
             if (NC > 1) {
                 issue_kq(1);
-                issue_g(1);
+                if (gate == 0) issue_g(1);
             }
             // next chunk for each kind of work
-            int ncs = 0, nap = 0, nuw = 0, nv = 1, nkq = 2, ng = 2;
+            int ncs = 0, nap = 0, nuw = 0, nv = 1, nkq = 2, ng = gate == 0 ? 2 : NC;
             long long idle_since = clock64();
             while ((ncs < NC || nap < NC || nuw < NC || nv < NC || nkq < NC || ng < NC) && !*s_abort) {
                 bool prog = false;
                 // [G; G] = [L; L] g: the tile landed and the previous chunk's A/P were read out
-                if (ncs < NC && mbar_test(bars + BAR_G + (ncs & 1), (uint32_t)(ncs >> 1)) &&
+                if (ncs < NC && (gate != 0 || mbar_test(bars + BAR_G + (ncs & 1), (uint32_t)(ncs >> 1))) &&
                     (ncs == 0 || mbar_test(bars + BAR_P4, (uint32_t)(ncs - 1)))) {
                     tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
+                    for (int kk = 0; kk < 4 && gate == 0; ++kk)
                         mma_bf16_ss(tmem + L::GC_COL, dadd(dLMAT, kk * 32),
                                     dadd(dCOLN, (ncs & 1) * 16384 + kk * 2048), ID_CS, kk > 0);
                     mma_commit(bars + BAR_CS);
@@ -640,9 +649,41 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const int t = m * kC + tid;
             return (tid < kC && m < NC && t < Tlen) ? __bfloat162float(beta[((size_t)b * Tlen + t) * H + h]) : 0.f;
         };
+        float* sGs = reinterpret_cast<float*>(sm + L::SGS);
         auto p2 = [&](int m) -> bool {
             const int par = m & 1, slot = m & 3;
             const uint32_t gaddr = lane_addr + L::GC_COL + 32 * cb;  // this thread's 32 channels of G
+            if (gate == 1) {  // per-token gate: prefix sums over the chunk's 64 tokens (one warp scans)
+                if (warp == 0) {
+                    const int t0 = m * kC;
+                    float g0 = (t0 + lane < Tlen) ? __bfloat162float(gate_tok[((size_t)b * Tlen + t0 + lane) * H + h]) : 0.f;
+                    float g1 = (t0 + 32 + lane < Tlen) ? __bfloat162float(gate_tok[((size_t)b * Tlen + t0 + 32 + lane) * H + h])
+                                                       : 0.f;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float x0 = __shfl_up_sync(0xffffffffu, g0, off), x1 = __shfl_up_sync(0xffffffffu, g1, off);
+                        if (lane >= off) {
+                            g0 += x0;
+                            g1 += x1;
+                        }
+                    }
+                    sGs[lane] = g0;
+                    sGs[32 + lane] = g1 + __shfl_sync(0xffffffffu, g0, 31);
+                }
+                nb_sync(NB_PREP, kPrep);
+            }
+            // G of 8 channels of this thread's token: from tensor memory (per-channel
+            // gate; warp-collective, the branch is uniform), the per-token sums, or 0
+            auto load_g8 = [&](int u4, uint32_t (&g8)[8]) {
+                if (gate == 0) {
+                    tmem_ld8(gaddr + 8 * u4, g8);
+                    tmem_ld_wait(g8);
+                } else {
+                    const uint32_t gv = gate == 1 ? __float_as_uint(sGs[tok]) : 0u;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) g8[e] = gv;
+                }
+            };
             // Rolled loops over groups of 8 channels keep the loop bodies
             // small: every chunk streams this code again, and what is not
             // in the instruction cache stalls the warp.
@@ -652,8 +693,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll 1
                 for (int u4 = 0; u4 < 4; ++u4) {
                     uint32_t g8[8];
-                    tmem_ld8(gaddr + 8 * u4, g8);
-                    tmem_ld_wait(g8);
+                    load_g8(u4, g8);
                     if (tok == 31 || tok == 63) {
                         *reinterpret_cast<float4*>(dst + 8 * u4) =
                             make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]), __uint_as_float(g8[2]),
@@ -670,8 +710,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll 1
             for (int u4 = 0; u4 < 4; ++u4) {
                 uint32_t g8[8];
-                tmem_ld8(gaddr + 8 * u4, g8);
-                tmem_ld_wait(g8);
+                load_g8(u4, g8);
                 const float4 ma = *reinterpret_cast<const float4*>(sGm + 32 * cb + 8 * u4);
                 const float4 mb = *reinterpret_cast<const float4*>(sGm + 32 * cb + 8 * u4 + 4);
                 const float gm8[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
@@ -703,8 +742,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll 1
                 for (int u4 = 0; u4 < 4; ++u4) {
                     uint32_t g8[8];
-                    tmem_ld8(gaddr + 8 * u4, g8);
-                    tmem_ld_wait(g8);
+                    load_g8(u4, g8);
                     float* dst = sG + tok * 128 + 32 * cb + 8 * u4;
                     *reinterpret_cast<float4*>(dst) = make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]),
                                                                   __uint_as_float(g8[2]), __uint_as_float(g8[3]));
@@ -735,7 +773,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         }
                         const int tr = m * kC + r;  // beta of chunk m (the scratch holds the previous chunk's)
                         const float br = tr < Tlen ? __bfloat162float(beta[((size_t)b * Tlen + tr) * H + h]) : 0.f;
-                        av[i] = (s < r) ? br * a : 0.f;
+                        av[i] = (s < r && erase) ? br * a : 0.f;  // no erase: A = 0
                         pv[i] = pp;
                     }
                 }
@@ -763,7 +801,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             for (int u4 = 0; u4 < 4; ++u4) {
                 const int c0 = 32 * cb + 8 * u4;
                 uint32_t g8[8];
-                tmem_ld8(gaddr + 8 * u4, g8);
+                load_g8(u4, g8);
                 const uint32_t ko = rop_off(tok, c0);
                 const uint32_t fo = (uint32_t)((c0 >> 6) * 8192 + tok * 128 + ((((c0 & 63) >> 3) ^ (tok & 7)) << 4));
                 const uint4 kv = ld_shared_v4(rop + ko);
@@ -771,7 +809,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 const float4 ra = *reinterpret_cast<const float4*>((exact ? sGl : sGm) + c0);
                 const float4 rb = *reinterpret_cast<const float4*>((exact ? sGl : sGm) + c0 + 4);
                 const float ref8[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-                tmem_ld_wait(g8);
                 const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w}, qw[4] = {qv.x, qv.y, qv.z, qv.w};
                 uint32_t ke[4], qe[4], kf[4];
 #pragma unroll
@@ -810,6 +847,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             tmem_ld32(lane_addr + L::GC_COL + 32 * hf, v);
             tmem_ld_wait(v);
             if (quad < 2) {
+                if (!erase) return;  // additive write: A is not used
                 const int r = 32 * quad + lane;
                 const float br = sBeta[r];
                 float* dst = sA + r * kLDA + 32 * hf;
@@ -844,6 +882,21 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             *reinterpret_cast<__nv_bfloat16*>(sm + L::TZP + km_off(r, s)) = __float2bfloat16_rn(t * sBeta[s]);
         };
         auto p5 = [&]() {
+            if (!erase) {  // A = 0: T = I, T' = Diag(beta); thread: row tid/4, 16 columns
+                const int r = tid >> 2, j0c = 2 * (tid & 3);
+#pragma unroll
+                for (int jc = 0; jc < 2; ++jc) {
+                    const int j = j0c + jc;  // 8-column chunk
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int s0 = 8 * j + 2 * u;
+                        w[u] = pack_bf16x2(s0 == r ? sBeta[r] : 0.f, s0 + 1 == r ? sBeta[r] : 0.f);
+                    }
+                    st_shared_v4(sb + L::TZP + r * 128 + ((j ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                }
+                return;
+            }
             {   // diagonal 16x16 blocks: four threads per column, rows q, q+4, q+8, q+12
                 const int a = tid >> 6, jc = (tid >> 2) & 15, q = tid & 3;
                 const float* Ab = sA + (16 * a) * kLDA + 16 * a;
@@ -902,6 +955,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         };
         // ---- P7: [W'; 0] (lanes 0-63) -> -W' over the KE rows
         auto p7 = [&](int par) {
+            if (quad < 2 && !erase) {  // additive write: delta = U, the W S term is zero
+                const int r = 32 * quad + lane;
+#pragma unroll
+                for (int jc = 0; jc < 8; ++jc)
+                    st_shared_v4(rowop(par) + hf * 16384 + r * 128 + ((jc ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
+                return;
+            }
             if (quad < 2) {
                 const int r = 32 * quad + lane;
 #pragma unroll 1
@@ -1016,14 +1076,15 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DVT>
+template <int DVT, int ERASE, int GATE>
 cudaError_t launch_dvt(const ChunkArgs& a, cudaStream_t stream) {
     using L = Layout<DVT>;
     CUtensorMap mk, mq, mg, mv;
     if (!make_map(&mk, a.k, a.B, a.T, a.H) || !make_map(&mq, a.q, a.B, a.T, a.H) ||
-        !make_map(&mg, a.log_alpha, a.B, a.T, a.H) || !make_map(&mv, a.v, a.B, a.T, a.H))
+        (a.gate == 0 && !make_map(&mg, a.log_alpha, a.B, a.T, a.H)) || !make_map(&mv, a.v, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    auto kern = kda_chunk_tc_kernel<DVT>;
+    if (a.gate != 0) mg = mk;  // no log_alpha tile is loaded; any valid map fills the parameter
+    auto kern = kda_chunk_tc_kernel<DVT, ERASE, GATE>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     unsigned* status = static_cast<unsigned*>(a.workspace);
@@ -1031,7 +1092,8 @@ cudaError_t launch_dvt(const ChunkArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     const unsigned grid = (unsigned)(a.B * a.H * (kD / DVT));
     kern<<<grid, kThreads, L::SMEM_BYTES, stream>>>(mk, mq, mg, mv, (const __nv_bfloat16*)a.beta, a.S0,
-                                                    (__nv_bfloat16*)a.o, a.ST, a.T, a.H, status);
+                                                    (__nv_bfloat16*)a.o, a.ST, a.T, a.H, status,
+                                                    GATE == 1 ? (const __nv_bfloat16*)a.log_alpha : nullptr);
     return cudaGetLastError();
 }
 
@@ -1052,8 +1114,22 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t stream) {
     }
     // One CTA per (batch, head) when there are enough heads to fill the
     // GPU; otherwise split the value channels in two.
-    if ((long)a.B * a.H >= 96) return launch_dvt<128>(a, stream);
-    return launch_dvt<64>(a, stream);
+    const bool wide = (long)a.B * a.H >= 96;
+    auto pick = [&](auto erase_c, auto gate_c) -> cudaError_t {
+        constexpr int E = decltype(erase_c)::value, G = decltype(gate_c)::value;
+        return wide ? launch_dvt<128, E, G>(a, stream) : launch_dvt<64, E, G>(a, stream);
+    };
+    using I0 = std::integral_constant<int, 0>;
+    using I1 = std::integral_constant<int, 1>;
+    using I2 = std::integral_constant<int, 2>;
+    if (a.erase) {
+        if (a.gate == 0) return pick(I1{}, I0{});
+        if (a.gate == 1) return pick(I1{}, I1{});
+        return pick(I1{}, I2{});
+    }
+    if (a.gate == 0) return pick(I0{}, I0{});
+    if (a.gate == 1) return pick(I0{}, I1{});
+    return pick(I0{}, I2{});
 }
 
 }  // namespace kda
@@ -1116,6 +1192,8 @@ extern "C" kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, cons
     kda::ChunkArgs a;
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
+    a.erase = 1;  // KDA: erase with a per-channel gate
+    a.gate = KDA_GATE_CHANNEL;
     if (!kda::chunk_tc_supported(a)) return KDA_ERR_UNSUPPORTED;
     if ((long long)B * T * H > 0) {
         const void* req[] = {q, k, v, log_alpha, beta, o};

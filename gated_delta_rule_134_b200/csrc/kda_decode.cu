@@ -5,6 +5,8 @@
 // the context length. Per (sequence, head), with S in R^{dk x dv}:
 //     S' = Diag(alpha) S,   delta = beta (v - S'^T k),
 //     S_out = S' + k delta^T,   o = S_out^T q = S'^T q + delta (k . q).
+// Variants (variant table of section 3.4): log_alpha per key channel, one per
+// head, or none; without the erase term delta = beta v.
 // The state is read once and written once: each CTA owns a 32-column slice of
 // one head's state, keeps it in registers between the two reductions
 // (S'^T k and S'^T q) and the rank-one update, and streams it with 16-byte
@@ -22,7 +24,7 @@ template <typename T, int DK>
 __global__ void __launch_bounds__(kDecodeThreads)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const T* __restrict__ log_alpha, const T* __restrict__ beta, const float* S_in,
-                   float* S_out, T* __restrict__ o, int dv) {
+                   float* S_out, T* __restrict__ o, int dv, int erase, int gate) {
     constexpr int RG = kDecodeThreads / 8;  // 16 row groups
     constexpr int ROWS = DK / RG;           // rows per thread
     const int nslices = dv / kDecodeCols;
@@ -43,7 +45,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     for (int i = t; i < DK; i += kDecodeThreads) {
         sk[i] = to_f32(k[head * DK + i]);
         sq[i] = to_f32(q[head * DK + i]);
-        sa[i] = expf(to_f32(log_alpha[head * DK + i]));
+        sa[i] = gate == 0 ? expf(to_f32(log_alpha[head * DK + i])) : (gate == 1 ? expf(to_f32(log_alpha[head])) : 1.f);
     }
     __syncthreads();
     if (warp == 0) {
@@ -87,10 +89,11 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     const float b = to_f32(beta[head]);
     const T* vh = v + head * dv + col0 + c4 * 4;
     float4 d;
-    d.x = b * (to_f32(vh[0]) - u.x);
-    d.y = b * (to_f32(vh[1]) - u.y);
-    d.z = b * (to_f32(vh[2]) - u.z);
-    d.w = b * (to_f32(vh[3]) - u.w);
+    const float er = erase ? 1.f : 0.f;  // no erase: delta = beta v
+    d.x = b * (to_f32(vh[0]) - er * u.x);
+    d.y = b * (to_f32(vh[1]) - er * u.y);
+    d.z = b * (to_f32(vh[2]) - er * u.z);
+    d.w = b * (to_f32(vh[3]) - er * u.w);
 
     float* Sout = S_out + head * DK * dv + col0 + c4 * 4;
 #pragma unroll
@@ -113,23 +116,24 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 
 template <typename T, int DK>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* la, const void* beta,
-                                   const float* S_in, float* S_out, void* o, int N, int H, int dv,
-                                   cudaStream_t stream) {
+                                   const float* S_in, float* S_out, void* o, int N, int H, int dv, int erase,
+                                   int gate, cudaStream_t stream) {
     const long blocks = (long)N * H * (dv / kDecodeCols);
     decode_step_kernel<T, DK><<<(unsigned)blocks, kDecodeThreads, 0, stream>>>(
-        (const T*)q, (const T*)k, (const T*)v, (const T*)la, (const T*)beta, S_in, S_out, (T*)o, dv);
+        (const T*)q, (const T*)k, (const T*)v, (const T*)la, (const T*)beta, S_in, S_out, (T*)o, dv, erase, gate);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* la, const void* beta,
                           const float* S_in, float* S_out, void* o, int N, int H, int dk, int dv, int bf16,
-                          cudaStream_t stream) {
+                          int erase, int gate, cudaStream_t stream) {
     if (bf16) {
-        if (dk == 64) return launch_decode_t<__nv_bfloat16, 64>(q, k, v, la, beta, S_in, S_out, o, N, H, dv, stream);
-        return launch_decode_t<__nv_bfloat16, 128>(q, k, v, la, beta, S_in, S_out, o, N, H, dv, stream);
+        if (dk == 64)
+            return launch_decode_t<__nv_bfloat16, 64>(q, k, v, la, beta, S_in, S_out, o, N, H, dv, erase, gate, stream);
+        return launch_decode_t<__nv_bfloat16, 128>(q, k, v, la, beta, S_in, S_out, o, N, H, dv, erase, gate, stream);
     }
-    if (dk == 64) return launch_decode_t<float, 64>(q, k, v, la, beta, S_in, S_out, o, N, H, dv, stream);
-    return launch_decode_t<float, 128>(q, k, v, la, beta, S_in, S_out, o, N, H, dv, stream);
+    if (dk == 64) return launch_decode_t<float, 64>(q, k, v, la, beta, S_in, S_out, o, N, H, dv, erase, gate, stream);
+    return launch_decode_t<float, 128>(q, k, v, la, beta, S_in, S_out, o, N, H, dv, erase, gate, stream);
 }
 
 }  // namespace kda

@@ -13,13 +13,15 @@ struct ChunkArgs {
     float* ST;
     int B, T, H, dk, dv, chunk;
     int bf16;
+    int erase;  // 1: delta-rule family (I - beta k k^T), 0: additive write beta k v^T
+    int gate;   // 0: log_alpha per key channel [.., dk]; 1: one per token and head [B, T, H]; 2: none
     void* workspace;
     size_t workspace_bytes;
 };
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* la, const void* beta,
                           const float* S_in, float* S_out, void* o, int N, int H, int dk, int dv, int bf16,
-                          cudaStream_t stream);
+                          int erase, int gate, cudaStream_t stream);
 
 cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t stream);
 

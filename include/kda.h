@@ -53,6 +53,21 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
  * kernel otherwise. */
 typedef enum { KDA_ALGO_AUTO = 0, KDA_ALGO_SIMT = 1, KDA_ALGO_TC = 2 } kda_algo_t;
 
+/* The variant table of "Decoding Hybrid Attention Architectures" (section
+ * 3.4, with sections 3.1-3.3 and the per-dimension gated linear attention it
+ * names) as two switches of the same kernels:
+ *   erase = 1: S_t = (I - beta_t k_t k_t^T) Diag(a_t) S_{t-1} + beta_t k_t v_t^T
+ *   erase = 0: S_t =                        Diag(a_t) S_{t-1} + beta_t k_t v_t^T
+ *   gate: how a_t = exp(log_alpha) is given (below).
+ * (erase, gate) = (1, CHANNEL) is KDA, (1, SCALAR) the scalar gated delta
+ * rule, (1, NONE) the delta rule, (0, CHANNEL) per-dimension gated linear
+ * attention, (0, NONE) with beta = 1 plain linear attention. */
+typedef enum {
+    KDA_GATE_CHANNEL = 0, /* log_alpha [B, T, H, dk]: one decay per key channel      */
+    KDA_GATE_SCALAR = 1,  /* log_alpha [B, T, H]: one decay per token and head        */
+    KDA_GATE_NONE = 2     /* no decay (a_t = 1); log_alpha is not read and may be NULL */
+} kda_gate_t;
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *kda_status_string(kda_status_t status);
 
@@ -102,6 +117,15 @@ kda_status_t kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const
                               int dk, int dv, int chunk, kda_dtype_t dtype, void *workspace,
                               size_t workspace_bytes, kda_algo_t algo, void *stream);
 
+/* kda_chunk_fwd_ex for any variant of the table above. With gate
+ * KDA_GATE_SCALAR, log_alpha is [B, T, H]; with KDA_GATE_NONE it may be NULL.
+ * erase must be 0 or 1 (else KDA_ERR_INVALID_ARG). Every algorithm supports
+ * every variant; the workspace size does not depend on the variant. */
+kda_status_t kda_chunk_fwd_v(const void *q, const void *k, const void *v, const void *log_alpha,
+                             const void *beta, const float *S0, void *o, float *S_T, int B, int T, int H,
+                             int dk, int dv, int chunk, kda_dtype_t dtype, int erase, kda_gate_t gate,
+                             void *workspace, size_t workspace_bytes, kda_algo_t algo, void *stream);
+
 /*
  * Device-side status left in `workspace` by the last kda_chunk_fwd_ex that
  * used it: synchronises `stream`, then returns KDA_OK, or KDA_ERR_TIMEOUT if
@@ -126,6 +150,14 @@ kda_status_t kda_workspace_status(const void *workspace, size_t workspace_bytes,
 kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const void *log_alpha,
                              const void *beta, const float *S_in, float *S_out, void *o, int N, int H,
                              int dk, int dv, kda_dtype_t dtype, void *stream);
+
+/* kda_decode_step for any variant: erase 0/1; log_alpha [N, H, dk]
+ * (KDA_GATE_CHANNEL), [N, H] (KDA_GATE_SCALAR) or NULL (KDA_GATE_NONE). Per
+ * head: S' = Diag(a) S; delta = beta (v - S'^T k) (erase = 1) or beta v
+ * (erase = 0); S_out = S' + k delta^T; o = S_out^T q. */
+kda_status_t kda_decode_step_v(const void *q, const void *k, const void *v, const void *log_alpha,
+                               const void *beta, const float *S_in, float *S_out, void *o, int N, int H,
+                               int dk, int dv, kda_dtype_t dtype, int erase, kda_gate_t gate, void *stream);
 
 /*
  * Allocation-free prefill (no counterpart in the paper; an addition of this

@@ -133,3 +133,41 @@ def test_binding_has_no_cpu_fallback():
         kda.chunk_fwd(x, x, v, x, b)
     with pytest.raises(ValueError, match="CUDA tensor"):
         kda.decode_step(x[:, 0], x[:, 0], v[:, 0], x[:, 0], b[:, 0], torch.zeros(1, 1, 64, 64))
+
+
+# ---------------------------------------------------------------- variant switches
+
+
+def _chunk_v(lib, ptrs, erase=1, gate=0, B=1, T=4, H=1, dk=64, dv=64, chunk=64, dtype=1, algo=0):
+    q, k, v, la, beta, S0, o, ST = ptrs
+    return lib.kda_chunk_fwd_v(q, k, v, la, beta, S0, o, ST, B, T, H, dk, dv, chunk, dtype, erase, gate, None, 0,
+                               algo, None)
+
+
+@pytest.mark.parametrize("erase,gate", [(2, 0), (-1, 0), (1, 3), (0, -1)])
+def test_variant_rejects_bad_switches(erase, gate):
+    assert _chunk_v(kda.load(), GOOD, erase=erase, gate=gate) == 1
+
+
+def test_variant_gate_needs_log_alpha():
+    lib = kda.load()
+    ptrs = list(GOOD)
+    ptrs[3] = None
+    for gate in (0, 1):
+        assert _chunk_v(lib, ptrs, gate=gate) == 1
+
+
+def test_variant_gate_none_accepts_null_log_alpha():
+    # passes pointer validation and stops at the next check (tensor-core
+    # algorithm with f32 inputs is unsupported), so nothing is launched
+    lib = kda.load()
+    ptrs = list(GOOD)
+    ptrs[3] = None
+    assert _chunk_v(lib, ptrs, gate=2, dtype=0, algo=2) == 2
+
+
+@pytest.mark.parametrize("erase,gate", [(2, 0), (1, 5)])
+def test_decode_variant_rejects_bad_switches(erase, gate):
+    lib = kda.load()
+    p = [ctypes.c_void_p(0x1000 * (i + 1)) for i in range(8)]
+    assert lib.kda_decode_step_v(*p, 2, 1, 64, 64, 1, erase, gate, None) == 1

@@ -249,3 +249,75 @@ def test_decode_full_1000_steps_sampled_heads(cuda_lib):
     torch.cuda.synchronize()
     assert worst <= TOL["bf16"]
     assert rel_err(S[nn.cuda(), hh.cuda()].cpu().numpy()[:, None], S_ref) <= TOL["bf16"]
+
+
+# ---------------------------------------------------------------- variants (erase / gate switches)
+
+VARIANTS = [(True, "scalar"), (True, "none"), (False, "channel"), (False, "scalar"), (False, "none")]
+
+
+def _variant_inputs(cfg, gate):
+    x = I.prefill_inputs(cfg)
+    la = x["log_alpha"]
+    x["log_alpha"] = {"channel": la, "scalar": la[..., 0].contiguous(), "none": None}[gate]
+    return x
+
+
+def check_variant(kda, cfg, algo, erase, gate):
+    x = _variant_inputs(cfg, gate)
+    xd = to_dev(x)
+    o, ST = kda.chunk_fwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["S0"], chunk=cfg.C, algo=algo,
+                          erase=erase, gate=gate)
+    torch.cuda.synchronize()
+    ref_o, ref_S = oracle.recurrent(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], erase=erase,
+                                    gate=gate)
+    eo, es = rel_err(o.float().cpu().numpy(), ref_o), rel_err(ST.cpu().numpy(), ref_S)
+    print(f"PARITY variant erase={int(erase)} gate={gate} {cfg.name} algo={algo} o={eo:.3e} S_T={es:.3e} "
+          f"bar={TOL[cfg.dtype]:.0e}")
+    assert np.isfinite(o.float().cpu().numpy()).all() and np.isfinite(ST.cpu().numpy()).all()
+    assert eo <= TOL[cfg.dtype] and es <= TOL[cfg.dtype], (cfg.name, algo, erase, gate, eo, es)
+
+
+@pytest.mark.parametrize("erase,gate", VARIANTS)
+@pytest.mark.parametrize("algo", ["simt", "tc"])
+@pytest.mark.parametrize("la", [(0.01, 1.0), (0.001, 0.1)])
+def test_prefill_variants_bf16(cuda_lib, algo, erase, gate, la):
+    check_variant(cuda_lib, small_cfg("bf16", 128, 64, 200, la=la, s0=0.3, seed=31), algo, erase, gate)
+
+
+@pytest.mark.parametrize("erase,gate", VARIANTS)
+def test_prefill_variants_f32(cuda_lib, erase, gate):
+    check_variant(cuda_lib, small_cfg("f32", 64, 32, 97, s0=0.3, seed=32), "simt", erase, gate)
+
+
+@pytest.mark.parametrize("erase,gate", [(True, "scalar"), (False, "channel")])
+def test_prefill_variants_tc_extreme_decay(cuda_lib, erase, gate):
+    # decays up to e^-6 per token: the guard sends chunks down the exact path
+    check_variant(cuda_lib, small_cfg("bf16", 128, 64, 150, la=(0.5, 6.0), seed=33), "tc", erase, gate)
+
+
+@pytest.mark.parametrize("erase,gate", VARIANTS)
+def test_prefill_variants_tc_many_chunks(cuda_lib, erase, gate):
+    check_variant(cuda_lib, small_cfg("bf16", 128, 64, 1536, B=2, H=16, la=(0.001, 0.1), s0=0.1, seed=34), "tc",
+                  erase, gate)
+
+
+@pytest.mark.parametrize("erase,gate", VARIANTS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_variants_chain(cuda_lib, erase, gate, dtype):
+    cfg = I.DecodeConfig("decode_variant", 3, 5, 128, 128, 6, dtype, 0.01, 1.0, 0.2, 35)
+    S = I.decode_state(cfg)
+    Sd = S.cuda()
+    S_ref = S.double().numpy()
+    for step in range(cfg.steps):
+        x = I.decode_step_inputs(cfg, step)
+        la = x["log_alpha"]
+        x["log_alpha"] = {"channel": la, "scalar": la[..., 0].contiguous(), "none": None}[gate]
+        xd = to_dev(x)
+        o, Sd = cuda_lib.decode_step(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], Sd, erase=erase,
+                                     gate=gate)
+        ref_o, S_ref = oracle.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S_ref, erase=erase,
+                                          gate=gate)
+        torch.cuda.synchronize()
+        assert rel_err(o.float().cpu().numpy(), ref_o) <= TOL[dtype]
+    assert rel_err(Sd.cpu().numpy(), S_ref) <= TOL[dtype]
