@@ -150,3 +150,28 @@ def decode_step(q, k, v, log_alpha, beta, S, nthreads: int = 0, erase: bool = Tr
     if rc:
         raise ValueError("kda_oracle_decode_step_v: bad sizes or switches")
     return o, Sn
+
+
+def recurrent_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, erase: bool = True, gate="channel"):
+    """Packed variable-length sequences: q,k [total_T,H,dk], v [total_T,H,dv],
+    beta [total_T,H], log_alpha [total_T,H,dk] / [total_T,H] / None, cu_seqlens
+    [N+1] offsets, S0 [N,H,dk,dv] or None. Each sequence is its own recurrence
+    (the definition of packing); returns (o [total_T,H,dv], S_T [N,H,dk,dv])."""
+    q, k, v, la, beta, S0 = map(_f64, (q, k, v, log_alpha, beta, S0))
+    cu = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    N = len(cu) - 1
+    H, dk = q.shape[1], q.shape[2]
+    dv = v.shape[-1]
+    o = np.zeros((q.shape[0], H, dv))
+    ST = np.zeros((N, H, dk, dv))
+    for n in range(N):
+        a, b = cu[n], cu[n + 1]
+        s0 = None if S0 is None else S0[n:n + 1]
+        if b == a:
+            ST[n] = 0.0 if S0 is None else S0[n]
+            continue
+        sl = (lambda x: None if x is None else x[None, a:b])
+        on, sn = recurrent(sl(q), sl(k), sl(v), sl(la), sl(beta), s0, erase=erase, gate=gate)
+        o[a:b] = on[0]
+        ST[n] = sn[0]
+    return o, ST

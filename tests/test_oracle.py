@@ -197,3 +197,22 @@ def test_variant_bad_switches():
         oracle.recurrent(q, k, v, None, beta, S0, gate="channel")  # a gate needs log_alpha
     with pytest.raises(ValueError):
         oracle.chunkwise(q, k, v, la, beta, S0, C=4, gate=3)
+
+
+def test_varlen_equal_lengths_equals_dense_batch():
+    """Packing B equal-length sequences back to back is the dense [B, T] batch."""
+    q, k, v, la, beta, S0 = pins.random_inputs(500, T=21, dk=6, dv=5, B_=3, H_=2)
+    o_d, s_d = oracle.recurrent(q, k, v, la, beta, S0)
+    pack = lambda x: x.reshape((-1,) + x.shape[2:])
+    o_v, s_v = oracle.recurrent_varlen(pack(q), pack(k), pack(v), pack(la), pack(beta), [0, 21, 42, 63], S0)
+    assert np.abs(o_v - pack(o_d)).max() < 1e-12 and np.abs(s_v - s_d).max() < 1e-12
+
+
+def test_varlen_empty_sequence_keeps_state():
+    q, k, v, la, beta, S0 = pins.random_inputs(501, T=10, dk=4, dv=4, B_=2, H_=1)
+    pack = lambda x: x.reshape((-1,) + x.shape[2:])
+    o_v, s_v = oracle.recurrent_varlen(pack(q), pack(k), pack(v), pack(la), pack(beta), [0, 0, 20], S0)
+    assert np.array_equal(s_v[0], S0[0])
+    o_1, s_1 = oracle.recurrent(q.reshape(1, 20, 1, 4), k.reshape(1, 20, 1, 4), v.reshape(1, 20, 1, 4),
+                                la.reshape(1, 20, 1, 4), beta.reshape(1, 20, 1), S0[1:2])
+    assert np.abs(s_v[1] - s_1[0]).max() < 1e-12
