@@ -10,7 +10,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["load", "chunk_fwd", "chunk_fwd_noalloc", "decode_step", "workspace_size", "workspace_status", "KDAError",
+__all__ = ["load", "chunk_fwd", "chunk_fwd_varlen", "chunk_fwd_noalloc", "decode_step", "workspace_size", "workspace_status", "KDAError",
            "library_path", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +70,8 @@ def load(build_if_stale: bool = True):
     lib.kda_chunk_fwd_v.restype = I
     lib.kda_decode_step_v.argtypes = [P] * 8 + [I] * 7 + [P]
     lib.kda_decode_step_v.restype = I
+    lib.kda_chunk_fwd_varlen.argtypes = [P] * 9 + [I] * 9 + [P, Z, I, P]
+    lib.kda_chunk_fwd_varlen.restype = I
     _lib = lib
     return lib
 
@@ -157,6 +159,49 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, chunk: int = 64, algo: str =
                                _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPE[dts], int(bool(erase)), GATES[gate],
                                _ptr(workspace), ws_len, _ALGO[algo], _stream(stream))
     _check("kda_chunk_fwd_v", code)
+    return o, S_T
+
+
+def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, chunk: int = 64, algo: str = "auto",
+                     output_final_state: bool = True, o=None, S_T=None, workspace=None, stream=None,
+                     erase: bool = True, gate: str = "channel"):
+    """kda_chunk_fwd_varlen: N packed sequences. q, k [total_T,H,dk]; v
+    [total_T,H,dv]; beta [total_T,H]; log_alpha [total_T,H,dk] / [total_T,H] /
+    None by gate; cu_seqlens int32 CUDA tensor [N+1]; S0 [N,H,dk,dv] float32
+    or None. Returns (o [total_T,H,dv], S_T [N,H,dk,dv] or None)."""
+    import torch
+    lib = load()
+    TT, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    dt, dev = q.dtype, q.device
+    _need(q, "q", (TT, H, dk), dt, dev)
+    _need(k, "k", (TT, H, dk), dt, dev)
+    gshape = _gate_shape(gate, (TT, H), dk)
+    if gshape is not None:
+        _need(log_alpha, "log_alpha", gshape, dt, dev)
+    _need(v, "v", (TT, H, dv), dt, dev)
+    _need(beta, "beta", (TT, H), dt, dev)
+    _need(cu_seqlens, "cu_seqlens", (N + 1,), torch.int32, dev)
+    if S0 is not None:
+        _need(S0, "S0", (N, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(TT, H, dv, dtype=dt, device=dev)
+    _need(o, "o", (TT, H, dv), dt, dev)
+    if output_final_state and S_T is None:
+        S_T = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", (N, H, dk, dv), torch.float32, dev)
+    dts = _dtype_of(q)
+    ws_bytes = workspace_size(N, TT, H, dk, dv, chunk, dts, algo)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    la = log_alpha if gshape is not None else None
+    code = lib.kda_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T),
+                                    _ptr(cu_seqlens), N, TT, H, dk, dv, chunk, _DTYPE[dts], int(bool(erase)),
+                                    GATES[gate], _ptr(workspace), ws_len, _ALGO[algo], _stream(stream))
+    _check("kda_chunk_fwd_varlen", code)
     return o, S_T
 
 

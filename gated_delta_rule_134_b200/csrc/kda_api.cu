@@ -11,6 +11,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool head_dims_ok(int dk, int dv) { return dk == dv && (dk == 64 || dk == 128); }
 
+kda_status_t run_chunk(const kda::ChunkArgs& a, kda_dtype_t dtype, kda_algo_t algo, void* stream);
+
 kda_status_t check_chunk_args(const kda::ChunkArgs& a, kda_dtype_t dtype) {
     if (a.B < 0 || a.T < 0 || a.H < 0) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
@@ -51,6 +53,7 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chu
                                     kda_algo_t algo) {
     kda::ChunkArgs a{};
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
+    a.erase = 1; a.gate = KDA_GATE_CHANNEL; a.cu_seqlens = nullptr;
     if (B < 0 || T < 0 || H < 0 || !head_dims_ok(dk, dv)) return 0;
     const bool tc = (algo == KDA_ALGO_TC) || (algo == KDA_ALGO_AUTO && kda::chunk_tc_supported(a));
     return tc ? kda::chunk_tc_workspace_bytes(B, T, H, dk, dv) : 0;
@@ -64,7 +67,36 @@ kda_status_t kda_chunk_fwd_v(const void* q, const void* k, const void* v, const 
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
     a.erase = erase; a.gate = (int)gate;
+    a.cu_seqlens = nullptr;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+    return run_chunk(a, dtype, algo, stream);
+}
+
+kda_status_t kda_chunk_fwd_varlen(const void* q, const void* k, const void* v, const void* log_alpha,
+                                  const void* beta, const float* S0, void* o, float* S_T, const int* cu_seqlens,
+                                  int N, int total_T, int H, int dk, int dv, int chunk, kda_dtype_t dtype, int erase,
+                                  kda_gate_t gate, void* workspace, size_t workspace_bytes, kda_algo_t algo,
+                                  void* stream) {
+    if (N < 0 || total_T < 0) return KDA_ERR_INVALID_ARG;
+    if (N > 0 && (cu_seqlens == nullptr || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0))
+        return KDA_ERR_INVALID_ARG;
+    kda::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
+    a.B = N; a.T = total_T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
+    a.erase = erase; a.gate = (int)gate;
+    a.cu_seqlens = cu_seqlens;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+    return run_chunk(a, dtype, algo, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+kda_status_t run_chunk(const kda::ChunkArgs& a, kda_dtype_t dtype, kda_algo_t algo, void* stream) {
+    const int B = a.B, T = a.T, H = a.H, dk = a.dk, dv = a.dv;
+    void* workspace = a.workspace;
+    const size_t workspace_bytes = a.workspace_bytes;
     kda_status_t st = check_chunk_args(a, dtype);
     if (st != KDA_OK) return st;
     if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TC) return KDA_ERR_INVALID_ARG;
@@ -81,6 +113,10 @@ kda_status_t kda_chunk_fwd_v(const void* q, const void* k, const void* v, const 
     const cudaError_t err = tc ? kda::launch_chunk_tc(a, s) : kda::launch_chunk_simt(a, s);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
+
+}  // namespace
+
+extern "C" {
 
 kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                               const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,

@@ -38,7 +38,8 @@ template <typename T, int DK, int C>
 __global__ void __launch_bounds__(kSimtThreads)
 chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const T* __restrict__ log_alpha, const T* __restrict__ beta, const float* S0,
-                  T* __restrict__ o, float* ST, int Tlen, int H, int dv, int erase, int gate) {
+                  T* __restrict__ o, float* ST, int Tlen, int H, int dv, int erase, int gate,
+                  const int* __restrict__ cu_seqlens) {
     constexpr int NT = kSimtThreads, DVT = kSimtDVT;
     extern __shared__ float smem[];
     float* sQ = smem;             // q, then q e^G
@@ -57,22 +58,34 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int j0 = blockIdx.y * DVT;
     const int tid = threadIdx.x;
+    // this sequence's tokens: [tok0, tok0 + len) of the token-major layout
+    // (dense: sequence b of a [B, T] batch; packed: offsets clamped into [0, T])
+    size_t tok0;
+    int len_seq;
+    if (cu_seqlens) {
+        const int s0 = min(max(cu_seqlens[b], 0), Tlen), s1 = min(max(cu_seqlens[b + 1], s0), Tlen);
+        tok0 = (size_t)s0;
+        len_seq = s1 - s0;
+    } else {
+        tok0 = (size_t)b * Tlen;
+        len_seq = Tlen;
+    }
 
     for (int e = tid; e < DK * DVT; e += NT) {
         const int c = e / DVT, j = e % DVT;
         sS[e] = S0 ? S0[((size_t)bh * DK + c) * dv + j0 + j] : 0.f;
     }
 
-    const int NC = (Tlen + C - 1) / C;
+    const int NC = (len_seq + C - 1) / C;
     for (int n = 0; n < NC; ++n) {
         const int t0 = n * C;
-        const int len = min(C, Tlen - t0);
+        const int len = min(C, len_seq - t0);
         __syncthreads();
         for (int e = tid; e < C * DK; e += NT) {
             const int r = e / DK, c = e % DK;
             float qv = 0.f, kv = 0.f, lv = 0.f;
             if (r < len) {
-                const size_t tok = ((size_t)b * Tlen + t0 + r) * H + h;
+                const size_t tok = (tok0 + t0 + r) * H + h;
                 const size_t off = tok * DK + c;
                 qv = to_f32(q[off]);
                 kv = to_f32(k[off]);
@@ -84,9 +97,9 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         }
         for (int e = tid; e < C * DVT; e += NT) {
             const int r = e / DVT, j = e % DVT;
-            sV[e] = r < len ? to_f32(v[(((size_t)b * Tlen + t0 + r) * H + h) * dv + j0 + j]) : 0.f;
+            sV[e] = r < len ? to_f32(v[((tok0 + t0 + r) * H + h) * dv + j0 + j]) : 0.f;
         }
-        for (int r = tid; r < C; r += NT) sB[r] = r < len ? to_f32(beta[((size_t)b * Tlen + t0 + r) * H + h]) : 0.f;
+        for (int r = tid; r < C; r += NT) sB[r] = r < len ? to_f32(beta[(tok0 + t0 + r) * H + h]) : 0.f;
         __syncthreads();
 
         // G: inclusive prefix sum over the chunk's tokens, per key channel.
@@ -177,7 +190,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             float acc = 0.f;
             for (int c = 0; c < DK; ++c) acc = fmaf(sQ[r * DK + c], sS[c * DVT + j], acc);
             for (int s = 0; s <= r; ++s) acc = fmaf(sP[r * C + s], sD[s * DVT + j], acc);
-            if (r < len) o[(((size_t)b * Tlen + t0 + r) * H + h) * dv + j0 + j] = from_f32<T>(acc);
+            if (r < len) o[((tok0 + t0 + r) * H + h) * dv + j0 + j] = from_f32<T>(acc);
         }
         __syncthreads();
 
@@ -207,7 +220,7 @@ static cudaError_t launch_simt_t(const ChunkArgs& a, cudaStream_t stream) {
     dim3 grid((unsigned)(a.B * a.H), (unsigned)(a.dv / kSimtDVT));
     kern<<<grid, kSimtThreads, smem, stream>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, (const T*)a.log_alpha,
                                                (const T*)a.beta, a.S0, (T*)a.o, a.ST, a.T, a.H, a.dv, a.erase,
-                                               a.gate);
+                                               a.gate, a.cu_seqlens);
     return cudaGetLastError();
 }
 

@@ -230,7 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
                     const __nv_bfloat16* __restrict__ beta, const float* S0, __nv_bfloat16* __restrict__ o,
-                    float* ST, int Tlen, int H, unsigned* status, const __nv_bfloat16* __restrict__ gate_tok) {
+                    float* ST, int Tlen, int H, unsigned* status, const __nv_bfloat16* __restrict__ gate_tok,
+                    const int* __restrict__ cu_seqlens) {
     constexpr int erase = ERASE, gate = GATE;
     using L = Layout<DVT>;
     extern __shared__ uint8_t smem_raw[];
@@ -244,8 +245,25 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const int nslices = kD / DVT;
     const int bh = blockIdx.x / nslices;
     const int b = bh / H, h = bh % H;
+    // This sequence's tokens: [tok0, tok0 + seq_len) of the token-major layout.
+    // Dense batch: sequence b of [B, T]; packed: offsets clamped into [0, T], and
+    // the tensor maps then describe one [1, T] sequence (tile origin tma_t0).
+    size_t tok0;
+    int seq_len, tma_t0, tma_b;
+    if (cu_seqlens) {
+        const int s0 = min(max(cu_seqlens[b], 0), Tlen), s1 = min(max(cu_seqlens[b + 1], s0), Tlen);
+        tok0 = (size_t)s0;
+        seq_len = s1 - s0;
+        tma_t0 = s0;
+        tma_b = 0;
+    } else {
+        tok0 = (size_t)b * Tlen;
+        seq_len = Tlen;
+        tma_t0 = 0;
+        tma_b = b;
+    }
     const int j0 = (blockIdx.x % nslices) * DVT;
-    const int NC = (Tlen + kC - 1) / kC;
+    const int NC = (seq_len + kC - 1) / kC;
     const int quad = warp & 3;  // tensor-memory lane quadrant this warp may access
 
     float* sBeta = reinterpret_cast<float*>(sm + L::SBETA);
@@ -340,19 +358,19 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         // inputs come from three roles in an order that varies from chunk to
         // chunk, so it polls the hand-over barriers and issues whatever is
         // ready; each kind of work goes out in chunk order.
-        if (lane == 0) {
+        if (lane == 0 && NC > 0) {
             auto issue_kq = [&](int m) {
                 const int par = m & 1;
                 uint8_t* dst = sm + L::ROWOP + par * 32768;
                 mbar_arrive_expect_tx(bars + BAR_KQ + par, 4 * 8192);
                 for (int x = 0; x < 2; ++x) {
-                    tma_load_4d(dst + x * 16384, &tm_k, bars + BAR_KQ + par, 64 * x, h, m * kC, b);
-                    tma_load_4d(dst + x * 16384 + 8192, &tm_q, bars + BAR_KQ + par, 64 * x, h, m * kC, b);
+                    tma_load_4d(dst + x * 16384, &tm_k, bars + BAR_KQ + par, 64 * x, h, tma_t0 + m * kC, tma_b);
+                    tma_load_4d(dst + x * 16384 + 8192, &tm_q, bars + BAR_KQ + par, 64 * x, h, tma_t0 + m * kC, tma_b);
                 }
                 if (m + 1 < NC) {  // the next chunk's tiles into L2: their loads wait for a free buffer
                     for (int x = 0; x < 2; ++x) {
-                        tma_prefetch_l2_4d(&tm_k, 64 * x, h, (m + 1) * kC, b);
-                        tma_prefetch_l2_4d(&tm_q, 64 * x, h, (m + 1) * kC, b);
+                        tma_prefetch_l2_4d(&tm_k, 64 * x, h, tma_t0 + (m + 1) * kC, tma_b);
+                        tma_prefetch_l2_4d(&tm_q, 64 * x, h, tma_t0 + (m + 1) * kC, tma_b);
                     }
                 }
             };
@@ -361,16 +379,17 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 uint8_t* dst = sm + L::COLOP + par * 16384;
                 mbar_arrive_expect_tx(bars + BAR_G + par, 2 * 8192);
                 for (int x = 0; x < 2; ++x)
-                    tma_load_4d(dst + x * 8192, &tm_g, bars + BAR_G + par, 64 * x, h, m * kC, b);
+                    tma_load_4d(dst + x * 8192, &tm_g, bars + BAR_G + par, 64 * x, h, tma_t0 + m * kC, tma_b);
                 if (m + 1 < NC)
-                    for (int x = 0; x < 2; ++x) tma_prefetch_l2_4d(&tm_g, 64 * x, h, (m + 1) * kC, b);
+                    for (int x = 0; x < 2; ++x) tma_prefetch_l2_4d(&tm_g, 64 * x, h, tma_t0 + (m + 1) * kC, tma_b);
             };
             auto issue_v = [&](int m) {
                 mbar_arrive_expect_tx(bars + BAR_V, (DVT / 64) * 8192);
                 for (int x = 0; x < DVT / 64; ++x)
-                    tma_load_4d(sm + L::RAWV + x * 8192, &tm_v, bars + BAR_V, j0 + 64 * x, h, m * kC, b);
+                    tma_load_4d(sm + L::RAWV + x * 8192, &tm_v, bars + BAR_V, j0 + 64 * x, h, tma_t0 + m * kC, tma_b);
                 if (m + 1 < NC)
-                    for (int x = 0; x < DVT / 64; ++x) tma_prefetch_l2_4d(&tm_v, j0 + 64 * x, h, (m + 1) * kC, b);
+                    for (int x = 0; x < DVT / 64; ++x)
+                        tma_prefetch_l2_4d(&tm_v, j0 + 64 * x, h, tma_t0 + (m + 1) * kC, tma_b);
             };
             // a per-token gate or none: no log_alpha tile and no prefix-sum MMA
             // (the prefix-sum barrier still completes, with an empty commit)
@@ -597,8 +616,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         uint32_t v[32];
                         tmem_ld32(lane_addr + L::D1_COL + 32 * gq, v);
                         tmem_ld_wait(v);
-                        if (t0 + r < Tlen) {
-                            uint4* dst = reinterpret_cast<uint4*>(o + (((size_t)b * Tlen + t0 + r) * H + h) * kD + j0 +
+                        if (t0 + r < seq_len) {
+                            uint4* dst = reinterpret_cast<uint4*>(o + ((tok0 + t0 + r) * H + h) * kD + j0 +
                                                                   32 * gq);
 #pragma unroll
                             for (int jc = 0; jc < 4; ++jc) {
@@ -620,7 +639,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
         }
         // ------------------------------------------------------------ final state S = e^{G_last - G_m} R
-        if (quad < 2) waitw(BAR_M2, (uint32_t)(NC - 1));
+        if (quad < 2 && NC > 0) waitw(BAR_M2, (uint32_t)(NC - 1));
         // one decision per warp: the tensor-memory loads below are warp-collective
         if (__shfl_sync(0xffffffffu, (ST && !*s_abort) ? 1 : 0, 0)) {
             const float ek = sEK[row];
@@ -647,7 +666,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const int cb = 2 * (quad >> 1) + hf;     // P2: 32-channel block of this thread
         auto load_beta = [&](int m) -> float {
             const int t = m * kC + tid;
-            return (tid < kC && m < NC && t < Tlen) ? __bfloat162float(beta[((size_t)b * Tlen + t) * H + h]) : 0.f;
+            return (tid < kC && m < NC && t < seq_len) ? __bfloat162float(beta[(tok0 + t) * H + h]) : 0.f;
         };
         float* sGs = reinterpret_cast<float*>(sm + L::SGS);
         auto p2 = [&](int m) -> bool {
@@ -656,9 +675,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             if (gate == 1) {  // per-token gate: prefix sums over the chunk's 64 tokens (one warp scans)
                 if (warp == 0) {
                     const int t0 = m * kC;
-                    float g0 = (t0 + lane < Tlen) ? __bfloat162float(gate_tok[((size_t)b * Tlen + t0 + lane) * H + h]) : 0.f;
-                    float g1 = (t0 + 32 + lane < Tlen) ? __bfloat162float(gate_tok[((size_t)b * Tlen + t0 + 32 + lane) * H + h])
-                                                       : 0.f;
+                    float g0 = (t0 + lane < seq_len) ? __bfloat162float(gate_tok[(tok0 + t0 + lane) * H + h]) : 0.f;
+                    float g1 = (t0 + 32 + lane < seq_len) ? __bfloat162float(gate_tok[(tok0 + t0 + 32 + lane) * H + h])
+                                                          : 0.f;
 #pragma unroll
                     for (int off = 1; off < 32; off <<= 1) {
                         const float x0 = __shfl_up_sync(0xffffffffu, g0, off), x1 = __shfl_up_sync(0xffffffffu, g1, off);
@@ -687,20 +706,28 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             // Rolled loops over groups of 8 channels keep the loop bodies
             // small: every chunk streams this code again, and what is not
             // in the instruction cache stalls the warp.
+            // Tokens of this chunk that belong to the sequence: [0, lim). Rows past
+            // it are zero (past the tensor) or the next packed sequence's.
+            const int lim = min(seq_len - m * kC, kC);
+            const bool live = tok < lim;
+            const int tm_tok = min(31, lim - 1), tl_tok = min(63, lim - 1);  // reference, last token
             {   // G_m, G_last of this thread's channels (tcgen05.ld is warp-collective:
-                // every lane loads, the lanes of tokens 31 and 63 store)
-                float* dst = (tok == 31 ? sGm : sGl) + 32 * cb;
+                // every lane loads, the lanes of the two tokens store)
 #pragma unroll 1
                 for (int u4 = 0; u4 < 4; ++u4) {
                     uint32_t g8[8];
                     load_g8(u4, g8);
-                    if (tok == 31 || tok == 63) {
-                        *reinterpret_cast<float4*>(dst + 8 * u4) =
-                            make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]), __uint_as_float(g8[2]),
-                                        __uint_as_float(g8[3]));
-                        *reinterpret_cast<float4*>(dst + 8 * u4 + 4) =
-                            make_float4(__uint_as_float(g8[4]), __uint_as_float(g8[5]), __uint_as_float(g8[6]),
-                                        __uint_as_float(g8[7]));
+                    const float4 lo = make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]), __uint_as_float(g8[2]),
+                                                  __uint_as_float(g8[3]));
+                    const float4 hi = make_float4(__uint_as_float(g8[4]), __uint_as_float(g8[5]), __uint_as_float(g8[6]),
+                                                  __uint_as_float(g8[7]));
+                    if (tok == tm_tok) {
+                        *reinterpret_cast<float4*>(sGm + 32 * cb + 8 * u4) = lo;
+                        *reinterpret_cast<float4*>(sGm + 32 * cb + 8 * u4 + 4) = hi;
+                    }
+                    if (tok == tl_tok) {
+                        *reinterpret_cast<float4*>(sGl + 32 * cb + 8 * u4) = lo;
+                        *reinterpret_cast<float4*>(sGl + 32 * cb + 8 * u4 + 4) = hi;
                     }
                     __syncwarp();
                 }
@@ -716,7 +743,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 const float gm8[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    bad |= !(fabsf(__uint_as_float(g8[e]) - gm8[e]) <= kGuard) || !(gm8[e] >= -kGuard);
+                    bad |= live && (!(fabsf(__uint_as_float(g8[e]) - gm8[e]) <= kGuard) || !(gm8[e] >= -kGuard));
             }
             const bool exact = nb_or(NB_OR, kPrep, bad);
             if (tid < kD) {
@@ -763,7 +790,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         while (r * (r + 1) / 2 > p) --r;
                         const int s = p - r * (r + 1) / 2;
                         float a = 0.f, pp = 0.f;
-                        for (int i2 = 0; i2 < kD; ++i2) {
+                        // rows past the sequence stay 0 (their gates may be another
+                        // sequence's and overflow the exponential)
+                        for (int i2 = 0; i2 < (r < lim ? kD : 0); ++i2) {
                             const int cc = (i2 + p) & (kD - 1);
                             const float ks = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(s, cc))) *
                                              __expf(sG[r * 128 + cc] - sG[s * 128 + cc]);
@@ -772,7 +801,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                                       ks, pp);
                         }
                         const int tr = m * kC + r;  // beta of chunk m (the scratch holds the previous chunk's)
-                        const float br = tr < Tlen ? __bfloat162float(beta[((size_t)b * Tlen + tr) * H + h]) : 0.f;
+                        const float br = tr < seq_len ? __bfloat162float(beta[(tok0 + tr) * H + h]) : 0.f;
                         av[i] = (s < r && erase) ? br * a : 0.f;  // no erase: A = 0
                         pv[i] = pp;
                     }
@@ -809,7 +838,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 const float4 ra = *reinterpret_cast<const float4*>((exact ? sGl : sGm) + c0);
                 const float4 rb = *reinterpret_cast<const float4*>((exact ? sGl : sGm) + c0 + 4);
                 const float ref8[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-                const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w}, qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                const uint32_t km = live ? 0xFFFFFFFFu : 0u;  // rows past the sequence: k = q = 0
+                const uint32_t kw[4] = {kv.x & km, kv.y & km, kv.z & km, kv.w & km};
+                const uint32_t qw[4] = {qv.x & km, qv.y & km, qv.z & km, qv.w & km};
                 uint32_t ke[4], qe[4], kf[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -826,6 +857,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         f0 = __expf(ref8[2 * u] - g0);
                         f1 = __expf(ref8[2 * u + 1] - g1);
                     }
+                    if (!live) e0 = e1 = f0 = f1 = 0.f;  // finite zeros, whatever the gate of a foreign row
                     // packed bf16 products: the factor pairs are rounded to bf16
                     // first, the products once more (both well inside the bf16
                     // rounding of the MMA operands)
@@ -995,11 +1027,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
             __syncwarp();
         };
-        waitw(BAR_CS, 0u);
-        waitw(BAR_KQ, 0u);
-        nb_sync(NB_PREP, kPrep);
-        bool exact_cur = p2(0);
-        p2_signal(0, exact_cur);
+        bool exact_cur = false;
+        if (NC > 0) {  // (an empty packed sequence has no chunk: its state passes through)
+            waitw(BAR_CS, 0u);
+            waitw(BAR_KQ, 0u);
+            nb_sync(NB_PREP, kPrep);
+            exact_cur = p2(0);
+            p2_signal(0, exact_cur);
+        }
         float beta_next = load_beta(0);
         for (int m = 0; m < NC; ++m) {
             const int par = m & 1;
@@ -1080,8 +1115,9 @@ template <int DVT, int ERASE, int GATE>
 cudaError_t launch_dvt(const ChunkArgs& a, cudaStream_t stream) {
     using L = Layout<DVT>;
     CUtensorMap mk, mq, mg, mv;
-    if (!make_map(&mk, a.k, a.B, a.T, a.H) || !make_map(&mq, a.q, a.B, a.T, a.H) ||
-        (a.gate == 0 && !make_map(&mg, a.log_alpha, a.B, a.T, a.H)) || !make_map(&mv, a.v, a.B, a.T, a.H))
+    const int mb = a.cu_seqlens ? 1 : a.B;  // packed sequences: one [1, T] token range
+    if (!make_map(&mk, a.k, mb, a.T, a.H) || !make_map(&mq, a.q, mb, a.T, a.H) ||
+        (a.gate == 0 && !make_map(&mg, a.log_alpha, mb, a.T, a.H)) || !make_map(&mv, a.v, mb, a.T, a.H))
         return cudaErrorInvalidValue;
     if (a.gate != 0) mg = mk;  // no log_alpha tile is loaded; any valid map fills the parameter
     auto kern = kda_chunk_tc_kernel<DVT, ERASE, GATE>;
@@ -1093,7 +1129,7 @@ cudaError_t launch_dvt(const ChunkArgs& a, cudaStream_t stream) {
     const unsigned grid = (unsigned)(a.B * a.H * (kD / DVT));
     kern<<<grid, kThreads, L::SMEM_BYTES, stream>>>(mk, mq, mg, mv, (const __nv_bfloat16*)a.beta, a.S0,
                                                     (__nv_bfloat16*)a.o, a.ST, a.T, a.H, status,
-                                                    GATE == 1 ? (const __nv_bfloat16*)a.log_alpha : nullptr);
+                                                    GATE == 1 ? (const __nv_bfloat16*)a.log_alpha : nullptr, a.cu_seqlens);
     return cudaGetLastError();
 }
 
@@ -1194,6 +1230,7 @@ extern "C" kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, cons
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
     a.erase = 1;  // KDA: erase with a per-channel gate
     a.gate = KDA_GATE_CHANNEL;
+    a.cu_seqlens = nullptr;
     if (!kda::chunk_tc_supported(a)) return KDA_ERR_UNSUPPORTED;
     if ((long long)B * T * H > 0) {
         const void* req[] = {q, k, v, log_alpha, beta, o};

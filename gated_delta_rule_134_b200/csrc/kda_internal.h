@@ -15,6 +15,11 @@ struct ChunkArgs {
     int bf16;
     int erase;  // 1: delta-rule family (I - beta k k^T), 0: additive write beta k v^T
     int gate;   // 0: log_alpha per key channel [.., dk]; 1: one per token and head [B, T, H]; 2: none
+    // Packed variable-length sequences (NULL: dense [B, T, H, .] batch). When
+    // set, B is the number of sequences, T the packed token count, and
+    // sequence b owns tokens [cu_seqlens[b], cu_seqlens[b+1]) of the [1, T, H, .]
+    // tensors; kernels clamp the offsets into [0, T].
+    const int* cu_seqlens;
     void* workspace;
     size_t workspace_bytes;
 };

@@ -167,3 +167,41 @@ def decode_step_inputs(cfg: DecodeConfig, step: int) -> dict:
     beta = torch.sigmoid(torch.randn(N, H, generator=g))
     dt = cfg.torch_dtype
     return dict(q=q.to(dt), k=k.to(dt), v=v.to(dt), log_alpha=la.to(dt), beta=beta.to(dt))
+
+
+def varlen_lengths(n: int, mean: int, seed: int, zero_frac: float = 0.0) -> list:
+    """A seeded length mix for packed batches: lengths ~ U(1, 2*mean - 1),
+    with about `zero_frac` of them set to 0 (empty sequences)."""
+    g = _gen(seed, 7)
+    ls = torch.randint(1, 2 * mean, (n,), generator=g)
+    z = torch.rand(n, generator=g) < zero_frac
+    return [0 if zz else int(x) for x, zz in zip(ls.tolist(), z.tolist())]
+
+
+def varlen_inputs(cfg: PrefillConfig, lengths) -> dict:
+    """Packed inputs for sequences of the given lengths: sequence n, head h is
+    prefill_head(cfg with T = lengths[n], n, h). Shapes: q,k,log_alpha
+    [total_T,H,dk], v [total_T,H,dv], beta [total_T,H], S0 [N,H,dk,dv] fp32
+    (None when s0_std == 0), cu_seqlens int32 [N+1]."""
+    lengths = [int(x) for x in lengths]
+    N, H, dk, dv, dt = len(lengths), cfg.H, cfg.dk, cfg.dv, cfg.torch_dtype
+    cu = [0]
+    for L in lengths:
+        cu.append(cu[-1] + L)
+    TT = cu[-1]
+    q = torch.empty(TT, H, dk, dtype=dt)
+    k = torch.empty(TT, H, dk, dtype=dt)
+    la = torch.empty(TT, H, dk, dtype=dt)
+    v = torch.empty(TT, H, dv, dtype=dt)
+    beta = torch.empty(TT, H, dtype=dt)
+    S0 = torch.zeros(N, H, dk, dv)
+    for n, L in enumerate(lengths):
+        cn = cfg.replace(T=L)
+        for h in range(H):
+            x = prefill_head(cn, n, h)
+            a, b = cu[n], cu[n + 1]
+            q[a:b, h], k[a:b, h], la[a:b, h] = x["q"], x["k"], x["log_alpha"]
+            v[a:b, h], beta[a:b, h] = x["v"], x["beta"]
+            S0[n, h] = x["S0"]
+    return dict(q=q, k=k, v=v, log_alpha=la, beta=beta, S0=S0 if cfg.s0_std > 0 else None,
+                cu_seqlens=torch.tensor(cu, dtype=torch.int32))

@@ -127,6 +127,35 @@ kda_status_t kda_chunk_fwd_v(const void *q, const void *k, const void *v, const 
                              void *workspace, size_t workspace_bytes, kda_algo_t algo, void *stream);
 
 /*
+ * Packed variable-length sequences (serving: many requests of different
+ * lengths in one call; "Decoding Hybrid Attention Architectures", section 5,
+ * inference side: fixed-size state per request under high concurrency). The
+ * operation per sequence is the one of kda_chunk_fwd_v. N sequences, their
+ * tokens packed back to back:
+ *   q, k            : [total_T, H, dk]   dtype
+ *   log_alpha       : [total_T, H, dk] (KDA_GATE_CHANNEL), [total_T, H]
+ *                     (KDA_GATE_SCALAR) or NULL (KDA_GATE_NONE)
+ *   v, o            : [total_T, H, dv]   dtype
+ *   beta            : [total_T, H]       dtype
+ *   cu_seqlens      : DEVICE int32 [N + 1], cu_seqlens[0] = 0, non-decreasing,
+ *                     cu_seqlens[N] = total_T; sequence n is tokens
+ *                     [cu_seqlens[n], cu_seqlens[n+1]). The contents are read
+ *                     on the device only: offsets outside [0, total_T] are
+ *                     clamped and a decreasing pair is an empty sequence, so a
+ *                     malformed array cannot make a kernel access memory
+ *                     outside these tensors.
+ *   S0, S_T         : [N, H, dk, dv] float (per sequence; NULL as above)
+ * Each sequence is computed exactly as kda_chunk_fwd_v would compute it
+ * alone (its own chunking from its first token; a zero-length sequence
+ * copies S0 to S_T). Workspace as for kda_chunk_fwd_v with B = N.
+ */
+kda_status_t kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const void *log_alpha,
+                                  const void *beta, const float *S0, void *o, float *S_T,
+                                  const int *cu_seqlens, int N, int total_T, int H, int dk, int dv, int chunk,
+                                  kda_dtype_t dtype, int erase, kda_gate_t gate, void *workspace,
+                                  size_t workspace_bytes, kda_algo_t algo, void *stream);
+
+/*
  * Device-side status left in `workspace` by the last kda_chunk_fwd_ex that
  * used it: synchronises `stream`, then returns KDA_OK, or KDA_ERR_TIMEOUT if
  * a bounded wait inside a kernel gave up (that kernel's outputs are then

@@ -171,3 +171,11 @@ def test_decode_variant_rejects_bad_switches(erase, gate):
     lib = kda.load()
     p = [ctypes.c_void_p(0x1000 * (i + 1)) for i in range(8)]
     assert lib.kda_decode_step_v(*p, 2, 1, 64, 64, 1, erase, gate, None) == 1
+
+
+def test_varlen_rejects_missing_or_misaligned_offsets():
+    lib = kda.load()
+    q, k, v, la, beta, S0, o, ST = GOOD
+    args = lambda cu: (q, k, v, la, beta, S0, o, ST, cu, 2, 8, 1, 64, 64, 64, 1, 1, 0, None, 0, 0, None)
+    assert lib.kda_chunk_fwd_varlen(*args(None)) == 1
+    assert lib.kda_chunk_fwd_varlen(*args(ctypes.c_void_p(0x5002))) == 1

@@ -321,3 +321,102 @@ def test_decode_variants_chain(cuda_lib, erase, gate, dtype):
         torch.cuda.synchronize()
         assert rel_err(o.float().cpu().numpy(), ref_o) <= TOL[dtype]
     assert rel_err(Sd.cpu().numpy(), S_ref) <= TOL[dtype]
+
+
+# ---------------------------------------------------------------- packed variable-length sequences
+
+
+def _gate_view(la, gate):
+    return {"channel": la, "scalar": None if la is None else la[..., 0].contiguous(), "none": None}[gate]
+
+
+def check_varlen(kda, cfg, lengths, algo, erase=True, gate="channel"):
+    x = I.varlen_inputs(cfg, lengths)
+    x["log_alpha"] = _gate_view(x["log_alpha"], gate)
+    xd = to_dev(x)
+    o, ST = kda.chunk_fwd_varlen(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["cu_seqlens"], xd["S0"],
+                                 chunk=cfg.C, algo=algo, erase=erase, gate=gate)
+    torch.cuda.synchronize()
+    ref_o, ref_S = oracle.recurrent_varlen(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["cu_seqlens"],
+                                           x["S0"], erase=erase, gate=gate)
+    got_o, got_S = o.float().cpu().numpy(), ST.cpu().numpy()
+    assert np.isfinite(got_o).all() and np.isfinite(got_S).all()
+    eo = rel_err(got_o, ref_o) if got_o.size else 0.0
+    es = rel_err(got_S, ref_S)
+    print(f"PARITY varlen {cfg.name} N={len(lengths)} total={sum(lengths)} algo={algo} erase={int(erase)} "
+          f"gate={gate} o={eo:.3e} S_T={es:.3e}")
+    assert eo <= TOL[cfg.dtype] and es <= TOL[cfg.dtype], (lengths, algo, eo, es)
+    return o, ST
+
+
+VARLEN_MIXES = [[0, 1, 63, 64, 65, 200], [300], [5, 0, 0, 129], [128, 1, 0], [0]]
+
+
+@pytest.mark.parametrize("lengths", VARLEN_MIXES)
+@pytest.mark.parametrize("algo", ["simt", "tc"])
+def test_varlen_mixes_bf16(cuda_lib, algo, lengths):
+    check_varlen(cuda_lib, small_cfg("bf16", 128, 64, 0, H=3, s0=0.3, seed=41), lengths, algo)
+
+
+@pytest.mark.parametrize("C", [16, 32, 64])
+def test_varlen_f32_simt(cuda_lib, C):
+    check_varlen(cuda_lib, small_cfg("f32", 64, C, 0, H=2, s0=0.3, seed=42), [17, 0, 33, 64, 1, 90], "simt")
+
+
+@pytest.mark.parametrize("algo", ["simt", "tc"])
+def test_varlen_many_sequences(cuda_lib, algo):
+    lengths = I.varlen_lengths(40, 150, seed=43, zero_frac=0.1)
+    check_varlen(cuda_lib, small_cfg("bf16", 128, 64, 0, H=4, s0=0.2, seed=43), lengths, algo)
+
+
+@pytest.mark.parametrize("erase,gate", VARIANTS)
+@pytest.mark.parametrize("algo", ["simt", "tc"])
+def test_varlen_variants(cuda_lib, algo, erase, gate):
+    check_varlen(cuda_lib, small_cfg("bf16", 128, 64, 0, H=2, s0=0.3, seed=44), [70, 0, 129, 3], algo, erase, gate)
+
+
+def test_varlen_tc_extreme_decay(cuda_lib):
+    # strong decay sends chunks down the exact path; tails end mid-chunk
+    check_varlen(cuda_lib, small_cfg("bf16", 128, 64, 0, H=2, la=(0.5, 6.0), seed=45), [100, 37, 64, 190], "tc")
+
+
+@pytest.mark.parametrize("algo", ["simt", "tc"])
+def test_varlen_equal_lengths_match_dense(cuda_lib, algo):
+    """Packing B equal-length sequences must give exactly the dense [B, T] result:
+    the same kernel does the same arithmetic on the same tokens."""
+    cfg = I.B2_H16_T4K if algo == "tc" else small_cfg("bf16", 128, 64, 777, B=3, H=4, s0=0.3, seed=46)
+    x = to_dev(I.prefill_inputs(cfg))
+    o_d, S_d = cuda_lib.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], chunk=64, algo=algo)
+    pack = lambda t: t.reshape((-1,) + tuple(t.shape[2:]))
+    cu = torch.arange(0, cfg.B + 1, dtype=torch.int32, device="cuda") * cfg.T
+    o_v, S_v = cuda_lib.chunk_fwd_varlen(pack(x["q"]), pack(x["k"]), pack(x["v"]), pack(x["log_alpha"]),
+                                         pack(x["beta"]), cu, x["S0"], chunk=64, algo=algo)
+    torch.cuda.synchronize()
+    assert torch.equal(pack(o_d), o_v) and torch.equal(S_d, S_v)
+
+
+def test_varlen_full_size_sampled(cuda_lib):
+    """A packed batch of 24 sequences (about 35K tokens, H32 d128, strong
+    decay) with mixed lengths; sampled (sequence, head) slices against the
+    oracle."""
+    lengths = I.varlen_lengths(24, 1365, seed=47, zero_frac=0.05)
+    cfg = I.B4_H32_T8K.replace(s0_std=0.05, seed=47)
+    x = I.varlen_inputs(cfg, lengths)
+    xd = to_dev(x)
+    o, ST = cuda_lib.chunk_fwd_varlen(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["cu_seqlens"],
+                                      xd["S0"], chunk=64, algo="auto")
+    torch.cuda.synchronize()
+    cu = x["cu_seqlens"].tolist()
+    rng = np.random.default_rng(47)
+    worst = 0.0
+    for n in rng.choice(len(lengths), 6, replace=False):
+        h = int(rng.integers(cfg.H))
+        a, b = cu[n], cu[n + 1]
+        sl = lambda t: t[a:b, h:h + 1][None]
+        s0 = None if x["S0"] is None else x["S0"][n:n + 1, h:h + 1]
+        ref_o, ref_S = oracle.recurrent(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["log_alpha"]), sl(x["beta"]), s0)
+        if b > a:
+            worst = max(worst, rel_err(o[a:b, h].float().cpu().numpy()[None, :, None], ref_o))
+        worst = max(worst, rel_err(ST[n, h].cpu().numpy()[None, None], ref_S))
+    print(f"PARITY varlen full-size sampled worst={worst:.3e}")
+    assert worst <= TOL["bf16"]
