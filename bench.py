@@ -395,6 +395,81 @@ def time_decode(args, ctx, kda, I, peaks, peak_kind):
             "clocks": clk.summary(), "inputs": "pre-generated on the device, fresh each step"}
 
 
+def _time_calls(ctx, fn, warmup, steps):
+    """Average device time (ms) of fn() over `steps` launches on ctx.stream,
+    after `warmup` untimed ones; max over ranks."""
+    torch = ctx.torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ctx.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(ctx.stream)
+    for _ in range(steps):
+        fn()
+    e1.record(ctx.stream)
+    torch.cuda.synchronize()
+    return ctx.max_over_ranks(e0.elapsed_time(e1) / steps)
+
+
+def time_widened(args, ctx, kda, I, pf, peaks):
+    """The widened rows, each on a workload of the headline's size:
+    packed variable-length sequences (about 32K tokens in 32 sequences of
+    mixed lengths, H32 d128, strong decay) and the four variants on the
+    B4 H32 T8192 inputs. Tokens/s and the HBM roofline fraction of each
+    (algorithmic bytes: q, k, v, the gate as the variant reads it, beta, o,
+    and the states)."""
+    torch = ctx.torch
+    steps = max(3, min(args.steps, 10))
+    hbm = peaks["hbm_gbs"]
+    out = {}
+    # packed sequences
+    lengths = I.varlen_lengths(32, 1024, seed=48 + ctx.rank)
+    vcfg = I.B4_H32_T8K.replace(seed=48 + ctx.rank)
+    xv = {k: (None if v is None else v.to(ctx.dev)) for k, v in I.varlen_inputs(vcfg, lengths).items()}
+    TT, N, H = sum(lengths), len(lengths), vcfg.H
+    ov = torch.empty(TT, H, vcfg.dv, dtype=torch.bfloat16, device=ctx.dev)
+    Sv = torch.empty(N, H, vcfg.dk, vcfg.dv, dtype=torch.float32, device=ctx.dev)
+    wsv = torch.empty(256, dtype=torch.uint8, device=ctx.dev)
+
+    def run_v():
+        kda.chunk_fwd_varlen(xv["q"], xv["k"], xv["v"], xv["log_alpha"], xv["beta"], xv["cu_seqlens"], xv["S0"],
+                             o=ov, S_T=Sv, workspace=wsv, stream=ctx.stream)
+    ms = _time_calls(ctx, run_v, args.warmup, steps)
+    nbytes = BYTES_PER_TOKEN_HEAD * TT * H + Sv.numel() * 4 + 4 * (N + 1)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out["varlen"] = {"workload": f"packed_n{N}_total{TT}_h32_d128_bf16_strong_decay", "lengths": "U(1, 2047)",
+                     "value": ctx.world * TT / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                                  "algorithmic_bytes_per_launch": nbytes}}
+    del xv, ov, Sv
+    # variants on the headline inputs
+    x = pf.x
+    cfg = pf.cfg
+    la_tok = x["log_alpha"][..., 0].contiguous()
+    per_gate = {"channel": 256, "scalar": 2, "none": 0}
+    variants = {"kda": (True, "channel"), "scalar_gated_delta": (True, "scalar"), "delta_rule": (True, "none"),
+                "gated_linear_attention": (False, "channel"), "linear_attention": (False, "none")}
+    res = {}
+    for name, (erase, gate) in variants.items():
+        la = {"channel": x["log_alpha"], "scalar": la_tok, "none": None}[gate]
+
+        def run_x():
+            kda.chunk_fwd(x["q"], x["k"], x["v"], la, x["beta"], x["S0"], chunk=cfg.C, algo=pf.algo, o=pf.o,
+                          S_T=pf.ST, workspace=pf.ws if pf.ws_bytes else None, stream=ctx.stream, erase=erase,
+                          gate=gate)
+        ms = _time_calls(ctx, run_x, args.warmup, steps)
+        ntok = cfg.B * cfg.T
+        nbytes = (3 * 256 + per_gate[gate] + 2 + 256) * ntok * cfg.H + pf.ST.numel() * 4
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[name] = {"erase": erase, "gate": gate, "value": ctx.world * ntok / (ms * 1e-3), "unit": "tokens/s",
+                     "ms_per_step": ms, "roofline_frac": gbs / hbm, "achieved_gbs": gbs}
+    out["variants"] = {"workload": cfg.name, "steps": steps, **res}
+    if pf.use_tc and kda.workspace_status(pf.ws, ctx.stream) != 0:
+        raise RuntimeError("device-side timeout reported by the prefill kernel")
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -406,8 +481,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-T", type=int, default=None,
                     help="shorter sequence for profiler captures (the printed line is then not a bench value)")
-    ap.add_argument("--parts", default="prefill,e2e,decode",
-                    help="comma list of prefill, e2e, decode (profiling runs select one)")
+    ap.add_argument("--parts", default="prefill,e2e,decode,widened",
+                    help="comma list of prefill, e2e, decode, widened (profiling runs select one)")
     args = ap.parse_args()
     args.parts = set(args.parts.split(","))
     if args.warmup < 3:
@@ -424,8 +499,9 @@ def main():
     line = {"metric": METRIC, "value": None, "unit": "tokens/s", "n_gpus": ctx.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": None, "data": "synthetic", "config": None, "roofline": None,
-            "cpu_baseline": None, "e2e": None, "gpu_launches": None, "clocks": None, "decode": None}
-    if "prefill" in args.parts or "e2e" in args.parts:
+            "cpu_baseline": None, "e2e": None, "gpu_launches": None, "clocks": None, "decode": None,
+            "widened": None}
+    if args.parts & {"prefill", "e2e", "widened"}:
         pf = Prefill(ctx, kda, I, args.algo, args.profile_T)
         line["config"] = {"workload": pf.name, "B": pf.cfg.B, "H": pf.cfg.H, "T": pf.cfg.T, "dk": pf.cfg.dk,
                           "dv": pf.cfg.dv, "chunk": pf.cfg.C, "algo": pf.algo_name,
@@ -438,6 +514,8 @@ def main():
                         clocks=clocks, gpu_launches=pf.launches_per_step * args.steps)
         if "e2e" in args.parts:
             line["e2e"] = time_e2e(args, ctx, pf)
+        if "widened" in args.parts:
+            line["widened"] = time_widened(args, ctx, kda, I, pf, peaks)
         del pf
     if "decode" in args.parts:
         line["decode"] = time_decode(args, ctx, kda, I, peaks, peak_kind)

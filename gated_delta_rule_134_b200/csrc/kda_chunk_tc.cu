@@ -743,9 +743,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 const float gm8[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    bad |= live && (!(fabsf(__uint_as_float(g8[e]) - gm8[e]) <= kGuard) || !(gm8[e] >= -kGuard));
+                    bad |= !(fabsf(__uint_as_float(g8[e]) - gm8[e]) <= kGuard) || !(gm8[e] >= -kGuard);
             }
-            const bool exact = nb_or(NB_OR, kPrep, bad);
+            const bool exact = nb_or(NB_OR, kPrep, bad && live);
             if (tid < kD) {
                 const int c = tid;
                 const float g_m = sGm[c], g_l = sGl[c], ek_prev = sEK[c];
@@ -839,8 +839,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 const float4 rb = *reinterpret_cast<const float4*>((exact ? sGl : sGm) + c0 + 4);
                 const float ref8[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
                 const uint32_t km = live ? 0xFFFFFFFFu : 0u;  // rows past the sequence: k = q = 0
-                const uint32_t kw[4] = {kv.x & km, kv.y & km, kv.z & km, kv.w & km};
-                const uint32_t qw[4] = {qv.x & km, qv.y & km, qv.z & km, qv.w & km};
+                const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+                const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
                 uint32_t ke[4], qe[4], kf[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -857,14 +857,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         f0 = __expf(ref8[2 * u] - g0);
                         f1 = __expf(ref8[2 * u + 1] - g1);
                     }
-                    if (!live) e0 = e1 = f0 = f1 = 0.f;  // finite zeros, whatever the gate of a foreign row
                     // packed bf16 products: the factor pairs are rounded to bf16
                     // first, the products once more (both well inside the bf16
                     // rounding of the MMA operands)
                     const uint32_t ep = pack_bf16x2(e0, e1), fp = pack_bf16x2(f0, f1);
-                    ke[u] = hmul2_bf16(kw[u], ep);
-                    qe[u] = hmul2_bf16(qw[u], ep);
-                    kf[u] = hmul2_bf16(kw[u], fp);
+                    ke[u] = hmul2_bf16(kw[u], ep) & km;
+                    qe[u] = hmul2_bf16(qw[u], ep) & km;
+                    kf[u] = hmul2_bf16(kw[u], fp) & km;
                 }
                 st_shared_v4(rop + ko, ke[0], ke[1], ke[2], ke[3]);
                 st_shared_v4(rop + ko + 8192, qe[0], qe[1], qe[2], qe[3]);
