@@ -175,3 +175,40 @@ def recurrent_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, erase: bool 
         o[a:b] = on[0]
         ST[n] = sn[0]
     return o, ST
+
+
+def segment_affine_map(k, v, log_alpha, beta, erase: bool = True, gate="channel"):
+    """The update is affine in the state ("Decoding Hybrid Attention
+    Architectures" section 3.4: S_t = A_t S_{t-1} + b_t k_t v_t^T with
+    A_t = (I - e b_t k_t k_t^T) Diag(a_t)), so a run of tokens maps S_in to
+    M S_in + c. One head, fp64, explicit matrices: k [T,dk], v [T,dv], beta [T],
+    log_alpha [T,dk] / [T] / None by gate. Returns (M [dk,dk], c [dk,dv])."""
+    k, v, beta = _f64(k), _f64(v), _f64(beta)
+    la = _f64(log_alpha)
+    T, dk = k.shape
+    dv = v.shape[1]
+    M = np.eye(dk)
+    c = np.zeros((dk, dv))
+    for t in range(T):
+        if gate == "channel":
+            a = np.exp(la[t])
+        elif gate == "scalar":
+            a = np.full(dk, np.exp(la[t]))
+        else:
+            a = np.ones(dk)
+        A = np.diag(a)
+        if erase:
+            A = (np.eye(dk) - beta[t] * np.outer(k[t], k[t])) @ A
+        M = A @ M
+        c = A @ c + beta[t] * np.outer(k[t], v[t])
+    return M, c
+
+
+def segment_scan(maps, S0):
+    """States entering each segment from the segments' affine maps:
+    S_in[0] = S0, S_in[j+1] = M_j S_in[j] + c_j. Returns the list of P+1
+    states (the last is the final state)."""
+    S = [np.asarray(S0, dtype=np.float64)]
+    for M, c in maps:
+        S.append(M @ S[-1] + c)
+    return S

@@ -216,3 +216,59 @@ def test_varlen_empty_sequence_keeps_state():
     o_1, s_1 = oracle.recurrent(q.reshape(1, 20, 1, 4), k.reshape(1, 20, 1, 4), v.reshape(1, 20, 1, 4),
                                 la.reshape(1, 20, 1, 4), beta.reshape(1, 20, 1), S0[1:2])
     assert np.abs(s_v[1] - s_1[0]).max() < 1e-12
+
+
+# ---------------------------------------------------------------- affine maps of token runs (chunk-parallel scan)
+
+
+def _one_head(seed, T, dk=6, dv=5, la_range=(0.01, 1.0)):
+    q, k, v, la, beta, S0 = pins.random_inputs(seed, T=T, dk=dk, dv=dv, la_range=la_range, B_=1, H_=1)
+    return q[0, :, 0], k[0, :, 0], v[0, :, 0], la[0, :, 0], beta[0, :, 0], S0[0, 0]
+
+
+@pytest.mark.parametrize("erase,gate", [(True, "channel"), (True, "scalar"), (True, "none"), (False, "channel"),
+                                        (False, "none")])
+def test_affine_map_reproduces_recurrence(erase, gate):
+    """M S0 + c equals the C recurrence's final state for several S0 (the map
+    is the run's action on any state), and o is unaffected by the split."""
+    q, k, v, la, beta, _ = _one_head(510, T=19)
+    lag = {"channel": la, "scalar": la[:, 0], "none": None}[gate]
+    M, c = oracle.segment_affine_map(k, v, lag, beta, erase=erase, gate=gate)
+    r = np.random.default_rng(511)
+    for _ in range(3):
+        S0 = r.standard_normal((6, 5))
+        x = lambda a: None if a is None else a[None, :, None]
+        _, ST = oracle.recurrent(x(q), x(k), x(v), x(lag), x(beta), S0[None, None], erase=erase, gate=gate)
+        assert np.abs(M @ S0 + c - ST[0, 0]).max() < 1e-12
+
+
+def test_affine_map_closed_forms():
+    """No erase: M = Diag(exp(sum log_alpha)) (identity without a gate) and
+    c = sum_t exp(G_T - G_t) b_t k_t v_t^T. beta = 0 with erase: M is the pure
+    decay and c = 0."""
+    _, k, v, la, beta, _ = _one_head(512, T=11)
+    M, c = oracle.segment_affine_map(k, v, la, beta, erase=False, gate="channel")
+    G = np.cumsum(la, axis=0)
+    assert np.abs(M - np.diag(np.exp(G[-1]))).max() < 1e-13
+    c_ref = sum(beta[t] * np.outer(np.exp(G[-1] - G[t]) * k[t], v[t]) for t in range(11))
+    assert np.abs(c - c_ref).max() < 1e-13
+    M, c = oracle.segment_affine_map(k, v, None, beta, erase=False, gate="none")
+    assert np.abs(M - np.eye(6)).max() == 0.0
+    M, c = oracle.segment_affine_map(k, v, la, np.zeros_like(beta), erase=True, gate="channel")
+    assert np.abs(M - np.diag(np.exp(G[-1]))).max() < 1e-13 and np.abs(c).max() == 0.0
+
+
+def test_segment_scan_composes_to_whole_run():
+    """Splitting a run into segments, scanning their maps from S0 and reading the
+    last state equals the whole run's map applied to S0; every entry state is
+    the recurrence's state at that segment boundary."""
+    q, k, v, la, beta, S0 = _one_head(513, T=40)
+    cuts = [0, 7, 8, 23, 40]
+    maps = [oracle.segment_affine_map(k[a:b], v[a:b], la[a:b], beta[a:b]) for a, b in zip(cuts, cuts[1:])]
+    states = oracle.segment_scan(maps, S0)
+    M, c = oracle.segment_affine_map(k, v, la, beta)
+    assert np.abs(states[-1] - (M @ S0 + c)).max() < 1e-12
+    for j, t in enumerate(cuts[1:-1], start=1):
+        _, St = oracle.recurrent(q[None, :t, None], k[None, :t, None], v[None, :t, None], la[None, :t, None],
+                                 beta[None, :t, None], S0[None, None])
+        assert np.abs(states[j] - St[0, 0]).max() < 1e-12
