@@ -415,8 +415,9 @@ def _time_calls(ctx, fn, warmup, steps):
 def time_widened(args, ctx, kda, I, pf, peaks):
     """The widened rows, each on a workload of the headline's size:
     packed variable-length sequences (about 32K tokens in 32 sequences of
-    mixed lengths, H32 d128, strong decay) and the four variants on the
-    B4 H32 T8192 inputs. Tokens/s and the HBM roofline fraction of each
+    mixed lengths, H32 d128, strong decay), the four variants on the
+    B4 H32 T8192 inputs, and the B1 H32 T131072 long-context prefill with
+    and without the chunk-parallel segment scan. Tokens/s and the HBM roofline fraction of each
     (algorithmic bytes: q, k, v, the gate as the variant reads it, beta, o,
     and the states)."""
     torch = ctx.torch
@@ -465,6 +466,40 @@ def time_widened(args, ctx, kda, I, pf, peaks):
         res[name] = {"erase": erase, "gate": gate, "value": ctx.world * ntok / (ms * 1e-3), "unit": "tokens/s",
                      "ms_per_step": ms, "roofline_frac": gbs / hbm, "achieved_gbs": gbs}
     out["variants"] = {"workload": cfg.name, "steps": steps, **res}
+    # long context, few heads: one pass per sequence against the segment scan
+    lc = I.B1_H32_T128K
+    g = torch.Generator(device=ctx.dev)
+    g.manual_seed(lc.seed + 1000 * ctx.rank)
+    shp = (lc.B, lc.T, lc.H)
+
+    def unit(z):
+        return (z / z.norm(dim=-1, keepdim=True)).bfloat16()
+    xl = {"q": unit(torch.randn(*shp, lc.dk, device=ctx.dev, generator=g)),
+          "k": unit(torch.randn(*shp, lc.dk, device=ctx.dev, generator=g)),
+          "v": torch.randn(*shp, lc.dv, device=ctx.dev, generator=g).bfloat16(),
+          "log_alpha": (-(lc.la_lo + (lc.la_hi - lc.la_lo) * torch.rand(*shp, lc.dk, device=ctx.dev,
+                                                                          generator=g))).bfloat16(),
+          "beta": torch.sigmoid(torch.randn(*shp, device=ctx.dev, generator=g)).bfloat16()}
+    ol = torch.empty(*shp, lc.dv, dtype=torch.bfloat16, device=ctx.dev)
+    Sl = torch.empty(lc.B, lc.H, lc.dk, lc.dv, dtype=torch.float32, device=ctx.dev)
+    ntok = lc.B * lc.T
+    nbytes = BYTES_PER_TOKEN_HEAD * ntok * lc.H + Sl.numel() * 4
+    long_ctx = {"workload": lc.name, "inputs": "drawn on the device (same distributions)"}
+    for algo in ("tc", "tc_scan"):
+        wsb = kda.workspace_size(lc.B, lc.T, lc.H, lc.dk, lc.dv, lc.C, "bf16", algo)
+        wsl = torch.empty(wsb, dtype=torch.uint8, device=ctx.dev)
+
+        def run_l():
+            kda.chunk_fwd(xl["q"], xl["k"], xl["v"], xl["log_alpha"], xl["beta"], None, chunk=lc.C, algo=algo,
+                          o=ol, S_T=Sl, workspace=wsl, stream=ctx.stream)
+        ms = _time_calls(ctx, run_l, 3, 3)
+        if kda.workspace_status(wsl, ctx.stream) != 0:
+            raise RuntimeError("device-side timeout reported by the prefill kernel")
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        long_ctx[algo] = {"value": ctx.world * ntok / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+                          "steps": 3, "roofline_frac": gbs / hbm, "achieved_gbs": gbs, "workspace_bytes": wsb}
+    out["long_context"] = long_ctx
+    del xl, ol, Sl
     if pf.use_tc and kda.workspace_status(pf.ws, ctx.stream) != 0:
         raise RuntimeError("device-side timeout reported by the prefill kernel")
     return out

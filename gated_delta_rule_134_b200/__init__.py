@@ -19,7 +19,7 @@ _LIB_PATH = os.path.join(_PKG, "libkda.so")
 STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA",
           4: "KDA_ERR_TIMEOUT"}
 _DTYPE = {"f32": 0, "bf16": 1}
-_ALGO = {"auto": 0, "simt": 1, "tc": 2}
+_ALGO = {"auto": 0, "simt": 1, "tc": 2, "tc_scan": 3}
 # Variant switches (include/kda.h): gate "channel" = log_alpha [.., dk], "scalar" =
 # one per token and head, "none" = no decay (log_alpha may be None).
 GATES = {"channel": 0, "scalar": 1, "none": 2}

@@ -11,6 +11,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool head_dims_ok(int dk, int dv) { return dk == dv && (dk == 64 || dk == 128); }
 
+// 0: one pass per sequence; 1: the segment scan where it pays; 2: the scan forced.
+int scan_mode_of(kda_algo_t algo) { return algo == KDA_ALGO_TC_SCAN ? 2 : (algo == KDA_ALGO_AUTO ? 1 : 0); }
+
 kda_status_t run_chunk(const kda::ChunkArgs& a, kda_dtype_t dtype, kda_algo_t algo, void* stream);
 
 kda_status_t check_chunk_args(const kda::ChunkArgs& a, kda_dtype_t dtype) {
@@ -55,8 +58,9 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chu
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
     a.erase = 1; a.gate = KDA_GATE_CHANNEL; a.cu_seqlens = nullptr;
     if (B < 0 || T < 0 || H < 0 || !head_dims_ok(dk, dv)) return 0;
-    const bool tc = (algo == KDA_ALGO_TC) || (algo == KDA_ALGO_AUTO && kda::chunk_tc_supported(a));
-    return tc ? kda::chunk_tc_workspace_bytes(B, T, H, dk, dv) : 0;
+    const bool tc = (algo == KDA_ALGO_TC) || (algo == KDA_ALGO_TC_SCAN) ||
+                    (algo == KDA_ALGO_AUTO && kda::chunk_tc_supported(a));
+    return tc ? kda::chunk_tc_workspace_bytes(a, scan_mode_of(algo)) : 0;
 }
 
 kda_status_t kda_chunk_fwd_v(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
@@ -99,18 +103,21 @@ kda_status_t run_chunk(const kda::ChunkArgs& a, kda_dtype_t dtype, kda_algo_t al
     const size_t workspace_bytes = a.workspace_bytes;
     kda_status_t st = check_chunk_args(a, dtype);
     if (st != KDA_OK) return st;
-    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TC) return KDA_ERR_INVALID_ARG;
-    const bool tc = (algo == KDA_ALGO_TC) || (algo == KDA_ALGO_AUTO && kda::chunk_tc_supported(a));
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TC && algo != KDA_ALGO_TC_SCAN)
+        return KDA_ERR_INVALID_ARG;
+    const bool tc = (algo == KDA_ALGO_TC) || (algo == KDA_ALGO_TC_SCAN) ||
+                    (algo == KDA_ALGO_AUTO && kda::chunk_tc_supported(a));
     if (tc && !kda::chunk_tc_supported(a)) return KDA_ERR_UNSUPPORTED;
+    if (algo == KDA_ALGO_TC_SCAN && a.cu_seqlens) return KDA_ERR_UNSUPPORTED;
     if (tc) {
-        const size_t need = kda::chunk_tc_workspace_bytes(B, T, H, dk, dv);
+        const size_t need = kda::chunk_tc_workspace_bytes(a, scan_mode_of(algo));
         if (need > 0 && (workspace == nullptr || workspace_bytes < need ||
                          (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
             return KDA_ERR_INVALID_ARG;
     }
     if ((long long)B * H == 0) return KDA_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const cudaError_t err = tc ? kda::launch_chunk_tc(a, s) : kda::launch_chunk_simt(a, s);
+    const cudaError_t err = tc ? kda::launch_chunk_tc(a, scan_mode_of(algo), s) : kda::launch_chunk_simt(a, s);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

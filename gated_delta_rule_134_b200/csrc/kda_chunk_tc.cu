@@ -59,6 +59,7 @@
 // Every wait on an mbarrier is bounded; on expiry the kernel records status 1
 // in the caller's workspace word and stops waiting (later waits are skipped,
 // so every role reaches the end), frees its tensor memory and returns.
+#include <algorithm>
 #include <type_traits>
 
 #include "kda_common.cuh"
@@ -225,13 +226,28 @@ __device__ __forceinline__ bool nb_or(int id, int nthreads, bool pred) {
 // ERASE: 1 delta-rule family, 0 additive write. GATE: 0 per-channel log_alpha,
 // 1 one per token and head, 2 none. Compile-time, so each variant is its own
 // kernel and the KDA instance carries no variant branches.
+// Chunk-parallel scan over segments of each sequence (few heads, long T).
+// The update is affine in the state, so a segment maps its entry state S_in
+// to M S_in + C. Phase 1 runs segment 0 in full and, for each middle segment
+// j = 1..P-2, its transition M_j (entry state I, v = 0) and offset C_j (entry
+// state 0); a scan then chains S_in of segments 1..P-1; phase 3 runs those
+// segments in full from their entry states. P = 0: whole sequences.
+struct SegJobs {
+    int P;       // segments per sequence (0: no scan)
+    int L;       // tokens per segment, a multiple of the chunk
+    int phase;   // 1 or 3
+    float* M;    // [B*H][P-2][dk][dv]
+    float* C;    // [B*H][P-2][dk][dv]
+    float* Sin;  // [B*H][P-1][dk][dv]: state entering segment j at [j-1]
+};
+
 template <int DVT, int ERASE, int GATE>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
                     const __nv_bfloat16* __restrict__ beta, const float* S0, __nv_bfloat16* __restrict__ o,
                     float* ST, int Tlen, int H, unsigned* status, const __nv_bfloat16* __restrict__ gate_tok,
-                    const int* __restrict__ cu_seqlens) {
+                    const int* __restrict__ cu_seqlens, const SegJobs sj) {
     constexpr int erase = ERASE, gate = GATE;
     using L = Layout<DVT>;
     extern __shared__ uint8_t smem_raw[];
@@ -243,13 +259,19 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nslices = kD / DVT;
-    const int bh = blockIdx.x / nslices;
+    const int unit = blockIdx.x / nslices;  // the (sequence-head, piece) of this CTA
+    const int per = sj.P == 0 ? 1 : (sj.phase == 1 ? 2 * sj.P - 3 : sj.P - 1);
+    const int bh = unit / per, piece = unit % per;
     const int b = bh / H, h = bh % H;
-    // This sequence's tokens: [tok0, tok0 + seq_len) of the token-major layout.
+    constexpr size_t kMat = (size_t)kD * kD;
+    // This piece's tokens: [tok0, tok0 + seq_len) of the token-major layout.
     // Dense batch: sequence b of [B, T]; packed: offsets clamped into [0, T], and
     // the tensor maps then describe one [1, T] sequence (tile origin tma_t0).
     size_t tok0;
     int seq_len, tma_t0, tma_b;
+    const float* s0m = S0 ? S0 + bh * kMat : nullptr;  // entry state [dk][dv] (NULL: zero)
+    float* stm = ST ? ST + bh * kMat : nullptr;        // final state destination (NULL: none)
+    bool s0_ident = false, v_zero = false, o_on = true;
     if (cu_seqlens) {
         const int s0 = min(max(cu_seqlens[b], 0), Tlen), s1 = min(max(cu_seqlens[b + 1], s0), Tlen);
         tok0 = (size_t)s0;
@@ -261,6 +283,28 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         seq_len = Tlen;
         tma_t0 = 0;
         tma_b = b;
+        if (sj.P > 0) {
+            // phase 1: piece 0 = segment 0 in full, then (M_j, C_j) pairs; phase 3: segments 1..P-1
+            const int j = sj.phase == 3 ? piece + 1 : (piece == 0 ? 0 : 1 + (piece - 1) / 2);
+            const int t_begin = j * sj.L;
+            seq_len = max(0, min(sj.L, Tlen - t_begin));
+            tok0 += (size_t)t_begin;
+            tma_t0 = t_begin;
+            if (sj.phase == 3) {
+                s0m = sj.Sin + ((size_t)bh * (sj.P - 1) + (j - 1)) * kMat;
+                if (j != sj.P - 1) stm = nullptr;
+            } else if (piece == 0) {
+                stm = sj.Sin + (size_t)bh * (sj.P - 1) * kMat;
+            } else {
+                const size_t off = ((size_t)bh * (sj.P - 2) + (j - 1)) * kMat;
+                const bool is_m = ((piece - 1) & 1) == 0;
+                o_on = false;
+                s0m = nullptr;
+                s0_ident = is_m;
+                v_zero = is_m;
+                stm = (is_m ? sj.M : sj.C) + off;
+            }
+        }
     }
     const int j0 = (blockIdx.x % nslices) * DVT;
     const int NC = (seq_len + kC - 1) / kC;
@@ -307,6 +351,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             st_shared_v4(sb + L::TZP + R * 128 + (j << 4), 0u, 0u, 0u, 0u);
         }
         for (int c = tid; c < kD; c += kThreads) sEK[c] = 1.f;
+        if (v_zero)  // transition run: v = 0 stays in the v tile, which is never loaded
+            for (int i = tid; i < (DVT / 64) * 8192 / 16; i += kThreads) st_shared_v4(sb + L::RAWV + 16 * i, 0u, 0u, 0u, 0u);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -384,6 +430,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     for (int x = 0; x < 2; ++x) tma_prefetch_l2_4d(&tm_g, 64 * x, h, tma_t0 + (m + 1) * kC, tma_b);
             };
             auto issue_v = [&](int m) {
+                if (v_zero) {  // the zero tile is already in place
+                    mbar_arrive(bars + BAR_V);
+                    return;
+                }
                 mbar_arrive_expect_tx(bars + BAR_V, (DVT / 64) * 8192);
                 for (int x = 0; x < DVT / 64; ++x)
                     tma_load_4d(sm + L::RAWV + x * 8192, &tm_v, bars + BAR_V, j0 + 64 * x, h, tma_t0 + m * kC, tma_b);
@@ -480,8 +530,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll 1
             for (int gq = 0; gq < DVT / 32; ++gq) {
                 uint32_t r[32];
-                if (S0) {
-                    const float4* src = reinterpret_cast<const float4*>(S0 + ((size_t)bh * kD + row) * kD + j0 + 32 * gq);
+                if (s0m) {
+                    const float4* src = reinterpret_cast<const float4*>(s0m + (size_t)row * kD + j0 + 32 * gq);
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const float4 v = src[u];
@@ -490,7 +540,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     }
                 } else {
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) r[u] = 0u;
+                    for (int u = 0; u < 32; ++u) r[u] = (s0_ident && row == j0 + 32 * gq + u) ? __float_as_uint(1.f) : 0u;
                 }
                 tmem_st32(lane_addr + L::S_COL + 32 * gq, r);
             }
@@ -616,7 +666,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         uint32_t v[32];
                         tmem_ld32(lane_addr + L::D1_COL + 32 * gq, v);
                         tmem_ld_wait(v);
-                        if (t0 + r < seq_len) {
+                        if (o_on && t0 + r < seq_len) {
                             uint4* dst = reinterpret_cast<uint4*>(o + ((tok0 + t0 + r) * H + h) * kD + j0 +
                                                                   32 * gq);
 #pragma unroll
@@ -641,14 +691,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         // ------------------------------------------------------------ final state S = e^{G_last - G_m} R
         if (quad < 2 && NC > 0) waitw(BAR_M2, (uint32_t)(NC - 1));
         // one decision per warp: the tensor-memory loads below are warp-collective
-        if (__shfl_sync(0xffffffffu, (ST && !*s_abort) ? 1 : 0, 0)) {
+        if (__shfl_sync(0xffffffffu, (stm && !*s_abort) ? 1 : 0, 0)) {
             const float ek = sEK[row];
 #pragma unroll 1
             for (int gq = 0; gq < DVT / 32; ++gq) {
                 uint32_t v[32];
                 tmem_ld32(lane_addr + L::S_COL + 32 * gq, v);
                 tmem_ld_wait(v);
-                float4* dst = reinterpret_cast<float4*>(ST + ((size_t)bh * kD + row) * kD + j0 + 32 * gq);
+                float4* dst = reinterpret_cast<float4*>(stm + (size_t)row * kD + j0 + 32 * gq);
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
                     dst[u] = make_float4(__uint_as_float(v[4 * u]) * ek, __uint_as_float(v[4 * u + 1]) * ek,
@@ -1110,8 +1160,47 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Chains the entry states of the segments: S_in[j+1] = M_j S_in[j] + C_j for
+// j = 1..P-2 (S_in[1] is segment 0's final state). The columns of a state are
+// independent, so each CTA carries 8 value columns of one sequence-head
+// through every segment, in fp32.
+__global__ void __launch_bounds__(256) segment_scan_kernel(const float* __restrict__ M, const float* __restrict__ C,
+                                                           float* Sin, int P) {
+    constexpr size_t kMat = (size_t)kD * kD;
+    const int bh = blockIdx.x, c0 = blockIdx.y * 8, tid = threadIdx.x;
+    const int i = tid >> 1, cc = (tid & 1) * 4;  // output row, first of 4 columns
+    __shared__ float s[kD][8];
+    const float* S1 = Sin + (size_t)bh * (P - 1) * kMat;
+    for (int e = tid; e < kD * 8; e += 256) s[e >> 3][e & 7] = S1[(size_t)(e >> 3) * kD + c0 + (e & 7)];
+    __syncthreads();
+    for (int j = 1; j <= P - 2; ++j) {
+        const size_t mj = ((size_t)bh * (P - 2) + (j - 1)) * kMat + (size_t)i * kD;
+        const float4 cv = *reinterpret_cast<const float4*>(C + mj + c0 + cc);
+        float a0 = cv.x, a1 = cv.y, a2 = cv.z, a3 = cv.w;
+        const float4* mrow = reinterpret_cast<const float4*>(M + mj);
+#pragma unroll 4
+        for (int k4 = 0; k4 < kD / 4; ++k4) {
+            const float4 m = mrow[k4];
+            const float mk[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float* sr = s[4 * k4 + u] + cc;
+                a0 = fmaf(mk[u], sr[0], a0);
+                a1 = fmaf(mk[u], sr[1], a1);
+                a2 = fmaf(mk[u], sr[2], a2);
+                a3 = fmaf(mk[u], sr[3], a3);
+            }
+        }
+        __syncthreads();  // every read of the previous state is done
+        s[i][cc] = a0; s[i][cc + 1] = a1; s[i][cc + 2] = a2; s[i][cc + 3] = a3;
+        *reinterpret_cast<float4*>(Sin + ((size_t)bh * (P - 1) + j) * kMat + (size_t)i * kD + c0 + cc) =
+            make_float4(a0, a1, a2, a3);
+        __syncthreads();
+    }
+}
+
 template <int DVT, int ERASE, int GATE>
-cudaError_t launch_dvt(const ChunkArgs& a, cudaStream_t stream) {
+cudaError_t launch_dvt(const ChunkArgs& a, cudaStream_t stream, const SegJobs& sj, long units) {
     using L = Layout<DVT>;
     CUtensorMap mk, mq, mg, mv;
     const int mb = a.cu_seqlens ? 1 : a.B;  // packed sequences: one [1, T] token range
@@ -1123,13 +1212,45 @@ cudaError_t launch_dvt(const ChunkArgs& a, cudaStream_t stream) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     unsigned* status = static_cast<unsigned*>(a.workspace);
-    err = cudaMemsetAsync(status, 0, sizeof(unsigned), stream);
-    if (err != cudaSuccess) return err;
-    const unsigned grid = (unsigned)(a.B * a.H * (kD / DVT));
+    const unsigned grid = (unsigned)(units * (kD / DVT));
     kern<<<grid, kThreads, L::SMEM_BYTES, stream>>>(mk, mq, mg, mv, (const __nv_bfloat16*)a.beta, a.S0,
                                                     (__nv_bfloat16*)a.o, a.ST, a.T, a.H, status,
-                                                    GATE == 1 ? (const __nv_bfloat16*)a.log_alpha : nullptr, a.cu_seqlens);
+                                                    GATE == 1 ? (const __nv_bfloat16*)a.log_alpha : nullptr,
+                                                    a.cu_seqlens, sj);
     return cudaGetLastError();
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess || n <= 0) {
+        cudaGetLastError();  // (no device: plan for a B200)
+        return 148;
+    }
+    return n;
+}
+
+// Segments for the chunk-parallel scan, or 0 when it does not pay.
+// Phase 1 holds B*H*(2P-3) CTAs; P is the largest count that keeps it to one
+// wave, with at least kMinSegChunks chunks per segment (forced: 2, and P >= 3).
+// L is then rounded to whole chunks and P recounted so no segment is empty.
+constexpr int kMinSegChunks = 8;
+void scan_plan(const ChunkArgs& a, int mode, int* P_out, int* L_out) {
+    *P_out = 0;
+    *L_out = 0;
+    if (mode == 0 || a.cu_seqlens || a.T <= 0) return;
+    const long bh = (long)a.B * a.H;
+    const int NC = (a.T + kC - 1) / kC;
+    if (bh <= 0) return;
+    long P = ((long)sm_count() / bh + 3) / 2;
+    P = std::min<long>(P, NC / (mode == 2 ? 2 : kMinSegChunks));
+    if (mode == 2) P = std::max<long>(P, 3);
+    if (P < 3 || NC < 3) return;
+    const int Lc = (int)((NC + P - 1) / P);
+    const int Pn = (NC + Lc - 1) / Lc;
+    if (Pn < 3) return;
+    *P_out = Pn;
+    *L_out = Lc * kC;
 }
 
 }  // namespace
@@ -1138,21 +1259,47 @@ bool chunk_tc_supported(const ChunkArgs& a) {
     return a.bf16 && a.dk == kD && a.dv == kD && a.chunk == kC;
 }
 
-size_t chunk_tc_workspace_bytes(int, int, int, int, int) { return 256; }
+size_t chunk_tc_workspace_bytes(const ChunkArgs& a, int scan_mode) {
+    int P, L;
+    scan_plan(a, scan_mode, &P, &L);
+    if (P == 0) return 256;
+    const size_t mat = (size_t)kD * kD * sizeof(float), bh = (size_t)a.B * a.H;
+    return 256 + bh * mat * (size_t)(2 * (P - 2) + (P - 1));
+}
 
-cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t stream) {
+cudaError_t launch_chunk_tc(const ChunkArgs& a, int scan_mode, cudaStream_t stream) {
+    cudaError_t err = cudaMemsetAsync(a.workspace, 0, sizeof(unsigned), stream);
+    if (err != cudaSuccess) return err;
     // An empty sequence has no chunk to load (and no tensor map can describe
     // it): the result is S_T = S0, which the SIMT kernel writes.
-    if (a.T == 0) {
-        cudaError_t err = cudaMemsetAsync(a.workspace, 0, sizeof(unsigned), stream);
-        return err != cudaSuccess ? err : launch_chunk_simt(a, stream);
-    }
-    // One CTA per (batch, head) when there are enough heads to fill the
-    // GPU; otherwise split the value channels in two.
-    const bool wide = (long)a.B * a.H >= 96;
+    if (a.T == 0) return launch_chunk_simt(a, stream);
+    const long bh = (long)a.B * a.H;
+    const int sms = sm_count();
+    int P, L;
+    scan_plan(a, scan_mode, &P, &L);
     auto pick = [&](auto erase_c, auto gate_c) -> cudaError_t {
         constexpr int E = decltype(erase_c)::value, G = decltype(gate_c)::value;
-        return wide ? launch_dvt<128, E, G>(a, stream) : launch_dvt<64, E, G>(a, stream);
+        if (P == 0) {
+            // One CTA per (batch, head) when there are enough heads to fill the
+            // GPU; otherwise split the value channels in two.
+            const bool wide = bh >= 96;
+            return wide ? launch_dvt<128, E, G>(a, stream, SegJobs{}, bh) : launch_dvt<64, E, G>(a, stream, SegJobs{}, bh);
+        }
+        const size_t mat = (size_t)kD * kD;
+        float* Mb = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + 256);
+        float* Cb = Mb + (size_t)bh * (P - 2) * mat;
+        float* Sin = Cb + (size_t)bh * (P - 2) * mat;
+        SegJobs sj{P, L, 1, Mb, Cb, Sin};
+        cudaError_t e = launch_dvt<128, E, G>(a, stream, sj, bh * (2 * P - 3));
+        if (e != cudaSuccess) return e;
+        if (P > 2) {
+            segment_scan_kernel<<<dim3((unsigned)bh, kD / 8), 256, 0, stream>>>(Mb, Cb, Sin, P);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+        sj.phase = 3;
+        const long units3 = bh * (P - 1);
+        return 2 * units3 <= sms ? launch_dvt<64, E, G>(a, stream, sj, units3) : launch_dvt<128, E, G>(a, stream, sj, units3);
     };
     using I0 = std::integral_constant<int, 0>;
     using I1 = std::integral_constant<int, 1>;
@@ -1238,13 +1385,13 @@ extern "C" kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, cons
     }
     if ((S0 && !noalloc_aligned16(S0)) || (S_T && !noalloc_aligned16(S_T))) return KDA_ERR_INVALID_ARG;
     // The kernel's scratch must fit the fixed array.
-    if (kda::chunk_tc_workspace_bytes(B, T, H, dk, dv) > sizeof(g_kda_noalloc_scratch)) return KDA_ERR_INVALID_ARG;
+    if (kda::chunk_tc_workspace_bytes(a, 0) > sizeof(g_kda_noalloc_scratch)) return KDA_ERR_INVALID_ARG;
     if ((long long)B * H == 0) return KDA_OK;
     void* scratch = nullptr;
     if (noalloc_scratch(&scratch) != cudaSuccess) return KDA_ERR_CUDA;
     a.workspace = scratch;
     a.workspace_bytes = sizeof(g_kda_noalloc_scratch);
     // launch_chunk_tc clears the status word before the kernel runs.
-    const cudaError_t err = kda::launch_chunk_tc(a, static_cast<cudaStream_t>(stream));
+    const cudaError_t err = kda::launch_chunk_tc(a, 0, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

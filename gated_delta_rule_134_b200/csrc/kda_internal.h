@@ -32,7 +32,9 @@ cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t stream);
 
 // Fused tensor-core prefill (bf16, dk = dv = 128, chunk = 64).
 bool chunk_tc_supported(const ChunkArgs& a);
-size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv);
-cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t stream);
+// scan_mode: 0 one pass per sequence; 1 the chunk-parallel segment scan where
+// it pays (dense batch, few heads, long T); 2 the scan whenever T has 3 chunks.
+size_t chunk_tc_workspace_bytes(const ChunkArgs& a, int scan_mode);
+cudaError_t launch_chunk_tc(const ChunkArgs& a, int scan_mode, cudaStream_t stream);
 
 }  // namespace kda

@@ -50,8 +50,21 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
 
 /* Which prefill kernels to run. AUTO picks the fused tensor-core kernel when
  * it supports the shape (bf16, dk = dv = 128, chunk = 64) and the SIMT fp32
- * kernel otherwise. */
-typedef enum { KDA_ALGO_AUTO = 0, KDA_ALGO_SIMT = 1, KDA_ALGO_TC = 2 } kda_algo_t;
+ * kernel otherwise; for a dense batch with few heads and a long T it adds the
+ * chunk-parallel segment scan when that shortens the run.
+ *
+ * KDA_ALGO_TC_SCAN: the tensor-core kernel with the segment scan whenever T
+ * spans at least 3 chunks (else plain KDA_ALGO_TC); dense batches only
+ * (KDA_ERR_UNSUPPORTED for packed sequences). The update is affine in the
+ * state ("Decoding Hybrid Attention Architectures" section 3.4; the chunk
+ * form of section 4 passes the state between chunks the same way), so each
+ * segment of a sequence maps its entry state S_in to M S_in + C. Segment 0
+ * and the maps (M, C) of the middle segments are computed in parallel, an
+ * fp32 scan chains the entry states, and segments 1..P-1 are then run in
+ * parallel from them. Work grows by about half; the sequential depth drops
+ * from T to about 2T/P tokens. The workspace holds the maps and entry states
+ * (B*H*(3P-5) fp32 [dk][dv] matrices; see kda_chunk_fwd_workspace_size). */
+typedef enum { KDA_ALGO_AUTO = 0, KDA_ALGO_SIMT = 1, KDA_ALGO_TC = 2, KDA_ALGO_TC_SCAN = 3 } kda_algo_t;
 
 /* The variant table of "Decoding Hybrid Attention Architectures" (section
  * 3.4, with sections 3.1-3.3 and the per-dimension gated linear attention it

@@ -179,3 +179,22 @@ def test_varlen_rejects_missing_or_misaligned_offsets():
     args = lambda cu: (q, k, v, la, beta, S0, o, ST, cu, 2, 8, 1, 64, 64, 64, 1, 1, 0, None, 0, 0, None)
     assert lib.kda_chunk_fwd_varlen(*args(None)) == 1
     assert lib.kda_chunk_fwd_varlen(*args(ctypes.c_void_p(0x5002))) == 1
+
+
+def test_scan_workspace_sizes():
+    """The segment scan keeps B*H*(3P-5) fp32 [128][128] matrices after the
+    256-byte status block; it is planned only where it pays (auto) and never
+    for 128 heads (one wave of whole sequences already fills 148 SMs)."""
+    mat = 128 * 128 * 4
+    # 32 heads, 2048 chunks: P = 3 -> 4 matrices per head
+    assert kda.workspace_size(1, 131072, 32, 128, 128, 64, "bf16", "tc_scan") == 256 + 32 * 4 * mat
+    assert kda.workspace_size(1, 131072, 32, 128, 128, 64, "bf16", "auto") == 256 + 32 * 4 * mat
+    assert kda.workspace_size(1, 131072, 32, 128, 128, 64, "bf16", "tc") == 256
+    assert kda.workspace_size(4, 8192, 32, 128, 128, 64, "bf16", "auto") == 256
+    # 2 heads, 65 chunks, forced: P = 32 -> Lc = 3 chunks -> 22 segments
+    assert kda.workspace_size(1, 4100, 2, 128, 128, 64, "bf16", "tc_scan") == 256 + 2 * (3 * 22 - 5) * mat
+    # forced on 3 chunks: one chunk per segment, P = 3
+    assert kda.workspace_size(1, 191, 1, 128, 128, 64, "bf16", "tc_scan") == 256 + 4 * mat
+    # too short to split (2 chunks): plain
+    assert kda.workspace_size(1, 100, 1, 128, 128, 64, "bf16", "tc_scan") == 256
+    assert kda.workspace_size(1, 1000, 1, 128, 128, 64, "bf16", "auto") == 256

@@ -177,7 +177,7 @@ def test_prefill_small_f32_full(cuda_lib):
     check_prefill(cuda_lib, I.SMALL_F32, "auto")
 
 
-@pytest.mark.parametrize("algo", ["auto", "simt"])
+@pytest.mark.parametrize("algo", ["auto", "tc", "simt"])
 def test_prefill_b2_h16_t4k(cuda_lib, algo):
     check_prefill(cuda_lib, I.B2_H16_T4K, algo, heads=[(0, 0), (0, 7), (1, 3), (1, 15)])
 
@@ -186,8 +186,10 @@ def test_prefill_b4_h32_t8k(cuda_lib):
     check_prefill(cuda_lib, I.B4_H32_T8K, "auto", heads=[(0, 0), (0, 31), (1, 5), (2, 17), (3, 2), (3, 30)])
 
 
-def test_prefill_b1_h32_t128k(cuda_lib):
-    check_prefill(cuda_lib, I.B1_H32_T128K, "auto", heads=[(0, 0), (0, 13), (0, 31)])
+@pytest.mark.parametrize("algo", ["auto", "tc"])
+def test_prefill_b1_h32_t128k(cuda_lib, algo):
+    # auto takes the segment scan here (32 heads, 2048 chunks)
+    check_prefill(cuda_lib, I.B1_H32_T128K, algo, heads=[(0, 0), (0, 13), (0, 31)])
 
 
 # ---------------------------------------------------------------- decode
@@ -420,3 +422,63 @@ def test_varlen_full_size_sampled(cuda_lib):
         worst = max(worst, rel_err(ST[n, h].cpu().numpy()[None, None], ref_S))
     print(f"PARITY varlen full-size sampled worst={worst:.3e}")
     assert worst <= TOL["bf16"]
+
+
+# ---------------------------------------------------------------- chunk-parallel segment scan (tc_scan)
+
+
+@pytest.mark.parametrize("B,H,T,s0", [(2, 3, 1000, 0.3), (1, 1, 777, 0.0), (1, 2, 4100, 0.2), (3, 2, 384, 0.3),
+                                      (1, 1, 191, 0.3), (1, 1, 100, 0.3)])
+def test_scan_small(cuda_lib, B, H, T, s0):
+    """Segments of 2+ chunks, a ragged last segment, many segments in the scan
+    chain (T=4100 on 2 heads: 22 segments), one-chunk segments (T=191) and the
+    plain fallback (T=100, two chunks)."""
+    check_prefill(cuda_lib, small_cfg("bf16", 128, 64, T, B=B, H=H, s0=s0, seed=60 + T), "tc_scan")
+
+
+@pytest.mark.parametrize("erase,gate", VARIANTS)
+def test_scan_variants(cuda_lib, erase, gate):
+    check_variant(cuda_lib, small_cfg("bf16", 128, 64, 1100, B=1, H=2, s0=0.3, seed=61), "tc_scan", erase, gate)
+
+
+@pytest.mark.parametrize("algo", ["tc_scan", "auto"])
+def test_scan_weak_decay(cuda_lib, algo):
+    """Weak decay over short segments: every segment's output depends on its
+    entry state, so errors in the maps or the scan would show everywhere."""
+    check_prefill(cuda_lib, small_cfg("bf16", 128, 64, 3000, B=1, H=2, la=(0.0001, 0.005), s0=0.3, seed=66), algo)
+
+
+def test_scan_extreme_decay(cuda_lib):
+    # strong decay: chunks take the exact path inside the segment runs too
+    check_prefill(cuda_lib, small_cfg("bf16", 128, 64, 900, B=1, H=2, la=(0.5, 6.0), s0=0.3, seed=62), "tc_scan")
+
+
+def test_scan_state_aliasing(cuda_lib):
+    """S_T may alias S0: segment 0 reads S0 in the first launch, the last
+    segment writes S_T in the last one."""
+    cfg = small_cfg("bf16", 128, 64, 1000, B=1, H=3, s0=0.3, seed=63)
+    x = I.prefill_inputs(cfg)
+    xd = to_dev(x)
+    S = xd["S0"].clone()
+    o, ST = cuda_lib.chunk_fwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], S, S_T=S, algo="tc_scan")
+    torch.cuda.synchronize()
+    ref_o, ref_S = oracle.recurrent(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"])
+    assert rel_err(o.float().cpu().numpy(), ref_o) <= TOL["bf16"]
+    assert rel_err(S.cpu().numpy(), ref_S) <= TOL["bf16"]
+
+
+def test_scan_deterministic(cuda_lib):
+    cfg = small_cfg("bf16", 128, 64, 2000, B=1, H=4, s0=0.3, seed=64)
+    x = to_dev(I.prefill_inputs(cfg))
+    outs = [cuda_lib.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], algo="tc_scan")
+            for _ in range(3)]
+    torch.cuda.synchronize()
+    for o, ST in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(ST, outs[0][1])
+
+
+def test_scan_varlen_unsupported(cuda_lib):
+    x = to_dev(I.varlen_inputs(small_cfg("bf16", 128, 64, 0, H=1, seed=65), [100, 200]))
+    with pytest.raises(RuntimeError):
+        cuda_lib.chunk_fwd_varlen(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["cu_seqlens"], x["S0"],
+                                  algo="tc_scan")
