@@ -212,3 +212,79 @@ def segment_scan(maps, S0):
     for M, c in maps:
         S.append(M @ S[-1] + c)
     return S
+
+
+def recurrent_bwd(q, k, v, log_alpha, beta, S0, do, dST=None, erase: bool = True, gate="channel",
+                  ckpt: int = 64):
+    """Gradients of the token recurrence, by reverse-mode differentiation of
+    each step (the pages give no backward pass; this is the chain rule applied
+    to the update of "Decoding Hybrid Attention Architectures" section 3.4).
+
+    Loss L with dL/do = do [B,T,H,dv] and dL/dS_T = dST [B,H,dk,dv] (None:
+    0). Per step, with Lam = dL/dS_t (the future part plus q_t do_t^T):
+        S~ = Diag(a_t) S_{t-1},  r = v_t - S~^T k_t,  delta = b_t r  (no erase: b_t v_t)
+        dq_t = S_t do_t,  g = Lam^T k_t,  dv_t = b_t g,  db_t = g . r (no erase: g . v_t)
+        dk_t = Lam delta - b_t S~ g   (second term only with the erase term)
+        Lam~ = Lam - b_t k_t g^T      (dL/dS~; no erase: Lam)
+        dlog_a_t = rowsum(Lam~ * S~)  (per channel; summed for a scalar gate)
+        dL/dS_{t-1} = Diag(a_t) Lam~
+    and dS0 = dL/dS_0. States are recomputed from checkpoints every `ckpt`
+    tokens (same arithmetic, less memory). fp64 numpy; small cases only.
+    Returns dict dq, dk, dv, dlog_alpha (shape of log_alpha, None without a
+    gate), dbeta, dS0."""
+    q, k, v, beta, do = map(_f64, (q, k, v, beta, do))
+    la = _f64(log_alpha)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    S0 = np.zeros((B, H, dk, dv)) if S0 is None else _f64(S0)
+    dST = np.zeros((B, H, dk, dv)) if dST is None else _f64(dST)
+    out = {n: np.zeros_like(x) for n, x in (("dq", q), ("dk", k), ("dv", v), ("dbeta", beta))}
+    out["dlog_alpha"] = None if gate == "none" else np.zeros_like(la)
+    out["dS0"] = np.zeros_like(S0)
+
+    def decay(b, t, h):
+        if gate == "channel":
+            return np.exp(la[b, t, h])
+        if gate == "scalar":
+            return np.full(dk, np.exp(la[b, t, h]))
+        return np.ones(dk)
+
+    def step(S, b, t, h):
+        St = decay(b, t, h)[:, None] * S
+        r = v[b, t, h] - St.T @ k[b, t, h]
+        delta = beta[b, t, h] * (r if erase else v[b, t, h])
+        return St, r, St + np.outer(k[b, t, h], delta)
+
+    for b in range(B):
+        for h in range(H):
+            # forward: states at the checkpoints
+            marks = {}
+            S = S0[b, h].copy()
+            for t in range(T):
+                if t % ckpt == 0:
+                    marks[t] = S.copy()
+                S = step(S, b, t, h)[2]
+            Lam = dST[b, h].copy()
+            for t0 in sorted(marks, reverse=True):
+                t1 = min(t0 + ckpt, T)
+                prev = [marks[t0]]
+                for t in range(t0, t1 - 1):
+                    prev.append(step(prev[-1], b, t, h)[2])
+                for t in range(t1 - 1, t0 - 1, -1):
+                    St, r, S_t = step(prev[t - t0], b, t, h)
+                    kt, bt = k[b, t, h], beta[b, t, h]
+                    Lam = Lam + np.outer(q[b, t, h], do[b, t, h])
+                    out["dq"][b, t, h] = S_t @ do[b, t, h]
+                    g = Lam.T @ kt
+                    delta = bt * (r if erase else v[b, t, h])
+                    out["dv"][b, t, h] = bt * g
+                    out["dbeta"][b, t, h] = g @ (r if erase else v[b, t, h])
+                    out["dk"][b, t, h] = Lam @ delta - (bt * (St @ g) if erase else 0.0)
+                    Lt = Lam - bt * np.outer(kt, g) if erase else Lam
+                    if gate == "channel":
+                        out["dlog_alpha"][b, t, h] = (Lt * St).sum(axis=1)
+                    elif gate == "scalar":
+                        out["dlog_alpha"][b, t, h] = (Lt * St).sum()
+                    Lam = decay(b, t, h)[:, None] * Lt
+            out["dS0"][b, h] = Lam
+    return out

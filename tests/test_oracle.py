@@ -272,3 +272,72 @@ def test_segment_scan_composes_to_whole_run():
         _, St = oracle.recurrent(q[None, :t, None], k[None, :t, None], v[None, :t, None], la[None, :t, None],
                                  beta[None, :t, None], S0[None, None])
         assert np.abs(states[j] - St[0, 0]).max() < 1e-12
+
+
+# ---------------------------------------------------------------- backward (gradients of the recurrence)
+
+
+def _loss_and_grads(seed, erase, gate, T=5, dk=3, dv=2):
+    q, k, v, la, beta, S0 = pins.random_inputs(seed, T=T, dk=dk, dv=dv, B_=1, H_=2)
+    lag = {"channel": la, "scalar": la[..., 0], "none": None}[gate]
+    r = np.random.default_rng(seed + 1)
+    Wo = r.standard_normal(v.shape)
+    WS = r.standard_normal(S0.shape)
+    inputs = {"q": q, "k": k, "v": v, "log_alpha": lag, "beta": beta, "S0": S0}
+
+    def loss(x):
+        o, ST = oracle.recurrent(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], erase=erase, gate=gate)
+        return float((o * Wo).sum() + (ST * WS).sum())
+
+    g = oracle.recurrent_bwd(q, k, v, lag, beta, S0, Wo, WS, erase=erase, gate=gate, ckpt=2)
+    return inputs, loss, g
+
+
+@pytest.mark.parametrize("erase,gate", [(True, "channel"), (True, "scalar"), (True, "none"), (False, "channel"),
+                                        (False, "scalar"), (False, "none")])
+def test_bwd_matches_finite_differences(erase, gate):
+    """Every gradient element against a central difference of the forward
+    oracle (a linear functional of o and S_T), for every variant."""
+    inputs, loss, g = _loss_and_grads(520, erase, gate)
+    names = {"q": "dq", "k": "dk", "v": "dv", "log_alpha": "dlog_alpha", "beta": "dbeta", "S0": "dS0"}
+    eps = 1e-6
+    for name, gname in names.items():
+        x = inputs[name]
+        if x is None:
+            assert g[gname] is None
+            continue
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp = {kk: (None if vv is None else vv.copy()) for kk, vv in inputs.items()}
+            xm = {kk: (None if vv is None else vv.copy()) for kk, vv in inputs.items()}
+            xp[name][idx] += eps
+            xm[name][idx] -= eps
+            fd[idx] = (loss(xp) - loss(xm)) / (2 * eps)
+        assert np.abs(g[gname] - fd).max() < 1e-7 * max(1.0, np.abs(fd).max()), (name, erase, gate)
+
+
+def test_bwd_linear_attention_closed_form():
+    """No erase, no gate: o_t = S0^T q_t + sum_{s<=t} (q_t . k_s) b_s v_s and
+    S_T = S0 + sum_s b_s k_s v_s^T, so dv_s = b_s (sum_{t>=s} (q_t . k_s) do_t
+    + dS_T^T k_s) and dq_t = S0 do_t + sum_{s<=t} k_s b_s (v_s . do_t)."""
+    q, k, v, _, beta, S0 = pins.random_inputs(521, T=9, dk=5, dv=4, B_=1, H_=1)
+    r = np.random.default_rng(522)
+    do = r.standard_normal(v.shape)
+    dST = r.standard_normal(S0.shape)
+    g = oracle.recurrent_bwd(q, k, v, None, beta, S0, do, dST, erase=False, gate="none", ckpt=4)
+    Q, K, V, Bt, DO = q[0, :, 0], k[0, :, 0], v[0, :, 0], beta[0, :, 0], do[0, :, 0]
+    for s in range(9):
+        dv_ref = Bt[s] * (sum((Q[t] @ K[s]) * DO[t] for t in range(s, 9)) + dST[0, 0].T @ K[s])
+        assert np.abs(g["dv"][0, s, 0] - dv_ref).max() < 1e-12
+        dq_ref = S0[0, 0] @ DO[s] + sum(K[u] * Bt[u] * (V[u] @ DO[s]) for u in range(s + 1))
+        assert np.abs(g["dq"][0, s, 0] - dq_ref).max() < 1e-12
+    assert np.abs(g["dS0"][0, 0] - (dST[0, 0] + Q.T @ DO)).max() < 1e-12
+
+
+def test_bwd_checkpoint_interval_invariant():
+    q, k, v, la, beta, S0 = pins.random_inputs(523, T=13, dk=4, dv=3, B_=1, H_=2)
+    do = np.random.default_rng(524).standard_normal(v.shape)
+    a = oracle.recurrent_bwd(q, k, v, la, beta, S0, do, ckpt=1)
+    b = oracle.recurrent_bwd(q, k, v, la, beta, S0, do, ckpt=64)
+    for n in a:
+        assert np.array_equal(a[n], b[n])
