@@ -416,8 +416,9 @@ def time_widened(args, ctx, kda, I, pf, peaks):
     """The widened rows, each on a workload of the headline's size:
     packed variable-length sequences (about 32K tokens in 32 sequences of
     mixed lengths, H32 d128, strong decay), the four variants on the
-    B4 H32 T8192 inputs, and the B1 H32 T131072 long-context prefill with
-    and without the chunk-parallel segment scan. Tokens/s and the HBM roofline fraction of each
+    B4 H32 T8192 inputs, the B1 H32 T131072 long-context prefill with
+    and without the chunk-parallel segment scan, and the backward pass on
+    the B4 H32 T8192 inputs. Tokens/s and the HBM roofline fraction of each
     (algorithmic bytes: q, k, v, the gate as the variant reads it, beta, o,
     and the states)."""
     torch = ctx.torch
@@ -500,6 +501,28 @@ def time_widened(args, ctx, kda, I, pf, peaks):
                           "steps": 3, "roofline_frac": gbs / hbm, "achieved_gbs": gbs, "workspace_bytes": wsb}
     out["long_context"] = long_ctx
     del xl, ol, Sl
+    # backward (gradients of o and S_T) on the headline inputs
+    gb = torch.Generator(device=ctx.dev)
+    gb.manual_seed(cfg.seed + 77 + 1000 * ctx.rank)
+    dO = torch.randn(cfg.B, cfg.T, cfg.H, cfg.dv, device=ctx.dev, generator=gb).bfloat16()
+    dST = torch.randn(cfg.B, cfg.H, cfg.dk, cfg.dv, device=ctx.dev, generator=gb)
+    wbb = int(kda.load().kda_chunk_bwd_workspace_size(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv))
+    wsb = torch.empty(wbb, dtype=torch.uint8, device=ctx.dev)
+
+    def run_b():
+        kda.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], dO, dST, workspace=wsb,
+                      stream=ctx.stream)
+    ms = _time_calls(ctx, run_b, 3, 3)
+    ntok = cfg.B * cfg.T
+    # read q, k, v, log_alpha, beta, dO; write dq, dk, dv, dlog_alpha, dbeta; dS_T read, dS0 written
+    nbytes = (5 * 256 + 2 + 4 * 256 + 2) * ntok * cfg.H + 2 * pf.ST.numel() * 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out["backward"] = {"workload": cfg.name, "kernel": "chunk_bwd_kernel", "value": ctx.world * ntok / (ms * 1e-3),
+                       "unit": "tokens/s", "ms_per_step": ms, "steps": 3, "workspace_bytes": wbb,
+                       "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                                    "algorithmic_bytes_per_launch": nbytes},
+                       "note": "fp32 SIMT, one CTA per (batch, head): latency bound"}
+    del dO, dST, wsb
     if pf.use_tc and kda.workspace_status(pf.ws, ctx.stream) != 0:
         raise RuntimeError("device-side timeout reported by the prefill kernel")
     return out

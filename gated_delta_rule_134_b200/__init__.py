@@ -10,7 +10,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["load", "chunk_fwd", "chunk_fwd_varlen", "chunk_fwd_noalloc", "decode_step", "workspace_size", "workspace_status", "KDAError",
+__all__ = ["load", "chunk_fwd", "chunk_fwd_varlen", "chunk_bwd", "chunk_fwd_noalloc", "decode_step", "workspace_size", "workspace_status", "KDAError",
            "library_path", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -72,6 +72,10 @@ def load(build_if_stale: bool = True):
     lib.kda_decode_step_v.restype = I
     lib.kda_chunk_fwd_varlen.argtypes = [P] * 9 + [I] * 9 + [P, Z, I, P]
     lib.kda_chunk_fwd_varlen.restype = I
+    lib.kda_chunk_bwd_workspace_size.argtypes = [I] * 5
+    lib.kda_chunk_bwd_workspace_size.restype = Z
+    lib.kda_chunk_bwd.argtypes = [P] * 14 + [I] * 8 + [P, Z, P]
+    lib.kda_chunk_bwd.restype = I
     _lib = lib
     return lib
 
@@ -203,6 +207,46 @@ def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, chunk: in
                                     GATES[gate], _ptr(workspace), ws_len, _ALGO[algo], _stream(stream))
     _check("kda_chunk_fwd_varlen", code)
     return o, S_T
+
+
+def chunk_bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None, *, erase: bool = True, gate: str = "channel",
+              want_dS0: bool = True, workspace=None, stream=None) -> dict:
+    """kda_chunk_bwd: gradients of a loss with dL/do = dO [B,T,H,dv] and
+    dL/dS_T = dS_T [B,H,dk,dv] (None: 0). Inputs as for chunk_fwd. Returns
+    dict dq, dk, dv, dlog_alpha (None without a gate), dbeta, dS0 (None
+    unless want_dS0)."""
+    import torch
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt, dev = q.dtype, q.device
+    _need(q, "q", (B, T, H, dk), dt, dev)
+    _need(k, "k", (B, T, H, dk), dt, dev)
+    gshape = _gate_shape(gate, (B, T, H), dk)
+    if gshape is not None:
+        _need(log_alpha, "log_alpha", gshape, dt, dev)
+    _need(v, "v", (B, T, H, dv), dt, dev)
+    _need(beta, "beta", (B, T, H), dt, dev)
+    _need(dO, "dO", (B, T, H, dv), dt, dev)
+    if S0 is not None:
+        _need(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    if dS_T is not None:
+        _need(dS_T, "dS_T", (B, H, dk, dv), torch.float32, dev)
+    g = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+         "dlog_alpha": None if gshape is None else torch.empty(gshape, dtype=dt, device=dev),
+         "dbeta": torch.empty_like(beta),
+         "dS0": torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev) if want_dS0 else None}
+    ws_bytes = int(lib.kda_chunk_bwd_workspace_size(B, T, H, dk, dv))
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    la = log_alpha if gshape is not None else None
+    code = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0), _ptr(dO), _ptr(dS_T),
+                             _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]),
+                             _ptr(g["dS0"]), B, T, H, dk, dv, _DTYPE[_dtype_of(q)], int(bool(erase)), GATES[gate],
+                             _ptr(workspace), ws_len, _stream(stream))
+    _check("kda_chunk_bwd", code)
+    return g
 
 
 def workspace_status(workspace, stream=None) -> int:

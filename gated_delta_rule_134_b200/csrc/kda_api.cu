@@ -175,4 +175,44 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
                              stream);
 }
 
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
+    if (B < 0 || T < 0 || H < 0 || !head_dims_ok(dk, dv)) return 0;
+    return kda::chunk_bwd_workspace_bytes(B, T, H, dk);
+}
+
+kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                           const float* S0, const void* dO, const float* dS_T, void* d_q, void* d_k, void* d_v,
+                           void* d_log_alpha, void* d_beta, float* d_S0, int B, int T, int H, int dk, int dv,
+                           kda_dtype_t dtype, int erase, kda_gate_t gate, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (!head_dims_ok(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if ((long long)B * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    if (erase != 0 && erase != 1) return KDA_ERR_INVALID_ARG;
+    if (gate < KDA_GATE_CHANNEL || gate > KDA_GATE_NONE) return KDA_ERR_INVALID_ARG;
+    if ((long long)B * T * H > 0) {
+        const void* req[] = {q, k, v, beta, dO, d_q, d_k, d_v, d_beta};
+        for (const void* p : req)
+            if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+        if (gate != KDA_GATE_NONE &&
+            (log_alpha == nullptr || !aligned16(log_alpha) || d_log_alpha == nullptr || !aligned16(d_log_alpha)))
+            return KDA_ERR_INVALID_ARG;
+    }
+    const float* opt[] = {S0, dS_T, d_S0};
+    for (const float* p : opt)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    const size_t need = kda::chunk_bwd_workspace_bytes(B, T, H, dk);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+        return KDA_ERR_INVALID_ARG;
+    if ((long long)B * H == 0) return KDA_OK;
+    kda::BwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.dO = dO; a.S0 = S0; a.dST = dS_T;
+    a.g_q = d_q; a.g_k = d_k; a.g_v = d_v; a.g_log_alpha = d_log_alpha; a.g_beta = d_beta; a.g_S0 = d_S0;
+    a.B = B; a.T = T; a.H = H; a.d = dk; a.bf16 = dtype == KDA_BF16; a.erase = erase; a.gate = (int)gate;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+    const cudaError_t err = kda::launch_chunk_bwd(a, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -37,4 +37,17 @@ bool chunk_tc_supported(const ChunkArgs& a);
 size_t chunk_tc_workspace_bytes(const ChunkArgs& a, int scan_mode);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, int scan_mode, cudaStream_t stream);
 
+// Backward of the chunkwise prefill (SIMT fp32, any variant, dk = dv = d in {64, 128}).
+struct BwdArgs {
+    const void *q, *k, *v, *log_alpha, *beta, *dO;
+    const float *S0, *dST;
+    void *g_q, *g_k, *g_v, *g_log_alpha, *g_beta;  // gradients (input dtype)
+    float* g_S0;
+    int B, T, H, d, bf16, erase, gate;
+    void* workspace;
+    size_t workspace_bytes;
+};
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int d);
+cudaError_t launch_chunk_bwd(const BwdArgs& a, cudaStream_t stream);
+
 }  // namespace kda

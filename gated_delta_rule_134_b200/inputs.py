@@ -205,3 +205,13 @@ def varlen_inputs(cfg: PrefillConfig, lengths) -> dict:
             S0[n, h] = x["S0"]
     return dict(q=q, k=k, v=v, log_alpha=la, beta=beta, S0=S0 if cfg.s0_std > 0 else None,
                 cu_seqlens=torch.tensor(cu, dtype=torch.int32))
+
+
+def bwd_cotangents(cfg: PrefillConfig, with_dST: bool = True) -> dict:
+    """Seeded upstream gradients for a backward pass over cfg's prefill:
+    dO ~ N(0, 1) [B,T,H,dv] in cfg's dtype, dS_T ~ N(0, 1) fp32 [B,H,dk,dv]
+    (None without it)."""
+    g = _gen(cfg.seed, 9)
+    dO = torch.randn(cfg.B, cfg.T, cfg.H, cfg.dv, generator=g).to(cfg.torch_dtype)
+    dST = torch.randn(cfg.B, cfg.H, cfg.dk, cfg.dv, generator=g) if with_dST else None
+    return {"dO": dO, "dST": dST}

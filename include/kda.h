@@ -169,6 +169,42 @@ kda_status_t kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
                                   size_t workspace_bytes, kda_algo_t algo, void *stream);
 
 /*
+ * Backward of the prefill (training): gradients of a loss L given
+ * dO = dL/do and dS_T = dL/dS_T, for any variant.
+ *
+ * The pages give no backward pass ("Decoding Hybrid Attention Architectures",
+ * section 5, names training throughput as a goal). This is the chain rule
+ * through the update of section 3.4, in the same chunked form as the forward
+ * pass: a forward sweep keeps the state every 64 tokens, a backward sweep
+ * walks 8-token chunks in reverse with the adjoint of the state on chip. The
+ * decay gradient comes from an identity of the update (a shift of log a at
+ * token t equals a rescaling of every later query and key), as one reverse
+ * running sum per channel.
+ *
+ *   inputs as for kda_chunk_fwd_v (q, k, log_alpha, v, beta, S0 may be NULL)
+ *   dO          : [B, T, H, dv]  dtype
+ *   dS_T        : [B, H, dk, dv] float, or NULL (zero)
+ *   d_q, d_k    : [B, T, H, dk]  dtype, written
+ *   d_v         : [B, T, H, dv]  dtype, written
+ *   d_log_alpha : shape of log_alpha, written (NULL allowed for KDA_GATE_NONE)
+ *   d_beta      : [B, T, H]      dtype, written
+ *   d_S0        : [B, H, dk, dv] float, written; NULL: not computed
+ *   dk == dv in {64, 128}
+ *   workspace   : device scratch of kda_chunk_bwd_workspace_size(...) bytes,
+ *                 16-byte aligned: fp32 [dk][dv] states, one per 64 tokens
+ *                 and 8 per (batch, head) for the block being reversed
+ * Arithmetic: fp32 throughout (exact per-pair decay exponentials, all with
+ * non-positive exponents), gradients rounded to dtype once. One CTA per
+ * (batch, head): the work is latency bound, not tuned.
+ */
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv);
+kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,
+                           const float *S0, const void *dO, const float *dS_T, void *d_q, void *d_k, void *d_v,
+                           void *d_log_alpha, void *d_beta, float *d_S0, int B, int T, int H, int dk, int dv,
+                           kda_dtype_t dtype, int erase, kda_gate_t gate, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/*
  * Device-side status left in `workspace` by the last kda_chunk_fwd_ex that
  * used it: synchronises `stream`, then returns KDA_OK, or KDA_ERR_TIMEOUT if
  * a bounded wait inside a kernel gave up (that kernel's outputs are then

@@ -198,3 +198,46 @@ def test_scan_workspace_sizes():
     # too short to split (2 chunks): plain
     assert kda.workspace_size(1, 100, 1, 128, 128, 64, "bf16", "tc_scan") == 256
     assert kda.workspace_size(1, 1000, 1, 128, 128, 64, "bf16", "auto") == 256
+
+
+def _bwd(lib, ptrs, ws=None, ws_bytes=0, gate=0, erase=1, d=64):
+    # q, k, v, log_alpha, beta, S0, dO, dS_T, d_q, d_k, d_v, d_log_alpha, d_beta, d_S0
+    return lib.kda_chunk_bwd(*ptrs, 1, 8, 1, d, d, 1, erase, gate, ws, ws_bytes, None)
+
+
+def _bwd_good():
+    p = [ctypes.c_void_p(0x1000 * (i + 1)) for i in range(14)]
+    p[5] = p[7] = p[13] = None  # S0, dS_T, d_S0 optional
+    return p
+
+
+def test_bwd_workspace_size():
+    d = 128
+    # one fp32 [d][d] state per 64 tokens plus 8 per (batch, head)
+    assert kda.load().kda_chunk_bwd_workspace_size(2, 130, 3, d, d) == 2 * 3 * (3 + 8) * d * d * 4
+    assert kda.load().kda_chunk_bwd_workspace_size(1, 8, 1, 96, 96) == 0
+
+
+@pytest.mark.parametrize("which", [0, 1, 2, 3, 4, 6, 8, 9, 10, 11, 12])
+def test_bwd_rejects_null(which):
+    lib = kda.load()
+    p = _bwd_good()
+    p[which] = None
+    ws_bytes = lib.kda_chunk_bwd_workspace_size(1, 8, 1, 64, 64)
+    assert _bwd(lib, p, ctypes.c_void_p(0x100000), ws_bytes) == 1
+
+
+def test_bwd_rejects_small_workspace_and_bad_switches():
+    lib = kda.load()
+    ws_bytes = lib.kda_chunk_bwd_workspace_size(1, 8, 1, 64, 64)
+    assert _bwd(lib, _bwd_good(), ctypes.c_void_p(0x100000), ws_bytes - 4) == 1
+    assert _bwd(lib, _bwd_good(), None, 0) == 1
+    assert _bwd(lib, _bwd_good(), ctypes.c_void_p(0x100000), ws_bytes, gate=3) == 1
+    assert _bwd(lib, _bwd_good(), ctypes.c_void_p(0x100000), ws_bytes, erase=2) == 1
+    assert _bwd(lib, _bwd_good(), ctypes.c_void_p(0x100000), ws_bytes, d=96) == 2
+    p = _bwd_good()
+    p[3] = p[11] = None  # no gate: log_alpha and its gradient may be NULL
+    # (valid arguments would launch: check only that validation passes the gate rule by
+    # making another required pointer misaligned)
+    p[0] = ctypes.c_void_p(0x1001)
+    assert _bwd(lib, p, ctypes.c_void_p(0x100000), ws_bytes, gate=2) == 1

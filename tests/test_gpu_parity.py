@@ -482,3 +482,98 @@ def test_scan_varlen_unsupported(cuda_lib):
     with pytest.raises(RuntimeError):
         cuda_lib.chunk_fwd_varlen(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["cu_seqlens"], x["S0"],
                                   algo="tc_scan")
+
+
+# ---------------------------------------------------------------- backward (kda_chunk_bwd)
+
+
+BWD_NAMES = ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0")
+
+
+def check_bwd(kda, cfg, erase=True, gate="channel", with_dST=True):
+    x = _variant_inputs(cfg, gate)
+    c = I.bwd_cotangents(cfg, with_dST)
+    xd, cd = to_dev(x), to_dev(c)
+    g = kda.chunk_bwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["S0"], cd["dO"], cd["dST"],
+                      erase=erase, gate=gate)
+    torch.cuda.synchronize()
+    ref = oracle.recurrent_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], c["dO"], c["dST"],
+                               erase=erase, gate=gate)
+    errs = {}
+    for n in BWD_NAMES:
+        if ref[n] is None:
+            assert g[n] is None
+            continue
+        got = g[n].float().cpu().numpy()
+        assert np.isfinite(got).all(), n
+        errs[n] = rel_err(got, ref[n]) if got.size else 0.0
+    print(f"PARITY bwd {cfg.name} erase={int(erase)} gate={gate} " + " ".join(f"{n}={e:.2e}" for n, e in errs.items()))
+    for n, e in errs.items():
+        assert e <= TOL[cfg.dtype], (cfg.name, erase, gate, n, e)
+    return g
+
+
+@pytest.mark.parametrize("T", [1, 9, 64, 77, 200])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_bwd_small(cuda_lib, dtype, d, T):
+    check_bwd(cuda_lib, small_cfg(dtype, d, 64, T, B=2, H=2, s0=0.3, seed=70 + T))
+
+
+@pytest.mark.parametrize("erase,gate", VARIANTS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_bwd_variants(cuda_lib, dtype, erase, gate):
+    d = 64 if dtype == "f32" else 128
+    check_bwd(cuda_lib, small_cfg(dtype, d, 64, 150, B=1, H=2, s0=0.3, seed=71), erase, gate)
+
+
+@pytest.mark.parametrize("la", [(0.5, 6.0), (0.0, 1e-4)])
+def test_bwd_decay_extremes(cuda_lib, la):
+    check_bwd(cuda_lib, small_cfg("f32", 128, 64, 130, B=1, H=2, la=la, s0=0.3, seed=72))
+
+
+def test_bwd_no_state_inputs(cuda_lib):
+    check_bwd(cuda_lib, small_cfg("bf16", 128, 64, 90, B=1, H=3, s0=0.0, seed=73), with_dST=False)
+
+
+def test_bwd_empty_sequence(cuda_lib):
+    """T = 0: dS0 = dS_T, nothing else is written."""
+    cfg = small_cfg("f32", 64, 64, 0, B=1, H=2, s0=0.3, seed=74)
+    x = to_dev(I.prefill_inputs(cfg))
+    c = to_dev(I.bwd_cotangents(cfg))
+    g = cuda_lib.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], c["dO"], c["dST"])
+    torch.cuda.synchronize()
+    assert torch.equal(g["dS0"], c["dST"])
+
+
+def test_bwd_deterministic(cuda_lib):
+    cfg = small_cfg("bf16", 128, 64, 300, B=2, H=2, s0=0.3, seed=75)
+    x = to_dev(I.prefill_inputs(cfg))
+    c = to_dev(I.bwd_cotangents(cfg))
+    outs = [cuda_lib.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], c["dO"], c["dST"])
+            for _ in range(2)]
+    torch.cuda.synchronize()
+    for n in BWD_NAMES:
+        assert torch.equal(outs[0][n], outs[1][n]), n
+
+
+def test_bwd_b4_h32_t8k_sampled(cuda_lib):
+    """The B4 H32 T8192 strong-decay workload; two (batch, head) slices against
+    the oracle (heads are independent, so the sample is exact)."""
+    cfg = I.B4_H32_T8K
+    x = to_dev(I.prefill_inputs(cfg))
+    c = to_dev(I.bwd_cotangents(cfg))
+    g = cuda_lib.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], c["dO"], c["dST"])
+    torch.cuda.synchronize()
+    cc = I.bwd_cotangents(cfg)
+    for b, h in [(0, 3), (3, 30)]:
+        xs = I.prefill_inputs(cfg, heads=[(b, h)])
+        dO = cc["dO"][b:b + 1, :, h:h + 1]
+        dST = cc["dST"][b:b + 1, h:h + 1]
+        ref = oracle.recurrent_bwd(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["beta"], xs["S0"], dO, dST)
+        for n in BWD_NAMES:
+            got = g[n][b, :, h] if n not in ("dS0",) else g[n][b, h]
+            want = ref[n][0, :, 0] if n != "dS0" else ref[n][0, 0]
+            e = rel_err(got.float().cpu().numpy(), want)
+            print(f"PARITY bwd full b={b} h={h} {n}={e:.2e}")
+            assert e <= TOL["bf16"], (b, h, n, e)
