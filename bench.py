@@ -133,7 +133,9 @@ KERNEL_SOURCES = {
     "decode": ["kda_decode.cu", "kda_common.cuh"],
     "simt": ["kda_chunk_simt.cu", "kda_common.cuh"],
     "tc": ["kda_chunk_tc.cu", "kda_common.cuh", "kda_sm100.cuh"],
+    "bwd": ["kda_chunk_bwd.cu", "kda_common.cuh"],
 }
+WIDENED = ("varlen", "variants", "long_context", "backward")
 
 
 def kernel_source_digest(kind: str) -> str:
@@ -421,11 +423,24 @@ def time_widened(args, ctx, kda, I, pf, peaks):
     the B4 H32 T8192 inputs. Tokens/s and the HBM roofline fraction of each
     (algorithmic bytes: q, k, v, the gate as the variant reads it, beta, o,
     and the states)."""
-    torch = ctx.torch
     steps = max(3, min(args.steps, 10))
     hbm = peaks["hbm_gbs"]
     out = {}
-    # packed sequences
+    if "varlen" in args.parts:
+        out["varlen"] = _time_varlen(args, ctx, kda, I, steps, hbm)
+    if "variants" in args.parts:
+        out["variants"] = _time_variants(args, ctx, kda, pf, steps, hbm)
+    if "long_context" in args.parts:
+        out["long_context"] = _time_long_context(ctx, kda, I, hbm)
+    if "backward" in args.parts:
+        out["backward"] = _time_backward(ctx, kda, pf, hbm)
+    if pf.use_tc and kda.workspace_status(pf.ws, ctx.stream) != 0:
+        raise RuntimeError("device-side timeout reported by the prefill kernel")
+    return out
+
+
+def _time_varlen(args, ctx, kda, I, steps, hbm):
+    torch = ctx.torch
     lengths = I.varlen_lengths(32, 1024, seed=48 + ctx.rank)
     vcfg = I.B4_H32_T8K.replace(seed=48 + ctx.rank)
     xv = {k: (None if v is None else v.to(ctx.dev)) for k, v in I.varlen_inputs(vcfg, lengths).items()}
@@ -440,12 +455,13 @@ def time_widened(args, ctx, kda, I, pf, peaks):
     ms = _time_calls(ctx, run_v, args.warmup, steps)
     nbytes = BYTES_PER_TOKEN_HEAD * TT * H + Sv.numel() * 4 + 4 * (N + 1)
     gbs = nbytes / (ms * 1e-3) / 1e9
-    out["varlen"] = {"workload": f"packed_n{N}_total{TT}_h32_d128_bf16_strong_decay", "lengths": "U(1, 2047)",
-                     "value": ctx.world * TT / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
-                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                                  "algorithmic_bytes_per_launch": nbytes}}
-    del xv, ov, Sv
-    # variants on the headline inputs
+    return {"workload": f"packed_n{N}_total{TT}_h32_d128_bf16_strong_decay", "lengths": "U(1, 2047)",
+            "value": ctx.world * TT / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "algorithmic_bytes_per_launch": nbytes}}
+
+
+def _time_variants(args, ctx, kda, pf, steps, hbm):
     x = pf.x
     cfg = pf.cfg
     la_tok = x["log_alpha"][..., 0].contiguous()
@@ -466,8 +482,12 @@ def time_widened(args, ctx, kda, I, pf, peaks):
         gbs = nbytes / (ms * 1e-3) / 1e9
         res[name] = {"erase": erase, "gate": gate, "value": ctx.world * ntok / (ms * 1e-3), "unit": "tokens/s",
                      "ms_per_step": ms, "roofline_frac": gbs / hbm, "achieved_gbs": gbs}
-    out["variants"] = {"workload": cfg.name, "steps": steps, **res}
-    # long context, few heads: one pass per sequence against the segment scan
+    return {"workload": cfg.name, "steps": steps, **res}
+
+
+def _time_long_context(ctx, kda, I, hbm):
+    """B1 H32 T131072: one pass per sequence against the segment scan."""
+    torch = ctx.torch
     lc = I.B1_H32_T128K
     g = torch.Generator(device=ctx.dev)
     g.manual_seed(lc.seed + 1000 * ctx.rank)
@@ -499,9 +519,14 @@ def time_widened(args, ctx, kda, I, pf, peaks):
         gbs = nbytes / (ms * 1e-3) / 1e9
         long_ctx[algo] = {"value": ctx.world * ntok / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
                           "steps": 3, "roofline_frac": gbs / hbm, "achieved_gbs": gbs, "workspace_bytes": wsb}
-    out["long_context"] = long_ctx
     del xl, ol, Sl
-    # backward (gradients of o and S_T) on the headline inputs
+    return long_ctx
+
+
+def _time_backward(ctx, kda, pf, hbm):
+    """Gradients of o and S_T on the prefill inputs (kda_chunk_bwd)."""
+    torch = ctx.torch
+    x, cfg = pf.x, pf.cfg
     gb = torch.Generator(device=ctx.dev)
     gb.manual_seed(cfg.seed + 77 + 1000 * ctx.rank)
     dO = torch.randn(cfg.B, cfg.T, cfg.H, cfg.dv, device=ctx.dev, generator=gb).bfloat16()
@@ -517,15 +542,12 @@ def time_widened(args, ctx, kda, I, pf, peaks):
     # read q, k, v, log_alpha, beta, dO; write dq, dk, dv, dlog_alpha, dbeta; dS_T read, dS0 written
     nbytes = (5 * 256 + 2 + 4 * 256 + 2) * ntok * cfg.H + 2 * pf.ST.numel() * 4
     gbs = nbytes / (ms * 1e-3) / 1e9
-    out["backward"] = {"workload": cfg.name, "kernel": "chunk_bwd_kernel", "value": ctx.world * ntok / (ms * 1e-3),
-                       "unit": "tokens/s", "ms_per_step": ms, "steps": 3, "workspace_bytes": wbb,
-                       "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                                    "algorithmic_bytes_per_launch": nbytes},
-                       "note": "fp32 SIMT, one CTA per (batch, head): latency bound"}
     del dO, dST, wsb
-    if pf.use_tc and kda.workspace_status(pf.ws, ctx.stream) != 0:
-        raise RuntimeError("device-side timeout reported by the prefill kernel")
-    return out
+    return {"workload": pf.name, "kernel": "chunk_bwd_kernel", "value": ctx.world * ntok / (ms * 1e-3),
+            "unit": "tokens/s", "ms_per_step": ms, "steps": 3, "workspace_bytes": wbb,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "algorithmic_bytes_per_launch": nbytes, "traffic": recorded_traffic(pf.name, "bwd")},
+            "note": "fp32 SIMT, one CTA per (batch, head): latency bound"}
 
 
 def main():
@@ -540,9 +562,12 @@ def main():
     ap.add_argument("--profile-T", type=int, default=None,
                     help="shorter sequence for profiler captures (the printed line is then not a bench value)")
     ap.add_argument("--parts", default="prefill,e2e,decode,widened",
-                    help="comma list of prefill, e2e, decode, widened (profiling runs select one)")
+                    help="comma list of prefill, e2e, decode, widened (= varlen, variants, long_context, "
+                         "backward) (profiling runs select one)")
     args = ap.parse_args()
     args.parts = set(args.parts.split(","))
+    if "widened" in args.parts:
+        args.parts |= set(WIDENED)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
@@ -559,7 +584,7 @@ def main():
             "vs_baseline": None, "dtype": None, "data": "synthetic", "config": None, "roofline": None,
             "cpu_baseline": None, "e2e": None, "gpu_launches": None, "clocks": None, "decode": None,
             "widened": None}
-    if args.parts & {"prefill", "e2e", "widened"}:
+    if args.parts & ({"prefill", "e2e"} | set(WIDENED)):
         pf = Prefill(ctx, kda, I, args.algo, args.profile_T)
         line["config"] = {"workload": pf.name, "B": pf.cfg.B, "H": pf.cfg.H, "T": pf.cfg.T, "dk": pf.cfg.dk,
                           "dv": pf.cfg.dv, "chunk": pf.cfg.C, "algo": pf.algo_name,
@@ -572,7 +597,7 @@ def main():
                         clocks=clocks, gpu_launches=pf.launches_per_step * args.steps)
         if "e2e" in args.parts:
             line["e2e"] = time_e2e(args, ctx, pf)
-        if "widened" in args.parts:
+        if args.parts & set(WIDENED):
             line["widened"] = time_widened(args, ctx, kda, I, pf, peaks)
         del pf
     if "decode" in args.parts:
