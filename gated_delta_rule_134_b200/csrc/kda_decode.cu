@@ -20,11 +20,14 @@ namespace kda {
 constexpr int kDecodeThreads = 128;
 constexpr int kDecodeCols = 32;  // value columns per CTA (8 threads x float4)
 
-template <typename T, int DK>
-__global__ void __launch_bounds__(kDecodeThreads)
+// ERASE / GATE: the variant switches, compile-time so each variant is its own
+// kernel and the KDA instance carries no variant branches.
+template <typename T, int DK, int ERASE, int GATE>
+__global__ void __launch_bounds__(kDecodeThreads, 8)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const T* __restrict__ log_alpha, const T* __restrict__ beta, const float* S_in,
-                   float* S_out, T* __restrict__ o, int dv, int erase, int gate) {
+                   float* S_out, T* __restrict__ o, int dv) {
+    constexpr int erase = ERASE, gate = GATE;
     constexpr int RG = kDecodeThreads / 8;  // 16 row groups
     constexpr int ROWS = DK / RG;           // rows per thread
     const int nslices = dv / kDecodeCols;
@@ -118,10 +121,20 @@ template <typename T, int DK>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* la, const void* beta,
                                    const float* S_in, float* S_out, void* o, int N, int H, int dv, int erase,
                                    int gate, cudaStream_t stream) {
-    const long blocks = (long)N * H * (dv / kDecodeCols);
-    decode_step_kernel<T, DK><<<(unsigned)blocks, kDecodeThreads, 0, stream>>>(
-        (const T*)q, (const T*)k, (const T*)v, (const T*)la, (const T*)beta, S_in, S_out, (T*)o, dv, erase, gate);
-    return cudaGetLastError();
+    const unsigned blocks = (unsigned)((long)N * H * (dv / kDecodeCols));
+    auto go = [&](auto kern) {
+        kern<<<blocks, kDecodeThreads, 0, stream>>>((const T*)q, (const T*)k, (const T*)v, (const T*)la,
+                                                    (const T*)beta, S_in, S_out, (T*)o, dv);
+        return cudaGetLastError();
+    };
+    if (erase) {
+        if (gate == 0) return go(decode_step_kernel<T, DK, 1, 0>);
+        if (gate == 1) return go(decode_step_kernel<T, DK, 1, 1>);
+        return go(decode_step_kernel<T, DK, 1, 2>);
+    }
+    if (gate == 0) return go(decode_step_kernel<T, DK, 0, 0>);
+    if (gate == 1) return go(decode_step_kernel<T, DK, 0, 1>);
+    return go(decode_step_kernel<T, DK, 0, 2>);
 }
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* la, const void* beta,
