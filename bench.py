@@ -212,21 +212,26 @@ def run_reference(args):
 
 
 class Ctx:
-    """Per-process distributed context (one rank per GPU)."""
+    """Per-process distributed context (one rank per GPU). The path shards by
+    replicas: ranks exchange nothing on the data path, only the barrier and
+    the max-over-ranks of the timings. backend="gloo" runs the same host logic
+    on CPU (tests)."""
 
-    def __init__(self):
+    def __init__(self, backend: str = "nccl", timeout_s: float = 120.0):
         import torch
         import torch.distributed as dist
         self.torch, self.dist = torch, dist
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
-        torch.cuda.set_device(self.local)
+        cuda = backend == "nccl"
+        if cuda:
+            torch.cuda.set_device(self.local)
         if self.world > 1:
             import datetime
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        self.dev = torch.device("cuda", self.local)
-        self.stream = torch.cuda.current_stream(self.dev)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+        self.dev = torch.device("cuda", self.local) if cuda else torch.device("cpu")
+        self.stream = torch.cuda.current_stream(self.dev) if cuda else None
 
     def barrier(self):
         if self.world > 1:
@@ -244,6 +249,17 @@ class Ctx:
             self.dist.destroy_process_group()
 
 
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Each replica draws its own inputs of the same workload."""
+    return base_seed + 1000 * rank
+
+
+def whole_job_rate(world: int, units_per_rank: float, ms_max: float) -> float:
+    """Units per second of the whole job: every rank processed units_per_rank
+    in at most ms_max milliseconds (the max over ranks)."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
 class Prefill:
     """The B=4, H=32, T=8192 bf16 prefill workload resident on this rank's GPU."""
 
@@ -251,7 +267,7 @@ class Prefill:
         torch = ctx.torch
         self.kda, self.ctx, self.algo = kda, ctx, algo
         base = I.B4_H32_T8K
-        self.cfg = cfg = base.replace(seed=base.seed + 1000 * ctx.rank, T=profile_T or base.T)
+        self.cfg = cfg = base.replace(seed=replica_seed(base.seed, ctx.rank), T=profile_T or base.T)
         self.name = base.name if not profile_T else f"{base.name}_profile_T{profile_T}"
         self.x = {k: (None if v is None else v.to(ctx.dev)) for k, v in I.prefill_inputs(cfg).items()}
         B, T, H, dk, dv = cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv
@@ -593,7 +609,7 @@ def main():
         line["dtype"] = "bf16" if pf.use_tc else "f32"
         if "prefill" in args.parts:
             ms, roof, clocks = time_prefill(args, ctx, pf, peaks, peak_kind)
-            line.update(value=ctx.world * pf.tokens_per_step / (ms * 1e-3), ms_per_step=ms, roofline=roof,
+            line.update(value=whole_job_rate(ctx.world, pf.tokens_per_step, ms), ms_per_step=ms, roofline=roof,
                         clocks=clocks, gpu_launches=pf.launches_per_step * args.steps)
         if "e2e" in args.parts:
             line["e2e"] = time_e2e(args, ctx, pf)
