@@ -563,7 +563,7 @@ def _time_backward(ctx, kda, pf, hbm):
             "unit": "tokens/s", "ms_per_step": ms, "steps": 3, "workspace_bytes": wbb,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                          "algorithmic_bytes_per_launch": nbytes, "traffic": recorded_traffic(pf.name, "bwd")},
-            "note": "fp32 SIMT, one CTA per (batch, head): latency bound"}
+            "note": "fp32 (tf32x3 warp MMAs for the products), one CTA per (batch, head): barrier and latency bound"}
 
 
 def main():

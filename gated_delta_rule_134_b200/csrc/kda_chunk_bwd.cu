@@ -29,13 +29,16 @@
 //   dlog_a_tau = sum_{t >= tau} (q dq - k dkw + k dkr)_t + rowsum(dS_T * S_T),
 // one reverse running sum per channel (a scalar gate sums it over channels).
 //
-// Design: one CTA per (batch, head), fp32 throughout, the state S and the
-// adjoint F ([dk][dv], rows padded by one float against bank conflicts) in
-// shared memory, chunks of 8 tokens with every decay factor an exact
-// exponential of a non-positive exponent. A forward sweep stores the state
-// every 8 chunks (64 tokens); the backward sweep recomputes the 8 entry
-// states of each such block into a per-CTA ring in global memory (L2) and
-// then walks the block in reverse.
+// Design: one CTA per (batch, head), the state S and the adjoint F
+// ([dk][dv] fp32, rows padded by 4 floats) in shared memory, chunks of 8
+// tokens with every decay factor an exact exponential of a non-positive
+// exponent. The six [8 x d] x [d x d] products per chunk run on warp-level
+// tensor-core MMAs (m16n8k8) with each fp32 operand split into a tf32 high
+// part and a tf32 remainder: hi*hi + hi*lo + lo*hi keeps the product at about
+// fp32 accuracy. A forward sweep stores the state every 8 chunks (64
+// tokens); the backward sweep recomputes the 8 entry states and deltas of
+// each such block into a per-CTA ring in global memory (L2) and then walks the
+// block in reverse.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -51,23 +54,26 @@ __host__ __device__ constexpr int pidx(int r, int s) { return r * (r + 1) / 2 + 
 
 template <int D>
 struct BwdLayout {  // offsets in floats
-    static constexpr int LD = D + 1;
+    static constexpr int LD = D + 4;          // row stride of S and F
+    static constexpr int TD = D + 4;          // row stride of the [8][D] tiles
+    static constexpr int TILE = kBC * TD;
     static constexpr int S = 0;
     static constexpr int F = S + D * LD;
     static constexpr int Q = F + D * LD;
-    static constexpr int K = Q + kBC * D;
-    static constexpr int G = K + kBC * D;     // log a, then inclusive prefix sums
-    static constexpr int GAM = G + kBC * D;   // e^{G}
-    static constexpr int V = GAM + kBC * D;
-    static constexpr int DO = V + kBC * D;
-    static constexpr int DL = DO + kBC * D;   // U, then delta
-    static constexpr int R = DL + kBC * D;    // W, then R, then S dO
-    static constexpr int X = R + kBC * D;     // k e^G / k e^{G_last-G}, X, then F delta
-    static constexpr int DD = X + kBC * D;    // d(delta)
-    static constexpr int DG = DD + kBC * D;   // S d(delta), then q dq - k dkw + k dkr
-    static constexpr int E = DG + kBC * D;    // [pair][D]: e^{G_r - G_s}
-    static constexpr int RED = E + kPairs * D;  // [kBT / D groups][8][D] partial sums
-    static constexpr int A0 = RED + kBT * kBC;
+    static constexpr int K = Q + TILE;
+    static constexpr int G = K + TILE;        // log a, then inclusive prefix sums
+    static constexpr int GAM = G + TILE;      // e^{G}
+    static constexpr int V = GAM + TILE;
+    static constexpr int DO = V + TILE;
+    static constexpr int DL = DO + TILE;      // U, then delta
+    static constexpr int R = DL + TILE;       // W, then R, then S dO
+    static constexpr int X = R + TILE;        // k e^G / k e^{G_last-G}, X, then F delta
+    static constexpr int DD = X + TILE;       // d(delta)
+    static constexpr int DG = DD + TILE;      // S d(delta), then q dq - k dkw + k dkr
+    static constexpr int E = DG + TILE;       // [pair][D]: e^{G_r - G_s}
+    static constexpr int RED = E + kPairs * D;  // [k-splits][8][D] partial sums
+    static constexpr int NKS = 256 / D;         // k-splits of a product over 16 warps
+    static constexpr int A0 = RED + NKS * kBC * D;
     static constexpr int P = A0 + 64;
     static constexpr int TM = P + 64;
     static constexpr int C1 = TM + 64;        // [r][s] delta_s . dO_r
@@ -77,12 +83,41 @@ struct BwdLayout {  // offsets in floats
     static constexpr int CARRY = BETA + kBC;  // running reverse sum of the decay gradient
     static constexpr int TOTAL = CARRY + D;
     static constexpr size_t BYTES = (size_t)TOTAL * sizeof(float);
+    static_assert(BYTES <= 232448, "shared memory budget");
 };
 
 __device__ __forceinline__ void pair_rs(int p, int& r, int& s) {
     r = 0;
     while (pidx(r + 1, 0) <= p) ++r;
     s = p - pidx(r, 0);
+}
+
+// fp32 -> (tf32 high part, tf32 remainder)
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+    const float rem = x - __uint_as_float(hi);
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(rem));
+}
+
+__device__ __forceinline__ void mma_16x8x8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// One 16 x 8 x 8 step at fp32 accuracy: A given by its four fp32 fragment
+// values, B by two.
+__device__ __forceinline__ void mma3_step(float (&d)[4], const float (&af)[4], float b0f, float b1f) {
+    uint32_t ah[4], al[4], bh0, bl0, bh1, bl1;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) split_tf32(af[e], ah[e], al[e]);
+    split_tf32(b0f, bh0, bl0);
+    split_tf32(b1f, bh1, bl1);
+    mma_16x8x8(d, al, bh0, bh1);
+    mma_16x8x8(d, ah, bl0, bl1);
+    mma_16x8x8(d, ah, bh0, bh1);
 }
 
 template <typename T, int D>
@@ -93,20 +128,23 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                  T* __restrict__ dv, T* __restrict__ dla, T* __restrict__ dbeta, float* __restrict__ dS0,
                  float* __restrict__ ckpt, float* __restrict__ ring, int Tlen, int H, int erase, int gate) {
     using L = BwdLayout<D>;
-    constexpr int LD = L::LD;
-    constexpr int NG = kBT / D;   // thread groups in the matrix-vector products
-    constexpr int RW = D / NG;    // rows (or columns) per group
+    constexpr int LD = L::LD, TD = L::TD, NKS = L::NKS;
+    constexpr int MT = D / 16;              // 16-row tiles of a product's output
+    constexpr int KSTEPS = D / 8 / NKS;     // 8-deep k steps per warp
     extern __shared__ float sm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g8 = lane >> 2, t4 = lane & 3;  // mma fragment coordinates
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const size_t tok0 = (size_t)b * Tlen;
     const int NB = (Tlen + kBC - 1) / kBC;
     const int NBLK = (NB + kBlk - 1) / kBlk;
     constexpr size_t kMat = (size_t)D * D;
+    constexpr size_t kRing = kMat + (size_t)kBC * D;  // ring slot: entry state, then delta
     float* ck = ckpt + (size_t)bh * NBLK * kMat;
-    float* rg = ring + (size_t)bh * kBlk * kMat;
+    float* rg = ring + (size_t)bh * kBlk * kRing;
     float* sS = sm + L::S;
     float* sF = sm + L::F;
+    auto tl = [&](int base, int r, int c) -> float& { return sm[base + r * TD + c]; };
 
     auto load_mat = [&](float* dst, const float* src) {
         for (int e = tid; e < D * D; e += kBT) dst[(e / D) * LD + e % D] = src ? src[e] : 0.f;
@@ -114,40 +152,78 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
     auto store_mat = [&](const float* src, float* dst) {
         for (int e = tid; e < D * D; e += kBT) dst[e] = src[(e / D) * LD + e % D];
     };
-    // out_v = sum_i x_v[i] M[i][.] (x from the left), 8 vectors; partials to RED
-    auto left_partials = [&](const float* M, const float* x) {
-        const int j = tid % D, g = tid / D;
-        float acc[kBC];
-#pragma unroll
-        for (int u = 0; u < kBC; ++u) acc[u] = 0.f;
-        for (int ii = 0; ii < RW; ++ii) {
-            const int i = g * RW + ii;
-            const float m = M[i * LD + j];
-#pragma unroll
-            for (int u = 0; u < kBC; ++u) acc[u] = fmaf(x[u * D + i], m, acc[u]);
+    // out_u[j] = sum_i x_u[i] M[i][j]  (x from the left), as out^T = M^T x^T:
+    // m = j, n = u, k = i. Warp w: output rows 16 (w % MT).., k split w / MT.
+    auto left_partials = [&](const float* M, int xb) {
+        const int j0 = 16 * (warp % MT), ks = warp / MT;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+        for (int st = 0; st < KSTEPS; ++st) {
+            const int i0 = 8 * (ks * KSTEPS + st);
+            const float af[4] = {M[(i0 + t4) * LD + j0 + g8], M[(i0 + t4) * LD + j0 + g8 + 8],
+                                 M[(i0 + t4 + 4) * LD + j0 + g8], M[(i0 + t4 + 4) * LD + j0 + g8 + 8]};
+            mma3_step(d, af, sm[xb + g8 * TD + i0 + t4], sm[xb + g8 * TD + i0 + t4 + 4]);
         }
-#pragma unroll
-        for (int u = 0; u < kBC; ++u) sm[L::RED + (g * kBC + u) * D + j] = acc[u];
+        float* red = sm + L::RED + ks * kBC * D;
+        red[(2 * t4) * D + j0 + g8] = d[0];
+        red[(2 * t4 + 1) * D + j0 + g8] = d[1];
+        red[(2 * t4) * D + j0 + g8 + 8] = d[2];
+        red[(2 * t4 + 1) * D + j0 + g8 + 8] = d[3];
     };
-    // out_v = M x_v (x from the right), 8 vectors; partials to RED
-    auto right_partials = [&](const float* M, const float* x) {
-        const int i = tid % D, g = tid / D;
-        float acc[kBC];
-#pragma unroll
-        for (int u = 0; u < kBC; ++u) acc[u] = 0.f;
-        for (int jj = 0; jj < RW; ++jj) {
-            const int j = g * RW + jj;
-            const float m = M[i * LD + j];
-#pragma unroll
-            for (int u = 0; u < kBC; ++u) acc[u] = fmaf(m, x[u * D + j], acc[u]);
+    // out_u[i] = sum_j M[i][j] x_u[j]  (x from the right): m = i, n = u, k = j
+    auto right_partials = [&](const float* M, int xb) {
+        const int i0 = 16 * (warp % MT), ks = warp / MT;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+        for (int st = 0; st < KSTEPS; ++st) {
+            const int j0 = 8 * (ks * KSTEPS + st);
+            const float af[4] = {M[(i0 + g8) * LD + j0 + t4], M[(i0 + g8 + 8) * LD + j0 + t4],
+                                 M[(i0 + g8) * LD + j0 + t4 + 4], M[(i0 + g8 + 8) * LD + j0 + t4 + 4]};
+            mma3_step(d, af, sm[xb + g8 * TD + j0 + t4], sm[xb + g8 * TD + j0 + t4 + 4]);
         }
-#pragma unroll
-        for (int u = 0; u < kBC; ++u) sm[L::RED + (g * kBC + u) * D + i] = acc[u];
+        float* red = sm + L::RED + ks * kBC * D;
+        red[(2 * t4) * D + i0 + g8] = d[0];
+        red[(2 * t4 + 1) * D + i0 + g8] = d[1];
+        red[(2 * t4) * D + i0 + g8 + 8] = d[2];
+        red[(2 * t4 + 1) * D + i0 + g8 + 8] = d[3];
+    };
+    // M[i][j] = rowscale[i] M[i][j] + sum_r a_r[i] b_r[j] over one or two 8-deep
+    // k steps: (a0, b0) with sign +1 and, if two, (a1, b1) with sign sgn1. a_r[i]
+    // is tile(a, r, i) times tile(am, r, i) when am >= 0; b_r[j] is tile(b, r, j)
+    // times beta_r when bb is set. Warp w owns the 16 x 8 output tiles w, w+16, ...
+    auto rank_update = [&](float* M, int rs, int a0b, int am0, int b0b, bool two, int a1b, int am1, int b1b,
+                           float sgn1, bool bb1) {
+        for (int tile = warp; tile < (D / 16) * (D / 8); tile += kBT / 32) {
+            const int i0 = 16 * (tile / (D / 8)), j0 = 8 * (tile % (D / 8));
+            float d[4];
+            const float sc0 = tl(rs, kBC - 1, i0 + g8), sc1 = tl(rs, kBC - 1, i0 + g8 + 8);
+            d[0] = sc0 * M[(i0 + g8) * LD + j0 + 2 * t4];
+            d[1] = sc0 * M[(i0 + g8) * LD + j0 + 2 * t4 + 1];
+            d[2] = sc1 * M[(i0 + g8 + 8) * LD + j0 + 2 * t4];
+            d[3] = sc1 * M[(i0 + g8 + 8) * LD + j0 + 2 * t4 + 1];
+            auto av = [&](int ab, int am, int r, int i) { return am >= 0 ? tl(ab, r, i) * tl(am, r, i) : tl(ab, r, i); };
+            {
+                const float af[4] = {av(a0b, am0, t4, i0 + g8), av(a0b, am0, t4, i0 + g8 + 8),
+                                     av(a0b, am0, t4 + 4, i0 + g8), av(a0b, am0, t4 + 4, i0 + g8 + 8)};
+                mma3_step(d, af, tl(b0b, t4, j0 + g8), tl(b0b, t4 + 4, j0 + g8));
+            }
+            if (two) {
+                const float af[4] = {sgn1 * av(a1b, am1, t4, i0 + g8), sgn1 * av(a1b, am1, t4, i0 + g8 + 8),
+                                     sgn1 * av(a1b, am1, t4 + 4, i0 + g8), sgn1 * av(a1b, am1, t4 + 4, i0 + g8 + 8)};
+                const float bf0 = tl(b1b, t4, j0 + g8) * (bb1 ? sm[L::BETA + t4] : 1.f);
+                const float bf1 = tl(b1b, t4 + 4, j0 + g8) * (bb1 ? sm[L::BETA + t4 + 4] : 1.f);
+                mma3_step(d, af, bf0, bf1);
+            }
+            M[(i0 + g8) * LD + j0 + 2 * t4] = d[0];
+            M[(i0 + g8) * LD + j0 + 2 * t4 + 1] = d[1];
+            M[(i0 + g8 + 8) * LD + j0 + 2 * t4] = d[2];
+            M[(i0 + g8 + 8) * LD + j0 + 2 * t4 + 1] = d[3];
+        }
     };
     auto red_sum = [&](int u, int c) -> float {
         float s = 0.f;
 #pragma unroll
-        for (int g = 0; g < NG; ++g) s += sm[L::RED + (g * kBC + u) * D + c];
+        for (int g = 0; g < NKS; ++g) s += sm[L::RED + (g * kBC + u) * D + c];
         return s;
     };
 
@@ -167,11 +243,11 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                     ov = to_f32(dO[tok * D + c]);
                 }
             }
-            sm[L::Q + e] = qv;
-            sm[L::K + e] = kv;
-            sm[L::G + e] = gv;
-            sm[L::V + e] = vv;
-            sm[L::DO + e] = ov;
+            tl(L::Q, r, c) = qv;
+            tl(L::K, r, c) = kv;
+            tl(L::G, r, c) = gv;
+            tl(L::V, r, c) = vv;
+            tl(L::DO, r, c) = ov;
         }
         if (tid < kBC) sm[L::BETA + tid] = tid < len ? to_f32(beta[(tok0 + (size_t)n * kBC + tid) * H + h]) : 0.f;
         __syncthreads();
@@ -183,9 +259,9 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             float acc = 0.f;
 #pragma unroll
             for (int r = 0; r < kBC; ++r) {
-                acc += sm[L::G + r * D + c];
-                sm[L::G + r * D + c] = acc;
-                sm[L::GAM + r * D + c] = expf(acc);
+                acc += tl(L::G, r, c);
+                tl(L::G, r, c) = acc;
+                tl(L::GAM, r, c) = expf(acc);
             }
         }
         __syncthreads();
@@ -193,7 +269,7 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             const int p = e / D, c = e % D;
             int r, s;
             pair_rs(p, r, s);
-            sm[L::E + e] = expf(sm[L::G + r * D + c] - sm[L::G + s * D + c]);
+            sm[L::E + e] = expf(tl(L::G, r, c) - tl(L::G, s, c));
         }
         __syncthreads();
         for (int p = warp; p < kPairs; p += kBT / 32) {
@@ -201,9 +277,9 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             pair_rs(p, r, s);
             float a = 0.f, pp = 0.f;
             for (int c = lane; c < D; c += 32) {
-                const float ks = sm[L::K + s * D + c] * sm[L::E + p * D + c];
-                a = fmaf(sm[L::K + r * D + c], ks, a);
-                if (want_p) pp = fmaf(sm[L::Q + r * D + c], ks, pp);
+                const float ks = tl(L::K, s, c) * sm[L::E + p * D + c];
+                a = fmaf(tl(L::K, r, c), ks, a);
+                if (want_p) pp = fmaf(tl(L::Q, r, c), ks, pp);
             }
             a = warp_sum(a);
             pp = warp_sum(pp);
@@ -232,80 +308,81 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             float w = 0.f, u = 0.f;
             for (int s = 0; s <= r; ++s) {
                 const float ts = sm[L::TM + r * kBC + s] * sm[L::BETA + s];
-                w = fmaf(ts, sm[L::K + s * D + c] * sm[L::GAM + s * D + c], w);
-                u = fmaf(ts, sm[L::V + s * D + c], u);
+                w = fmaf(ts, tl(L::K, s, c) * tl(L::GAM, s, c), w);
+                u = fmaf(ts, tl(L::V, s, c), u);
             }
-            sm[L::R + e] = erase ? w : 0.f;
-            sm[L::DL + e] = u;
+            tl(L::R, r, c) = erase ? w : 0.f;
+            tl(L::DL, r, c) = u;
         }
         __syncthreads();
         if (erase) {
-            left_partials(sS, sm + L::R);
+            left_partials(sS, L::R);
             __syncthreads();
-            for (int e = tid; e < kBC * D; e += kBT) sm[L::DL + e] -= red_sum(e / D, e % D);
+            for (int e = tid; e < kBC * D; e += kBT) tl(L::DL, e / D, e % D) -= red_sum(e / D, e % D);
             __syncthreads();
         }
     };
-    // one chunk forward: S <- Gamma_last S + (k e^{G_last - G})^T delta
+    // S <- Gamma_last S + (k e^{G_last - G})^T delta
+    auto state_update = [&]() {
+        for (int e = tid; e < kBC * D; e += kBT) {
+            const int r = e / D, c = e % D;
+            tl(L::X, r, c) = tl(L::K, r, c) * expf(tl(L::G, kBC - 1, c) - tl(L::G, r, c));
+        }
+        __syncthreads();
+        rank_update(sS, L::GAM, L::X, -1, L::DL, false, 0, -1, 0, 0.f, false);
+        __syncthreads();
+    };
     auto fwd_step = [&](int n) {
         load_chunk(n, false);
         prep(false);
         make_delta();
-        for (int e = tid; e < kBC * D; e += kBT) {
-            const int r = e / D, c = e % D;
-            sm[L::X + e] = sm[L::K + e] * expf(sm[L::G + (kBC - 1) * D + c] - sm[L::G + r * D + c]);
-        }
-        __syncthreads();
-        for (int e = tid; e < D * D; e += kBT) {
-            const int i = e / D, j = e % D;
-            float acc = sm[L::GAM + (kBC - 1) * D + i] * sS[i * LD + j];
-#pragma unroll
-            for (int r = 0; r < kBC; ++r) acc = fmaf(sm[L::X + r * D + i], sm[L::DL + r * D + j], acc);
-            sS[i * LD + j] = acc;
-        }
-        __syncthreads();
+        state_update();
     };
 
-    auto bwd_step = [&](int n) {
+    auto bwd_step = [&](int n, const float* delta_g) {
         const int len = load_chunk(n, true);
         prep(true);
-        make_delta();
+        for (int e = tid; e < kBC * D; e += kBT) tl(L::DL, e / D, e % D) = delta_g[e];  // delta of the recompute
         // R = v - (k e^G) S - A0 delta  (additive write: R = v)
+        for (int e = tid; e < kBC * D; e += kBT) {
+            const int r = e / D, c = e % D;
+            tl(L::X, r, c) = tl(L::K, r, c) * tl(L::GAM, r, c);
+        }
+        __syncthreads();
         if (erase) {
-            for (int e = tid; e < kBC * D; e += kBT) sm[L::X + e] = sm[L::K + e] * sm[L::GAM + e];
-            __syncthreads();
-            left_partials(sS, sm + L::X);
+            left_partials(sS, L::X);
             __syncthreads();
             for (int e = tid; e < kBC * D; e += kBT) {
                 const int r = e / D, c = e % D;
-                float acc = sm[L::V + e] - red_sum(r, c);
-                for (int s = 0; s < r; ++s) acc = fmaf(-sm[L::A0 + r * kBC + s], sm[L::DL + s * D + c], acc);
-                sm[L::R + e] = acc;
+                float acc = tl(L::V, r, c) - red_sum(r, c);
+                for (int s = 0; s < r; ++s) acc = fmaf(-sm[L::A0 + r * kBC + s], tl(L::DL, s, c), acc);
+                tl(L::R, r, c) = acc;
             }
         } else {
-            for (int e = tid; e < kBC * D; e += kBT) sm[L::R + e] = sm[L::V + e];
+            for (int e = tid; e < kBC * D; e += kBT) tl(L::R, e / D, e % D) = tl(L::V, e / D, e % D);
         }
+        __syncthreads();
         // X = (k e^{G_last - G}) F + P^T dO
         for (int e = tid; e < kBC * D; e += kBT) {
             const int r = e / D, c = e % D;
-            sm[L::X + e] = sm[L::K + e] * expf(sm[L::G + (kBC - 1) * D + c] - sm[L::G + r * D + c]);
+            tl(L::X, r, c) = tl(L::K, r, c) * expf(tl(L::G, kBC - 1, c) - tl(L::G, r, c));
         }
         __syncthreads();
-        left_partials(sF, sm + L::X);
+        left_partials(sF, L::X);
         __syncthreads();
         for (int e = tid; e < kBC * D; e += kBT) {
             const int r = e / D, c = e % D;
             float acc = red_sum(r, c);
-            for (int s = r; s < kBC; ++s) acc = fmaf(sm[L::P + s * kBC + r], sm[L::DO + s * D + c], acc);
-            sm[L::X + e] = acc;
+            for (int s = r; s < kBC; ++s) acc = fmaf(sm[L::P + s * kBC + r], tl(L::DO, s, c), acc);
+            tl(L::X, r, c) = acc;
         }
         __syncthreads();
         // d(delta) = T^T X; dv = b d(delta)
         for (int e = tid; e < kBC * D; e += kBT) {
             const int r = e / D, c = e % D;
             float acc = 0.f;
-            for (int s = r; s < kBC; ++s) acc = fmaf(sm[L::TM + s * kBC + r], sm[L::X + s * D + c], acc);
-            sm[L::DD + e] = acc;
+            for (int s = r; s < kBC; ++s) acc = fmaf(sm[L::TM + s * kBC + r], tl(L::X, s, c), acc);
+            tl(L::DD, r, c) = acc;
             if (r < len) dv[((tok0 + (size_t)n * kBC + r) * H + h) * D + c] = from_f32<T>(sm[L::BETA + r] * acc);
         }
         __syncthreads();
@@ -313,17 +390,17 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         if (warp < kBC) {
             const int r = warp;
             float acc = 0.f;
-            for (int c = lane; c < D; c += 32) acc = fmaf(sm[L::DD + r * D + c], sm[L::R + r * D + c], acc);
+            for (int c = lane; c < D; c += 32) acc = fmaf(tl(L::DD, r, c), tl(L::R, r, c), acc);
             acc = warp_sum(acc);
             if (lane == 0 && r < len) dbeta[(tok0 + (size_t)n * kBC + r) * H + h] = from_f32<T>(acc);
         }
-        for (int d = warp; d < 3 * kBC * kBC; d += kBT / 32) {
-            const int tbl = d / (kBC * kBC), r = (d / kBC) % kBC, s = d % kBC;
+        for (int dd = warp; dd < 3 * kBC * kBC; dd += kBT / 32) {
+            const int tbl = dd / (kBC * kBC), r = (dd / kBC) % kBC, s = dd % kBC;
             // C1: delta_s . dO_r;  C2: delta_s . d(delta)_r;  C3: delta_r . d(delta)_s (times b_s)
-            const float* x = sm + L::DL + (tbl == 2 ? r : s) * D;
-            const float* y = tbl == 0 ? sm + L::DO + r * D : sm + L::DD + (tbl == 1 ? r : s) * D;
+            const int xb = L::DL + (tbl == 2 ? r : s) * TD;
+            const int yb = tbl == 0 ? L::DO + r * TD : L::DD + (tbl == 1 ? r : s) * TD;
             float acc = 0.f;
-            for (int c = lane; c < D; c += 32) acc = fmaf(x[c], y[c], acc);
+            for (int c = lane; c < D; c += 32) acc = fmaf(sm[xb + c], sm[yb + c], acc);
             acc = warp_sum(acc);
             if (lane == 0) {
                 if (tbl == 0) sm[L::C1 + r * kBC + s] = acc;
@@ -333,44 +410,44 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         }
         __syncthreads();
         // right products: S dO -> R, S d(delta) -> DG, F delta -> X
-        right_partials(sS, sm + L::DO);
+        right_partials(sS, L::DO);
         __syncthreads();
-        for (int e = tid; e < kBC * D; e += kBT) sm[L::R + e] = red_sum(e / D, e % D);
+        for (int e = tid; e < kBC * D; e += kBT) tl(L::R, e / D, e % D) = red_sum(e / D, e % D);
         __syncthreads();
-        right_partials(sS, sm + L::DD);
+        right_partials(sS, L::DD);
         __syncthreads();
-        for (int e = tid; e < kBC * D; e += kBT) sm[L::DG + e] = red_sum(e / D, e % D);
+        for (int e = tid; e < kBC * D; e += kBT) tl(L::DG, e / D, e % D) = red_sum(e / D, e % D);
         __syncthreads();
-        right_partials(sF, sm + L::DL);
+        right_partials(sF, L::DL);
         __syncthreads();
-        for (int e = tid; e < kBC * D; e += kBT) sm[L::X + e] = red_sum(e / D, e % D);
+        for (int e = tid; e < kBC * D; e += kBT) tl(L::X, e / D, e % D) = red_sum(e / D, e % D);
         __syncthreads();
         // per (token, channel): dq, dk, and q dq - k dkw + k dkr
         for (int e = tid; e < kBC * D; e += kBT) {
             const int r = e / D, c = e % D;
-            const float gam = sm[L::GAM + e], kr = sm[L::K + e], qr = sm[L::Q + e];
-            float gq = gam * sm[L::R + e];
+            const float gam = tl(L::GAM, r, c), kr = tl(L::K, r, c), qr = tl(L::Q, r, c);
+            float gq = gam * tl(L::R, r, c);
             for (int s = 0; s <= r; ++s)
-                gq = fmaf(sm[L::E + pidx(r, s) * D + c] * sm[L::K + s * D + c], sm[L::C1 + r * kBC + s], gq);
+                gq = fmaf(sm[L::E + pidx(r, s) * D + c] * tl(L::K, s, c), sm[L::C1 + r * kBC + s], gq);
             float gkr = 0.f;
             if (erase) {
-                gkr = gam * sm[L::DG + e];
+                gkr = gam * tl(L::DG, r, c);
                 for (int s = 0; s < r; ++s)
-                    gkr = fmaf(sm[L::E + pidx(r, s) * D + c] * sm[L::K + s * D + c], sm[L::C2 + r * kBC + s], gkr);
+                    gkr = fmaf(sm[L::E + pidx(r, s) * D + c] * tl(L::K, s, c), sm[L::C2 + r * kBC + s], gkr);
                 gkr *= -sm[L::BETA + r];
             }
-            float gkw = expf(sm[L::G + (kBC - 1) * D + c] - sm[L::G + e]) * sm[L::X + e];
+            float gkw = expf(tl(L::G, kBC - 1, c) - tl(L::G, r, c)) * tl(L::X, r, c);
             for (int s = r; s < kBC; ++s) {
                 const float es = sm[L::E + pidx(s, r) * D + c];
-                gkw = fmaf(es * sm[L::Q + s * D + c], sm[L::C1 + s * kBC + r], gkw);
-                if (erase && s > r) gkw = fmaf(-es * sm[L::K + s * D + c], sm[L::C3 + r * kBC + s], gkw);
+                gkw = fmaf(es * tl(L::Q, s, c), sm[L::C1 + s * kBC + r], gkw);
+                if (erase && s > r) gkw = fmaf(-es * tl(L::K, s, c), sm[L::C3 + r * kBC + s], gkw);
             }
             if (r < len) {
                 const size_t off = ((tok0 + (size_t)n * kBC + r) * H + h) * D + c;
                 dq[off] = from_f32<T>(gq);
                 dk[off] = from_f32<T>(gkw + gkr);
             }
-            sm[L::DG + e] = qr * gq - kr * gkw + kr * gkr;
+            tl(L::DG, r, c) = qr * gq - kr * gkw + kr * gkr;
         }
         __syncthreads();
         // decay gradient: reverse running sum per channel
@@ -378,11 +455,11 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             for (int c = tid; c < D; c += kBT) {
                 float acc = sm[L::CARRY + c];
                 for (int r = kBC - 1; r >= 0; --r) {
-                    acc += sm[L::DG + r * D + c];
+                    acc += tl(L::DG, r, c);
                     if (gate == 0) {
                         if (r < len) dla[((tok0 + (size_t)n * kBC + r) * H + h) * D + c] = from_f32<T>(acc);
                     } else {
-                        sm[L::DG + r * D + c] = acc;
+                        tl(L::DG, r, c) = acc;
                     }
                 }
                 sm[L::CARRY + c] = acc;
@@ -392,24 +469,14 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                 if (warp < kBC) {
                     const int r = warp;
                     float acc = 0.f;
-                    for (int c = lane; c < D; c += 32) acc += sm[L::DG + r * D + c];
+                    for (int c = lane; c < D; c += 32) acc += tl(L::DG, r, c);
                     acc = warp_sum(acc);
                     if (lane == 0 && r < len) dla[(tok0 + (size_t)n * kBC + r) * H + h] = from_f32<T>(acc);
                 }
             }
         }
         // F <- Gamma_last F + (q e^G)^T dO - (k e^G)^T dv
-        for (int e = tid; e < D * D; e += kBT) {
-            const int i = e / D, j = e % D;
-            float acc = sm[L::GAM + (kBC - 1) * D + i] * sF[i * LD + j];
-#pragma unroll
-            for (int r = 0; r < kBC; ++r) {
-                const float gr = sm[L::GAM + r * D + i];
-                acc = fmaf(sm[L::Q + r * D + i] * gr, sm[L::DO + r * D + j], acc);
-                if (erase) acc = fmaf(-sm[L::K + r * D + i] * gr, sm[L::BETA + r] * sm[L::DD + r * D + j], acc);
-            }
-            sF[i * LD + j] = acc;
-        }
+        rank_update(sF, L::GAM, L::Q, L::GAM, L::DO, erase != 0, L::K, L::GAM, L::DD, -1.f, true);
         __syncthreads();
     };
 
@@ -439,15 +506,21 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         const int n0 = blk * kBlk, n1 = min(n0 + kBlk, NB);
         load_mat(sS, ck + (size_t)blk * kMat);
         __syncthreads();
-        for (int n = n0; n < n1; ++n) {
-            store_mat(sS, rg + (size_t)(n - n0) * kMat);
+        for (int n = n0; n < n1; ++n) {  // recompute: entry state and delta of each chunk
+            float* slot = rg + (size_t)(n - n0) * kRing;
+            store_mat(sS, slot);
+            load_chunk(n, false);
+            prep(false);
+            make_delta();
+            for (int e = tid; e < kBC * D; e += kBT) slot[kMat + e] = tl(L::DL, e / D, e % D);
+            if (n + 1 < n1) state_update();
             __syncthreads();
-            if (n + 1 < n1) fwd_step(n);
         }
         for (int n = n1 - 1; n >= n0; --n) {
-            load_mat(sS, rg + (size_t)(n - n0) * kMat);
+            const float* slot = rg + (size_t)(n - n0) * kRing;
+            load_mat(sS, slot);
             __syncthreads();
-            bwd_step(n);
+            bwd_step(n, slot + kMat);
         }
     }
     if (dS0) store_mat(sF, dS0 + (size_t)bh * kMat);
@@ -461,7 +534,7 @@ cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     const size_t NBLK = ((size_t)(a.T + kBC - 1) / kBC + kBlk - 1) / kBlk;
     float* ckpt = static_cast<float*>(a.workspace);
-    float* ring = ckpt + (size_t)a.B * a.H * NBLK * D * D;
+    float* ring = ckpt + (size_t)a.B * a.H * NBLK * D * D;  // then B*H*kBlk slots of (state, delta)
     kern<<<(unsigned)(a.B * a.H), kBT, L::BYTES, stream>>>(
         (const T*)a.q, (const T*)a.k, (const T*)a.v, (const T*)a.log_alpha, (const T*)a.beta, a.S0, (const T*)a.dO,
         a.dST, (T*)a.g_q, (T*)a.g_k, (T*)a.g_v, (T*)a.g_log_alpha, (T*)a.g_beta, a.g_S0, ckpt, ring, a.T, a.H,
@@ -473,7 +546,7 @@ cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t stream) {
 
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int d) {
     const size_t NBLK = ((size_t)(T + kBC - 1) / kBC + kBlk - 1) / kBlk;
-    return (size_t)B * H * (NBLK + kBlk) * d * d * sizeof(float);
+    return (size_t)B * H * (NBLK * d * d + kBlk * ((size_t)d * d + (size_t)kBC * d)) * sizeof(float);
 }
 
 cudaError_t launch_chunk_bwd(const BwdArgs& a, cudaStream_t stream) {

@@ -213,8 +213,8 @@ def _bwd_good():
 
 def test_bwd_workspace_size():
     d = 128
-    # one fp32 [d][d] state per 64 tokens plus 8 per (batch, head)
-    assert kda.load().kda_chunk_bwd_workspace_size(2, 130, 3, d, d) == 2 * 3 * (3 + 8) * d * d * 4
+    # one fp32 [d][d] state per 64 tokens, plus a ring of 8 (state, [8][d] delta) slots per (batch, head)
+    assert kda.load().kda_chunk_bwd_workspace_size(2, 130, 3, d, d) == 2 * 3 * (3 * d * d + 8 * (d * d + 8 * d)) * 4
     assert kda.load().kda_chunk_bwd_workspace_size(1, 8, 1, 96, 96) == 0
 
 
