@@ -193,9 +193,10 @@ kda_status_t kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
  *   workspace   : device scratch of kda_chunk_bwd_workspace_size(...) bytes,
  *                 16-byte aligned: fp32 [dk][dv] states, one per 64 tokens
  *                 and 8 per (batch, head) for the block being reversed
- * Arithmetic: fp32 throughout (exact per-pair decay exponentials, all with
- * non-positive exponents), gradients rounded to dtype once. One CTA per
- * (batch, head): the work is latency bound, not tuned.
+ * Arithmetic: fp32 (exact per-pair decay exponentials, all with non-positive
+ * exponents; the matrix products on tensor cores with each fp32 operand split
+ * into two tf32 parts, which keeps fp32-level accuracy), gradients rounded to
+ * dtype once. One CTA per (batch, head).
  */
 size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv);
 kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,
