@@ -332,24 +332,59 @@ def time_prefill(args, ctx, pf, peaks, peak_kind):
     return ms_per_step, roofline, clk.summary()
 
 
-def time_e2e(args, ctx, pf):
-    """Same metric through the C ABI with host buffers: every step copies its
-    inputs host->device from pinned memory and reads o and S_T back."""
+def time_e2e(args, ctx, pf, pieces_per_seq: int = 8):
+    """Same metric through the C ABI with host buffers: every step copies all
+    of its inputs host->device from pinned memory and reads o and S_T back.
+    The batch is cut into pieces of whole chunks along T (each sequence in
+    order, its state passed from piece to piece through S0 / S_T), and three
+    streams overlap the copy of piece p+1, the prefill of piece p and the
+    read-back of piece p-1; the copy engines then set the pace."""
     torch = ctx.torch
+    cfg = pf.cfg
+    B, T = cfg.B, cfg.T
     pin = {k: (None if v is None else v.cpu().pin_memory()) for k, v in pf.x.items()}
     dbuf = {k: (None if v is None else torch.empty_like(v)) for k, v in pf.x.items()}
     o_host = torch.empty(pf.o.shape, dtype=pf.o.dtype, pin_memory=True)
     ST_host = torch.empty(pf.ST.shape, dtype=pf.ST.dtype, pin_memory=True)
     h2d = sum(v.numel() * v.element_size() for v in pin.values() if v is not None)
     d2h = o_host.numel() * o_host.element_size() + ST_host.numel() * ST_host.element_size()
+    LT = max(cfg.C, (T // pieces_per_seq + cfg.C - 1) // cfg.C * cfg.C)  # tokens per piece, whole chunks
+    cuts = [(b, t0, min(t0 + LT, T)) for b in range(B) for t0 in range(0, T, LT)]
+    s_in, s_run, s_out = torch.cuda.Stream(ctx.dev), torch.cuda.Stream(ctx.dev), torch.cuda.Stream(ctx.dev)
+    dts = "bf16" if pf.x["q"].dtype == torch.bfloat16 else "f32"
+    ws_piece = max(pf.kda.workspace_size(1, t1 - t0, cfg.H, cfg.dk, cfg.dv, cfg.C, dts, pf.algo)
+                   for _, t0, t1 in cuts)
+    ws = torch.empty(max(ws_piece, 256), dtype=torch.uint8, device=ctx.dev)
 
     def step():
-        for k in pin:
-            if pin[k] is not None:
-                dbuf[k].copy_(pin[k], non_blocking=True)
-        pf.run(dbuf)
-        o_host.copy_(pf.o, non_blocking=True)
-        ST_host.copy_(pf.ST, non_blocking=True)
+        start = torch.cuda.Event()
+        start.record(ctx.stream)
+        for st in (s_in, s_run, s_out):
+            st.wait_event(start)
+        for b, t0, t1 in cuts:
+            with torch.cuda.stream(s_in):
+                for k in ("q", "k", "v", "log_alpha", "beta"):
+                    dbuf[k][b, t0:t1].copy_(pin[k][b, t0:t1], non_blocking=True)
+                if t0 == 0 and pin["S0"] is not None:
+                    dbuf["S0"][b].copy_(pin["S0"][b], non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(s_in)
+            s_run.wait_event(landed)
+            sl = lambda key: dbuf[key][b:b + 1, t0:t1]
+            S0 = (dbuf["S0"][b:b + 1] if pin["S0"] is not None else None) if t0 == 0 else pf.ST[b:b + 1]
+            pf.kda.chunk_fwd(sl("q"), sl("k"), sl("v"), sl("log_alpha"), sl("beta"), S0, chunk=cfg.C,
+                             algo=pf.algo, o=pf.o[b:b + 1, t0:t1], S_T=pf.ST[b:b + 1], workspace=ws,
+                             stream=s_run)
+            done = torch.cuda.Event()
+            done.record(s_run)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                o_host[b, t0:t1].copy_(pf.o[b, t0:t1], non_blocking=True)
+                if t1 == T:
+                    ST_host[b].copy_(pf.ST[b], non_blocking=True)
+        fin = torch.cuda.Event()
+        fin.record(s_out)
+        ctx.stream.wait_event(fin)
 
     n = max(3, min(args.steps, 10))
     for _ in range(3):
@@ -363,9 +398,23 @@ def time_e2e(args, ctx, pf):
     e1.record(ctx.stream)
     torch.cuda.synchronize()
     ms = ctx.max_over_ranks(e0.elapsed_time(e1) / n)
-    return {"value": ctx.world * pf.tokens_per_step / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n,
-            "path": "pinned host -> device copies, kda_chunk_fwd, device -> pinned host copies of o and S_T"}
+    if pf.use_tc and pf.kda.workspace_status(ws, s_run) != 0:
+        raise RuntimeError("device-side timeout reported by the prefill kernel")
+    # the pieces must reproduce one call over the whole batch (up to rounding)
+    o_one, S_one = pf.o.clone(), pf.ST.clone()
+    pf.run()
+    torch.cuda.synchronize()
+    den_o, den_s = pf.o.float().abs().max().item(), pf.ST.abs().max().item()
+    diff = max((o_host.to(ctx.dev).float() - pf.o.float()).abs().max().item() / max(den_o, 1e-30),
+               (ST_host.to(ctx.dev) - pf.ST).abs().max().item() / max(den_s, 1e-30))
+    del o_one, S_one
+    if not diff < 2e-2:
+        raise RuntimeError(f"pipelined end-to-end result differs from one call: {diff}")
+    return {"value": whole_job_rate(ctx.world, pf.tokens_per_step, ms), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n,
+            "pieces": len(cuts), "tokens_per_piece": LT, "max_rel_diff_vs_one_call": diff,
+            "path": "pinned host -> device copies, kda_chunk_fwd per piece (state chained through S0/S_T), "
+                    "device -> pinned host copies of o and S_T; copy, compute and read-back on three streams"}
 
 
 def time_decode(args, ctx, kda, I, peaks, peak_kind):
