@@ -332,7 +332,7 @@ def time_prefill(args, ctx, pf, peaks, peak_kind):
     return ms_per_step, roofline, clk.summary()
 
 
-def time_e2e(args, ctx, pf, pieces_per_seq: int = 8):
+def time_e2e(args, ctx, pf, pieces_per_seq: int = 4):
     """Same metric through the C ABI with host buffers: every step copies all
     of its inputs host->device from pinned memory and reads o and S_T back.
     The batch is cut into pieces of whole chunks along T (each sequence in
