@@ -76,6 +76,10 @@ def load(build_if_stale: bool = True):
     lib.kda_chunk_bwd_workspace_size.restype = Z
     lib.kda_chunk_bwd.argtypes = [P] * 14 + [I] * 8 + [P, Z, P]
     lib.kda_chunk_bwd.restype = I
+    lib.kda_chunk_bwd_ex.argtypes = [P] * 14 + [I] * 9 + [P, Z, P]
+    lib.kda_chunk_bwd_ex.restype = I
+    lib.kda_chunk_bwd_workspace_size_ex.argtypes = [I] * 6
+    lib.kda_chunk_bwd_workspace_size_ex.restype = Z
     _lib = lib
     return lib
 
@@ -209,12 +213,16 @@ def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, chunk: in
     return o, S_T
 
 
+BWD_MODES = {"auto": 0, "all": 1, "low": 2}
+
+
 def chunk_bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None, *, erase: bool = True, gate: str = "channel",
-              want_dS0: bool = True, workspace=None, stream=None) -> dict:
-    """kda_chunk_bwd: gradients of a loss with dL/do = dO [B,T,H,dv] and
-    dL/dS_T = dS_T [B,H,dk,dv] (None: 0). Inputs as for chunk_fwd. Returns
-    dict dq, dk, dv, dlog_alpha (None without a gate), dbeta, dS0 (None
-    unless want_dS0)."""
+              want_dS0: bool = True, workspace=None, stream=None, memory: str = "auto") -> dict:
+    """kda_chunk_bwd_ex: gradients of a loss with dL/do = dO [B,T,H,dv] and
+    dL/dS_T = dS_T [B,H,dk,dv] (None: 0). Inputs as for chunk_fwd. memory:
+    "auto", "all" (keep every chunk's state) or "low" (one per 64 tokens and a
+    recompute sweep). Returns dict dq, dk, dv, dlog_alpha (None without a
+    gate), dbeta, dS0 (None unless want_dS0)."""
     import torch
     lib = load()
     B, T, H, dk = q.shape
@@ -236,16 +244,17 @@ def chunk_bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None, *, erase: bool = True
          "dlog_alpha": None if gshape is None else torch.empty(gshape, dtype=dt, device=dev),
          "dbeta": torch.empty_like(beta),
          "dS0": torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev) if want_dS0 else None}
-    ws_bytes = int(lib.kda_chunk_bwd_workspace_size(B, T, H, dk, dv))
+    mode = BWD_MODES[memory]
+    ws_bytes = int(lib.kda_chunk_bwd_workspace_size_ex(B, T, H, dk, dv, mode))
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
     la = log_alpha if gshape is not None else None
-    code = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0), _ptr(dO), _ptr(dS_T),
-                             _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]),
-                             _ptr(g["dS0"]), B, T, H, dk, dv, _DTYPE[_dtype_of(q)], int(bool(erase)), GATES[gate],
-                             _ptr(workspace), ws_len, _stream(stream))
-    _check("kda_chunk_bwd", code)
+    code = lib.kda_chunk_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0), _ptr(dO), _ptr(dS_T),
+                                _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]),
+                                _ptr(g["dS0"]), B, T, H, dk, dv, _DTYPE[_dtype_of(q)], int(bool(erase)), GATES[gate],
+                                mode, _ptr(workspace), ws_len, _stream(stream))
+    _check("kda_chunk_bwd_ex", code)
     return g
 
 

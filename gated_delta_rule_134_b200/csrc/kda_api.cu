@@ -175,9 +175,14 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
                              stream);
 }
 
-size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
+size_t kda_chunk_bwd_workspace_size_ex(int B, int T, int H, int dk, int dv, kda_bwd_mode_t mode) {
     if (B < 0 || T < 0 || H < 0 || !head_dims_ok(dk, dv)) return 0;
-    return kda::chunk_bwd_workspace_bytes(B, T, H, dk);
+    if (mode < KDA_BWD_AUTO || mode > KDA_BWD_LOW_MEMORY) return 0;
+    return kda::chunk_bwd_workspace_bytes(B, T, H, dk, (int)mode);
+}
+
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
+    return kda_chunk_bwd_workspace_size_ex(B, T, H, dk, dv, KDA_BWD_AUTO);
 }
 
 kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
@@ -185,7 +190,17 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const vo
                            void* d_log_alpha, void* d_beta, float* d_S0, int B, int T, int H, int dk, int dv,
                            kda_dtype_t dtype, int erase, kda_gate_t gate, void* workspace, size_t workspace_bytes,
                            void* stream) {
+    return kda_chunk_bwd_ex(q, k, v, log_alpha, beta, S0, dO, dS_T, d_q, d_k, d_v, d_log_alpha, d_beta, d_S0, B, T,
+                            H, dk, dv, dtype, erase, gate, KDA_BWD_AUTO, workspace, workspace_bytes, stream);
+}
+
+kda_status_t kda_chunk_bwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                              const float* S0, const void* dO, const float* dS_T, void* d_q, void* d_k, void* d_v,
+                              void* d_log_alpha, void* d_beta, float* d_S0, int B, int T, int H, int dk, int dv,
+                              kda_dtype_t dtype, int erase, kda_gate_t gate, kda_bwd_mode_t mode, void* workspace,
+                              size_t workspace_bytes, void* stream) {
     if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+    if (mode < KDA_BWD_AUTO || mode > KDA_BWD_LOW_MEMORY) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (!head_dims_ok(dk, dv)) return KDA_ERR_UNSUPPORTED;
     if ((long long)B * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
@@ -202,7 +217,7 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const vo
     const float* opt[] = {S0, dS_T, d_S0};
     for (const float* p : opt)
         if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
-    const size_t need = kda::chunk_bwd_workspace_bytes(B, T, H, dk);
+    const size_t need = kda::chunk_bwd_workspace_bytes(B, T, H, dk, (int)mode);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
         return KDA_ERR_INVALID_ARG;
     if ((long long)B * H == 0) return KDA_OK;
@@ -210,6 +225,7 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const vo
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.dO = dO; a.S0 = S0; a.dST = dS_T;
     a.g_q = d_q; a.g_k = d_k; a.g_v = d_v; a.g_log_alpha = d_log_alpha; a.g_beta = d_beta; a.g_S0 = d_S0;
     a.B = B; a.T = T; a.H = H; a.d = dk; a.bf16 = dtype == KDA_BF16; a.erase = erase; a.gate = (int)gate;
+    a.mode = (int)mode;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
     const cudaError_t err = kda::launch_chunk_bwd(a, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;

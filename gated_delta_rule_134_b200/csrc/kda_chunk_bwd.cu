@@ -35,10 +35,12 @@
 // exponent. The six [8 x d] x [d x d] products per chunk run on warp-level
 // tensor-core MMAs (m16n8k8) with each fp32 operand split into a tf32 high
 // part and a tf32 remainder: hi*hi + hi*lo + lo*hi keeps the product at about
-// fp32 accuracy. A forward sweep stores the state every 8 chunks (64
-// tokens); the backward sweep recomputes the 8 entry states and deltas of
-// each such block into a per-CTA ring in global memory (L2) and then walks the
-// block in reverse.
+// fp32 accuracy. A forward sweep keeps every chunk's entry state and delta
+// in the workspace (up to 16 GB of it), and the backward sweep walks the
+// chunks in reverse from there. Beyond that size the forward sweep keeps the
+// state every 8 chunks (64 tokens), and the backward sweep recomputes the 8
+// entry states and deltas of each such block into a per-CTA ring in global
+// memory, then walks the block in reverse.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -126,7 +128,8 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                  const T* __restrict__ log_alpha, const T* __restrict__ beta, const float* __restrict__ S0,
                  const T* __restrict__ dO, const float* __restrict__ dST, T* __restrict__ dq, T* __restrict__ dk,
                  T* __restrict__ dv, T* __restrict__ dla, T* __restrict__ dbeta, float* __restrict__ dS0,
-                 float* __restrict__ ckpt, float* __restrict__ ring, int Tlen, int H, int erase, int gate) {
+                 float* __restrict__ ckpt, float* __restrict__ ring, int Tlen, int H, int erase, int gate,
+                 int store_all) {
     using L = BwdLayout<D>;
     constexpr int LD = L::LD, TD = L::TD, NKS = L::NKS;
     constexpr int MT = D / 16;              // 16-row tiles of a product's output
@@ -332,11 +335,16 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         rank_update(sS, L::GAM, L::X, -1, L::DL, false, 0, -1, 0, 0.f, false);
         __syncthreads();
     };
-    auto fwd_step = [&](int n) {
+    // one chunk forward; its delta also goes to dslot when given, and the state
+    // update is skipped when the next entry state is not needed
+    auto fwd_step = [&](int n, float* dslot, bool update) {
         load_chunk(n, false);
         prep(false);
         make_delta();
-        state_update();
+        if (dslot)
+            for (int e = tid; e < kBC * D; e += kBT) dslot[e] = tl(L::DL, e / D, e % D);
+        if (update) state_update();
+        __syncthreads();
     };
 
     auto bwd_step = [&](int n, const float* delta_g) {
@@ -480,15 +488,22 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         __syncthreads();
     };
 
-    // ---- forward sweep: the state every kBlk chunks, and S_T
+    // the (entry state, delta) slot of every chunk, when they are all kept
+    float* all = ckpt + (size_t)bh * NB * kRing;
+    // ---- forward sweep: every chunk's entry state and delta, or the state
+    // every kBlk chunks; and S_T
     load_mat(sS, S0 ? S0 + (size_t)bh * kMat : nullptr);
     __syncthreads();
     for (int n = 0; n < NB; ++n) {
-        if (n % kBlk == 0) {
+        float* dslot = nullptr;
+        if (store_all) {
+            store_mat(sS, all + (size_t)n * kRing);
+            dslot = all + (size_t)n * kRing + kMat;
+        } else if (n % kBlk == 0) {
             store_mat(sS, ck + (size_t)(n / kBlk) * kMat);
-            __syncthreads();
         }
-        fwd_step(n);
+        __syncthreads();
+        fwd_step(n, dslot, true);
     }
     // ---- F = dS_T; carry = rowsum(dS_T * S_T)
     const float* dst_h = dST ? dST + (size_t)bh * kMat : nullptr;
@@ -501,29 +516,47 @@ chunk_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         if (lane == 0) sm[L::CARRY + c] = acc;
     }
     __syncthreads();
-    // ---- backward sweep, one block of kBlk chunks at a time
-    for (int blk = NBLK - 1; blk >= 0; --blk) {
-        const int n0 = blk * kBlk, n1 = min(n0 + kBlk, NB);
-        load_mat(sS, ck + (size_t)blk * kMat);
+    // ---- backward sweep over the chunks in reverse. Without every slot kept,
+    // the top chunk of each block of kBlk first recomputes the block's entry
+    // states and deltas into the ring.
+    int n0 = 0;
+    for (int n = NB - 1; n >= 0; --n) {
+        const float* slot;
+        if (store_all) {
+            slot = all + (size_t)n * kRing;
+        } else {
+            if (n == NB - 1 || n % kBlk == kBlk - 1) {
+                n0 = n - n % kBlk;
+                load_mat(sS, ck + (size_t)(n0 / kBlk) * kMat);
+                __syncthreads();
+                for (int r = n0; r <= n; ++r) {
+                    float* rs = rg + (size_t)(r - n0) * kRing;
+                    store_mat(sS, rs);
+                    __syncthreads();
+                    fwd_step(r, rs + kMat, r < n);
+                }
+            }
+            slot = rg + (size_t)(n - n0) * kRing;
+        }
+        load_mat(sS, slot);
         __syncthreads();
-        for (int n = n0; n < n1; ++n) {  // recompute: entry state and delta of each chunk
-            float* slot = rg + (size_t)(n - n0) * kRing;
-            store_mat(sS, slot);
-            load_chunk(n, false);
-            prep(false);
-            make_delta();
-            for (int e = tid; e < kBC * D; e += kBT) slot[kMat + e] = tl(L::DL, e / D, e % D);
-            if (n + 1 < n1) state_update();
-            __syncthreads();
-        }
-        for (int n = n1 - 1; n >= n0; --n) {
-            const float* slot = rg + (size_t)(n - n0) * kRing;
-            load_mat(sS, slot);
-            __syncthreads();
-            bwd_step(n, slot + kMat);
-        }
+        bwd_step(n, slot + kMat);
     }
     if (dS0) store_mat(sF, dS0 + (size_t)bh * kMat);
+}
+
+// Keep every chunk's entry state and delta (no recompute sweep) while that
+// takes at most this much workspace; beyond it, one state per 64 tokens and a
+// per-CTA ring of recomputed ones.
+constexpr size_t kStoreAllCap = (size_t)16 << 30;
+
+size_t bwd_bytes_all(int B, int T, int H, int d) {
+    const size_t NB = (size_t)(T + kBC - 1) / kBC;
+    return (size_t)B * H * NB * ((size_t)d * d + (size_t)kBC * d) * sizeof(float);
+}
+
+bool bwd_store_all(int B, int T, int H, int d, int mode) {
+    return mode == 1 || (mode == 0 && bwd_bytes_all(B, T, H, d) <= kStoreAllCap);
 }
 
 template <typename T, int D>
@@ -533,18 +566,20 @@ cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t stream) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::BYTES);
     if (err != cudaSuccess) return err;
     const size_t NBLK = ((size_t)(a.T + kBC - 1) / kBC + kBlk - 1) / kBlk;
+    const int store_all = bwd_store_all(a.B, a.T, a.H, D, a.mode) ? 1 : 0;
     float* ckpt = static_cast<float*>(a.workspace);
     float* ring = ckpt + (size_t)a.B * a.H * NBLK * D * D;  // then B*H*kBlk slots of (state, delta)
     kern<<<(unsigned)(a.B * a.H), kBT, L::BYTES, stream>>>(
         (const T*)a.q, (const T*)a.k, (const T*)a.v, (const T*)a.log_alpha, (const T*)a.beta, a.S0, (const T*)a.dO,
         a.dST, (T*)a.g_q, (T*)a.g_k, (T*)a.g_v, (T*)a.g_log_alpha, (T*)a.g_beta, a.g_S0, ckpt, ring, a.T, a.H,
-        a.erase, a.gate);
+        a.erase, a.gate, store_all);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t chunk_bwd_workspace_bytes(int B, int T, int H, int d) {
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int d, int mode) {
+    if (bwd_store_all(B, T, H, d, mode)) return bwd_bytes_all(B, T, H, d);
     const size_t NBLK = ((size_t)(T + kBC - 1) / kBC + kBlk - 1) / kBlk;
     return (size_t)B * H * (NBLK * d * d + kBlk * ((size_t)d * d + (size_t)kBC * d)) * sizeof(float);
 }

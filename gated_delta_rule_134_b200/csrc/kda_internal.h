@@ -44,10 +44,11 @@ struct BwdArgs {
     void *g_q, *g_k, *g_v, *g_log_alpha, *g_beta;  // gradients (input dtype)
     float* g_S0;
     int B, T, H, d, bf16, erase, gate;
+    int mode;  // 0: keep every chunk's state while that fits 16 GB; 1: always; 2: one per 64 tokens
     void* workspace;
     size_t workspace_bytes;
 };
-size_t chunk_bwd_workspace_bytes(int B, int T, int H, int d);
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int d, int mode);
 cudaError_t launch_chunk_bwd(const BwdArgs& a, cudaStream_t stream);
 
 }  // namespace kda

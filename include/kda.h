@@ -191,19 +191,33 @@ kda_status_t kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
  *   d_S0        : [B, H, dk, dv] float, written; NULL: not computed
  *   dk == dv in {64, 128}
  *   workspace   : device scratch of kda_chunk_bwd_workspace_size(...) bytes,
- *                 16-byte aligned: fp32 [dk][dv] states, one per 64 tokens
- *                 and 8 per (batch, head) for the block being reversed
+ *                 16-byte aligned. By default (KDA_BWD_AUTO) it keeps every
+ *                 8-token chunk's entry state and delta (fp32) when that is at
+ *                 most 16 GB, and otherwise one state per 64 tokens plus 8
+ *                 (state, delta) slots per (batch, head), recomputing each
+ *                 block before reversing it
  * Arithmetic: fp32 (exact per-pair decay exponentials, all with non-positive
  * exponents; the matrix products on tensor cores with each fp32 operand split
  * into two tf32 parts, which keeps fp32-level accuracy), gradients rounded to
  * dtype once. One CTA per (batch, head).
  */
 size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv);
+
+/* Workspace policy of the backward pass: AUTO (as above), STORE_ALL (every
+ * chunk's state, whatever the size), LOW_MEMORY (one state per 64 tokens and
+ * a recompute sweep, about a third more time). */
+typedef enum { KDA_BWD_AUTO = 0, KDA_BWD_STORE_ALL = 1, KDA_BWD_LOW_MEMORY = 2 } kda_bwd_mode_t;
+size_t kda_chunk_bwd_workspace_size_ex(int B, int T, int H, int dk, int dv, kda_bwd_mode_t mode);
 kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,
                            const float *S0, const void *dO, const float *dS_T, void *d_q, void *d_k, void *d_v,
                            void *d_log_alpha, void *d_beta, float *d_S0, int B, int T, int H, int dk, int dv,
                            kda_dtype_t dtype, int erase, kda_gate_t gate, void *workspace, size_t workspace_bytes,
                            void *stream);
+kda_status_t kda_chunk_bwd_ex(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,
+                              const float *S0, const void *dO, const float *dS_T, void *d_q, void *d_k, void *d_v,
+                              void *d_log_alpha, void *d_beta, float *d_S0, int B, int T, int H, int dk, int dv,
+                              kda_dtype_t dtype, int erase, kda_gate_t gate, kda_bwd_mode_t mode, void *workspace,
+                              size_t workspace_bytes, void *stream);
 
 /*
  * Device-side status left in `workspace` by the last kda_chunk_fwd_ex that

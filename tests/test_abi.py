@@ -213,8 +213,11 @@ def _bwd_good():
 
 def test_bwd_workspace_size():
     d = 128
-    # one fp32 [d][d] state per 64 tokens, plus a ring of 8 (state, [8][d] delta) slots per (batch, head)
-    assert kda.load().kda_chunk_bwd_workspace_size(2, 130, 3, d, d) == 2 * 3 * (3 * d * d + 8 * (d * d + 8 * d)) * 4
+    # small enough to keep every 8-token chunk's (state, [8][d] delta): 17 chunks per (batch, head)
+    assert kda.load().kda_chunk_bwd_workspace_size(2, 130, 3, d, d) == 2 * 3 * 17 * (d * d + 8 * d) * 4
+    # beyond 16 GB: one state per 64 tokens plus a ring of 8 (state, delta) slots per (batch, head)
+    B, T, H = 1, 131072, 32
+    assert kda.load().kda_chunk_bwd_workspace_size(B, T, H, d, d) == B * H * (2048 * d * d + 8 * (d * d + 8 * d)) * 4
     assert kda.load().kda_chunk_bwd_workspace_size(1, 8, 1, 96, 96) == 0
 
 
@@ -241,3 +244,16 @@ def test_bwd_rejects_small_workspace_and_bad_switches():
     # making another required pointer misaligned)
     p[0] = ctypes.c_void_p(0x1001)
     assert _bwd(lib, p, ctypes.c_void_p(0x100000), ws_bytes, gate=2) == 1
+
+
+def test_bwd_workspace_modes():
+    lib = kda.load()
+    d = 64
+    all_b = 1 * 2 * 10 * (d * d + 8 * d) * 4                 # 77 tokens: 10 chunks of 8
+    low_b = 1 * 2 * (2 * d * d + 8 * (d * d + 8 * d)) * 4    # 2 stored states + 8 ring slots
+    assert lib.kda_chunk_bwd_workspace_size_ex(1, 77, 2, d, d, 0) == all_b
+    assert lib.kda_chunk_bwd_workspace_size_ex(1, 77, 2, d, d, 1) == all_b
+    assert lib.kda_chunk_bwd_workspace_size_ex(1, 77, 2, d, d, 2) == low_b
+    assert lib.kda_chunk_bwd_workspace_size_ex(1, 77, 2, d, d, 3) == 0
+    p = _bwd_good()
+    assert lib.kda_chunk_bwd_ex(*p, 1, 8, 1, 64, 64, 1, 1, 0, 7, ctypes.c_void_p(0x100000), 1 << 20, None) == 1

@@ -490,12 +490,12 @@ def test_scan_varlen_unsupported(cuda_lib):
 BWD_NAMES = ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0")
 
 
-def check_bwd(kda, cfg, erase=True, gate="channel", with_dST=True):
+def check_bwd(kda, cfg, erase=True, gate="channel", with_dST=True, memory="auto"):
     x = _variant_inputs(cfg, gate)
     c = I.bwd_cotangents(cfg, with_dST)
     xd, cd = to_dev(x), to_dev(c)
     g = kda.chunk_bwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["S0"], cd["dO"], cd["dST"],
-                      erase=erase, gate=gate)
+                      erase=erase, gate=gate, memory=memory)
     torch.cuda.synchronize()
     ref = oracle.recurrent_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], c["dO"], c["dST"],
                                erase=erase, gate=gate)
@@ -507,7 +507,7 @@ def check_bwd(kda, cfg, erase=True, gate="channel", with_dST=True):
         got = g[n].float().cpu().numpy()
         assert np.isfinite(got).all(), n
         errs[n] = rel_err(got, ref[n]) if got.size else 0.0
-    print(f"PARITY bwd {cfg.name} erase={int(erase)} gate={gate} " + " ".join(f"{n}={e:.2e}" for n, e in errs.items()))
+    print(f"PARITY bwd {cfg.name} erase={int(erase)} gate={gate} memory={memory} " + " ".join(f"{n}={e:.2e}" for n, e in errs.items()))
     for n, e in errs.items():
         assert e <= TOL[cfg.dtype], (cfg.name, erase, gate, n, e)
     return g
@@ -577,3 +577,29 @@ def test_bwd_b4_h32_t8k_sampled(cuda_lib):
             e = rel_err(got.float().cpu().numpy(), want)
             print(f"PARITY bwd full b={b} h={h} {n}={e:.2e}")
             assert e <= TOL["bf16"], (b, h, n, e)
+
+
+@pytest.mark.parametrize("T", [77, 200, 512])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_bwd_low_memory_mode(cuda_lib, dtype, T):
+    """One stored state per 64 tokens and the per-block recompute sweep
+    (the default for workspaces above 16 GB)."""
+    d = 64 if dtype == "f32" else 128
+    check_bwd(cuda_lib, small_cfg(dtype, d, 64, T, B=1, H=2, s0=0.3, seed=76), memory="low")
+
+
+@pytest.mark.parametrize("erase,gate", [(True, "scalar"), (False, "channel")])
+def test_bwd_low_memory_variants(cuda_lib, erase, gate):
+    check_bwd(cuda_lib, small_cfg("bf16", 128, 64, 150, B=1, H=2, s0=0.3, seed=77), erase, gate, memory="low")
+
+
+def test_bwd_modes_agree(cuda_lib):
+    """Both workspace policies run the same arithmetic: bitwise-equal gradients."""
+    cfg = small_cfg("bf16", 128, 64, 300, B=2, H=2, s0=0.3, seed=78)
+    x = to_dev(I.prefill_inputs(cfg))
+    c = to_dev(I.bwd_cotangents(cfg))
+    ga = cuda_lib.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], c["dO"], c["dST"], memory="all")
+    gl = cuda_lib.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], c["dO"], c["dST"], memory="low")
+    torch.cuda.synchronize()
+    for n in BWD_NAMES:
+        assert torch.equal(ga[n], gl[n]), n
