@@ -152,7 +152,8 @@ def decode_step(q, k, v, log_alpha, beta, S, nthreads: int = 0, erase: bool = Tr
     return o, Sn
 
 
-def recurrent_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, erase: bool = True, gate="channel"):
+def recurrent_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, erase: bool = True, gate="channel",
+                     mutation: str | None = None):
     """Packed variable-length sequences: q,k [total_T,H,dk], v [total_T,H,dv],
     beta [total_T,H], log_alpha [total_T,H,dk] / [total_T,H] / None, cu_seqlens
     [N+1] offsets, S0 [N,H,dk,dv] or None. Each sequence is its own recurrence
@@ -167,6 +168,8 @@ def recurrent_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, erase: bool 
     for n in range(N):
         a, b = cu[n], cu[n + 1]
         s0 = None if S0 is None else S0[n:n + 1]
+        if mutation == "state_leaks_between_sequences" and n > 0:
+            s0 = ST[n - 1:n]
         if b == a:
             ST[n] = 0.0 if S0 is None else S0[n]
             continue
@@ -177,7 +180,7 @@ def recurrent_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, erase: bool 
     return o, ST
 
 
-def segment_affine_map(k, v, log_alpha, beta, erase: bool = True, gate="channel"):
+def segment_affine_map(k, v, log_alpha, beta, erase: bool = True, gate="channel", mutation: str | None = None):
     """The update is affine in the state ("Decoding Hybrid Attention
     Architectures" section 3.4: S_t = A_t S_{t-1} + b_t k_t v_t^T with
     A_t = (I - e b_t k_t k_t^T) Diag(a_t)), so a run of tokens maps S_in to
@@ -199,8 +202,11 @@ def segment_affine_map(k, v, log_alpha, beta, erase: bool = True, gate="channel"
         A = np.diag(a)
         if erase:
             A = (np.eye(dk) - beta[t] * np.outer(k[t], k[t])) @ A
-        M = A @ M
-        c = A @ c + beta[t] * np.outer(k[t], v[t])
+        M = M @ A if mutation == "map_order_swapped" else A @ M
+        if mutation == "write_before_erase":
+            c = A @ (c + beta[t] * np.outer(k[t], v[t]))
+        else:
+            c = A @ c + beta[t] * np.outer(k[t], v[t])
     return M, c
 
 
@@ -214,8 +220,15 @@ def segment_scan(maps, S0):
     return S
 
 
+# Planted mistakes in the Python oracle functions, used only by the mutation
+# tests (each must make a pin fail); None = correct.
+BWD_MUTATIONS = ("no_read_key_grad", "decay_before_erase", "lam_for_lam_tilde", "beta_missing_in_dv")
+AFFINE_MUTATIONS = ("write_before_erase", "map_order_swapped")
+VARLEN_MUTATIONS = ("state_leaks_between_sequences",)
+
+
 def recurrent_bwd(q, k, v, log_alpha, beta, S0, do, dST=None, erase: bool = True, gate="channel",
-                  ckpt: int = 64):
+                  ckpt: int = 64, mutation: str | None = None):
     """Gradients of the token recurrence, by reverse-mode differentiation of
     each step (the pages give no backward pass; this is the chain rule applied
     to the update of "Decoding Hybrid Attention Architectures" section 3.4).
@@ -277,14 +290,20 @@ def recurrent_bwd(q, k, v, log_alpha, beta, S0, do, dST=None, erase: bool = True
                     out["dq"][b, t, h] = S_t @ do[b, t, h]
                     g = Lam.T @ kt
                     delta = bt * (r if erase else v[b, t, h])
-                    out["dv"][b, t, h] = bt * g
+                    out["dv"][b, t, h] = (1.0 if mutation == "beta_missing_in_dv" else bt) * g
                     out["dbeta"][b, t, h] = g @ (r if erase else v[b, t, h])
-                    out["dk"][b, t, h] = Lam @ delta - (bt * (St @ g) if erase else 0.0)
+                    read = bt * (St @ g) if erase and mutation != "no_read_key_grad" else 0.0
+                    out["dk"][b, t, h] = Lam @ delta - read
                     Lt = Lam - bt * np.outer(kt, g) if erase else Lam
+                    Ld = Lam if mutation == "lam_for_lam_tilde" else Lt
                     if gate == "channel":
-                        out["dlog_alpha"][b, t, h] = (Lt * St).sum(axis=1)
+                        out["dlog_alpha"][b, t, h] = (Ld * St).sum(axis=1)
                     elif gate == "scalar":
-                        out["dlog_alpha"][b, t, h] = (Lt * St).sum()
-                    Lam = decay(b, t, h)[:, None] * Lt
+                        out["dlog_alpha"][b, t, h] = (Ld * St).sum()
+                    if mutation == "decay_before_erase" and erase:
+                        La = decay(b, t, h)[:, None] * Lam
+                        Lam = La - bt * np.outer(kt, La.T @ kt)
+                    else:
+                        Lam = decay(b, t, h)[:, None] * Lt
             out["dS0"][b, h] = Lam
     return out

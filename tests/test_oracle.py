@@ -341,3 +341,55 @@ def test_bwd_checkpoint_interval_invariant():
     b = oracle.recurrent_bwd(q, k, v, la, beta, S0, do, ckpt=64)
     for n in a:
         assert np.array_equal(a[n], b[n])
+
+
+# ---------------------------------------------------------------- planted mistakes in the Python oracle functions
+
+
+@pytest.mark.parametrize("mutation", oracle.BWD_MUTATIONS)
+def test_bwd_pins_catch_planted_mistakes(mutation):
+    """Each planted mistake in the backward oracle breaks the finite-difference
+    pin (in at least one variant)."""
+    caught = False
+    for erase, gate in [(True, "channel"), (True, "scalar")]:
+        q, k, v, la, beta, S0 = pins.random_inputs(530, T=5, dk=3, dv=2, B_=1, H_=1)
+        lag = la if gate == "channel" else la[..., 0]
+        r = np.random.default_rng(531)
+        Wo, WS = r.standard_normal(v.shape), r.standard_normal(S0.shape)
+        g = oracle.recurrent_bwd(q, k, v, lag, beta, S0, Wo, WS, erase=erase, gate=gate, mutation=mutation)
+        inputs = {"q": q, "k": k, "v": v, "log_alpha": lag, "beta": beta, "S0": S0}
+        names = {"q": "dq", "k": "dk", "v": "dv", "log_alpha": "dlog_alpha", "beta": "dbeta", "S0": "dS0"}
+        for name, gname in names.items():
+            x = inputs[name]
+            fd = np.zeros_like(x)
+            for idx in np.ndindex(x.shape):
+                xp = {kk: vv.copy() for kk, vv in inputs.items()}
+                xm = {kk: vv.copy() for kk, vv in inputs.items()}
+                xp[name][idx] += 1e-6
+                xm[name][idx] -= 1e-6
+                lp = oracle.recurrent(xp["q"], xp["k"], xp["v"], xp["log_alpha"], xp["beta"], xp["S0"], gate=gate)
+                lm = oracle.recurrent(xm["q"], xm["k"], xm["v"], xm["log_alpha"], xm["beta"], xm["S0"], gate=gate)
+                fd[idx] = ((lp[0] * Wo).sum() + (lp[1] * WS).sum() - (lm[0] * Wo).sum() - (lm[1] * WS).sum()) / 2e-6
+            if np.abs(g[gname] - fd).max() > 1e-5:
+                caught = True
+    assert caught, mutation
+
+
+@pytest.mark.parametrize("mutation", oracle.AFFINE_MUTATIONS)
+def test_affine_pins_catch_planted_mistakes(mutation):
+    q, k, v, la, beta, _ = _one_head(532, T=9)
+    M, c = oracle.segment_affine_map(k, v, la, beta, mutation=mutation)
+    S0 = np.random.default_rng(533).standard_normal((6, 5))
+    _, ST = oracle.recurrent(q[None, :, None], k[None, :, None], v[None, :, None], la[None, :, None],
+                             beta[None, :, None], S0[None, None])
+    assert np.abs(M @ S0 + c - ST[0, 0]).max() > 1e-6, mutation
+
+
+@pytest.mark.parametrize("mutation", oracle.VARLEN_MUTATIONS)
+def test_varlen_pins_catch_planted_mistakes(mutation):
+    q, k, v, la, beta, S0 = pins.random_inputs(534, T=21, dk=6, dv=5, B_=3, H_=2)
+    o_d, s_d = oracle.recurrent(q, k, v, la, beta, S0)
+    pack = lambda x: x.reshape((-1,) + x.shape[2:])
+    o_v, s_v = oracle.recurrent_varlen(pack(q), pack(k), pack(v), pack(la), pack(beta), [0, 21, 42, 63], S0,
+                                       mutation=mutation)
+    assert max(np.abs(o_v - pack(o_d)).max(), np.abs(s_v - s_d).max()) > 1e-6, mutation
