@@ -257,3 +257,30 @@ def test_bwd_workspace_modes():
     assert lib.kda_chunk_bwd_workspace_size_ex(1, 77, 2, d, d, 3) == 0
     p = _bwd_good()
     assert lib.kda_chunk_bwd_ex(*p, 1, 8, 1, 64, 64, 1, 1, 0, 7, ctypes.c_void_p(0x100000), 1 << 20, None) == 1
+
+
+def declared_arity():
+    """Number of parameters of every function declared in include/*.h."""
+    arity = {}
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            for name, params in re.findall(r"\b(kda_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", src):
+                params = params.strip()
+                arity[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return arity
+
+
+def test_binding_argtypes_match_declarations():
+    """Every argtypes the Python binding sets has the arity of the C
+    declaration (a missing or extra argument would shift every later one)."""
+    lib = kda.load()
+    arity = declared_arity()
+    checked = 0
+    for name, n in arity.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is not None:
+            assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+            checked += 1
+    assert checked >= 10, checked
