@@ -201,7 +201,9 @@ def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, chunk: in
     if S_T is not None:
         _need(S_T, "S_T", (N, H, dk, dv), torch.float32, dev)
     dts = _dtype_of(q)
-    ws_bytes = workspace_size(N, TT, H, dk, dv, chunk, dts, algo)
+    # packed batches never take the segment scan: size the workspace for one pass
+    ws_bytes = workspace_size(N, TT, H, dk, dv, chunk, dts, "tc" if algo == "auto" and dts == "bf16" and
+                              dk == dv == 128 and chunk == 64 else algo)
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
