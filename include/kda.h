@@ -1,6 +1,9 @@
 /*
  * kda.h -- C ABI of libkda.so: KDA (fine-grained gated delta rule) chunkwise
- * prefill and single-token decode on NVIDIA B200 (sm_100a).
+ * prefill (dense or packed batches, optional chunk-parallel segment scan), its
+ * backward pass, and the single-token decode step on NVIDIA B200 (sm_100a);
+ * the delta-rule and gated-linear-attention variants run through the same
+ * calls.
  *
  * The operation (pages: "Decoding Hybrid Attention Architectures", section
  * 3.4 and its variant table; "Technical Analysis ... Novel Hybrid Linear
