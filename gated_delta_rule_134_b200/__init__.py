@@ -10,8 +10,8 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["load", "chunk_fwd", "chunk_fwd_varlen", "chunk_bwd", "chunk_fwd_noalloc", "decode_step", "workspace_size", "workspace_status", "KDAError",
-           "library_path", "STATUS"]
+__all__ = ["load", "chunk_fwd", "chunk_fwd_varlen", "chunk_bwd", "chunk_fwd_noalloc", "noalloc_status", "decode_step",
+           "workspace_size", "workspace_status", "KDAError", "library_path", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libkda.so")
@@ -66,6 +66,8 @@ def load(build_if_stale: bool = True):
     lib.kda_decode_step.restype = I
     lib.kda_chunk_fwd_noalloc.argtypes = [P] * 8 + [I] * 7 + [P]
     lib.kda_chunk_fwd_noalloc.restype = I
+    lib.kda_noalloc_status.argtypes = [P]
+    lib.kda_noalloc_status.restype = I
     lib.kda_chunk_fwd_v.argtypes = [P] * 8 + [I] * 9 + [P, Z, I, P]
     lib.kda_chunk_fwd_v.restype = I
     lib.kda_decode_step_v.argtypes = [P] * 8 + [I] * 7 + [P]
@@ -102,10 +104,20 @@ def _dtype_of(t) -> str:
     raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
 
 
-def _stream(stream):
+def _stream(stream, device=None):
+    """The stream handle to pass: the given torch stream, else the current
+    stream of `device` (the tensors' device), else of the current device."""
     import torch
-    s = stream if stream is not None else torch.cuda.current_stream()
+    s = stream if stream is not None else torch.cuda.current_stream(device)
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _on(device):
+    """Make the tensors' device current for the call: the library launches on
+    the current device (and the allocation-free entry point looks up its
+    scratch array there), so it must be the device the pointers live on."""
+    import torch
+    return torch.cuda.device(device)
 
 
 def _need(t, name, shape, dtype, device):
@@ -163,9 +175,10 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, chunk: int = 64, algo: str =
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
     la = log_alpha if gshape is not None else None
-    code = lib.kda_chunk_fwd_v(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0), _ptr(o),
-                               _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPE[dts], int(bool(erase)), GATES[gate],
-                               _ptr(workspace), ws_len, _ALGO[algo], _stream(stream))
+    with _on(dev):
+        code = lib.kda_chunk_fwd_v(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0), _ptr(o),
+                                   _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPE[dts], int(bool(erase)), GATES[gate],
+                                   _ptr(workspace), ws_len, _ALGO[algo], _stream(stream, dev))
     _check("kda_chunk_fwd_v", code)
     return o, S_T
 
@@ -208,9 +221,11 @@ def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, chunk: in
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
     la = log_alpha if gshape is not None else None
-    code = lib.kda_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T),
-                                    _ptr(cu_seqlens), N, TT, H, dk, dv, chunk, _DTYPE[dts], int(bool(erase)),
-                                    GATES[gate], _ptr(workspace), ws_len, _ALGO[algo], _stream(stream))
+    with _on(dev):
+        code = lib.kda_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0), _ptr(o),
+                                        _ptr(S_T), _ptr(cu_seqlens), N, TT, H, dk, dv, chunk, _DTYPE[dts],
+                                        int(bool(erase)), GATES[gate], _ptr(workspace), ws_len, _ALGO[algo],
+                                        _stream(stream, dev))
     _check("kda_chunk_fwd_varlen", code)
     return o, S_T
 
@@ -252,10 +267,12 @@ def chunk_bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None, *, erase: bool = True
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
     la = log_alpha if gshape is not None else None
-    code = lib.kda_chunk_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0), _ptr(dO), _ptr(dS_T),
-                                _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]),
-                                _ptr(g["dS0"]), B, T, H, dk, dv, _DTYPE[_dtype_of(q)], int(bool(erase)), GATES[gate],
-                                mode, _ptr(workspace), ws_len, _stream(stream))
+    with _on(dev):
+        code = lib.kda_chunk_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S0), _ptr(dO),
+                                    _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]),
+                                    _ptr(g["dbeta"]), _ptr(g["dS0"]), B, T, H, dk, dv, _DTYPE[_dtype_of(q)],
+                                    int(bool(erase)), GATES[gate], mode, _ptr(workspace), ws_len,
+                                    _stream(stream, dev))
     _check("kda_chunk_bwd_ex", code)
     return g
 
@@ -263,7 +280,9 @@ def chunk_bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None, *, erase: bool = True
 def workspace_status(workspace, stream=None) -> int:
     """Synchronise and return the device-side status word of a workspace."""
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    return int(load().kda_workspace_status(_ptr(workspace), ws_len, _stream(stream)))
+    dev = None if workspace is None else workspace.device
+    with _on(dev):
+        return int(load().kda_workspace_status(_ptr(workspace), ws_len, _stream(stream, dev)))
 
 
 def decode_step(q, k, v, log_alpha, beta, S, *, S_out=None, o=None, stream=None, erase: bool = True,
@@ -292,9 +311,10 @@ def decode_step(q, k, v, log_alpha, beta, S, *, S_out=None, o=None, stream=None,
         o = torch.empty(N, H, dv, dtype=dt, device=dev)
     _need(o, "o", (N, H, dv), dt, dev)
     la = log_alpha if gshape is not None else None
-    code = lib.kda_decode_step_v(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S), _ptr(S_out),
-                                 _ptr(o), N, H, dk, dv, _DTYPE[_dtype_of(q)], int(bool(erase)), GATES[gate],
-                                 _stream(stream))
+    with _on(dev):
+        code = lib.kda_decode_step_v(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(S), _ptr(S_out),
+                                     _ptr(o), N, H, dk, dv, _DTYPE[_dtype_of(q)], int(bool(erase)), GATES[gate],
+                                     _stream(stream, dev))
     _check("kda_decode_step_v", code)
     return o, S_out
 
@@ -306,7 +326,8 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0=None, *, o, S_T=None, chunk: 
     prefill: the library keeps the kernel's small scratch in a fixed array of
     its own, so only inputs and caller-owned outputs (o, and S_T if wanted)
     are passed. bf16 inputs, dk = dv = 128, chunk = 64. Calls that overlap on
-    the GPU share that array and race. Returns (o, S_T)."""
+    the GPU share that array and race; noalloc_status reads its status word.
+    Returns (o, S_T)."""
     import torch
     lib = load()
     B, T, H, dk = q.shape
@@ -322,7 +343,19 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0=None, *, o, S_T=None, chunk: 
         _need(S0, "S0", (B, H, dk, dv), torch.float32, dev)
     if S_T is not None:
         _need(S_T, "S_T", (B, H, dk, dv), torch.float32, dev)
-    code = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(o),
-                                     _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPE[_dtype_of(q)], _stream(stream))
+    with _on(dev):
+        code = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                                         _ptr(o), _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPE[_dtype_of(q)],
+                                         _stream(stream, dev))
     _check("kda_chunk_fwd_noalloc", code)
     return o, S_T
+
+
+def noalloc_status(device=None, stream=None) -> int:
+    """kda_noalloc_status: synchronise and return the status word the last
+    chunk_fwd_noalloc on `device` left in the library's own scratch array
+    (0 = KDA_OK, 4 = KDA_ERR_TIMEOUT). Allocates nothing."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with _on(dev):
+        return int(load().kda_noalloc_status(_stream(stream, dev)))

@@ -16,7 +16,9 @@ int scan_mode_of(kda_algo_t algo) { return algo == KDA_ALGO_TC_SCAN ? 2 : (algo 
 
 kda_status_t run_chunk(const kda::ChunkArgs& a, kda_dtype_t dtype, kda_algo_t algo, void* stream);
 
-kda_status_t check_chunk_args(const kda::ChunkArgs& a, kda_dtype_t dtype) {
+}  // namespace
+
+kda_status_t kda::check_chunk_args(const kda::ChunkArgs& a, kda_dtype_t dtype) {
     if (a.B < 0 || a.T < 0 || a.H < 0) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (!head_dims_ok(a.dk, a.dv)) return KDA_ERR_UNSUPPORTED;
@@ -36,8 +38,6 @@ kda_status_t check_chunk_args(const kda::ChunkArgs& a, kda_dtype_t dtype) {
     if (a.ST && !aligned16(a.ST)) return KDA_ERR_INVALID_ARG;
     return KDA_OK;
 }
-
-}  // namespace
 
 extern "C" {
 
@@ -101,7 +101,7 @@ kda_status_t run_chunk(const kda::ChunkArgs& a, kda_dtype_t dtype, kda_algo_t al
     const int B = a.B, T = a.T, H = a.H, dk = a.dk, dv = a.dv;
     void* workspace = a.workspace;
     const size_t workspace_bytes = a.workspace_bytes;
-    kda_status_t st = check_chunk_args(a, dtype);
+    kda_status_t st = kda::check_chunk_args(a, dtype);
     if (st != KDA_OK) return st;
     if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TC && algo != KDA_ALGO_TC_SCAN)
         return KDA_ERR_INVALID_ARG;

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 
+#include "kda.h"
+
 namespace kda {
 
 struct ChunkArgs {
@@ -23,6 +25,11 @@ struct ChunkArgs {
     void* workspace;
     size_t workspace_bytes;
 };
+
+// Synchronous argument validation shared by every prefill entry point
+// (sizes, dtype, head and chunk sizes, variant switches, required pointers
+// and their 16-byte alignment). Launches nothing.
+kda_status_t check_chunk_args(const ChunkArgs& a, kda_dtype_t dtype);
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* la, const void* beta,
                           const float* S_in, float* S_out, void* o, int N, int H, int dk, int dv, int bf16,

@@ -46,7 +46,7 @@ typedef enum {
     KDA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, workspace too small */
     KDA_ERR_UNSUPPORTED = 2, /* valid but not implemented (head size, chunk size, dtype) */
     KDA_ERR_CUDA = 3,        /* a CUDA launch or query failed; see cudaGetLastError */
-    KDA_ERR_TIMEOUT = 4      /* a bounded device-side wait expired (reported by kda_workspace_status) */
+    KDA_ERR_TIMEOUT = 4      /* a bounded device-side wait expired (kda_workspace_status, kda_noalloc_status) */
 } kda_status_t;
 
 typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
@@ -223,10 +223,22 @@ kda_status_t kda_chunk_bwd_ex(const void *q, const void *k, const void *v, const
                               size_t workspace_bytes, void *stream);
 
 /*
- * Device-side status left in `workspace` by the last kda_chunk_fwd_ex that
- * used it: synchronises `stream`, then returns KDA_OK, or KDA_ERR_TIMEOUT if
- * a bounded wait inside a kernel gave up (that kernel's outputs are then
- * invalid), or KDA_ERR_CUDA if the stream reported an error.
+ * Device-side status left in `workspace` by the last prefill call
+ * (kda_chunk_fwd, _ex, _v, _varlen) that used it: synchronises `stream`,
+ * then returns KDA_OK, or KDA_ERR_TIMEOUT if a bounded wait inside a kernel
+ * gave up (that kernel's outputs are then invalid), or KDA_ERR_CUDA if the
+ * stream reported an error.
+ *
+ * Which calls can report KDA_ERR_TIMEOUT: only the prefill calls that run the
+ * tensor-core kernel (KDA_ALGO_TC, KDA_ALGO_TC_SCAN, or AUTO where it picks
+ * them). Its warps hand work to one another through shared-memory barriers;
+ * every wait on one gives up after about one second of SM clock, writes 1
+ * into the first 4 bytes of the workspace, skips every later wait and frees
+ * its tensor memory, so the kernel always returns. The call itself cannot see
+ * this (it returns once the work is enqueued): read it here, or with
+ * kda_noalloc_status for kda_chunk_fwd_noalloc. The SIMT prefill, the decode
+ * step and the backward pass have no waits between warps that could run out
+ * (only block-wide barriers) and never report it.
  */
 kda_status_t kda_workspace_status(const void *workspace, size_t workspace_bytes, void *stream);
 
@@ -269,19 +281,31 @@ kda_status_t kda_decode_step_v(const void *q, const void *k, const void *v, cons
  *     dk = dv = 128, chunk = 64 (else KDA_ERR_UNSUPPORTED). A shape whose
  *     scratch would exceed the 256-byte array is refused with
  *     KDA_ERR_INVALID_ARG (no supported shape needs more than 256 bytes).
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before capturing any CUDA graph.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress,
+ *     a host-side query) with the caller's current device, which must be the
+ *     device of the tensors. The very first call in a process may also load
+ *     the library's device code; make that first call before capturing any
+ *     CUDA graph.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind; each call clears the status word before its kernel runs. Calls
  *     that overlap on the GPU (different streams, no ordering) race on the
- *     array. A device-side timeout is recorded in the array and is not
- *     reported back through kda_workspace_status; callers that need that
- *     report use kda_chunk_fwd with their own workspace.
+ *     array. A device-side timeout is recorded in the array and read back by
+ *     kda_noalloc_status.
  */
 kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *log_alpha,
                                    const void *beta, const float *S0, void *o, float *S_T, int B, int T,
                                    int H, int dk, int dv, int chunk, kda_dtype_t dtype, void *stream);
+
+/*
+ * Device-side status of the last kda_chunk_fwd_noalloc on the current device
+ * (the counterpart of kda_workspace_status for the library's own array; no
+ * counterpart in the paper). Synchronises `stream`, then copies the 4-byte
+ * status word out of the array (no allocation): KDA_OK, KDA_ERR_TIMEOUT if a
+ * bounded wait in that call's kernel gave up (its outputs are then invalid),
+ * or KDA_ERR_CUDA if the stream or the copy reported an error. Racy in the
+ * same way as the calls themselves when they overlap on the GPU.
+ */
+kda_status_t kda_noalloc_status(void *stream);
 
 #ifdef __cplusplus
 }
