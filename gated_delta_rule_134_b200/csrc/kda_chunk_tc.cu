@@ -17,40 +17,45 @@
 // Reference-point factorisation. With G_m the gate at the chunk's middle token
 // and E_r = e^{G_r - G_m}, F_r = e^{G_m - G_r} (per channel):
 //   e^{G_r - G_s} = E_r F_s,  k e^G = (k E) e^{G_m},  k e^{G_last-G} = (k F) e^{G_last-G_m}.
-// So three bf16 tiles, KE = k E, QE = q E and KF = k F, feed every MMA:
-//   G = [L; L] g            -> gate prefix sums (L: lower-triangular ones)
-//   [KE; QE] KF^T           -> A and P (one M=128 MMA)
-//   [T'; 0] [v | KE]        -> [U; 0] and W' = T' KE, W = W' Diag(e^{G_m})
-//   D1 += [-W'; QE] (e^{G_m} S)   -> rows 0-63: U - W S = delta, rows 64-127: (q e^G) S
+// Three bf16 tiles, KE = k E, QE = q E and KF = k F, feed every MMA. The
+// output is regrouped so that P never meets the state: with PT = P T',
+//   O = QE S^ + P (U - W' S^) = (QE - P W') S^ + P T' v,   S^ = e^{G_m} S, W' = T' KE,
+// so per chunk the state-independent MMAs are
+//   G = [L; L] g                  -> gate prefix sums (L: lower-triangular ones)
+//   [A; P] = [KE; QE] KF^T        (one M=128 MMA)
+//   PT = P T'
+//   [W'; P W'] = [T'; PT] KE      -> row operand [-W'; QE - P W']
+//   [U; P T' v] = [T'; PT] v      -> the chunk's accumulator
+// and the state chain needs only two:
+//   D += [-W'; QE - P W'] S^      -> rows 0-63: delta, rows 64-127: O
 //   R  = e^{G_m} S + KF^T delta   -> S_next = Diag(e^{G_last-G_m}) R
-//   D1 += [* ; P] delta     -> rows 64-127: O (rows 0-63, already read, take junk)
-// The tensor memory therefore holds R, and the next chunk rescales it per
-// channel while it copies the state into the bf16 MMA operand. Each factor is
-// a single exponential, finite as long as |G_r - G_m| <= 80 and G_m >= -80;
-// a block-wide guard checks that per chunk. A chunk that fails the guard uses
-// exact per-pair exponentials e^{G_r - G_s} (exponent <= 0) for A and P and the
+// The tensor memory holds R, and the next chunk rescales it per channel while
+// it copies the state into the bf16 MMA operand. Each factor is a single
+// exponential, finite as long as |G_r - G_m| <= 80 and |G_m| <= 80; a vote of
+// the tile warps checks that per chunk. A chunk that fails it uses exact
+// per-pair exponentials e^{G_r - G_s} (exponent <= 0) for A and P and the
 // plain tiles k e^G, q e^G, k e^{G_last-G} (with G_m := 0); the same MMAs then
 // produce the same quantities.
 //
 // Schedule. One CTA owns one (batch, head) and a DVT-wide slice of value
-// channels; its state stays in tensor memory for the whole sequence. Three
-// warp roles run concurrently and hand work over through mbarriers:
-//   prep  (warps 0-7)  per chunk m: A/P readout, (I + A)^{-1} -> T'; then the
-//                      operand tiles of chunk m+1 (prefix sums out of tensor
-//                      memory, guard, KE/QE in place over the raw k/q rows, KF
-//                      over the log_alpha tile), which covers the U/W MMAs of
-//                      chunk m; then -W' of chunk m over its KE rows.
-//   chain (warps 8-11) per chunk n, the state-dependent part: state -> bf16
-//                      operand, MMA1 (two halves of the key channels, so one
-//                      16 KB operand buffer serves both), delta -> bf16,
-//                      MMA2, O -> global. Warp 8 issues these MMAs.
-//   control (warp 12)  every TMA load (plus an L2 prefetch of the next
-//                      chunk's tiles) and the state-independent MMAs, issued
-//                      from a polling loop in the order their inputs appear.
-// k/q tiles and the operand tiles built from them are double-buffered by
-// chunk parity, the per-channel scales by chunk mod 4. A/P land in the
-// prefix-sum columns once those are read, so the A/P MMA of chunk m+1 runs
-// while the prep warps finish chunk m.
+// channels; its state stays in tensor memory for the whole sequence. Each
+// chunk m lives in one of three tensor-memory slots (m mod 3) from its prefix
+// sums to its output, so the state-independent work of chunks m+1 and m+2
+// runs while the chain works on chunk m. Three warp groups hand work over
+// through mbarriers:
+//   chain (warps 0-3)   state -> bf16 operand, MMA1 (two halves of the key
+//                       channels through one 16 KB operand buffer), delta ->
+//                       bf16, MMA2, O -> global; it also issues the TMA loads
+//                       of k/q and log_alpha into the buffers its MMAs free.
+//   tile  (warps 4-7)   prefix sums out of tensor memory, KE/QE in place over
+//                       the raw k/q rows, KF over the log_alpha tile, the
+//                       overflow vote, per-channel scales; issues the [A; P]
+//                       MMA and the next chunk's prefix-sum MMA.
+//   inverse (warps 8-15) A/P readout, (I + A)^{-1} -> T', the PT, W and U
+//                       MMAs and their readouts into the row operand; issues
+//                       the v loads.
+// k/q tiles are double-buffered, the log_alpha/KF tiles triple-buffered, the
+// per-channel scales kept by chunk mod 4.
 // (I + A)^{-1}: 16x16 diagonal blocks by forward substitution (four threads per
 // column), then one column chain per warp, T_ab = -T_aa sum_k A_ak T_kb, on
 // m16n8k8 tf32 MMAs; T' = T Diag(beta) is written as bf16 by the thread that
@@ -58,7 +63,8 @@
 //
 // Every wait on an mbarrier is bounded; on expiry the kernel records status 1
 // in the caller's workspace word and stops waiting (later waits are skipped,
-// so every role reaches the end), frees its tensor memory and returns.
+// so every role reaches the end), waits for its copies and MMAs in flight,
+// frees its tensor memory and returns.
 #include <algorithm>
 #include <type_traits>
 
@@ -72,82 +78,81 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kPrep = 256;                    // warps 0-7: operand tiles, A/P readout, UT inverse, -W'
-constexpr int kChainWarp0 = kPrep / 32;       // warps 8-11: state chain
-constexpr int kCtrlWarp = kChainWarp0 + 4;    // warp 12: loads and state-independent MMAs
-constexpr int kThreads = 32 * (kCtrlWarp + 1);
+constexpr int kTileWarp0 = 4;   // warps 0-3: chain; 4-7: tiles; 8-15: inverse and W/U side
+constexpr int kInvWarp0 = 8;
+constexpr int kThreads = 512;
 // named barriers (0 is __syncthreads)
-constexpr int NB_PREP = 1;  // prep warps
-constexpr int NB_OR = 2;    // prep warps, OR-reduction
-constexpr int NB_CHA = 5;   // chain warps 8-9
-constexpr int NB_CHB = 6;   // chain warps 10-11 -> warp 8: second half of the state operand stored
-constexpr int NB_CHC = 7;   // chain warps 10-11
-constexpr int NB_CH = 8;    // all chain warps
+constexpr int NB_TILE = 1;  // tile warps
+constexpr int NB_TOR = 2;   // tile warps, OR-vote
+constexpr int NB_INV = 3;   // inverse warps
+constexpr int NB_CHLO = 4;  // chain warps 0-1
+constexpr int NB_CHB = 5;   // chain warps 2-3 -> warp 0: second half of the state operand stored
+constexpr int NB_CHHI = 6;  // chain warps 2-3
+constexpr int NB_CH = 7;    // all chain warps
 constexpr int kC = 64;    // chunk
 constexpr int kD = 128;   // dk = dv
 constexpr int kLDA = 68;  // fp32 row stride of the A / T scratch (bank spread)
-constexpr float kGuard = 80.f;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kGuardL = 80.f * kLog2e;      // |G_r - G_m| <= 80, in log2 units
 constexpr long long kWaitBudget = 1ll << 31;  // SM cycles (~1 s)
+constexpr long long kDrainBudget = 1ll << 24;
 
 template <int DVT>
 struct Layout {
     // shared memory, bytes from a 1024-aligned base
-    static constexpr uint32_t ROWOP = 0;            // 2 x 32 KB, K-major: per 64-channel box x (x * 16 KB)
-                                                    //   rows 0-63: k -> KE -> -W', rows 64-127: q -> QE
-    static constexpr uint32_t COLOP = 65536;        // 2 x 16 KB: log_alpha tile, then KF (box x at x * 8 KB)
-    static constexpr uint32_t RAWV = 98304;         // v slice: DVT/64 boxes of [64 tok][64 ch]
-    static constexpr uint32_t LMAT = 114688;        // [L; L] K-major 128 x 64
-    static constexpr uint32_t TZP = 131072;         // [T'; 0] K-major 128 x 64
-    static constexpr uint32_t SP = TZP + 16384;     // 2 x P, K-major 64 x 64 bf16 (8 KB each)
-    static constexpr uint32_t SCR = SP + 16384;     // A, T fp32 [64][kLDA] (exact path: G fp32 [64][128])
+    static constexpr uint32_t ROW = 0;          // 2 x 32 KB, K-major: per 64-channel box x (x * 16 KB)
+                                                //   rows 0-63: k -> KE -> -W', rows 64-127: q -> QE -> QE - P W'
+    static constexpr uint32_t COL = 65536;      // 3 x 16 KB: log_alpha tile, then KF (box x at x * 8 KB)
+    static constexpr uint32_t RAWV = 114688;    // v slice: DVT/64 boxes of [64 tok][64 ch]
+    static constexpr uint32_t LMAT = 131072;    // [L; L] K-major 128 x 64
+    static constexpr uint32_t TP = 147456;      // [T'; PT] K-major 128 x 64
+    static constexpr uint32_t SP = TP + 16384;  // P, K-major 64 x 64 bf16 (rows 64-127 of [Y; P], Y = TP rows 64-127)
+    static constexpr uint32_t SOP = SP + 8192;  // S half (64 channels) x DVT, bf16 MN-major, then delta
+    static constexpr uint32_t SCR = SOP + 64 * DVT * 2;  // A, T fp32 [64][kLDA]; exact path: staging
     static constexpr uint32_t SA = SCR;
     static constexpr uint32_t ST = SCR + 64 * kLDA * 4;
-    static constexpr uint32_t SOP = SCR + 2 * 64 * kLDA * 4;  // S half (64 channels) x DVT, bf16 MN-major
-    static constexpr uint32_t DOP = SOP;                      //   then delta (64 tokens) x DVT
-    static constexpr uint32_t SMALL = SOP + 64 * DVT * 2;
-    static constexpr uint32_t SBETA = SMALL;        // 64 f32: beta of the chunk the prep warps work on
+    static constexpr uint32_t SMALL = SCR + 2 * 64 * kLDA * 4;
+    static constexpr uint32_t SBETA = SMALL;        // 64 f32: beta of the inverse warps' chunk
     static constexpr uint32_t SOPS = SBETA + 256;   // 4 x 128 f32: operand scale per channel (by chunk mod 4)
     static constexpr uint32_t STMS = SOPS + 2048;   // 4 x 128 f32: tensor-memory scale per channel
     static constexpr uint32_t SEK = STMS + 2048;    // 128 f32: e^{G_last - G_m} of the last prepared chunk
-    static constexpr uint32_t SGM = SEK + 512;      // 128 f32: G_m of the chunk being prepared
+    static constexpr uint32_t SGM = SEK + 512;      // 128 f32: G_m of the tile warps' chunk
     static constexpr uint32_t SGL = SGM + 512;      // 128 f32: G_last
-    static constexpr uint32_t SGS = SGL + 512;      // 64 f32: prefix sums of a per-token gate
-    static constexpr uint32_t BARS = SGS + 256;     // mbarriers
-    static constexpr uint32_t MISC = BARS + 256;    // tmem base, abort flag, guard verdicts
-    static constexpr uint32_t END = MISC + 16;
+    static constexpr uint32_t SGML = SGL + 512;     // 128 f32: -G_m log2(e)
+    static constexpr uint32_t BARS = SGML + 512;    // mbarriers
+    static constexpr uint32_t MISC = BARS + 512;    // tmem base, abort flag
+    static constexpr uint32_t END = MISC + 64;
     static constexpr uint32_t SMEM_BYTES = END + 1024;   // + alignment slack
     static constexpr uint32_t SBO_V = 1024 * (DVT / 64); // K-group stride of the S / delta operands
-    static_assert(SOP % 1024 == 0, "operand alignment");
+    static_assert(SOP % 1024 == 0 && TP % 1024 == 0 && LMAT % 1024 == 0, "operand alignment");
     static_assert(64 * 128 * 4 <= 2 * 64 * kLDA * 4, "exact-path gate staging overflows the scratch");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    // tensor memory columns
-    static constexpr uint32_t S_COL = 0;     // R (fp32, lane = key channel)
-    static constexpr uint32_t D1_COL = 128;  // [U; 0] -> [delta; O] (lane = token row)
-    static constexpr uint32_t W_COL = 256;   // [W'; 0]
-    static constexpr uint32_t GC_COL = 384;  // [G; G] (lane = token, col = channel), then [A; P] (64 cols)
+    // tensor memory columns: R (fp32, lane = key channel) and three chunk slots
+    static constexpr uint32_t S_COL = 0;
+    static constexpr uint32_t SLOT0 = 128;
     static constexpr uint32_t TMEM_COLS = 512;
 };
 
 // mbarrier slots
 enum : int {
-    BAR_KQ = 0,      // 2: k/q tiles landed (by chunk parity)
-    BAR_G = 2,       // 2: log_alpha tile landed
-    BAR_V = 4,       // v tile landed
-    BAR_CS = 5,      // prefix-sum MMA done
-    BAR_AP = 6,      // A/P MMA done
-    BAR_UW = 7,      // U/W MMA done
-    BAR_M1A = 8,     // MMA1, first half, done
-    BAR_M1 = 9,      // MMA1 done
-    BAR_M2 = 10,     // MMA2 done
-    BAR_M1B = 11,    // 2: MMA1 of the chunk of this parity done (row operand free)
-    BAR_M2B = 13,    // 2: MMA2 of the chunk of this parity done (KF, P free)
-    BAR_D1 = 15,     // delta and O read out of tensor memory (D1 free)
-    BAR_SC = 16,     // 4: per-channel scales of the chunk (mod 4) stored
-    BAR_RR = 20,     // 2: row operand [-W'; QE] of the chunk of this parity stored
-    BAR_P2 = 22,     // operand tiles of a chunk stored, its prefix sums read
-    BAR_P4 = 23,     // A/P of a chunk read out (tensor-memory columns free)
-    BAR_P5 = 24,     // T' of a chunk stored, A/T scratch free
-    NUM_BARS = 25
+    B_KQ = 0,     // 2: k/q tiles landed (by chunk parity)
+    B_G = 2,      // 3: log_alpha tile (or per-token gate row) of the chunk (mod 3) in place
+    B_V = 5,      // v tile landed
+    B_CS = 6,     // 3: prefix-sum MMA of the slot's chunk done
+    B_AP = 9,     // 3: [A; P] of the slot's chunk in tensor memory
+    B_PT = 12,    // PT MMA done
+    B_WB = 13,    // [W'; P W'] MMA done
+    B_UO = 14,    // 3: [U; P T' v] MMA of the slot's chunk done (also frees [T'; PT] and the v tile)
+    B_RR = 17,    // 2: row operand [-W'; QE - P W'] of the chunk of this parity stored
+    B_SC = 19,    // 4: per-channel scales of the chunk (mod 4) stored
+    B_M1A = 23,   // MMA1, first half, done
+    B_M1 = 24,    // MMA1 done (row operand free)
+    B_M2 = 25,    // MMA2 done (KF and delta operand free, R updated)
+    B_SF = 28,    // 3: the slot's chunk read out by the chain (count 2)
+    B_SCRF = 31,  // A/T scratch of the inverse warps' chunk free
+    B_EXKQ = 32,  // k/q reloaded for an exact chunk
+    B_FIN = 33,   // 3: final drain of each MMA-issuing thread
+    NUM_BARS = 36
 };
 
 // offset of element (row R, channel c) of a row-operand buffer (K-major, two
@@ -161,11 +166,10 @@ __device__ __forceinline__ uint32_t km_off(int r, int s) {
     return (uint32_t)(r * 128 + ((((s >> 3) ^ (r & 7))) << 4) + ((s & 7) << 1));
 }
 
-// 1/x by the hardware reciprocal approximation (one MUFU operation; the
-// FMA pipe stays free for the products around it)
-__device__ __forceinline__ float rcp_approx(float x) {
+// 2^x by the hardware approximation (one MUFU operation)
+__device__ __forceinline__ float ex2(float x) {
     float r;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
     return r;
 }
 
@@ -223,9 +227,14 @@ __device__ __forceinline__ bool nb_or(int id, int nthreads, bool pred) {
     return r != 0;
 }
 
-// ERASE: 1 delta-rule family, 0 additive write. GATE: 0 per-channel log_alpha,
-// 1 one per token and head, 2 none. Compile-time, so each variant is its own
-// kernel and the KDA instance carries no variant branches.
+// 32 lanes x 1 column (the x1 form of tmem_ld32)
+__device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait1(uint32_t& r) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r) : : "memory");
+}
+
 // Chunk-parallel scan over segments of each sequence (few heads, long T).
 // The update is affine in the state, so a segment maps its entry state S_in
 // to M S_in + C. Phase 1 runs segment 0 in full and, for each middle segment
@@ -241,6 +250,9 @@ struct SegJobs {
     float* Sin;  // [B*H][P-1][dk][dv]: state entering segment j at [j-1]
 };
 
+// ERASE: 1 delta-rule family, 0 additive write. GATE: 0 per-channel log_alpha,
+// 1 one per token and head, 2 none. Compile-time, so each variant is its own
+// kernel and the KDA instance carries no variant branches.
 template <int DVT, int ERASE, int GATE>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
@@ -248,7 +260,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     const __nv_bfloat16* __restrict__ beta, const float* S0, __nv_bfloat16* __restrict__ o,
                     float* ST, int Tlen, int H, unsigned* status, const __nv_bfloat16* __restrict__ gate_tok,
                     const int* __restrict__ cu_seqlens, const SegJobs sj) {
-    constexpr int erase = ERASE, gate = GATE;
+    constexpr int erase = ERASE;
     using L = Layout<DVT>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base (the 128-byte swizzle repeats every 1024 bytes);
@@ -258,6 +270,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const uint32_t sb = smem_u32(sm);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3;  // tensor-memory lane quadrant this warp may access
     const int nslices = kD / DVT;
     const int unit = blockIdx.x / nslices;  // the (sequence-head, piece) of this CTA
     const int per = sj.P == 0 ? 1 : (sj.phase == 1 ? 2 * sj.P - 3 : sj.P - 1);
@@ -308,7 +321,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
     const int j0 = (blockIdx.x % nslices) * DVT;
     const int NC = (seq_len + kC - 1) / kC;
-    const int quad = warp & 3;  // tensor-memory lane quadrant this warp may access
 
     float* sBeta = reinterpret_cast<float*>(sm + L::SBETA);
     float* sOpS = reinterpret_cast<float*>(sm + L::SOPS);
@@ -316,16 +328,16 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     float* sEK = reinterpret_cast<float*>(sm + L::SEK);
     float* sGm = reinterpret_cast<float*>(sm + L::SGM);
     float* sGl = reinterpret_cast<float*>(sm + L::SGL);
+    float* sGmL = reinterpret_cast<float*>(sm + L::SGML);
     float* sA = reinterpret_cast<float*>(sm + L::SA);
     float* sT = reinterpret_cast<float*>(sm + L::ST);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BARS);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
-    volatile int* s_exact = reinterpret_cast<volatile int*>(sm + L::MISC + 8);  // 2: guard verdict by parity
 
     // ---------------------------------------------------------------- setup
     if (tid == 0) {
-        for (int i = 0; i < NUM_BARS; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < NUM_BARS; ++i) mbar_init(bars + i, (i >= B_SF && i < B_SF + 3) ? 2u : 1u);
         *s_abort = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_k);
@@ -337,8 +349,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         tmem_alloc(s_tmem, L::TMEM_COLS);
         tmem_relinquish();
     }
-    {   // constants: [L; L] (row R: ones in columns 0..R%64) and [T'; 0], whose
-        // blocks above the diagonal and zero half are never written again
+    {   // constants: [L; L] (row R: ones in columns 0..R%64) and the T' half of
+        // [T'; PT], whose blocks above the diagonal are never written again
         for (int i = tid; i < 128 * 8; i += kThreads) {
             const int R = i >> 3, j = i & 7, r = R & 63;
             uint32_t w[4];
@@ -348,7 +360,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 w[u] = pack_bf16x2(s <= r ? 1.f : 0.f, s + 1 <= r ? 1.f : 0.f);
             }
             st_shared_v4(sb + L::LMAT + R * 128 + ((j ^ (R & 7)) << 4), w[0], w[1], w[2], w[3]);
-            st_shared_v4(sb + L::TZP + R * 128 + (j << 4), 0u, 0u, 0u, 0u);
+            if (R < 64) st_shared_v4(sb + L::TP + R * 128 + (j << 4), 0u, 0u, 0u, 0u);
         }
         for (int c = tid; c < kD; c += kThreads) sEK[c] = 1.f;
         if (v_zero)  // transition run: v = 0 stays in the v tile, which is never loaded
@@ -375,157 +387,111 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         __syncwarp();
         tc_fence_after();
     };
-    auto rowop = [&](int par) -> uint32_t { return sb + L::ROWOP + (uint32_t)par * 32768; };
-    auto colop = [&](int par) -> uint32_t { return sb + L::COLOP + (uint32_t)par * 16384; };
+    // After an abort: wait (bounded) for the last phase a barrier was armed for,
+    // so no copy or MMA is still writing when the CTA exits.
+    auto drain = [&](int slot, int count) {
+        if (*s_abort && count > 0) mbar_wait_bounded(bars + slot, (uint32_t)(count - 1) & 1u, kDrainBudget);
+    };
 
-    constexpr uint32_t ID_CS = idesc_bf16(128, 128, 0, 1);
+    constexpr uint32_t ID_CS = idesc_bf16(128, 128, 0, 1);   // [L; L] x g (MN-major)
+    constexpr uint32_t ID_CS1 = idesc_bf16(128, 16, 0, 0);   // [L; L] x per-token gate row (K-major)
     constexpr uint32_t ID_AP = idesc_bf16(128, 64, 0, 0);
-    constexpr uint32_t ID_U = idesc_bf16(128, DVT, 0, 1);
+    constexpr uint32_t ID_PT = idesc_bf16(128, 64, 0, 1);    // [Y; P] x T' (MN-major)
     constexpr uint32_t ID_W = idesc_bf16(128, 128, 0, 1);
+    constexpr uint32_t ID_U = idesc_bf16(128, DVT, 0, 1);
     constexpr uint32_t ID_M1 = idesc_bf16(128, DVT, 0, 1);
-    constexpr uint32_t ID_M2S = idesc_bf16(128, DVT, 1, 1);
-    constexpr uint32_t ID_M2P = idesc_bf16(128, DVT, 0, 1);
+    constexpr uint32_t ID_M2 = idesc_bf16(128, DVT, 1, 1);
     // Shared-memory descriptors, built once: the address field holds addr >> 4,
     // so an offset of x bytes inside a tile is a plain add of x >> 4.
     auto dadd = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
     const uint64_t dLMAT = sdesc_sw128(sb + L::LMAT, 16, 1024);          // K-major A
-    const uint64_t dTZP = sdesc_sw128(sb + L::TZP, 16, 1024);            // K-major A
-    const uint64_t dROWK = sdesc_sw128(sb + L::ROWOP, 16, 1024);         // row operand as K-major A
-    const uint64_t dROWN = sdesc_sw128(sb + L::ROWOP, 16384, 1024);      // its KE rows as MN-major B
-    const uint64_t dCOLK = sdesc_sw128(sb + L::COLOP, 16, 1024);         // KF as K-major B
-    const uint64_t dCOLN = sdesc_sw128(sb + L::COLOP, 8192, 1024);       // g as MN-major B, KF^T as MN-major A
+    const uint64_t dTP = sdesc_sw128(sb + L::TP, 16, 1024);              // [T'; PT] as K-major A
+    const uint64_t dTPN = sdesc_sw128(sb + L::TP, 8192, 1024);           // T' as MN-major B
+    const uint64_t dYP = sdesc_sw128(sb + L::SP - 8192, 16, 1024);       // [Y; P] as K-major A
+    const uint64_t dROWK = sdesc_sw128(sb + L::ROW, 16, 1024);           // row operand as K-major A
+    const uint64_t dROWN = sdesc_sw128(sb + L::ROW, 16384, 1024);        // its KE rows as MN-major B
+    const uint64_t dCOLK = sdesc_sw128(sb + L::COL, 16, 1024);           // KF / gate row as K-major B
+    const uint64_t dCOLN = sdesc_sw128(sb + L::COL, 8192, 1024);         // g as MN-major B, KF^T as MN-major A
     const uint64_t dV = sdesc_sw128(sb + L::RAWV, 8192, 1024);           // MN-major B
     const uint64_t dSOP = sdesc_sw128(sb + L::SOP, 1024, L::SBO_V);      // MN-major B (S, then delta)
-    const uint64_t dYP = sdesc_sw128(sb + L::SP - 8192, 16, 1024);       // [Y; P] as K-major A
 
-    if (warp == kCtrlWarp) {
-        // ============================================================ control warp
-        // One thread issues every TMA load and the state-independent MMAs. Their
-        // inputs come from three roles in an order that varies from chunk to
-        // chunk, so it polls the hand-over barriers and issues whatever is
-        // ready; each kind of work goes out in chunk order.
-        if (lane == 0 && NC > 0) {
-            auto issue_kq = [&](int m) {
-                const int par = m & 1;
-                uint8_t* dst = sm + L::ROWOP + par * 32768;
-                mbar_arrive_expect_tx(bars + BAR_KQ + par, 4 * 8192);
-                for (int x = 0; x < 2; ++x) {
-                    tma_load_4d(dst + x * 16384, &tm_k, bars + BAR_KQ + par, 64 * x, h, tma_t0 + m * kC, tma_b);
-                    tma_load_4d(dst + x * 16384 + 8192, &tm_q, bars + BAR_KQ + par, 64 * x, h, tma_t0 + m * kC, tma_b);
-                }
-                if (m + 1 < NC) {  // the next chunk's tiles into L2: their loads wait for a free buffer
-                    for (int x = 0; x < 2; ++x) {
-                        tma_prefetch_l2_4d(&tm_k, 64 * x, h, tma_t0 + (m + 1) * kC, tma_b);
-                        tma_prefetch_l2_4d(&tm_q, 64 * x, h, tma_t0 + (m + 1) * kC, tma_b);
-                    }
-                }
-            };
-            auto issue_g = [&](int m) {
-                const int par = m & 1;
-                uint8_t* dst = sm + L::COLOP + par * 16384;
-                mbar_arrive_expect_tx(bars + BAR_G + par, 2 * 8192);
-                for (int x = 0; x < 2; ++x)
-                    tma_load_4d(dst + x * 8192, &tm_g, bars + BAR_G + par, 64 * x, h, tma_t0 + m * kC, tma_b);
-                if (m + 1 < NC)
-                    for (int x = 0; x < 2; ++x) tma_prefetch_l2_4d(&tm_g, 64 * x, h, tma_t0 + (m + 1) * kC, tma_b);
-            };
-            auto issue_v = [&](int m) {
-                if (v_zero) {  // the zero tile is already in place
-                    mbar_arrive(bars + BAR_V);
-                    return;
-                }
-                mbar_arrive_expect_tx(bars + BAR_V, (DVT / 64) * 8192);
-                for (int x = 0; x < DVT / 64; ++x)
-                    tma_load_4d(sm + L::RAWV + x * 8192, &tm_v, bars + BAR_V, j0 + 64 * x, h, tma_t0 + m * kC, tma_b);
-                if (m + 1 < NC)
-                    for (int x = 0; x < DVT / 64; ++x)
-                        tma_prefetch_l2_4d(&tm_v, j0 + 64 * x, h, tma_t0 + (m + 1) * kC, tma_b);
-            };
-            // a per-token gate or none: no log_alpha tile and no prefix-sum MMA
-            // (the prefix-sum barrier still completes, with an empty commit)
-            issue_kq(0);
-            if (gate == 0) issue_g(0);
-            issue_v(0);
-            if (NC > 1) {
-                issue_kq(1);
-                if (gate == 0) issue_g(1);
-            }
-            // next chunk for each kind of work
-            int ncs = 0, nap = 0, nuw = 0, nv = 1, nkq = 2, ng = gate == 0 ? 2 : NC;
-            long long idle_since = clock64();
-            while ((ncs < NC || nap < NC || nuw < NC || nv < NC || nkq < NC || ng < NC) && !*s_abort) {
-                bool prog = false;
-                // [G; G] = [L; L] g: the tile landed and the previous chunk's A/P were read out
-                if (ncs < NC && (gate != 0 || mbar_test(bars + BAR_G + (ncs & 1), (uint32_t)(ncs >> 1))) &&
-                    (ncs == 0 || mbar_test(bars + BAR_P4, (uint32_t)(ncs - 1)))) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 4 && gate == 0; ++kk)
-                        mma_bf16_ss(tmem + L::GC_COL, dadd(dLMAT, kk * 32),
-                                    dadd(dCOLN, (ncs & 1) * 16384 + kk * 2048), ID_CS, kk > 0);
-                    mma_commit(bars + BAR_CS);
-                    ++ncs;
-                    prog = true;
-                }
-                // [A; P] = [KE; QE] KF^T over the prefix-sum columns, once the operand tiles are stored
-                if (nap < ncs && mbar_test(bars + BAR_P2, (uint32_t)nap)) {
-                    const int par = nap & 1;
-                    tc_fence_after();
-                    if (!s_exact[par]) {
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_bf16_ss(tmem + L::GC_COL,
-                                        dadd(dROWK, par * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32),
-                                        dadd(dCOLK, par * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32), ID_AP, kk > 0);
-                    }
-                    mma_commit(bars + BAR_AP);
-                    ++nap;
-                    prog = true;
-                }
-                // [U; 0] = [T'; 0] v and [W'; 0] = [T'; 0] KE: T' stored, v landed, D1 read out
-                if (nuw < nap && mbar_test(bars + BAR_P5, (uint32_t)nuw) && mbar_test(bars + BAR_V, (uint32_t)nuw) &&
-                    (nuw == 0 || mbar_test(bars + BAR_D1, (uint32_t)(nuw - 1)))) {
-                    const int par = nuw & 1;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + L::D1_COL, dadd(dTZP, kk * 32), dadd(dV, kk * 2048), ID_U, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + L::W_COL, dadd(dTZP, kk * 32), dadd(dROWN, par * 32768 + kk * 2048), ID_W,
-                                    kk > 0);
-                    mma_commit(bars + BAR_UW);
-                    ++nuw;
-                    prog = true;
-                }
-                // loads into buffers freed by completed MMAs
-                if (nv < NC && nv <= nuw && mbar_test(bars + BAR_UW, (uint32_t)(nv - 1))) {
-                    issue_v(nv++);
-                    prog = true;
-                }
-                if (nkq < NC && mbar_test(bars + BAR_M1B + (nkq & 1), (uint32_t)((nkq - 2) >> 1))) {
-                    issue_kq(nkq++);
-                    prog = true;
-                }
-                if (ng < NC && mbar_test(bars + BAR_M2B + (ng & 1), (uint32_t)((ng - 2) >> 1))) {
-                    issue_g(ng++);
-                    prog = true;
-                }
-                if (prog) {
-                    idle_since = clock64();
-                } else if (clock64() - idle_since > kWaitBudget) {
-                    fail();
-                } else {
-                    __nanosleep(32);
-                }
-            }
+    // TMA issue helpers (one thread)
+    auto load_kq = [&](int m, int bar) {  // k/q tiles of chunk m into the row buffer of its parity
+        uint8_t* dst = sm + L::ROW + (m & 1) * 32768;
+        mbar_arrive_expect_tx(bars + bar, 4 * 8192);
+        for (int x = 0; x < 2; ++x) {
+            tma_load_4d(dst + x * 16384, &tm_k, bars + bar, 64 * x, h, tma_t0 + m * kC, tma_b);
+            tma_load_4d(dst + x * 16384 + 8192, &tm_q, bars + bar, 64 * x, h, tma_t0 + m * kC, tma_b);
         }
+    };
+    auto pf_kq = [&](int m) {  // into L2: the load itself waits for a free buffer
+        if (m < NC)
+            for (int x = 0; x < 2; ++x) {
+                tma_prefetch_l2_4d(&tm_k, 64 * x, h, tma_t0 + m * kC, tma_b);
+                tma_prefetch_l2_4d(&tm_q, 64 * x, h, tma_t0 + m * kC, tma_b);
+            }
+    };
+    auto load_g = [&](int m) {
+        mbar_arrive_expect_tx(bars + B_G + m % 3, 2 * 8192);
+        for (int x = 0; x < 2; ++x)
+            tma_load_4d(sm + L::COL + (m % 3) * 16384 + x * 8192, &tm_g, bars + B_G + m % 3, 64 * x, h,
+                        tma_t0 + m * kC, tma_b);
+    };
+    auto pf_g = [&](int m) {
+        if (m < NC)
+            for (int x = 0; x < 2; ++x) tma_prefetch_l2_4d(&tm_g, 64 * x, h, tma_t0 + m * kC, tma_b);
+    };
+    auto load_v = [&](int m) {
+        if (v_zero) {  // the zero tile is already in place
+            mbar_arrive(bars + B_V);
+            return;
+        }
+        mbar_arrive_expect_tx(bars + B_V, (DVT / 64) * 8192);
+        for (int x = 0; x < DVT / 64; ++x)
+            tma_load_4d(sm + L::RAWV + x * 8192, &tm_v, bars + B_V, j0 + 64 * x, h, tma_t0 + m * kC, tma_b);
+    };
+    auto pf_v = [&](int m) {
+        if (m < NC && !v_zero)
+            for (int x = 0; x < DVT / 64; ++x) tma_prefetch_l2_4d(&tm_v, j0 + 64 * x, h, tma_t0 + m * kC, tma_b);
+    };
+    // per-token gate (GATE == 1): the chunk's 64 gates as row 0 of a K-major
+    // B tile at the start of its log_alpha/KF buffer (rows 1-15 feed prefix-sum
+    // columns that are never read). Lane l holds tokens 2l, 2l+1.
+    auto gate_row_load = [&](int m) -> uint32_t {
+        const int t = m * kC + 2 * lane;
+        const float a = (m < NC && t < seq_len) ? __bfloat162float(gate_tok[(tok0 + t) * H + h]) : 0.f;
+        const float c = (m < NC && t + 1 < seq_len) ? __bfloat162float(gate_tok[(tok0 + t + 1) * H + h]) : 0.f;
+        return pack_bf16x2(a, c);
+    };
+    auto gate_row_store = [&](int m, uint32_t w) {  // warp-collective
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sb + L::COL + (uint32_t)(m % 3) * 16384 + 4u * lane), "r"(w)
+                     : "memory");
+        fence_proxy_async_smem();
         __syncwarp();
-    } else if (warp >= kChainWarp0 && warp < kCtrlWarp) {
+        if (lane == 0) mbar_arrive(bars + B_G + m % 3);
+    };
+    auto cumsum_mma = [&](int m) {  // prefix sums of chunk m into its slot (one thread)
+        const int s = m % 3;
+        if (GATE == 0) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dLMAT, kk * 32), dadd(dCOLN, s * 16384 + kk * 2048),
+                            ID_CS, kk > 0);
+        } else if (GATE == 1) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dLMAT, kk * 32), dadd(dCOLK, s * 16384 + kk * 32),
+                            ID_CS1, kk > 0);
+        }
+        mma_commit(bars + B_CS + s);  // (no gate: an empty commit completes the phase)
+    };
+
+    if (warp < kTileWarp0) {
         // ============================================================ chain warps
-        // lane row = 32 * quad + lane: a key channel of the state, a token row of D1
+        // lane row = 32 * quad + lane: a key channel of the state, a token row of the slot
         const int row = 32 * quad + lane;
-        const bool issuer = (quad == 0) && (lane == 0);
+        const bool issuer = warp == 0 && lane == 0;
+        int n_kq[2] = {0, 0}, n_g[3] = {0, 0, 0};  // loads issued per barrier (issuer)
         {   // initial state into TMEM (fp32, lane = key channel)
 #pragma unroll 1
             for (int gq = 0; gq < DVT / 32; ++gq) {
@@ -549,126 +515,159 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             nb_sync(NB_CH, 128);
             tc_fence_after();
         }
-        // state rows -> bf16 operand (times the operand scale), R *= tensor-memory scale
-        auto s1 = [&](int slot) {
-            const float os = sOpS[slot * 128 + row], ts = sTmS[slot * 128 + row];
-            const int i = row & 63;
-#pragma unroll 1
-            for (int gq = 0; gq < DVT / 32; ++gq) {
-                uint32_t v[32];
-                tmem_ld32(lane_addr + L::S_COL + 32 * gq, v);
-                tmem_ld_wait(v);
-#pragma unroll
-                for (int jc = 0; jc < 4; ++jc) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]) * os,
-                                           __uint_as_float(v[8 * jc + 2 * u + 1]) * os);
-                    const int j = 32 * gq + 8 * jc;
-                    const uint32_t off = (uint32_t)(i >> 3) * L::SBO_V + (uint32_t)(j >> 6) * 1024 +
-                                         (uint32_t)(i & 7) * 128 + ((uint32_t)(((j & 63) >> 3) ^ (i & 7)) << 4);
-                    st_shared_v4(sb + L::SOP + off, w[0], w[1], w[2], w[3]);
+        uint32_t gnext = 0;  // per-token gate row of the next chunk to place (warp 0)
+        if (NC > 0) {
+            if (issuer) {
+                load_kq(0, B_KQ);
+                ++n_kq[0];
+                if (NC > 1) {
+                    load_kq(1, B_KQ + 1);
+                    ++n_kq[1];
                 }
-#pragma unroll
-                for (int u = 0; u < 32; ++u) v[u] = __float_as_uint(__uint_as_float(v[u]) * ts);
-                tmem_st32(lane_addr + L::S_COL + 32 * gq, v);
+                pf_kq(2);
+                if (GATE == 0) {
+                    for (int j = 0; j < 3 && j < NC; ++j) {
+                        load_g(j);
+                        ++n_g[j];
+                    }
+                    pf_g(3);
+                }
             }
-            tmem_st_wait();
+            if (GATE == 1 && warp == 0) {
+                for (int j = 0; j < 3 && j < NC; ++j) gate_row_store(j, gate_row_load(j));
+                gnext = gate_row_load(3);
+            }
+        }
+        // s1 body for one 32-column group: state rows -> bf16 operand words (times
+        // the operand scale), R *= tensor-memory scale
+        auto s1_group = [&](int gq, float os, float ts, uint32_t (&pk)[16]) {
+            uint32_t v[32];
+            tmem_ld32(lane_addr + L::S_COL + 32 * gq, v);
+            tmem_ld_wait(v);
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                pk[u] = pack_bf16x2(__uint_as_float(v[2 * u]) * os, __uint_as_float(v[2 * u + 1]) * os);
+#pragma unroll
+            for (int u = 0; u < 32; ++u) v[u] = __float_as_uint(__uint_as_float(v[u]) * ts);
+            tmem_st32(lane_addr + L::S_COL + 32 * gq, v);
+        };
+        // operand words of one 32-column group of channel row i -> the S/delta operand
+        auto sop_store = [&](int i, int gq, const uint32_t (&pk)[16]) {
+#pragma unroll
+            for (int jc = 0; jc < 4; ++jc) {
+                const int j = 32 * gq + 8 * jc;
+                const uint32_t off = (uint32_t)(i >> 3) * L::SBO_V + (uint32_t)(j >> 6) * 1024 + (uint32_t)(i & 7) * 128 +
+                                     ((uint32_t)(((j & 63) >> 3) ^ (i & 7)) << 4);
+                st_shared_v4(sb + L::SOP + off, pk[4 * jc], pk[4 * jc + 1], pk[4 * jc + 2], pk[4 * jc + 3]);
+            }
         };
         for (int n = 0; n < NC; ++n) {
-            const int par = n & 1;
-            const uint32_t ph = (uint32_t)(n >> 1);
+            const int s = n % 3, rb = n & 1;
+            const uint32_t slot = lane_addr + L::SLOT0 + 128 * s;
+            if (n > 0) {
+                waitw(B_M2, (uint32_t)(n - 1));  // state update of the previous chunk done
+                if (n + 2 < NC) {  // its log_alpha/KF buffer is free: the gate tile of chunk n+2
+                    if (GATE == 0 && issuer) {
+                        load_g(n + 2);
+                        ++n_g[(n + 2) % 3];
+                        pf_g(n + 3);
+                    }
+                    if (GATE == 1 && warp == 0) {
+                        gate_row_store(n + 2, gnext);
+                        gnext = gate_row_load(n + 3);
+                    }
+                }
+            }
+            waitw(B_SC + (n & 3), (uint32_t)(n >> 2));
+            const float os = sOpS[(n & 3) * 128 + row], ts = sTmS[(n & 3) * 128 + row];
             if (quad < 2) {
-                if (n > 0) waitw(BAR_M2, (uint32_t)(n - 1));  // state update of the previous chunk done
-                waitw(BAR_SC + (n & 3), (uint32_t)(n >> 2));
-                s1(n & 3);  // key channels 0-63
+#pragma unroll 1
+                for (int gq = 0; gq < DVT / 32; ++gq) {  // key channels 0-63
+                    uint32_t pk[16];
+                    s1_group(gq, os, ts, pk);
+                    sop_store(row, gq, pk);
+                }
+                tmem_st_wait();
                 fence_proxy_async_smem();
                 tc_fence_before();
-                nb_sync(NB_CHA, 64);
-                if (quad == 0) {
-                    if (issuer) {
-                        wait1(BAR_RR + par, ph);  // row operand of chunk n stored
+                nb_sync(NB_CHLO, 64);
+                if (warp == 0) {
+                    if (lane == 0) {
+                        wait1(B_RR + rb, (uint32_t)(n >> 1));  // row operand of chunk n stored
+                        wait1(B_UO + s, (uint32_t)(n / 3));    // its accumulator holds [U; P T' v]
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16_ss(tmem + L::D1_COL, dadd(dROWK, par * 32768 + kk * 32),
+                            mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dROWK, rb * 32768 + kk * 32),
                                         dadd(dSOP, kk * 2 * L::SBO_V), ID_M1, 1);
-                        mma_commit(bars + BAR_M1A);
+                        mma_commit(bars + B_M1A);
                     }
                     __syncwarp();
                     nb_sync(NB_CHB, 96);  // key channels 64-127 stored
-                    if (issuer) {
+                    if (lane == 0) {
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16_ss(tmem + L::D1_COL, dadd(dROWK, par * 32768 + 16384 + kk * 32),
+                            mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dROWK, rb * 32768 + 16384 + kk * 32),
                                         dadd(dSOP, kk * 2 * L::SBO_V), ID_M1, 1);
-                        mma_commit(bars + BAR_M1);
-                        mma_commit(bars + BAR_M1B + par);
+                        mma_commit(bars + B_M1);
                     }
                     __syncwarp();
                 }
-                waitw(BAR_M1, (uint32_t)n);
-                {   // delta (D1 rows 0-63) -> bf16 operand over the state operand
-                    const int r = row;
+                waitw(B_M1, (uint32_t)n);
+                if (issuer && n + 2 < NC) {  // the row buffer of this parity is free
+                    load_kq(n + 2, B_KQ + rb);
+                    ++n_kq[rb];
+                    pf_kq(n + 3);
+                }
+                {   // delta (slot rows 0-63) -> bf16 operand over the state operand
 #pragma unroll 1
                     for (int gq = 0; gq < DVT / 32; ++gq) {
                         uint32_t v[32];
-                        tmem_ld32(lane_addr + L::D1_COL + 32 * gq, v);
+                        tmem_ld32(slot + 32 * gq, v);
                         tmem_ld_wait(v);
+                        uint32_t pk[16];
 #pragma unroll
-                        for (int jc = 0; jc < 4; ++jc) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]),
-                                                   __uint_as_float(v[8 * jc + 2 * u + 1]));
-                            const int j = 32 * gq + 8 * jc;
-                            const uint32_t off = (uint32_t)(r >> 3) * L::SBO_V + (uint32_t)(j >> 6) * 1024 +
-                                                 (uint32_t)(r & 7) * 128 +
-                                                 ((uint32_t)(((j & 63) >> 3) ^ (r & 7)) << 4);
-                            st_shared_v4(sb + L::DOP + off, w[0], w[1], w[2], w[3]);
-                        }
+                        for (int u = 0; u < 16; ++u)
+                            pk[u] = pack_bf16x2(__uint_as_float(v[2 * u]), __uint_as_float(v[2 * u + 1]));
+                        sop_store(row, gq, pk);
                     }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                nb_sync(NB_CHA, 64);
+                nb_sync(NB_CHLO, 64);
                 if (issuer) {
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // R += KF^T delta
-                        mma_bf16_ss(tmem + L::S_COL, dadd(dCOLN, par * 16384 + kk * 2048), dadd(dSOP, kk * 2 * L::SBO_V),
-                                    ID_M2S, 1);
-                    // [Y; P]: Y, the 8 KB before P, only feeds D1 rows 0-63, already read out
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // D1 rows 64-127 += P delta
-                        mma_bf16_ss(tmem + L::D1_COL, dadd(dYP, par * 8192 + kk * 32), dadd(dSOP, kk * 2 * L::SBO_V),
-                                    ID_M2P, 1);
-                    mma_commit(bars + BAR_M2);
-                    mma_commit(bars + BAR_M2B + par);
+                        mma_bf16_ss(tmem + L::S_COL, dadd(dCOLN, s * 16384 + kk * 2048), dadd(dSOP, kk * 2 * L::SBO_V),
+                                    ID_M2, 1);
+                    mma_commit(bars + B_M2);
+                    mbar_arrive(bars + B_SF + s);  // slot rows 0-63 read
                 }
                 __syncwarp();
             } else {
-                waitw(BAR_SC + (n & 3), (uint32_t)(n >> 2));
-                waitw(BAR_M1A, (uint32_t)n);  // first half of the state operand consumed
-                s1(n & 3);                      // key channels 64-127
+                uint32_t pk[DVT / 32][16];  // key channels 64-127, staged until the operand buffer is free
+#pragma unroll
+                for (int gq = 0; gq < DVT / 32; ++gq) s1_group(gq, os, ts, pk[gq]);
+                tmem_st_wait();
+                waitw(B_M1A, (uint32_t)n);  // first half of the state operand consumed
+#pragma unroll
+                for (int gq = 0; gq < DVT / 32; ++gq) sop_store(row - 64, gq, pk[gq]);
                 fence_proxy_async_smem();
                 tc_fence_before();
                 nb_arrive(NB_CHB, 96);
-                waitw(BAR_M2, (uint32_t)n);
-                {   // O (D1 rows 64-127) -> global bf16
+                waitw(B_M1, (uint32_t)n);
+                {   // O (slot rows 64-127) -> global bf16
                     const int r = row - 64;
                     const int t0 = n * kC;
 #pragma unroll 1
                     for (int gq = 0; gq < DVT / 32; ++gq) {
                         uint32_t v[32];
-                        tmem_ld32(lane_addr + L::D1_COL + 32 * gq, v);
+                        tmem_ld32(slot + 32 * gq, v);
                         tmem_ld_wait(v);
                         if (o_on && t0 + r < seq_len) {
-                            uint4* dst = reinterpret_cast<uint4*>(o + ((tok0 + t0 + r) * H + h) * kD + j0 +
-                                                                  32 * gq);
+                            uint4* dst = reinterpret_cast<uint4*>(o + ((tok0 + t0 + r) * H + h) * kD + j0 + 32 * gq);
 #pragma unroll
                             for (int jc = 0; jc < 4; ++jc) {
                                 uint4 w;
@@ -683,13 +682,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     }
                 }
                 tc_fence_before();
-                nb_sync(NB_CHC, 64);
-                if (quad == 2 && lane == 0) mbar_arrive(bars + BAR_D1);
+                nb_sync(NB_CHHI, 64);
+                if (warp == 2 && lane == 0) mbar_arrive(bars + B_SF + s);  // slot rows 64-127 read
                 __syncwarp();
             }
         }
         // ------------------------------------------------------------ final state S = e^{G_last - G_m} R
-        if (quad < 2 && NC > 0) waitw(BAR_M2, (uint32_t)(NC - 1));
+        if (NC > 0) waitw(B_M2, (uint32_t)(NC - 1));
         // one decision per warp: the tensor-memory loads below are warp-collective
         if (__shfl_sync(0xffffffffu, (stm && !*s_abort) ? 1 : 0, 0)) {
             const float ek = sEK[row];
@@ -705,230 +704,337 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                                          __uint_as_float(v[4 * u + 2]) * ek, __uint_as_float(v[4 * u + 3]) * ek);
             }
         }
-    } else if (warp < kChainWarp0) {
-        // ============================================================ prep warps
-        // Per chunk m: A/P readout and (I + A)^{-1} -> T'; then the operand
-        // tiles of chunk m+1 (which covers the U/W round trip of chunk m);
-        // then -W' over the KE rows of chunk m (the A/P MMA of chunk m+1 runs
-        // meanwhile).
-        const int hf = warp >> 2;
-        const int tok = 32 * (quad & 1) + lane;  // P2: token of this thread
-        const int cb = 2 * (quad >> 1) + hf;     // P2: 32-channel block of this thread
-        auto load_beta = [&](int m) -> float {
-            const int t = m * kC + tid;
-            return (tid < kC && m < NC && t < seq_len) ? __bfloat162float(beta[(tok0 + t) * H + h]) : 0.f;
-        };
-        float* sGs = reinterpret_cast<float*>(sm + L::SGS);
-        auto p2 = [&](int m) -> bool {
-            const int par = m & 1, slot = m & 3;
-            const uint32_t gaddr = lane_addr + L::GC_COL + 32 * cb;  // this thread's 32 channels of G
-            if (gate == 1) {  // per-token gate: prefix sums over the chunk's 64 tokens (one warp scans)
-                if (warp == 0) {
-                    const int t0 = m * kC;
-                    float g0 = (t0 + lane < seq_len) ? __bfloat162float(gate_tok[(tok0 + t0 + lane) * H + h]) : 0.f;
-                    float g1 = (t0 + 32 + lane < seq_len) ? __bfloat162float(gate_tok[(tok0 + t0 + 32 + lane) * H + h])
-                                                          : 0.f;
-#pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const float x0 = __shfl_up_sync(0xffffffffu, g0, off), x1 = __shfl_up_sync(0xffffffffu, g1, off);
-                        if (lane >= off) {
-                            g0 += x0;
-                            g1 += x1;
-                        }
-                    }
-                    sGs[lane] = g0;
-                    sGs[32 + lane] = g1 + __shfl_sync(0xffffffffu, g0, 31);
-                }
-                nb_sync(NB_PREP, kPrep);
+        if (issuer) {
+            for (int x = 0; x < 2; ++x) drain(B_KQ + x, n_kq[x]);
+            for (int x = 0; x < 3; ++x) drain(B_G + x, n_g[x]);
+            if (*s_abort) {
+                mma_commit(bars + B_FIN);
+                mbar_wait_bounded(bars + B_FIN, 0u, kDrainBudget);
             }
-            // G of 8 channels of this thread's token: from tensor memory (per-channel
-            // gate; warp-collective, the branch is uniform), the per-token sums, or 0
-            auto load_g8 = [&](int u4, uint32_t (&g8)[8]) {
-                if (gate == 0) {
-                    tmem_ld8(gaddr + 8 * u4, g8);
+        }
+    } else if (warp < kInvWarp0) {
+        // ============================================================ tile warps
+        // thread: token tok (lanes of its quadrant, both halves of [L; L] hold the
+        // chunk's 64 tokens), 64 channels from ch0
+        const int ttid = tid - 32 * kTileWarp0;
+        const int tok = 32 * (quad & 1) + lane, ch0 = 64 * (quad >> 1);
+        int nex = 0;
+        if (NC > 0 && ttid == 0) {
+            if (GATE != 2) wait1(B_G, 0u);
+            tc_fence_after();
+            cumsum_mma(0);
+        }
+        // Exact path of a chunk that fails the vote: reload the raw k/q rows, per-pair
+        // exponentials for A and P (raw sums, staged and stored into the slot where
+        // the [A; P] MMA would have put them), plain tiles k e^G, q e^G, k e^{G_last-G}.
+        auto exact_chunk = [&](int m, int s, int rb, int cb, int lim) {
+            const uint32_t slotq = lane_addr + L::SLOT0 + 128 * s;
+            if (ttid == 0) load_kq(m, B_EXKQ);
+            waitw(B_EXKQ, (uint32_t)nex);
+            if (m > 0) waitw(B_SCRF, (uint32_t)(m - 1));  // the inverse warps are done with the scratch
+            float* sG = reinterpret_cast<float*>(sm + L::SCR);
+            const bool live = tok < lim;
+#pragma unroll 1
+            for (int u8 = 0; u8 < 8; ++u8) {  // G -> fp32 [64][128] staging
+                uint32_t g8[8];
+                if (GATE == 0) {
+                    tmem_ld8(slotq + ch0 + 8 * u8, g8);
                     tmem_ld_wait(g8);
                 } else {
-                    const uint32_t gv = gate == 1 ? __float_as_uint(sGs[tok]) : 0u;
+                    uint32_t g1;
+                    tmem_ld1(slotq, g1);
+                    tmem_ld_wait1(g1);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) g8[e] = gv;
+                    for (int e = 0; e < 8; ++e) g8[e] = g1;
                 }
-            };
-            // Rolled loops over groups of 8 channels keep the loop bodies
-            // small: every chunk streams this code again, and what is not
-            // in the instruction cache stalls the warp.
+                float* dst = sG + tok * 128 + ch0 + 8 * u8;
+                *reinterpret_cast<float4*>(dst) = make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]),
+                                                              __uint_as_float(g8[2]), __uint_as_float(g8[3]));
+                *reinterpret_cast<float4*>(dst + 4) = make_float4(__uint_as_float(g8[4]), __uint_as_float(g8[5]),
+                                                                  __uint_as_float(g8[6]), __uint_as_float(g8[7]));
+            }
+            nb_sync(NB_TILE, 128);
+            const uint8_t* rk = sm + L::ROW + rb * 32768;
+            constexpr int kPairs = kC * (kC + 1) / 2, kPer = (kPairs + 127) / 128;
+            float av[kPer], pv[kPer];
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                av[i] = 0.f;
+                pv[i] = 0.f;
+                const int p = ttid + 128 * i;
+                if (p < kPairs) {
+                    int r = (int)((sqrtf(8.f * (float)p + 1.f) - 1.f) * 0.5f);
+                    while ((r + 1) * (r + 2) / 2 <= p) ++r;
+                    while (r * (r + 1) / 2 > p) --r;
+                    const int s2 = p - r * (r + 1) / 2;
+                    float a = 0.f, pp = 0.f;
+                    // rows past the sequence stay 0 (their gates may be another
+                    // sequence's and overflow the exponential)
+                    for (int i2 = 0; i2 < (r < lim ? kD : 0); ++i2) {
+                        const int cc = (i2 + p) & (kD - 1);
+                        const float ks = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(s2, cc))) *
+                                         ex2((sG[r * 128 + cc] - sG[s2 * 128 + cc]) * kLog2e);
+                        a = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(r, cc))), ks, a);
+                        pp = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(64 + r, cc))),
+                                  ks, pp);
+                    }
+                    av[i] = a;
+                    pv[i] = pp;
+                }
+            }
+            nb_sync(NB_TILE, 128);  // raw rows read
+            {   // plain tiles in place
+                const uint32_t rop = sb + L::ROW + rb * 32768;
+                const uint32_t colp = sb + L::COL + cb * 16384;
+#pragma unroll 1
+                for (int u8 = 0; u8 < 8; ++u8) {
+                    const int c0 = ch0 + 8 * u8;
+                    uint32_t g8[8];
+                    if (GATE == 0) {
+                        tmem_ld8(slotq + c0, g8);
+                        tmem_ld_wait(g8);
+                    } else {
+                        uint32_t g1;
+                        tmem_ld1(slotq, g1);
+                        tmem_ld_wait1(g1);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) g8[e] = g1;
+                    }
+                    const uint32_t ko = rop_off(tok, c0);
+                    const uint32_t fo = (uint32_t)((c0 >> 6) * 8192 + tok * 128 + ((((c0 & 63) >> 3) ^ (tok & 7)) << 4));
+                    const uint4 kv = ld_shared_v4(rop + ko);
+                    const uint4 qv = ld_shared_v4(rop + ko + 8192);
+                    const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+                    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                    uint32_t ke[4], qe[4], kf[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float g0 = __uint_as_float(g8[2 * u]), g1 = __uint_as_float(g8[2 * u + 1]);
+                        const float gl0 = GATE == 0 ? sGl[c0 + 2 * u] : sGl[0];
+                        const float gl1 = GATE == 0 ? sGl[c0 + 2 * u + 1] : sGl[0];
+                        const uint32_t ep = pack_bf16x2(ex2(g0 * kLog2e), ex2(g1 * kLog2e));
+                        const uint32_t fp = pack_bf16x2(ex2((gl0 - g0) * kLog2e), ex2((gl1 - g1) * kLog2e));
+                        ke[u] = live ? hmul2_bf16(kw[u], ep) : 0u;
+                        qe[u] = live ? hmul2_bf16(qw[u], ep) : 0u;
+                        kf[u] = live ? hmul2_bf16(kw[u], fp) : 0u;
+                    }
+                    st_shared_v4(rop + ko, ke[0], ke[1], ke[2], ke[3]);
+                    st_shared_v4(rop + ko + 8192, qe[0], qe[1], qe[2], qe[3]);
+                    st_shared_v4(colp + fo, kf[0], kf[1], kf[2], kf[3]);
+                }
+            }
+            // raw A and P sums -> fp32 [64][64] staging (over the gate staging), then
+            // into the slot: quadrant 0/1 rows are A rows, 2/3 rows are P rows
+            float* stA = sG;
+            float* stP = sG + 64 * 64;
+            for (int i = ttid; i < 2 * 64 * 64 / 4; i += 128)
+                reinterpret_cast<float4*>(stA)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            nb_sync(NB_TILE, 128);
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                const int p = ttid + 128 * i;
+                if (p < kPairs) {
+                    int r = (int)((sqrtf(8.f * (float)p + 1.f) - 1.f) * 0.5f);
+                    while ((r + 1) * (r + 2) / 2 <= p) ++r;
+                    while (r * (r + 1) / 2 > p) --r;
+                    const int s2 = p - r * (r + 1) / 2;
+                    stA[r * 64 + s2] = av[i];
+                    stP[r * 64 + s2] = pv[i];
+                }
+            }
+            nb_sync(NB_TILE, 128);
+            {
+                const float* src = quad < 2 ? stA + (32 * quad + lane) * 64 : stP + (32 * (quad - 2) + lane) * 64;
+#pragma unroll 1
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t r32[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) r32[u] = __float_as_uint(src[32 * h2 + u]);
+                    tmem_st32(slotq + 32 * h2, r32);
+                }
+                tmem_st_wait();
+            }
+            ++nex;
+        };
+        for (int m = 0; m < NC; ++m) {
+            const int s = m % 3, rb = m & 1, cb = m % 3;
+            const uint32_t slotq = lane_addr + L::SLOT0 + 128 * s;
+            waitw(B_CS + s, (uint32_t)(m / 3));
+            waitw(B_KQ + rb, (uint32_t)(m >> 1));
             // Tokens of this chunk that belong to the sequence: [0, lim). Rows past
             // it are zero (past the tensor) or the next packed sequence's.
             const int lim = min(seq_len - m * kC, kC);
             const bool live = tok < lim;
-            const int tm_tok = min(31, lim - 1), tl_tok = min(63, lim - 1);  // reference, last token
-            {   // G_m, G_last of this thread's channels (tcgen05.ld is warp-collective:
-                // every lane loads, the lanes of the two tokens store)
+            const int tm_tok = min(31, lim - 1), tl_tok = lim - 1;  // reference, last token
+            uint32_t g1 = 0;  // per-token gate: this token's prefix sum
+            if (GATE == 0) {  // G_m, G_last of this thread's channels (every lane loads, the owners store)
 #pragma unroll 1
-                for (int u4 = 0; u4 < 4; ++u4) {
+                for (int u8 = 0; u8 < 8; ++u8) {
                     uint32_t g8[8];
-                    load_g8(u4, g8);
-                    const float4 lo = make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]), __uint_as_float(g8[2]),
-                                                  __uint_as_float(g8[3]));
-                    const float4 hi = make_float4(__uint_as_float(g8[4]), __uint_as_float(g8[5]), __uint_as_float(g8[6]),
-                                                  __uint_as_float(g8[7]));
+                    tmem_ld8(slotq + ch0 + 8 * u8, g8);
+                    tmem_ld_wait(g8);
+                    const int c0 = ch0 + 8 * u8;
                     if (tok == tm_tok) {
-                        *reinterpret_cast<float4*>(sGm + 32 * cb + 8 * u4) = lo;
-                        *reinterpret_cast<float4*>(sGm + 32 * cb + 8 * u4 + 4) = hi;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            sGm[c0 + e] = __uint_as_float(g8[e]);
+                            sGmL[c0 + e] = -__uint_as_float(g8[e]) * kLog2e;
+                        }
                     }
                     if (tok == tl_tok) {
-                        *reinterpret_cast<float4*>(sGl + 32 * cb + 8 * u4) = lo;
-                        *reinterpret_cast<float4*>(sGl + 32 * cb + 8 * u4 + 4) = hi;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) sGl[c0 + e] = __uint_as_float(g8[e]);
                     }
                     __syncwarp();
                 }
+            } else if (GATE == 1) {
+                tmem_ld1(slotq, g1);
+                tmem_ld_wait1(g1);
+                if (tok == tm_tok) {
+                    sGm[0] = __uint_as_float(g1);
+                    sGmL[0] = -__uint_as_float(g1) * kLog2e;
+                }
+                if (tok == tl_tok) sGl[0] = __uint_as_float(g1);
             }
-            nb_sync(NB_PREP, kPrep);
-            bool bad = false;
+            nb_sync(NB_TILE, 128);
+            // operand tiles, in place: 8 groups of 8 channels of this thread's row;
+            // amax tracks the largest |exponent| (and |G_m|) for the vote
+            float amax = 0.f;
+            {
+                const uint32_t rop = sb + L::ROW + rb * 32768;
+                const uint32_t colp = sb + L::COL + cb * 16384;
+                uint32_t ep1 = 0, fp1 = 0;
+                if (GATE == 1) {
+                    const float nl = sGmL[0];
+                    const float a = fmaf(__uint_as_float(g1), kLog2e, nl);
+                    amax = fmaxf(fabsf(a), fabsf(nl));
+                    const float e = ex2(a), f = ex2(-a);
+                    ep1 = pack_bf16x2(e, e);
+                    fp1 = pack_bf16x2(f, f);
+                }
+                const uint32_t km = live ? 0xFFFFFFFFu : 0u;  // rows past the sequence: k = q = 0
 #pragma unroll 1
-            for (int u4 = 0; u4 < 4; ++u4) {
-                uint32_t g8[8];
-                load_g8(u4, g8);
-                const float4 ma = *reinterpret_cast<const float4*>(sGm + 32 * cb + 8 * u4);
-                const float4 mb = *reinterpret_cast<const float4*>(sGm + 32 * cb + 8 * u4 + 4);
-                const float gm8[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+                for (int u8 = 0; u8 < 8; ++u8) {
+                    const int c0 = ch0 + 8 * u8;
+                    const uint32_t ko = rop_off(tok, c0);
+                    const uint32_t fo = (uint32_t)((c0 >> 6) * 8192 + tok * 128 + ((((c0 & 63) >> 3) ^ (tok & 7)) << 4));
+                    const uint4 kv = ld_shared_v4(rop + ko);
+                    const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+                    uint32_t ke[4], qe[4], kf[4];
+                    if (GATE == 2) {  // no decay: KE = k, QE = q, KF = k
+                        if (!live) {
+                            st_shared_v4(rop + ko, 0u, 0u, 0u, 0u);
+                            st_shared_v4(rop + ko + 8192, 0u, 0u, 0u, 0u);
+                        }
+                        st_shared_v4(colp + fo, kw[0] & km, kw[1] & km, kw[2] & km, kw[3] & km);
+                        continue;
+                    }
+                    const uint4 qv = ld_shared_v4(rop + ko + 8192);
+                    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                    if (GATE == 0) {
+                        uint32_t g8[8];
+                        tmem_ld8(slotq + c0, g8);
+                        const float4 na = *reinterpret_cast<const float4*>(sGmL + c0);
+                        const float4 nb = *reinterpret_cast<const float4*>(sGmL + c0 + 4);
+                        const float nl8[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
+                        tmem_ld_wait(g8);
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    bad |= !(fabsf(__uint_as_float(g8[e]) - gm8[e]) <= kGuard) || !(gm8[e] >= -kGuard);
+                        for (int u = 0; u < 4; ++u) {
+                            // E = 2^{(G - G_m) log2 e}, F = 1/E
+                            const float a0 = fmaf(__uint_as_float(g8[2 * u]), kLog2e, nl8[2 * u]);
+                            const float a1 = fmaf(__uint_as_float(g8[2 * u + 1]), kLog2e, nl8[2 * u + 1]);
+                            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(a0), fabsf(a1)), fmaxf(fabsf(nl8[2 * u]), fabsf(nl8[2 * u + 1]))));
+                            // packed bf16 products: the factor pairs are rounded to bf16
+                            // first, the products once more (both well inside the bf16
+                            // rounding of the MMA operands)
+                            const uint32_t ep = pack_bf16x2(ex2(a0), ex2(a1));
+                            const uint32_t fp = pack_bf16x2(ex2(-a0), ex2(-a1));
+                            ke[u] = hmul2_bf16(kw[u], ep) & km;
+                            qe[u] = hmul2_bf16(qw[u], ep) & km;
+                            kf[u] = hmul2_bf16(kw[u], fp) & km;
+                        }
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            ke[u] = hmul2_bf16(kw[u], ep1) & km;
+                            qe[u] = hmul2_bf16(qw[u], ep1) & km;
+                            kf[u] = hmul2_bf16(kw[u], fp1) & km;
+                        }
+                    }
+                    st_shared_v4(rop + ko, ke[0], ke[1], ke[2], ke[3]);
+                    st_shared_v4(rop + ko + 8192, qe[0], qe[1], qe[2], qe[3]);
+                    st_shared_v4(colp + fo, kf[0], kf[1], kf[2], kf[3]);
+                }
             }
-            const bool exact = nb_or(NB_OR, kPrep, bad && live);
-            if (tid < kD) {
-                const int c = tid;
-                const float g_m = sGm[c], g_l = sGl[c], ek_prev = sEK[c];
+            // every factor finite and normal? (NaN counts as a failure)
+            const bool exact = GATE != 2 && nb_or(NB_TOR, 128, live && !(amax <= kGuardL));
+            if (exact) exact_chunk(m, s, rb, cb, lim);
+            {   // per-channel scales of this chunk
+                const int c = ttid;
+                const float g_m = GATE == 0 ? sGm[c] : (GATE == 1 ? sGm[0] : 0.f);
+                const float g_l = GATE == 0 ? sGl[c] : (GATE == 1 ? sGl[0] : 0.f);
+                const float ek_prev = sEK[c];
+                const int slot4 = m & 3;
                 if (!exact) {
-                    const float s = __expf(g_m) * ek_prev;
-                    sOpS[slot * 128 + c] = s;
-                    sTmS[slot * 128 + c] = s;
+                    const float sc = __expf(g_m) * ek_prev;
+                    sOpS[slot4 * 128 + c] = sc;
+                    sTmS[slot4 * 128 + c] = sc;
                     sEK[c] = __expf(g_l - g_m);
                 } else {
-                    sOpS[slot * 128 + c] = ek_prev;
-                    sTmS[slot * 128 + c] = __expf(g_l) * ek_prev;
+                    sOpS[slot4 * 128 + c] = ek_prev;
+                    sTmS[slot4 * 128 + c] = __expf(g_l) * ek_prev;
                     sEK[c] = 1.f;
                 }
             }
-            const uint32_t rop = rowop(par);
-            if (exact) {
-                // gate as fp32 [64][128] in the A/T scratch (free: the inverse of the
-                // previous chunk is done); P of chunk m-2 must be consumed first
-                if (m >= 2) waitw(BAR_M2B + par, (uint32_t)((m >> 1) - 1));
-                float* sG = reinterpret_cast<float*>(sm + L::SCR);
-#pragma unroll 1
-                for (int u4 = 0; u4 < 4; ++u4) {
-                    uint32_t g8[8];
-                    load_g8(u4, g8);
-                    float* dst = sG + tok * 128 + 32 * cb + 8 * u4;
-                    *reinterpret_cast<float4*>(dst) = make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]),
-                                                                  __uint_as_float(g8[2]), __uint_as_float(g8[3]));
-                    *reinterpret_cast<float4*>(dst + 4) = make_float4(__uint_as_float(g8[4]), __uint_as_float(g8[5]),
-                                                                      __uint_as_float(g8[6]), __uint_as_float(g8[7]));
-                }
-                nb_sync(NB_PREP, kPrep);
-                const uint8_t* rk = sm + L::ROWOP + par * 32768;
-                float av[9], pv[9];
+            fence_proxy_async_smem();
+            tc_fence_before();
+            nb_sync(NB_TILE, 128);
+            if (ttid == 0) {
+                mbar_arrive(bars + B_SC + (m & 3));
+                tc_fence_after();
+                if (!exact) {  // [A; P] = [KE; QE] KF^T over the prefix-sum columns (read)
 #pragma unroll
-                for (int i = 0; i < 9; ++i) {
-                    av[i] = 0.f;
-                    pv[i] = 0.f;
-                    const int p = tid + kPrep * i;
-                    if (p < kC * (kC + 1) / 2) {
-                        int r = (int)((sqrtf(8.f * (float)p + 1.f) - 1.f) * 0.5f);
-                        while ((r + 1) * (r + 2) / 2 <= p) ++r;
-                        while (r * (r + 1) / 2 > p) --r;
-                        const int s = p - r * (r + 1) / 2;
-                        float a = 0.f, pp = 0.f;
-                        // rows past the sequence stay 0 (their gates may be another
-                        // sequence's and overflow the exponential)
-                        for (int i2 = 0; i2 < (r < lim ? kD : 0); ++i2) {
-                            const int cc = (i2 + p) & (kD - 1);
-                            const float ks = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(s, cc))) *
-                                             __expf(sG[r * 128 + cc] - sG[s * 128 + cc]);
-                            a = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(r, cc))), ks, a);
-                            pp = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(64 + r, cc))),
-                                      ks, pp);
-                        }
-                        const int tr = m * kC + r;  // beta of chunk m (the scratch holds the previous chunk's)
-                        const float br = tr < seq_len ? __bfloat162float(beta[(tok0 + tr) * H + h]) : 0.f;
-                        av[i] = (s < r && erase) ? br * a : 0.f;  // no erase: A = 0
-                        pv[i] = pp;
-                    }
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dROWK, rb * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32),
+                                    dadd(dCOLK, cb * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32), ID_AP, kk > 0);
                 }
-                nb_sync(NB_PREP, kPrep);  // gate staging read
-                for (int i = tid; i < 64 * kLDA; i += kPrep) sA[i] = 0.f;
-                for (int i = tid; i < 8192 / 16; i += kPrep)
-                    st_shared_v4(sb + L::SP + par * 8192 + 16 * i, 0u, 0u, 0u, 0u);
-                nb_sync(NB_PREP, kPrep);
-#pragma unroll
-                for (int i = 0; i < 9; ++i) {
-                    const int p = tid + kPrep * i;
-                    if (p < kC * (kC + 1) / 2) {
-                        int r = (int)((sqrtf(8.f * (float)p + 1.f) - 1.f) * 0.5f);
-                        while ((r + 1) * (r + 2) / 2 <= p) ++r;
-                        while (r * (r + 1) / 2 > p) --r;
-                        const int s = p - r * (r + 1) / 2;
-                        sA[r * kLDA + s] = av[i];
-                        *reinterpret_cast<__nv_bfloat16*>(sm + L::SP + par * 8192 + km_off(r, s)) =
-                            __float2bfloat16_rn(pv[i]);
-                    }
+                mma_commit(bars + B_AP + s);
+                if (m + 1 < NC) {  // next chunk's prefix sums, once its slot is read out and its gate is in place
+                    const int s1 = (m + 1) % 3;
+                    if (m + 1 >= 3) wait1(B_SF + s1, (uint32_t)((m + 1) / 3 - 1));
+                    if (GATE != 2) wait1(B_G + s1, (uint32_t)((m + 1) / 3));
+                    tc_fence_after();
+                    cumsum_mma(m + 1);
                 }
             }
-            // operand tiles, in place: 4 groups of 8 channels of this thread's row
-#pragma unroll 1
-            for (int u4 = 0; u4 < 4; ++u4) {
-                const int c0 = 32 * cb + 8 * u4;
-                uint32_t g8[8];
-                load_g8(u4, g8);
-                const uint32_t ko = rop_off(tok, c0);
-                const uint32_t fo = (uint32_t)((c0 >> 6) * 8192 + tok * 128 + ((((c0 & 63) >> 3) ^ (tok & 7)) << 4));
-                const uint4 kv = ld_shared_v4(rop + ko);
-                const uint4 qv = ld_shared_v4(rop + ko + 8192);
-                const float4 ra = *reinterpret_cast<const float4*>((exact ? sGl : sGm) + c0);
-                const float4 rb = *reinterpret_cast<const float4*>((exact ? sGl : sGm) + c0 + 4);
-                const float ref8[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-                const uint32_t km = live ? 0xFFFFFFFFu : 0u;  // rows past the sequence: k = q = 0
-                const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
-                const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-                uint32_t ke[4], qe[4], kf[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float g0 = __uint_as_float(g8[2 * u]), g1 = __uint_as_float(g8[2 * u + 1]);
-                    float e0, e1, f0, f1;
-                    if (!exact) {  // E = e^{G - G_m}, F = 1/E
-                        e0 = __expf(g0 - ref8[2 * u]);
-                        e1 = __expf(g1 - ref8[2 * u + 1]);
-                        f0 = rcp_approx(e0);
-                        f1 = rcp_approx(e1);
-                    } else {       // e^G and e^{G_last - G}
-                        e0 = __expf(g0);
-                        e1 = __expf(g1);
-                        f0 = __expf(ref8[2 * u] - g0);
-                        f1 = __expf(ref8[2 * u + 1] - g1);
-                    }
-                    // packed bf16 products: the factor pairs are rounded to bf16
-                    // first, the products once more (both well inside the bf16
-                    // rounding of the MMA operands)
-                    const uint32_t ep = pack_bf16x2(e0, e1), fp = pack_bf16x2(f0, f1);
-                    ke[u] = hmul2_bf16(kw[u], ep) & km;
-                    qe[u] = hmul2_bf16(qw[u], ep) & km;
-                    kf[u] = hmul2_bf16(kw[u], fp) & km;
-                }
-                st_shared_v4(rop + ko, ke[0], ke[1], ke[2], ke[3]);
-                st_shared_v4(rop + ko + 8192, qe[0], qe[1], qe[2], qe[3]);
-                st_shared_v4(colop(par) + fo, kf[0], kf[1], kf[2], kf[3]);
+            __syncwarp();
+        }
+        if (ttid == 0) {
+            drain(B_EXKQ, nex);
+            if (*s_abort) {
+                mma_commit(bars + B_FIN + 1);
+                mbar_wait_bounded(bars + B_FIN + 1, 0u, kDrainBudget);
             }
-            return exact;
+        }
+    } else {
+        // ============================================================ inverse warps
+        // Per chunk m: A/P readout, (I + A)^{-1} -> T', then the PT, W and U MMAs
+        // with the readouts between them (PT -> [T'; PT], [W'; P W'] -> row operand).
+        const int iw = warp - kInvWarp0;  // 0..7
+        const int hf = iw >> 2;           // which 32-column half of a readout this warp takes
+        const int itid = tid - 32 * kInvWarp0;
+        int n_v = 0;
+        auto load_beta = [&](int m) -> float {
+            const int t = m * kC + itid;
+            return (itid < kC && m < NC && t < seq_len) ? __bfloat162float(beta[(tok0 + t) * H + h]) : 0.f;
         };
-        // ---- P4: A (lanes 0-63 of the prefix-sum columns) -> fp32 scratch (beta_r, strictly lower);
-        // P (lanes 64-127) -> bf16 K-major tile of this parity (lower incl.)
-        auto p4 = [&](int par) {
+        // ---- A (slot rows 0-63) -> fp32 scratch (beta_r, strictly lower); P (rows 64-127) -> bf16 K-major tile (lower incl.)
+        auto p4 = [&](uint32_t slot) {
+            if (quad < 2 && !erase) return;  // additive write: A is not used
             uint32_t v[32];
-            tmem_ld32(lane_addr + L::GC_COL + 32 * hf, v);
+            tmem_ld32(slot + 32 * hf, v);
             tmem_ld_wait(v);
             if (quad < 2) {
-                if (!erase) return;  // additive write: A is not used
                 const int r = 32 * quad + lane;
                 const float br = sBeta[r];
                 float* dst = sA + r * kLDA + 32 * hf;
@@ -953,18 +1059,17 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         const float p1 = (s + 1 <= r) ? __uint_as_float(v[8 * jc + 2 * u + 1]) : 0.f;
                         w[u] = pack_bf16x2(p0, p1);
                     }
-                    st_shared_v4(sb + L::SP + par * 8192 + r * 128 + (((4 * hf + jc) ^ (r & 7)) << 4), w[0], w[1],
-                                 w[2], w[3]);
+                    st_shared_v4(sb + L::SP + r * 128 + (((4 * hf + jc) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
                 }
             }
         };
-        // ---- P5: T = (I + A)^{-1} -> T' = T Diag(beta), bf16, rows 0-63 of [T'; 0]
+        // ---- P5: T = (I + A)^{-1} -> T' = T Diag(beta), bf16, rows 0-63 of [T'; PT]
         auto store_tprime = [&](int r, int s, float t) {
-            *reinterpret_cast<__nv_bfloat16*>(sm + L::TZP + km_off(r, s)) = __float2bfloat16_rn(t * sBeta[s]);
+            *reinterpret_cast<__nv_bfloat16*>(sm + L::TP + km_off(r, s)) = __float2bfloat16_rn(t * sBeta[s]);
         };
         auto p5 = [&]() {
-            if (!erase) {  // A = 0: T = I, T' = Diag(beta); thread: row tid/4, 16 columns
-                const int r = tid >> 2, j0c = 2 * (tid & 3);
+            if (!erase) {  // A = 0: T = I, T' = Diag(beta); thread: row itid/4, 16 columns
+                const int r = itid >> 2, j0c = 2 * (itid & 3);
 #pragma unroll
                 for (int jc = 0; jc < 2; ++jc) {
                     const int j = j0c + jc;  // 8-column chunk
@@ -974,12 +1079,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         const int s0 = 8 * j + 2 * u;
                         w[u] = pack_bf16x2(s0 == r ? sBeta[r] : 0.f, s0 + 1 == r ? sBeta[r] : 0.f);
                     }
-                    st_shared_v4(sb + L::TZP + r * 128 + ((j ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                    st_shared_v4(sb + L::TP + r * 128 + ((j ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
                 }
                 return;
             }
             {   // diagonal 16x16 blocks: four threads per column, rows q, q+4, q+8, q+12
-                const int a = tid >> 6, jc = (tid >> 2) & 15, q = tid & 3;
+                const int a = itid >> 6, jc = (itid >> 2) & 15, q = itid & 3;
                 const float* Ab = sA + (16 * a) * kLDA + 16 * a;
                 float acc[4] = {0.f, 0.f, 0.f, 0.f}, colv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -998,14 +1103,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     store_tprime(r, s, colv[i]);
                 }
             }
-            nb_sync(NB_PREP, kPrep);
+            nb_sync(NB_INV, 256);
             // Blocks below the diagonal, one column chain per warp (block column
             // bb, 8-column half nt), on the tensor cores (m16n8k8, tf32). For
             // a = bb+1..3: X = sum_{k=bb}^{a-1} A_ak T_kb, then T_ab = -T_aa X.
             // Every operand is either a diagonal block or a block this warp
             // wrote before, so the chain needs no block-wide barrier.
             {
-                const int bb = warp >> 1, nt = warp & 1;
+                const int bb = iw >> 1, nt = iw & 1;
                 const int g = lane >> 2, t = lane & 3;
                 const int s0 = 16 * bb + 8 * nt + 2 * t;
 #pragma unroll 1
@@ -1027,95 +1132,148 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         const int r = 16 * a + g + 8 * hh;
                         const float v0 = -tx[2 * hh], v1 = -tx[2 * hh + 1];
                         *reinterpret_cast<float2*>(sT + r * kLDA + s0) = make_float2(v0, v1);
-                        *reinterpret_cast<uint32_t*>(sm + L::TZP + km_off(r, s0)) =
+                        *reinterpret_cast<uint32_t*>(sm + L::TP + km_off(r, s0)) =
                             pack_bf16x2(v0 * sBeta[s0], v1 * sBeta[s0 + 1]);
                     }
                     __syncwarp();
                 }
             }
         };
-        // ---- P7: [W'; 0] (lanes 0-63) -> -W' over the KE rows
-        auto p7 = [&](int par) {
-            if (quad < 2 && !erase) {  // additive write: delta = U, the W S term is zero
-                const int r = 32 * quad + lane;
+        // ---- PT (slot rows 64-127, columns 64-127) -> bf16 rows 64-127 of [T'; PT]
+        auto p6 = [&](uint32_t slot) {
+            if (quad < 2) return;
+            const int r = 32 * (quad - 2) + lane;
+            uint32_t v[32];
+            tmem_ld32(slot + 64 + 32 * hf, v);
+            tmem_ld_wait(v);
 #pragma unroll
-                for (int jc = 0; jc < 8; ++jc)
-                    st_shared_v4(rowop(par) + hf * 16384 + r * 128 + ((jc ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
-                return;
+            for (int jc = 0; jc < 4; ++jc) {
+                uint32_t w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]), __uint_as_float(v[8 * jc + 2 * u + 1]));
+                const int R = 64 + r;
+                st_shared_v4(sb + L::TP + R * 128 + (((4 * hf + jc) ^ (R & 7)) << 4), w[0], w[1], w[2], w[3]);
             }
+        };
+        // ---- P7: [W'; P W'] -> row operand: rows 0-63 -W' over KE, rows 64-127 QE - P W'
+        auto p7 = [&](uint32_t slot, int rb) {
+            const uint32_t rop = sb + L::ROW + rb * 32768;
             if (quad < 2) {
                 const int r = 32 * quad + lane;
+                if (!erase) {  // additive write: delta = U, the W S term is zero
+#pragma unroll
+                    for (int jc = 0; jc < 8; ++jc)
+                        st_shared_v4(rop + hf * 16384 + r * 128 + ((jc ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
+                    return;
+                }
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t v[32];
-                    tmem_ld32(lane_addr + L::W_COL + 64 * hf + 32 * hh, v);
+                    tmem_ld32(slot + 64 * hf + 32 * hh, v);
                     tmem_ld_wait(v);
 #pragma unroll
                     for (int jc = 0; jc < 4; ++jc) {
                         uint32_t w[4];
 #pragma unroll
                         for (int u = 0; u < 4; ++u)
-                            w[u] = pack_bf16x2(-__uint_as_float(v[8 * jc + 2 * u]),
-                                               -__uint_as_float(v[8 * jc + 2 * u + 1]));
-                        st_shared_v4(rowop(par) + hf * 16384 + r * 128 + (((4 * hh + jc) ^ (r & 7)) << 4), w[0],
-                                     w[1], w[2], w[3]);
+                            w[u] = pack_bf16x2(-__uint_as_float(v[8 * jc + 2 * u]), -__uint_as_float(v[8 * jc + 2 * u + 1]));
+                        st_shared_v4(rop + hf * 16384 + r * 128 + (((4 * hh + jc) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                    }
+                }
+            } else {
+                if (!erase) return;  // W = 0: the rows keep QE
+                const int r = 32 * (quad - 2) + lane, R = 64 + r;
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t v[32];
+                    tmem_ld32(slot + 64 * hf + 32 * hh, v);
+                    tmem_ld_wait(v);
+#pragma unroll
+                    for (int jc = 0; jc < 4; ++jc) {
+                        const uint32_t addr = rop + hf * 16384 + R * 128 + (((4 * hh + jc) ^ (R & 7)) << 4);
+                        const uint4 qv = ld_shared_v4(addr);
+                        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                        uint32_t w[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            w[u] = pack_bf16x2(bf16_lo(qw[u]) - __uint_as_float(v[8 * jc + 2 * u]),
+                                               bf16_hi(qw[u]) - __uint_as_float(v[8 * jc + 2 * u + 1]));
+                        st_shared_v4(addr, w[0], w[1], w[2], w[3]);
                     }
                 }
             }
         };
-
-
-        auto p2_signal = [&](int m, bool exact) {
-            fence_proxy_async_smem();
-            tc_fence_before();
-            nb_sync(NB_PREP, kPrep);
-            if (tid == 0) {
-                s_exact[m & 1] = exact;
-                mbar_arrive(bars + BAR_SC + (m & 3));
-                mbar_arrive(bars + BAR_P2);
-            }
-            __syncwarp();
-        };
-        bool exact_cur = false;
-        if (NC > 0) {  // (an empty packed sequence has no chunk: its state passes through)
-            waitw(BAR_CS, 0u);
-            waitw(BAR_KQ, 0u);
-            nb_sync(NB_PREP, kPrep);
-            exact_cur = p2(0);
-            p2_signal(0, exact_cur);
+        if (NC > 0 && itid == 0) {
+            load_v(0);
+            ++n_v;
+            pf_v(1);
         }
         float beta_next = load_beta(0);
         for (int m = 0; m < NC; ++m) {
-            const int par = m & 1;
-            if (tid < kC) sBeta[tid] = beta_next;
+            const int s = m % 3, rb = m & 1;
+            const uint32_t slot = lane_addr + L::SLOT0 + 128 * s;
+            if (itid < kC) sBeta[itid] = beta_next;
             beta_next = load_beta(m + 1);
-            waitw(BAR_AP, (uint32_t)m);
-            if (!exact_cur && m >= 2) waitw(BAR_M2B + par, (uint32_t)((m >> 1) - 1));  // P of chunk m-2 consumed
-            nb_sync(NB_PREP, kPrep);  // beta of chunk m visible
-            if (!exact_cur) p4(par);
-            fence_proxy_async_smem();
-            tc_fence_before();
-            nb_sync(NB_PREP, kPrep);
-            if (tid == 0) mbar_arrive(bars + BAR_P4);  // prefix-sum columns free
+            waitw(B_AP + s, (uint32_t)(m / 3));
+            if (m > 0 && itid == 0) {  // [T'; PT] and the v tile of the previous chunk are free
+                wait1(B_UO + (m - 1) % 3, (uint32_t)((m - 1) / 3));
+                load_v(m);
+                ++n_v;
+                pf_v(m + 1);
+            }
+            nb_sync(NB_INV, 256);  // beta of chunk m visible, [T'; PT] free
+            p4(slot);
+            nb_sync(NB_INV, 256);
             p5();
             fence_proxy_async_smem();
             tc_fence_before();
-            nb_sync(NB_PREP, kPrep);
-            if (tid == 0) mbar_arrive(bars + BAR_P5);  // T' stored
-            bool exact_next = false;
-            if (m + 1 < NC) {
-                waitw(BAR_CS, (uint32_t)(m + 1));
-                waitw(BAR_KQ + (par ^ 1), (uint32_t)((m + 1) >> 1));
-                exact_next = p2(m + 1);
-                p2_signal(m + 1, exact_next);
+            nb_sync(NB_INV, 256);
+            if (itid == 0) {
+                mbar_arrive(bars + B_SCRF);  // A/T scratch free
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // PT = P T' into columns 64-127 (rows 0-63 take junk)
+                    mma_bf16_ss(tmem + L::SLOT0 + 128 * s + 64, dadd(dYP, kk * 32), dadd(dTPN, kk * 2048), ID_PT, kk > 0);
+                mma_commit(bars + B_PT);
             }
-            waitw(BAR_UW, (uint32_t)m);
-            p7(par);
+            waitw(B_PT, (uint32_t)m);
+            p6(slot);
             fence_proxy_async_smem();
             tc_fence_before();
-            nb_sync(NB_PREP, kPrep);
-            if (tid == 0) mbar_arrive(bars + BAR_RR + par);
-            exact_cur = exact_next;
+            nb_sync(NB_INV, 256);
+            if (erase) {
+                if (itid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)  // [W'; P W'] = [T'; PT] KE
+                        mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dTP, kk * 32), dadd(dROWN, rb * 32768 + kk * 2048),
+                                    ID_W, kk > 0);
+                    mma_commit(bars + B_WB);
+                }
+                waitw(B_WB, (uint32_t)m);
+            }
+            p7(slot, rb);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            nb_sync(NB_INV, 256);
+            if (itid == 0) {
+                mbar_arrive(bars + B_RR + rb);  // row operand of chunk m stored
+                wait1(B_V, (uint32_t)m);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // [U; P T' v] = [T'; PT] v: the chunk's accumulator
+                    mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dTP, kk * 32), dadd(dV, kk * 2048), ID_U, kk > 0);
+                mma_commit(bars + B_UO + s);
+            }
+            __syncwarp();
+        }
+        if (itid == 0) {
+            drain(B_V, n_v);
+            if (*s_abort) {
+                mma_commit(bars + B_FIN + 2);
+                mbar_wait_bounded(bars + B_FIN + 2, 0u, kDrainBudget);
+            }
         }
     }
     tc_fence_before();
@@ -1326,41 +1484,26 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int scan_mode, cudaStream_t stre
 // code running inside a memory allocator's own callbacks, host applications
 // that forbid cudaMalloc on their worker threads, or runtimes that expose
 // only the tensors they already own.
-#include <mutex>
-
 #include "kda.h"
 
 // Scratch of the allocation-free entry point; every GPU that loads this
 // library holds these bytes until the process exits. In host code this name
 // is only a stand-in for the symbol: its device address comes from
-// cudaGetSymbolAddress, once per device.
+// cudaGetSymbolAddress, looked up on every call with the caller's device
+// current (a host-side query, so a device reset cannot leave a stale address
+// behind).
 static __device__ __align__(256) unsigned char g_kda_noalloc_scratch[256];
 
 namespace {
 
-constexpr int kNoAllocMaxDevices = 128;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_scratch_addr[kNoAllocMaxDevices] = {};
-
-// Device address of the scratch array on the current device, looked up on
-// the first call made with that device current.
+// Device address of the scratch array on the current device.
 cudaError_t noalloc_scratch(void** out) {
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t err = cudaGetSymbolAddress(&p, g_kda_noalloc_scratch);
     if (err != cudaSuccess) return err;
-    if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_scratch_addr[dev] == nullptr) {
-        void* p = nullptr;
-        err = cudaGetSymbolAddress(&p, g_kda_noalloc_scratch);
-        if (err != cudaSuccess) return err;
-        g_noalloc_scratch_addr[dev] = p;
-    }
-    *out = g_noalloc_scratch_addr[dev];
+    *out = p;
     return cudaSuccess;
 }
-
-bool noalloc_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 
@@ -1368,22 +1511,15 @@ extern "C" kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, cons
                                               const void* beta, const float* S0, void* o, float* S_T, int B,
                                               int T, int H, int dk, int dv, int chunk, kda_dtype_t dtype,
                                               void* stream) {
-    if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
-    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
-    if ((long long)B * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
     kda::ChunkArgs a;
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
     a.erase = 1;  // KDA: erase with a per-channel gate
     a.gate = KDA_GATE_CHANNEL;
     a.cu_seqlens = nullptr;
+    const kda_status_t st = kda::check_chunk_args(a, dtype);
+    if (st != KDA_OK) return st;
     if (!kda::chunk_tc_supported(a)) return KDA_ERR_UNSUPPORTED;
-    if ((long long)B * T * H > 0) {
-        const void* req[] = {q, k, v, log_alpha, beta, o};
-        for (const void* p : req)
-            if (p == nullptr || !noalloc_aligned16(p)) return KDA_ERR_INVALID_ARG;
-    }
-    if ((S0 && !noalloc_aligned16(S0)) || (S_T && !noalloc_aligned16(S_T))) return KDA_ERR_INVALID_ARG;
     // The kernel's scratch must fit the fixed array.
     if (kda::chunk_tc_workspace_bytes(a, 0) > sizeof(g_kda_noalloc_scratch)) return KDA_ERR_INVALID_ARG;
     if ((long long)B * H == 0) return KDA_OK;
@@ -1394,4 +1530,14 @@ extern "C" kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, cons
     // launch_chunk_tc clears the status word before the kernel runs.
     const cudaError_t err = kda::launch_chunk_tc(a, 0, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" kda_status_t kda_noalloc_status(void* stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
+    void* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return KDA_ERR_CUDA;
+    unsigned flag = 0;
+    if (cudaMemcpy(&flag, scratch, sizeof(flag), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+    return flag ? KDA_ERR_TIMEOUT : KDA_OK;
 }
