@@ -91,7 +91,8 @@ constexpr int NB_CHHI = 6;  // chain warps 2-3
 constexpr int NB_CH = 7;    // all chain warps
 constexpr int kC = 64;    // chunk
 constexpr int kD = 128;   // dk = dv
-constexpr int kLDA = 68;  // fp32 row stride of the A / T scratch (bank spread)
+constexpr int kLDA = 68;  // fp32 row stride of the A scratch (bank spread)
+constexpr int kLDT = 20;  // fp32 row stride of the diagonal blocks of T (bank spread)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kGuardL = 80.f * kLog2e;      // |G_r - G_m| <= 80, in log2 units
 constexpr long long kWaitBudget = 1ll << 31;  // SM cycles (~1 s)
@@ -108,10 +109,12 @@ struct Layout {
     static constexpr uint32_t TP = 147456;      // [T'; PT] K-major 128 x 64
     static constexpr uint32_t SP = TP + 16384;  // P, K-major 64 x 64 bf16 (rows 64-127 of [Y; P], Y = TP rows 64-127)
     static constexpr uint32_t SOP = SP + 8192;  // S half (64 channels) x DVT, bf16 MN-major, then delta
-    static constexpr uint32_t SCR = SOP + 64 * DVT * 2;  // A, T fp32 [64][kLDA]; exact path: staging
-    static constexpr uint32_t SA = SCR;
-    static constexpr uint32_t ST = SCR + 64 * kLDA * 4;
-    static constexpr uint32_t SMALL = SCR + 2 * 64 * kLDA * 4;
+    static constexpr uint32_t OST = SOP + 64 * DVT * 2;  // 2 x [32 tok][32 ch] bf16 (64-byte swizzle): O stores
+    static constexpr uint32_t SCR = OST + 4096;          // A fp32 [64][kLDA], T diagonal blocks [4][16][kLDT]
+    static constexpr uint32_t SA = SCR;                  //   (exact path: 16 KB staging)
+    static constexpr uint32_t STD = SCR + 64 * kLDA * 4;
+    static constexpr uint32_t SCR_BYTES = 64 * kLDA * 4 + 4 * 16 * kLDT * 4;
+    static constexpr uint32_t SMALL = SCR + SCR_BYTES;
     static constexpr uint32_t SBETA = SMALL;        // 64 f32: beta of the inverse warps' chunk
     static constexpr uint32_t SOPS = SBETA + 256;   // 4 x 128 f32: operand scale per channel (by chunk mod 4)
     static constexpr uint32_t STMS = SOPS + 2048;   // 4 x 128 f32: tensor-memory scale per channel
@@ -124,8 +127,8 @@ struct Layout {
     static constexpr uint32_t END = MISC + 64;
     static constexpr uint32_t SMEM_BYTES = END + 1024;   // + alignment slack
     static constexpr uint32_t SBO_V = 1024 * (DVT / 64); // K-group stride of the S / delta operands
-    static_assert(SOP % 1024 == 0 && TP % 1024 == 0 && LMAT % 1024 == 0, "operand alignment");
-    static_assert(64 * 128 * 4 <= 2 * 64 * kLDA * 4, "exact-path gate staging overflows the scratch");
+    static_assert(SOP % 1024 == 0 && TP % 1024 == 0 && LMAT % 1024 == 0 && OST % 1024 == 0, "operand alignment");
+    static_assert(64 * 64 * 4 <= SCR_BYTES, "exact-path staging overflows the scratch");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     // tensor memory columns: R (fp32, lane = key channel) and three chunk slots
     static constexpr uint32_t S_COL = 0;
@@ -188,26 +191,6 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// acc += X Y restricted to columns [8*nt, 8*nt+8) of the 16x16 product; X and
-// Y are 16x16 fp32 tiles (row stride kLDA) in shared memory, rounded to tf32
-// (the resulting T' is stored as bf16, which dominates its rounding error).
-// Fragment mapping of m16n8k8 (g = lane/4, t = lane%4): A (g|g+8, t|t+4),
-// B (t|t+4, g), C (g|g+8, 2t|2t+1).
-__device__ __forceinline__ void mm16_ntile(float (&acc)[4], const float* X, const float* Y, int nt, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-    float part[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-        const uint32_t a[4] = {to_tf32(X[g * kLDA + 8 * ks + t]), to_tf32(X[(g + 8) * kLDA + 8 * ks + t]),
-                               to_tf32(X[g * kLDA + 8 * ks + t + 4]), to_tf32(X[(g + 8) * kLDA + 8 * ks + t + 4])};
-        const uint32_t bq[2] = {to_tf32(Y[(8 * ks + t) * kLDA + 8 * nt + g]),
-                                to_tf32(Y[(8 * ks + t + 4) * kLDA + 8 * nt + g])};
-        mma_tf32_16x8x8(part[ks], a, bq);  // two independent accumulators
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[e] += part[0][e] + part[1][e];
-}
-
 __device__ __forceinline__ void nb_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -257,7 +240,7 @@ template <int DVT, int ERASE, int GATE>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
-                    const __nv_bfloat16* __restrict__ beta, const float* S0, __nv_bfloat16* __restrict__ o,
+                    const __grid_constant__ CUtensorMap tm_o, const __nv_bfloat16* __restrict__ beta, const float* S0, __nv_bfloat16* __restrict__ o,
                     float* ST, int Tlen, int H, unsigned* status, const __nv_bfloat16* __restrict__ gate_tok,
                     const int* __restrict__ cu_seqlens, const SegJobs sj) {
     constexpr int erase = ERASE;
@@ -330,7 +313,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     float* sGl = reinterpret_cast<float*>(sm + L::SGL);
     float* sGmL = reinterpret_cast<float*>(sm + L::SGML);
     float* sA = reinterpret_cast<float*>(sm + L::SA);
-    float* sT = reinterpret_cast<float*>(sm + L::ST);
+    float* sTd = reinterpret_cast<float*>(sm + L::STD);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BARS);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
@@ -344,6 +327,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_g);
         tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_o);
     }
     if (warp == 0) {
         tmem_alloc(s_tmem, L::TMEM_COLS);
@@ -658,15 +642,36 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 tc_fence_before();
                 nb_arrive(NB_CHB, 96);
                 waitw(B_M1, (uint32_t)n);
-                {   // O (slot rows 64-127) -> global bf16
+                {   // O (slot rows 64-127) -> global bf16: a full chunk through a swizzled
+                    // [32 tok][32 ch] stage and a tensor store per 32 columns (coalesced,
+                    // asynchronous); a partial chunk by plain stores (rows past a packed
+                    // sequence belong to the next one)
                     const int r = row - 64;
                     const int t0 = n * kC;
+                    const bool full = t0 + kC <= seq_len;
+                    uint8_t* stg = sm + L::OST + (quad - 2) * 2048;
 #pragma unroll 1
                     for (int gq = 0; gq < DVT / 32; ++gq) {
                         uint32_t v[32];
                         tmem_ld32(slot + 32 * gq, v);
                         tmem_ld_wait(v);
-                        if (o_on && t0 + r < seq_len) {
+                        if (o_on && full) {
+                            if (lane == 0) bulk_wait_read0();  // the stage's previous store has read it
+                            __syncwarp();
+#pragma unroll
+                            for (int jc = 0; jc < 4; ++jc)
+                                st_shared_v4(smem_u32(stg) + lane * 64 + ((jc ^ ((lane >> 1) & 3)) << 4),
+                                             pack_bf16x2(__uint_as_float(v[8 * jc + 0]), __uint_as_float(v[8 * jc + 1])),
+                                             pack_bf16x2(__uint_as_float(v[8 * jc + 2]), __uint_as_float(v[8 * jc + 3])),
+                                             pack_bf16x2(__uint_as_float(v[8 * jc + 4]), __uint_as_float(v[8 * jc + 5])),
+                                             pack_bf16x2(__uint_as_float(v[8 * jc + 6]), __uint_as_float(v[8 * jc + 7])));
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_4d(&tm_o, stg, j0 + 32 * gq, h, tma_t0 + t0 + 32 * (quad - 2), tma_b);
+                                bulk_commit();
+                            }
+                        } else if (o_on && t0 + r < seq_len) {
                             uint4* dst = reinterpret_cast<uint4*>(o + ((tok0 + t0 + r) * H + h) * kD + j0 + 32 * gq);
 #pragma unroll
                             for (int jc = 0; jc < 4; ++jc) {
@@ -704,6 +709,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                                          __uint_as_float(v[4 * u + 2]) * ek, __uint_as_float(v[4 * u + 3]) * ek);
             }
         }
+        if (quad >= 2 && lane == 0) bulk_wait0();  // every tensor store of O complete
         if (issuer) {
             for (int x = 0; x < 2; ++x) drain(B_KQ + x, n_kq[x]);
             for (int x = 0; x < 3; ++x) drain(B_G + x, n_g[x]);
@@ -732,28 +738,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             if (ttid == 0) load_kq(m, B_EXKQ);
             waitw(B_EXKQ, (uint32_t)nex);
             if (m > 0) waitw(B_SCRF, (uint32_t)(m - 1));  // the inverse warps are done with the scratch
-            float* sG = reinterpret_cast<float*>(sm + L::SCR);
+            float* stg = reinterpret_cast<float*>(sm + L::SCR);  // 16 KB: G of 64 channels, then A, then P
             const bool live = tok < lim;
-#pragma unroll 1
-            for (int u8 = 0; u8 < 8; ++u8) {  // G -> fp32 [64][128] staging
-                uint32_t g8[8];
-                if (GATE == 0) {
-                    tmem_ld8(slotq + ch0 + 8 * u8, g8);
-                    tmem_ld_wait(g8);
-                } else {
-                    uint32_t g1;
-                    tmem_ld1(slotq, g1);
-                    tmem_ld_wait1(g1);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) g8[e] = g1;
-                }
-                float* dst = sG + tok * 128 + ch0 + 8 * u8;
-                *reinterpret_cast<float4*>(dst) = make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]),
-                                                              __uint_as_float(g8[2]), __uint_as_float(g8[3]));
-                *reinterpret_cast<float4*>(dst + 4) = make_float4(__uint_as_float(g8[4]), __uint_as_float(g8[5]),
-                                                                  __uint_as_float(g8[6]), __uint_as_float(g8[7]));
-            }
-            nb_sync(NB_TILE, 128);
             const uint8_t* rk = sm + L::ROW + rb * 32768;
             constexpr int kPairs = kC * (kC + 1) / 2, kPer = (kPairs + 127) / 128;
             float av[kPer], pv[kPer];
@@ -761,29 +747,62 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             for (int i = 0; i < kPer; ++i) {
                 av[i] = 0.f;
                 pv[i] = 0.f;
-                const int p = ttid + 128 * i;
-                if (p < kPairs) {
-                    int r = (int)((sqrtf(8.f * (float)p + 1.f) - 1.f) * 0.5f);
-                    while ((r + 1) * (r + 2) / 2 <= p) ++r;
-                    while (r * (r + 1) / 2 > p) --r;
-                    const int s2 = p - r * (r + 1) / 2;
-                    float a = 0.f, pp = 0.f;
-                    // rows past the sequence stay 0 (their gates may be another
-                    // sequence's and overflow the exponential)
-                    for (int i2 = 0; i2 < (r < lim ? kD : 0); ++i2) {
-                        const int cc = (i2 + p) & (kD - 1);
-                        const float ks = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(s2, cc))) *
-                                         ex2((sG[r * 128 + cc] - sG[s2 * 128 + cc]) * kLog2e);
-                        a = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(r, cc))), ks, a);
-                        pp = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(64 + r, cc))),
-                                  ks, pp);
-                    }
-                    av[i] = a;
-                    pv[i] = pp;
-                }
             }
-            nb_sync(NB_TILE, 128);  // raw rows read
-            {   // plain tiles in place
+            auto pair_rs = [](int p, int& r, int& s2) {
+                r = (int)((sqrtf(8.f * (float)p + 1.f) - 1.f) * 0.5f);
+                while ((r + 1) * (r + 2) / 2 <= p) ++r;
+                while (r * (r + 1) / 2 > p) --r;
+                s2 = p - r * (r + 1) / 2;
+            };
+#pragma unroll 1
+            for (int hc = 0; hc < 2; ++hc) {  // channels [64 hc, 64 hc + 64)
+                if ((ch0 >> 6) == hc) {       // this thread's channels: G -> fp32 [64 tok][64 ch]
+#pragma unroll 1
+                    for (int u8 = 0; u8 < 8; ++u8) {
+                        uint32_t g8[8];
+                        if (GATE == 0) {
+                            tmem_ld8(slotq + ch0 + 8 * u8, g8);
+                            tmem_ld_wait(g8);
+                        } else {
+                            uint32_t g1;
+                            tmem_ld1(slotq, g1);
+                            tmem_ld_wait1(g1);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) g8[e] = g1;
+                        }
+                        float* dst = stg + tok * 64 + 8 * u8;
+                        *reinterpret_cast<float4*>(dst) = make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]),
+                                                                      __uint_as_float(g8[2]), __uint_as_float(g8[3]));
+                        *reinterpret_cast<float4*>(dst + 4) = make_float4(__uint_as_float(g8[4]), __uint_as_float(g8[5]),
+                                                                          __uint_as_float(g8[6]), __uint_as_float(g8[7]));
+                    }
+                }
+                nb_sync(NB_TILE, 128);
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) {
+                    const int p = ttid + 128 * i;
+                    if (p < kPairs) {
+                        int r, s2;
+                        pair_rs(p, r, s2);
+                        float a = av[i], pp = pv[i];
+                        // rows past the sequence stay 0 (their gates may be another
+                        // sequence's and overflow the exponential)
+                        for (int i2 = 0; i2 < (r < lim ? 64 : 0); ++i2) {
+                            const int c = (i2 + p) & 63, cc = 64 * hc + c;
+                            const float ks =
+                                __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(s2, cc))) *
+                                ex2((stg[r * 64 + c] - stg[s2 * 64 + c]) * kLog2e);
+                            a = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(r, cc))), ks, a);
+                            pp = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(64 + r, cc))),
+                                      ks, pp);
+                        }
+                        av[i] = a;
+                        pv[i] = pp;
+                    }
+                }
+                nb_sync(NB_TILE, 128);  // staging read
+            }
+            {   // plain tiles in place (the raw rows are no longer needed)
                 const uint32_t rop = sb + L::ROW + rb * 32768;
                 const uint32_t colp = sb + L::COL + cb * 16384;
 #pragma unroll 1
@@ -823,36 +842,35 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     st_shared_v4(colp + fo, kf[0], kf[1], kf[2], kf[3]);
                 }
             }
-            // raw A and P sums -> fp32 [64][64] staging (over the gate staging), then
-            // into the slot: quadrant 0/1 rows are A rows, 2/3 rows are P rows
-            float* stA = sG;
-            float* stP = sG + 64 * 64;
-            for (int i = ttid; i < 2 * 64 * 64 / 4; i += 128)
-                reinterpret_cast<float4*>(stA)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            nb_sync(NB_TILE, 128);
-#pragma unroll
-            for (int i = 0; i < kPer; ++i) {
-                const int p = ttid + 128 * i;
-                if (p < kPairs) {
-                    int r = (int)((sqrtf(8.f * (float)p + 1.f) - 1.f) * 0.5f);
-                    while ((r + 1) * (r + 2) / 2 <= p) ++r;
-                    while (r * (r + 1) / 2 > p) --r;
-                    const int s2 = p - r * (r + 1) / 2;
-                    stA[r * 64 + s2] = av[i];
-                    stP[r * 64 + s2] = pv[i];
-                }
-            }
-            nb_sync(NB_TILE, 128);
-            {
-                const float* src = quad < 2 ? stA + (32 * quad + lane) * 64 : stP + (32 * (quad - 2) + lane) * 64;
+            // raw A sums, then raw P sums -> fp32 [64][64] staging -> the slot
+            // (quadrants 0/1 hold the A rows, 2/3 the P rows)
 #pragma unroll 1
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t r32[32];
+            for (int w = 0; w < 2; ++w) {
+                for (int i = ttid; i < 64 * 64 / 4; i += 128)
+                    reinterpret_cast<float4*>(stg)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                nb_sync(NB_TILE, 128);
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) r32[u] = __float_as_uint(src[32 * h2 + u]);
-                    tmem_st32(slotq + 32 * h2, r32);
+                for (int i = 0; i < kPer; ++i) {
+                    const int p = ttid + 128 * i;
+                    if (p < kPairs) {
+                        int r, s2;
+                        pair_rs(p, r, s2);
+                        stg[r * 64 + s2] = w == 0 ? av[i] : pv[i];
+                    }
                 }
-                tmem_st_wait();
+                nb_sync(NB_TILE, 128);
+                if ((quad >> 1) == w) {
+                    const float* src = stg + (32 * (quad & 1) + lane) * 64;
+#pragma unroll 1
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        uint32_t r32[32];
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) r32[u] = __float_as_uint(src[32 * h2 + u]);
+                        tmem_st32(slotq + 32 * h2, r32);
+                    }
+                    tmem_st_wait();
+                }
+                nb_sync(NB_TILE, 128);  // staging read before the next pass overwrites it
             }
             ++nex;
         };
@@ -1098,44 +1116,80 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int r = 16 * a + q + 4 * i, s = 16 * a + jc;
-                    sT[r * kLDA + s] = colv[i];
-                    store_tprime(r, s, colv[i]);
+                    const int r = q + 4 * i;  // row inside the block
+                    sTd[(a * 16 + r) * kLDT + jc] = colv[i];
+                    store_tprime(16 * a + r, 16 * a + jc, colv[i]);
                 }
             }
             nb_sync(NB_INV, 256);
             // Blocks below the diagonal, one column chain per warp (block column
-            // bb, 8-column half nt), on the tensor cores (m16n8k8, tf32). For
-            // a = bb+1..3: X = sum_{k=bb}^{a-1} A_ak T_kb, then T_ab = -T_aa X.
-            // Every operand is either a diagonal block or a block this warp
-            // wrote before, so the chain needs no block-wide barrier.
-            {
-                const int bb = iw >> 1, nt = iw & 1;
+            // bb, 8-column half nt), held in registers: for a = bb+1..3,
+            // X = sum_{k=bb}^{a-1} A_ak T_kb, then T_ab = -T_aa X, on m16n8k8 tf32
+            // MMAs. A product's accumulator fragment becomes the right-hand operand
+            // of the next product by shuffles; A and the diagonal blocks come from
+            // shared memory.
+            const int bb = iw >> 1, nt = iw & 1;
+            if (bb < 3) {
                 const int g = lane >> 2, t = lane & 3;
-                const int s0 = 16 * bb + 8 * nt + 2 * t;
-#pragma unroll 1
-                for (int a = bb + 1; a < 4; ++a) {
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                    for (int kb = bb; kb < a; ++kb)
-                        mm16_ntile(acc, sA + (16 * a) * kLDA + 16 * kb, sT + (16 * kb) * kLDA + 16 * bb, nt, lane);
-                    float* xb = sT + (16 * a) * kLDA + 16 * bb;  // X staged where T_ab goes
+                const int sc = 16 * bb + 8 * nt;  // first column of this warp's half
+                // accumulator (rows g | g+8, columns 2t | 2t+1) -> right operand
+                // fragments of the two 8-row k-steps (rows t | t+4, column g)
+                auto c2b = [&](const float (&c)[4], uint32_t (&bf)[2][2]) {
+                    const int src0 = 4 * t + (g >> 1), src1 = 4 * (t + 4) + (g >> 1);
+                    const bool odd = (g & 1) != 0;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const float e0 = __shfl_sync(0xffffffffu, c[2 * j], src0);
+                        const float o0 = __shfl_sync(0xffffffffu, c[2 * j + 1], src0);
+                        const float e1 = __shfl_sync(0xffffffffu, c[2 * j], src1);
+                        const float o1 = __shfl_sync(0xffffffffu, c[2 * j + 1], src1);
+                        bf[j][0] = to_tf32(odd ? o0 : e0);
+                        bf[j][1] = to_tf32(odd ? o1 : e1);
+                    }
+                };
+                uint32_t tb[3][2][2];  // right operand fragments of T_kb, k = bb..2
+                {
+                    const float* D = sTd + bb * 16 * kLDT + 8 * nt;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        tb[0][j][0] = to_tf32(D[(8 * j + t) * kLDT + g]);
+                        tb[0][j][1] = to_tf32(D[(8 * j + t + 4) * kLDT + g]);
+                    }
+                }
+#pragma unroll
+                for (int a = 1; a < 4; ++a) {
+                    if (a <= bb) continue;
+                    float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) {
+                        if (k < bb || k >= a) continue;
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const float* Ar = sA + (16 * a) * kLDA + 16 * k + 8 * j;
+                            const uint32_t af[4] = {to_tf32(Ar[g * kLDA + t]), to_tf32(Ar[(g + 8) * kLDA + t]),
+                                                    to_tf32(Ar[g * kLDA + t + 4]), to_tf32(Ar[(g + 8) * kLDA + t + 4])};
+                            mma_tf32_16x8x8(x, af, tb[k - bb][j]);
+                        }
+                    }
+                    uint32_t xb[2][2];
+                    c2b(x, xb);
+                    float y[4] = {0.f, 0.f, 0.f, 0.f};
+                    const float* D = sTd + a * 16 * kLDT;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const uint32_t af[4] = {to_tf32(D[g * kLDT + 8 * j + t]), to_tf32(D[(g + 8) * kLDT + 8 * j + t]),
+                                                to_tf32(D[g * kLDT + 8 * j + t + 4]),
+                                                to_tf32(D[(g + 8) * kLDT + 8 * j + t + 4])};
+                        mma_tf32_16x8x8(y, af, xb[j]);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) y[e] = -y[e];
+                    const int s0 = sc + 2 * t;
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh)
-                        *reinterpret_cast<float2*>(xb + (g + 8 * hh) * kLDA + 8 * nt + 2 * t) =
-                            make_float2(acc[2 * hh], acc[2 * hh + 1]);
-                    __syncwarp();
-                    float tx[4] = {0.f, 0.f, 0.f, 0.f};
-                    mm16_ntile(tx, sT + (16 * a) * kLDA + 16 * a, xb, nt, lane);
-                    __syncwarp();  // X read before T_ab overwrites it
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int r = 16 * a + g + 8 * hh;
-                        const float v0 = -tx[2 * hh], v1 = -tx[2 * hh + 1];
-                        *reinterpret_cast<float2*>(sT + r * kLDA + s0) = make_float2(v0, v1);
-                        *reinterpret_cast<uint32_t*>(sm + L::TP + km_off(r, s0)) =
-                            pack_bf16x2(v0 * sBeta[s0], v1 * sBeta[s0 + 1]);
-                    }
-                    __syncwarp();
+                        *reinterpret_cast<uint32_t*>(sm + L::TP + km_off(16 * a + g + 8 * hh, s0)) =
+                            pack_bf16x2(y[2 * hh] * sBeta[s0], y[2 * hh + 1] * sBeta[s0 + 1]);
+                    if (a < 3) c2b(y, tb[a - bb]);
                 }
             }
         };
@@ -1303,19 +1357,20 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [B, T, H, 128] bf16 viewed as a 4-D tensor (channel, head, token, batch);
-// box = 64 channels x 1 head x 64 tokens x 1 batch, 128-byte swizzle. Tokens
-// past T read as zero.
-bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
+// [B, T, H, 128] bf16 viewed as a 4-D tensor (channel, head, token, batch).
+// Loads: box = 64 channels x 1 head x 64 tokens x 1 batch, 128-byte swizzle;
+// tokens past T read as zero. Output stores (out = true): box = 32 channels
+// x 1 x 32 tokens x 1, 64-byte swizzle; tokens past T are not written.
+bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, bool out = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)T * H * kD * 2};
-    const cuuint32_t box[4] = {64, 1, 64, 1};
+    const cuuint32_t box_in[4] = {64, 1, 64, 1}, box_out[4] = {32, 1, 32, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, out ? box_out : box_in,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, out ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Chains the entry states of the segments: S_in[j+1] = M_j S_in[j] + C_j for
@@ -1360,10 +1415,11 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(const float* __restri
 template <int DVT, int ERASE, int GATE>
 cudaError_t launch_dvt(const ChunkArgs& a, cudaStream_t stream, const SegJobs& sj, long units) {
     using L = Layout<DVT>;
-    CUtensorMap mk, mq, mg, mv;
+    CUtensorMap mk, mq, mg, mv, mo;
     const int mb = a.cu_seqlens ? 1 : a.B;  // packed sequences: one [1, T] token range
     if (!make_map(&mk, a.k, mb, a.T, a.H) || !make_map(&mq, a.q, mb, a.T, a.H) ||
-        (a.gate == 0 && !make_map(&mg, a.log_alpha, mb, a.T, a.H)) || !make_map(&mv, a.v, mb, a.T, a.H))
+        (a.gate == 0 && !make_map(&mg, a.log_alpha, mb, a.T, a.H)) || !make_map(&mv, a.v, mb, a.T, a.H) ||
+        !make_map(&mo, a.o, mb, a.T, a.H, true))
         return cudaErrorInvalidValue;
     if (a.gate != 0) mg = mk;  // no log_alpha tile is loaded; any valid map fills the parameter
     auto kern = kda_chunk_tc_kernel<DVT, ERASE, GATE>;
@@ -1371,7 +1427,7 @@ cudaError_t launch_dvt(const ChunkArgs& a, cudaStream_t stream, const SegJobs& s
     if (err != cudaSuccess) return err;
     unsigned* status = static_cast<unsigned*>(a.workspace);
     const unsigned grid = (unsigned)(units * (kD / DVT));
-    kern<<<grid, kThreads, L::SMEM_BYTES, stream>>>(mk, mq, mg, mv, (const __nv_bfloat16*)a.beta, a.S0,
+    kern<<<grid, kThreads, L::SMEM_BYTES, stream>>>(mk, mq, mg, mv, mo, (const __nv_bfloat16*)a.beta, a.S0,
                                                     (__nv_bfloat16*)a.o, a.ST, a.T, a.H, status,
                                                     GATE == 1 ? (const __nv_bfloat16*)a.log_alpha : nullptr,
                                                     a.cu_seqlens, sj);
