@@ -135,7 +135,7 @@ KERNEL_SOURCES = {
     "tc": ["kda_chunk_tc.cu", "kda_common.cuh", "kda_sm100.cuh"],
     "bwd": ["kda_chunk_bwd.cu", "kda_common.cuh"],
 }
-WIDENED = ("varlen", "variants", "long_context", "backward")
+WIDENED = ("varlen", "variants", "b2_h16_t4k", "exact_path", "long_context", "backward")
 
 
 def kernel_source_digest(kind: str) -> str:
@@ -495,6 +495,10 @@ def time_widened(args, ctx, kda, I, pf, peaks):
         out["varlen"] = _time_varlen(args, ctx, kda, I, steps, hbm)
     if "variants" in args.parts:
         out["variants"] = _time_variants(args, ctx, kda, pf, steps, hbm)
+    if "b2_h16_t4k" in args.parts:
+        out["b2_h16_t4k"] = _time_b2_h16(ctx, kda, I, hbm)
+    if "exact_path" in args.parts:
+        out["exact_path"] = _time_exact_path(args, ctx, kda, pf, steps, hbm)
     if "long_context" in args.parts:
         out["long_context"] = _time_long_context(ctx, kda, I, hbm)
     if "backward" in args.parts:
@@ -548,6 +552,59 @@ def _time_variants(args, ctx, kda, pf, steps, hbm):
         res[name] = {"erase": erase, "gate": gate, "value": ctx.world * ntok / (ms * 1e-3), "unit": "tokens/s",
                      "ms_per_step": ms, "roofline_frac": gbs / hbm, "achieved_gbs": gbs}
     return {"workload": cfg.name, "steps": steps, **res}
+
+
+def _time_b2_h16(ctx, kda, I, hbm):
+    """B2 H16 T4096 (few heads: 32 (batch, head) units on the GPU): AUTO, the
+    one-pass tensor-core kernel and the segment scan, with the algorithm AUTO
+    picked (it adds the scan when the workspace it asks for holds segment
+    maps)."""
+    torch = ctx.torch
+    cfg = I.B2_H16_T4K.replace(seed=I.B2_H16_T4K.seed + 1000 * ctx.rank)
+    x = {k: (None if v is None else v.to(ctx.dev)) for k, v in I.prefill_inputs(cfg).items()}
+    o = torch.empty(cfg.B, cfg.T, cfg.H, cfg.dv, dtype=torch.bfloat16, device=ctx.dev)
+    S = torch.empty(cfg.B, cfg.H, cfg.dk, cfg.dv, dtype=torch.float32, device=ctx.dev)
+    ntok = cfg.B * cfg.T
+    nbytes = BYTES_PER_TOKEN_HEAD * ntok * cfg.H + 2 * S.numel() * 4  # S0 read, S_T written
+    res = {"workload": cfg.name, "units": cfg.B * cfg.H}
+    for algo in ("auto", "tc", "tc_scan"):
+        wsb = kda.workspace_size(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.C, "bf16", algo)
+        ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=ctx.dev)
+
+        def run_b():
+            kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], chunk=cfg.C, algo=algo, o=o,
+                          S_T=S, workspace=ws, stream=ctx.stream)
+        ms = _time_calls(ctx, run_b, 5, 20)
+        if kda.workspace_status(ws, ctx.stream) != 0:
+            raise RuntimeError("device-side timeout reported by the prefill kernel")
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[algo] = {"value": ctx.world * ntok / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": 20,
+                     "roofline_frac": gbs / hbm, "achieved_gbs": gbs, "workspace_bytes": wsb}
+    res["auto_picked"] = "tc_scan" if res["auto"]["workspace_bytes"] > 256 else "tc"
+    del x, o, S
+    return res
+
+
+def _time_exact_path(args, ctx, kda, pf, steps, hbm):
+    """The B4 H32 T8192 shapes with a decay of -U(1.5, 3) per token and channel:
+    every full chunk then fails the overflow vote of the reference-point
+    factorisation and takes the exact per-pair path."""
+    torch = ctx.torch
+    x, cfg = pf.x, pf.cfg
+    g = torch.Generator(device=ctx.dev)
+    g.manual_seed(cfg.seed + 555 + 1000 * ctx.rank)
+    la = (-(1.5 + 1.5 * torch.rand(cfg.B, cfg.T, cfg.H, cfg.dk, device=ctx.dev, generator=g))).bfloat16()
+
+    def run_e():
+        kda.chunk_fwd(x["q"], x["k"], x["v"], la, x["beta"], x["S0"], chunk=cfg.C, algo=pf.algo, o=pf.o,
+                      S_T=pf.ST, workspace=pf.ws if pf.ws_bytes else None, stream=ctx.stream)
+    ms = _time_calls(ctx, run_e, 3, 3)
+    ntok = cfg.B * cfg.T
+    nbytes = BYTES_PER_TOKEN_HEAD * ntok * cfg.H + pf.ST.numel() * 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del la
+    return {"workload": cfg.name + "_decay_U1.5_3", "value": ctx.world * ntok / (ms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": 3, "roofline_frac": gbs / hbm, "achieved_gbs": gbs}
 
 
 def _time_long_context(ctx, kda, I, hbm):
@@ -627,7 +684,7 @@ def main():
     ap.add_argument("--profile-T", type=int, default=None,
                     help="shorter sequence for profiler captures (the printed line is then not a bench value)")
     ap.add_argument("--parts", default="prefill,e2e,decode,widened",
-                    help="comma list of prefill, e2e, decode, widened (= varlen, variants, long_context, "
+                    help="comma list of prefill, e2e, decode, widened (= varlen, variants, b2_h16_t4k, exact_path, long_context, "
                          "backward) (profiling runs select one)")
     args = ap.parse_args()
     args.parts = set(args.parts.split(","))

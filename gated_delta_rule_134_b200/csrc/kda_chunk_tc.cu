@@ -84,7 +84,9 @@ constexpr int kThreads = 512;
 // named barriers (0 is __syncthreads)
 constexpr int NB_TILE = 1;  // tile warps
 constexpr int NB_TOR = 2;   // tile warps, OR-vote
-constexpr int NB_INV = 3;   // inverse warps
+constexpr int NB_INVA = 3;  // inverse warps
+constexpr int NB_INVA2 = 8; // inverse warps 0-1 (A readout)
+constexpr int NB_INVB = 9;  // U/W warps
 constexpr int NB_CHLO = 4;  // chain warps 0-1
 constexpr int NB_CHB = 5;   // chain warps 2-3 -> warp 0: second half of the state operand stored
 constexpr int NB_CHHI = 6;  // chain warps 2-3
@@ -110,7 +112,8 @@ struct Layout {
     static constexpr uint32_t SP = TP + 16384;  // P, K-major 64 x 64 bf16 (rows 64-127 of [Y; P], Y = TP rows 64-127)
     static constexpr uint32_t SOP = SP + 8192;  // S half (64 channels) x DVT, bf16 MN-major, then delta
     static constexpr uint32_t OST = SOP + 64 * DVT * 2;  // 2 x [32 tok][32 ch] bf16 (64-byte swizzle): O stores
-    static constexpr uint32_t SCR = OST + 4096;          // A fp32 [64][kLDA], T diagonal blocks [4][16][kLDT]
+    static constexpr uint32_t TPS = OST + 4096;          // T' staging, K-major 64 x 64 bf16
+    static constexpr uint32_t SCR = TPS + 8192;          // A fp32 [64][kLDA], T diagonal blocks [4][16][kLDT]
     static constexpr uint32_t SA = SCR;                  //   (exact path: 16 KB staging)
     static constexpr uint32_t STD = SCR + 64 * kLDA * 4;
     static constexpr uint32_t SCR_BYTES = 64 * kLDA * 4 + 4 * 16 * kLDT * 4;
@@ -119,15 +122,14 @@ struct Layout {
     static constexpr uint32_t SOPS = SBETA + 256;   // 4 x 128 f32: operand scale per channel (by chunk mod 4)
     static constexpr uint32_t STMS = SOPS + 2048;   // 4 x 128 f32: tensor-memory scale per channel
     static constexpr uint32_t SEK = STMS + 2048;    // 128 f32: e^{G_last - G_m} of the last prepared chunk
-    static constexpr uint32_t SGM = SEK + 512;      // 128 f32: G_m of the tile warps' chunk
-    static constexpr uint32_t SGL = SGM + 512;      // 128 f32: G_last
-    static constexpr uint32_t SGML = SGL + 512;     // 128 f32: -G_m log2(e)
-    static constexpr uint32_t BARS = SGML + 512;    // mbarriers
+    static constexpr uint32_t SGL = SEK + 512;      // 128 f32: G_last of the tile warps' chunk
+    static constexpr uint32_t BARS = SGL + 512;     // mbarriers
     static constexpr uint32_t MISC = BARS + 512;    // tmem base, abort flag
     static constexpr uint32_t END = MISC + 64;
     static constexpr uint32_t SMEM_BYTES = END + 1024;   // + alignment slack
     static constexpr uint32_t SBO_V = 1024 * (DVT / 64); // K-group stride of the S / delta operands
-    static_assert(SOP % 1024 == 0 && TP % 1024 == 0 && LMAT % 1024 == 0 && OST % 1024 == 0, "operand alignment");
+    static_assert(SOP % 1024 == 0 && TP % 1024 == 0 && LMAT % 1024 == 0 && OST % 1024 == 0 && TPS % 1024 == 0,
+                  "operand alignment");
     static_assert(64 * 64 * 4 <= SCR_BYTES, "exact-path staging overflows the scratch");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     // tensor memory columns: R (fp32, lane = key channel) and three chunk slots
@@ -155,7 +157,9 @@ enum : int {
     B_SCRF = 31,  // A/T scratch of the inverse warps' chunk free
     B_EXKQ = 32,  // k/q reloaded for an exact chunk
     B_FIN = 33,   // 3: final drain of each MMA-issuing thread
-    NUM_BARS = 36
+    B_TPR = 36,   // T' of the chunk staged by the inverse warps
+    B_TPSF = 37,  // staging tile copied into [T'; PT] by the U/W warps
+    NUM_BARS = 38
 };
 
 // offset of element (row R, channel c) of a row-operand buffer (K-major, two
@@ -309,9 +313,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     float* sOpS = reinterpret_cast<float*>(sm + L::SOPS);
     float* sTmS = reinterpret_cast<float*>(sm + L::STMS);
     float* sEK = reinterpret_cast<float*>(sm + L::SEK);
-    float* sGm = reinterpret_cast<float*>(sm + L::SGM);
     float* sGl = reinterpret_cast<float*>(sm + L::SGL);
-    float* sGmL = reinterpret_cast<float*>(sm + L::SGML);
     float* sA = reinterpret_cast<float*>(sm + L::SA);
     float* sTd = reinterpret_cast<float*>(sm + L::STD);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BARS);
@@ -333,8 +335,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         tmem_alloc(s_tmem, L::TMEM_COLS);
         tmem_relinquish();
     }
-    {   // constants: [L; L] (row R: ones in columns 0..R%64) and the T' half of
-        // [T'; PT], whose blocks above the diagonal are never written again
+    {   // constants: [L; L] (row R: ones in columns 0..R%64) and the T' staging
+        // tile, whose blocks above the diagonal are never written again
         for (int i = tid; i < 128 * 8; i += kThreads) {
             const int R = i >> 3, j = i & 7, r = R & 63;
             uint32_t w[4];
@@ -344,7 +346,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 w[u] = pack_bf16x2(s <= r ? 1.f : 0.f, s + 1 <= r ? 1.f : 0.f);
             }
             st_shared_v4(sb + L::LMAT + R * 128 + ((j ^ (R & 7)) << 4), w[0], w[1], w[2], w[3]);
-            if (R < 64) st_shared_v4(sb + L::TP + R * 128 + (j << 4), 0u, 0u, 0u, 0u);
+            if (R < 64) st_shared_v4(sb + L::TPS + R * 128 + (j << 4), 0u, 0u, 0u, 0u);
         }
         for (int c = tid; c < kD; c += kThreads) sEK[c] = 1.f;
         if (v_zero)  // transition run: v = 0 stays in the v tile, which is never loaded
@@ -475,7 +477,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         // lane row = 32 * quad + lane: a key channel of the state, a token row of the slot
         const int row = 32 * quad + lane;
         const bool issuer = warp == 0 && lane == 0;
-        int n_kq[2] = {0, 0}, n_g[3] = {0, 0, 0};  // loads issued per barrier (issuer)
         {   // initial state into TMEM (fp32, lane = key channel)
 #pragma unroll 1
             for (int gq = 0; gq < DVT / 32; ++gq) {
@@ -503,21 +504,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (NC > 0) {
             if (issuer) {
                 load_kq(0, B_KQ);
-                ++n_kq[0];
-                if (NC > 1) {
-                    load_kq(1, B_KQ + 1);
-                    ++n_kq[1];
-                }
+                if (NC > 1) load_kq(1, B_KQ + 1);
                 pf_kq(2);
                 if (GATE == 0) {
-                    for (int j = 0; j < 3 && j < NC; ++j) {
-                        load_g(j);
-                        ++n_g[j];
-                    }
+                    for (int j = 0; j < 3 && j < NC; ++j) load_g(j);
                     pf_g(3);
                 }
             }
-            if (GATE == 1 && warp == 0) {
+            if (GATE == 1 && warp == 3) {
                 for (int j = 0; j < 3 && j < NC; ++j) gate_row_store(j, gate_row_load(j));
                 gnext = gate_row_load(3);
             }
@@ -528,11 +522,26 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             uint32_t v[32];
             tmem_ld32(lane_addr + L::S_COL + 32 * gq, v);
             tmem_ld_wait(v);
+            if (os == ts) {  // (every factored chunk) the operand is the rescaled state itself
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
-                pk[u] = pack_bf16x2(__uint_as_float(v[2 * u]) * os, __uint_as_float(v[2 * u + 1]) * os);
+                for (int u = 0; u < 16; ++u) {
+                    float x0, x1;
+                    mul_f32x2(x0, x1, __uint_as_float(v[2 * u]), __uint_as_float(v[2 * u + 1]), ts, ts);
+                    v[2 * u] = __float_as_uint(x0);
+                    v[2 * u + 1] = __float_as_uint(x1);
+                    pk[u] = pack_bf16x2(x0, x1);
+                }
+            } else {
 #pragma unroll
-            for (int u = 0; u < 32; ++u) v[u] = __float_as_uint(__uint_as_float(v[u]) * ts);
+                for (int u = 0; u < 16; ++u) {
+                    float x0, x1, y0, y1;
+                    mul_f32x2(x0, x1, __uint_as_float(v[2 * u]), __uint_as_float(v[2 * u + 1]), os, os);
+                    mul_f32x2(y0, y1, __uint_as_float(v[2 * u]), __uint_as_float(v[2 * u + 1]), ts, ts);
+                    pk[u] = pack_bf16x2(x0, x1);
+                    v[2 * u] = __float_as_uint(y0);
+                    v[2 * u + 1] = __float_as_uint(y1);
+                }
+            }
             tmem_st32(lane_addr + L::S_COL + 32 * gq, v);
         };
         // operand words of one 32-column group of channel row i -> the S/delta operand
@@ -550,13 +559,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const uint32_t slot = lane_addr + L::SLOT0 + 128 * s;
             if (n > 0) {
                 waitw(B_M2, (uint32_t)(n - 1));  // state update of the previous chunk done
-                if (n + 2 < NC) {  // its log_alpha/KF buffer is free: the gate tile of chunk n+2
-                    if (GATE == 0 && issuer) {
+                if (n + 2 < NC) {  // its log_alpha/KF buffer is free: the gate tile of chunk n+2 (warp 3)
+                    if (GATE == 0 && warp == 3 && lane == 0) {
                         load_g(n + 2);
-                        ++n_g[(n + 2) % 3];
                         pf_g(n + 3);
                     }
-                    if (GATE == 1 && warp == 0) {
+                    if (GATE == 1 && warp == 3) {
                         gate_row_store(n + 2, gnext);
                         gnext = gate_row_load(n + 3);
                     }
@@ -599,11 +607,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     __syncwarp();
                 }
                 waitw(B_M1, (uint32_t)n);
-                if (issuer && n + 2 < NC) {  // the row buffer of this parity is free
-                    load_kq(n + 2, B_KQ + rb);
-                    ++n_kq[rb];
-                    pf_kq(n + 3);
-                }
                 {   // delta (slot rows 0-63) -> bf16 operand over the state operand
 #pragma unroll 1
                     for (int gq = 0; gq < DVT / 32; ++gq) {
@@ -631,17 +634,30 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
                 __syncwarp();
             } else {
-                uint32_t pk[DVT / 32][16];  // key channels 64-127, staged until the operand buffer is free
+                // key channels 64-127: the first half of the columns staged in registers
+                // until the operand buffer is free, the rest converted after
+                constexpr int kStaged = DVT / 64;
+                uint32_t pk[kStaged][16];
 #pragma unroll
-                for (int gq = 0; gq < DVT / 32; ++gq) s1_group(gq, os, ts, pk[gq]);
-                tmem_st_wait();
+                for (int gq = 0; gq < kStaged; ++gq) s1_group(gq, os, ts, pk[gq]);
                 waitw(B_M1A, (uint32_t)n);  // first half of the state operand consumed
 #pragma unroll
-                for (int gq = 0; gq < DVT / 32; ++gq) sop_store(row - 64, gq, pk[gq]);
+                for (int gq = 0; gq < kStaged; ++gq) sop_store(row - 64, gq, pk[gq]);
+#pragma unroll 1
+                for (int gq = kStaged; gq < DVT / 32; ++gq) {
+                    uint32_t pq[16];
+                    s1_group(gq, os, ts, pq);
+                    sop_store(row - 64, gq, pq);
+                }
+                tmem_st_wait();
                 fence_proxy_async_smem();
                 tc_fence_before();
                 nb_arrive(NB_CHB, 96);
                 waitw(B_M1, (uint32_t)n);
+                if (warp == 2 && lane == 0 && n + 2 < NC) {  // the row buffer of this parity is free
+                    load_kq(n + 2, B_KQ + rb);
+                    pf_kq(n + 3);
+                }
                 {   // O (slot rows 64-127) -> global bf16: a full chunk through a swizzled
                     // [32 tok][32 ch] stage and a tensor store per 32 columns (coalesced,
                     // asynchronous); a partial chunk by plain stores (rows past a packed
@@ -710,9 +726,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
         }
         if (quad >= 2 && lane == 0) bulk_wait0();  // every tensor store of O complete
-        if (issuer) {
-            for (int x = 0; x < 2; ++x) drain(B_KQ + x, n_kq[x]);
-            for (int x = 0; x < 3; ++x) drain(B_G + x, n_g[x]);
+        if (issuer) {  // (chunk m's k/q load arms B_KQ + m % 2, its log_alpha load B_G + m % 3)
+            for (int x = 0; x < 2; ++x) drain(B_KQ + x, (NC - x + 1) / 2);
+            if (GATE == 0)
+                for (int x = 0; x < 3; ++x) drain(B_G + x, (NC - x + 2) / 3);
             if (*s_abort) {
                 mma_commit(bars + B_FIN);
                 mbar_wait_bounded(bars + B_FIN, 0u, kDrainBudget);
@@ -883,54 +900,27 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             // it are zero (past the tensor) or the next packed sequence's.
             const int lim = min(seq_len - m * kC, kC);
             const bool live = tok < lim;
-            const int tm_tok = min(31, lim - 1), tl_tok = lim - 1;  // reference, last token
-            uint32_t g1 = 0;  // per-token gate: this token's prefix sum
-            if (GATE == 0) {  // G_m, G_last of this thread's channels (every lane loads, the owners store)
-#pragma unroll 1
-                for (int u8 = 0; u8 < 8; ++u8) {
-                    uint32_t g8[8];
-                    tmem_ld8(slotq + ch0 + 8 * u8, g8);
-                    tmem_ld_wait(g8);
-                    const int c0 = ch0 + 8 * u8;
-                    if (tok == tm_tok) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            sGm[c0 + e] = __uint_as_float(g8[e]);
-                            sGmL[c0 + e] = -__uint_as_float(g8[e]) * kLog2e;
-                        }
-                    }
-                    if (tok == tl_tok) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) sGl[c0 + e] = __uint_as_float(g8[e]);
-                    }
-                    __syncwarp();
-                }
-            } else if (GATE == 1) {
-                tmem_ld1(slotq, g1);
-                tmem_ld_wait1(g1);
-                if (tok == tm_tok) {
-                    sGm[0] = __uint_as_float(g1);
-                    sGmL[0] = -__uint_as_float(g1) * kLog2e;
-                }
-                if (tok == tl_tok) sGl[0] = __uint_as_float(g1);
-            }
-            nb_sync(NB_TILE, 128);
+            const int tl_tok = lim - 1;  // last token: publishes G_last for the scales
             // operand tiles, in place: 8 groups of 8 channels of this thread's row;
-            // amax tracks the largest |exponent| (and |G_m|) for the vote
+            // amax tracks the largest |exponent| for the vote
             float amax = 0.f;
             {
                 const uint32_t rop = sb + L::ROW + rb * 32768;
                 const uint32_t colp = sb + L::COL + cb * 16384;
                 uint32_t ep1 = 0, fp1 = 0;
-                if (GATE == 1) {
-                    const float nl = sGmL[0];
-                    const float a = fmaf(__uint_as_float(g1), kLog2e, nl);
-                    amax = fmaxf(fabsf(a), fabsf(nl));
+                if (GATE == 1) {  // per-token gate: one factor pair per token
+                    uint32_t g1;
+                    tmem_ld1(slotq, g1);
+                    tmem_ld_wait1(g1);
+                    if (tok == tl_tok) sGl[0] = __uint_as_float(g1);
+                    const float a = __uint_as_float(g1) * kLog2e;
+                    amax = fabsf(a);
                     const float e = ex2(a), f = ex2(-a);
                     ep1 = pack_bf16x2(e, e);
                     fp1 = pack_bf16x2(f, f);
                 }
                 const uint32_t km = live ? 0xFFFFFFFFu : 0u;  // rows past the sequence: k = q = 0
+                const bool masked = !__all_sync(0xffffffffu, live);
 #pragma unroll 1
                 for (int u8 = 0; u8 < 8; ++u8) {
                     const int c0 = ch0 + 8 * u8;
@@ -952,31 +942,42 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     if (GATE == 0) {
                         uint32_t g8[8];
                         tmem_ld8(slotq + c0, g8);
-                        const float4 na = *reinterpret_cast<const float4*>(sGmL + c0);
-                        const float4 nb = *reinterpret_cast<const float4*>(sGmL + c0 + 4);
-                        const float nl8[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
                         tmem_ld_wait(g8);
+                        if (tok == tl_tok) {
+                            *reinterpret_cast<float4*>(sGl + c0) = make_float4(
+                                __uint_as_float(g8[0]), __uint_as_float(g8[1]), __uint_as_float(g8[2]), __uint_as_float(g8[3]));
+                            *reinterpret_cast<float4*>(sGl + c0 + 4) = make_float4(
+                                __uint_as_float(g8[4]), __uint_as_float(g8[5]), __uint_as_float(g8[6]), __uint_as_float(g8[7]));
+                        }
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            // E = 2^{(G - G_m) log2 e}, F = 1/E
-                            const float a0 = fmaf(__uint_as_float(g8[2 * u]), kLog2e, nl8[2 * u]);
-                            const float a1 = fmaf(__uint_as_float(g8[2 * u + 1]), kLog2e, nl8[2 * u + 1]);
-                            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(a0), fabsf(a1)), fmaxf(fabsf(nl8[2 * u]), fabsf(nl8[2 * u + 1]))));
+                            // E = e^G = 2^{G log2 e}, F = 1/E
+                            float a0, a1;
+                            mul_f32x2(a0, a1, __uint_as_float(g8[2 * u]), __uint_as_float(g8[2 * u + 1]), kLog2e, kLog2e);
+                            amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
                             // packed bf16 products: the factor pairs are rounded to bf16
                             // first, the products once more (both well inside the bf16
                             // rounding of the MMA operands)
                             const uint32_t ep = pack_bf16x2(ex2(a0), ex2(a1));
                             const uint32_t fp = pack_bf16x2(ex2(-a0), ex2(-a1));
-                            ke[u] = hmul2_bf16(kw[u], ep) & km;
-                            qe[u] = hmul2_bf16(qw[u], ep) & km;
-                            kf[u] = hmul2_bf16(kw[u], fp) & km;
+                            ke[u] = hmul2_bf16(kw[u], ep);
+                            qe[u] = hmul2_bf16(qw[u], ep);
+                            kf[u] = hmul2_bf16(kw[u], fp);
                         }
                     } else {
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            ke[u] = hmul2_bf16(kw[u], ep1) & km;
-                            qe[u] = hmul2_bf16(qw[u], ep1) & km;
-                            kf[u] = hmul2_bf16(kw[u], fp1) & km;
+                            ke[u] = hmul2_bf16(kw[u], ep1);
+                            qe[u] = hmul2_bf16(qw[u], ep1);
+                            kf[u] = hmul2_bf16(kw[u], fp1);
+                        }
+                    }
+                    if (masked) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            ke[u] &= km;
+                            qe[u] &= km;
+                            kf[u] &= km;
                         }
                     }
                     st_shared_v4(rop + ko, ke[0], ke[1], ke[2], ke[3]);
@@ -984,22 +985,22 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     st_shared_v4(colp + fo, kf[0], kf[1], kf[2], kf[3]);
                 }
             }
-            // every factor finite and normal? (NaN counts as a failure)
+            // every factor finite and normal? (NaN counts as a failure); the vote also
+            // makes G_last visible to every tile thread
             const bool exact = GATE != 2 && nb_or(NB_TOR, 128, live && !(amax <= kGuardL));
             if (exact) exact_chunk(m, s, rb, cb, lim);
-            {   // per-channel scales of this chunk
+            {   // per-channel scales of this chunk. The tensor memory holds R with
+                // S = Diag(ek) R; the chain feeds S^ = Diag(os) R to MMA1 and keeps
+                // Diag(ts) R + KF^T delta, whose true state is Diag(ek_new) times it.
                 const int c = ttid;
-                const float g_m = GATE == 0 ? sGm[c] : (GATE == 1 ? sGm[0] : 0.f);
                 const float g_l = GATE == 0 ? sGl[c] : (GATE == 1 ? sGl[0] : 0.f);
                 const float ek_prev = sEK[c];
                 const int slot4 = m & 3;
-                if (!exact) {
-                    const float sc = __expf(g_m) * ek_prev;
-                    sOpS[slot4 * 128 + c] = sc;
-                    sTmS[slot4 * 128 + c] = sc;
-                    sEK[c] = __expf(g_l - g_m);
-                } else {
-                    sOpS[slot4 * 128 + c] = ek_prev;
+                sOpS[slot4 * 128 + c] = ek_prev;
+                if (!exact) {  // reference at the chunk start: S^ = S, KF = k e^{-G}
+                    sTmS[slot4 * 128 + c] = ek_prev;
+                    sEK[c] = __expf(g_l);
+                } else {       // KF = k e^{G_last - G}
                     sTmS[slot4 * 128 + c] = __expf(g_l) * ek_prev;
                     sEK[c] = 1.f;
                 }
@@ -1034,104 +1035,112 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 mbar_wait_bounded(bars + B_FIN + 1, 0u, kDrainBudget);
             }
         }
-    } else {
+    } else if (warp < kInvWarp0 + 4) {
         // ============================================================ inverse warps
-        // Per chunk m: A/P readout, (I + A)^{-1} -> T', then the PT, W and U MMAs
-        // with the readouts between them (PT -> [T'; PT], [W'; P W'] -> row operand).
-        const int iw = warp - kInvWarp0;  // 0..7
-        const int hf = iw >> 2;           // which 32-column half of a readout this warp takes
-        const int itid = tid - 32 * kInvWarp0;
-        int n_v = 0;
+        // Per chunk m: A readout, (I + A)^{-1} -> T' into the staging tile (the
+        // U/W warps copy it into [T'; PT] once that is free).
+        const int itid = tid - 32 * kInvWarp0;  // 0..127
+        const int iw = warp - kInvWarp0;        // 0..3
         auto load_beta = [&](int m) -> float {
             const int t = m * kC + itid;
             return (itid < kC && m < NC && t < seq_len) ? __bfloat162float(beta[(tok0 + t) * H + h]) : 0.f;
         };
-        // ---- A (slot rows 0-63) -> fp32 scratch (beta_r, strictly lower); P (rows 64-127) -> bf16 K-major tile (lower incl.)
-        auto p4 = [&](uint32_t slot) {
-            if (quad < 2 && !erase) return;  // additive write: A is not used
-            uint32_t v[32];
-            tmem_ld32(slot + 32 * hf, v);
-            tmem_ld_wait(v);
-            if (quad < 2) {
+        // T' (bf16) entry into the staging tile (K-major 64 x 64, 128-byte swizzle)
+        auto store_tprime = [&](int r, int s, float t) {
+            *reinterpret_cast<__nv_bfloat16*>(sm + L::TPS + km_off(r, s)) = __float2bfloat16_rn(t * sBeta[s]);
+        };
+        float beta_next = load_beta(0);
+        for (int m = 0; m < NC; ++m) {
+            const int s = m % 3;
+            const uint32_t slot = lane_addr + L::SLOT0 + 128 * s;
+            if (itid < kC) sBeta[itid] = beta_next;
+            beta_next = load_beta(m + 1);
+            waitw(B_AP + s, (uint32_t)(m / 3));
+            if (erase && quad < 2) {  // A (slot rows 0-63) -> fp32 scratch: beta_r, strictly lower
                 const int r = 32 * quad + lane;
-                const float br = sBeta[r];
-                float* dst = sA + r * kLDA + 32 * hf;
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t v[32];
+                    tmem_ld32(slot + 32 * hh, v);
+                    tmem_ld_wait(v);
+                    nb_sync(NB_INVA2, 64);  // (first pass: beta of chunk m visible)
+                    const float br = sBeta[r];
+                    float* dst = sA + r * kLDA + 32 * hh;
 #pragma unroll
-                for (int u = 0; u < 32; u += 4) {
-                    float4 f;
-                    f.x = (32 * hf + u + 0 < r) ? br * __uint_as_float(v[u + 0]) : 0.f;
-                    f.y = (32 * hf + u + 1 < r) ? br * __uint_as_float(v[u + 1]) : 0.f;
-                    f.z = (32 * hf + u + 2 < r) ? br * __uint_as_float(v[u + 2]) : 0.f;
-                    f.w = (32 * hf + u + 3 < r) ? br * __uint_as_float(v[u + 3]) : 0.f;
-                    *reinterpret_cast<float4*>(dst + u) = f;
-                }
-            } else {
-                const int r = 32 * (quad - 2) + lane;
-#pragma unroll
-                for (int jc = 0; jc < 4; ++jc) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int s = 32 * hf + 8 * jc + 2 * u;
-                        const float p0 = (s <= r) ? __uint_as_float(v[8 * jc + 2 * u]) : 0.f;
-                        const float p1 = (s + 1 <= r) ? __uint_as_float(v[8 * jc + 2 * u + 1]) : 0.f;
-                        w[u] = pack_bf16x2(p0, p1);
+                    for (int u = 0; u < 32; u += 4) {
+                        float4 f;
+                        f.x = (32 * hh + u + 0 < r) ? br * __uint_as_float(v[u + 0]) : 0.f;
+                        f.y = (32 * hh + u + 1 < r) ? br * __uint_as_float(v[u + 1]) : 0.f;
+                        f.z = (32 * hh + u + 2 < r) ? br * __uint_as_float(v[u + 2]) : 0.f;
+                        f.w = (32 * hh + u + 3 < r) ? br * __uint_as_float(v[u + 3]) : 0.f;
+                        *reinterpret_cast<float4*>(dst + u) = f;
                     }
-                    st_shared_v4(sb + L::SP + r * 128 + (((4 * hf + jc) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
                 }
             }
-        };
-        // ---- P5: T = (I + A)^{-1} -> T' = T Diag(beta), bf16, rows 0-63 of [T'; PT]
-        auto store_tprime = [&](int r, int s, float t) {
-            *reinterpret_cast<__nv_bfloat16*>(sm + L::TP + km_off(r, s)) = __float2bfloat16_rn(t * sBeta[s]);
-        };
-        auto p5 = [&]() {
-            if (!erase) {  // A = 0: T = I, T' = Diag(beta); thread: row itid/4, 16 columns
-                const int r = itid >> 2, j0c = 2 * (itid & 3);
+            // the staging tile of the previous chunk has been copied out
+            if (m > 0) waitw(B_TPSF, (uint32_t)(m - 1));
+            nb_sync(NB_INVA, 128);  // A and beta of chunk m visible
+            if (!erase) {  // A = 0: T = I, T' = Diag(beta); thread: row itid/2, 32 columns
+                const int r = itid >> 1;
 #pragma unroll
-                for (int jc = 0; jc < 2; ++jc) {
-                    const int j = j0c + jc;  // 8-column chunk
+                for (int jc = 0; jc < 4; ++jc) {
+                    const int j = 4 * (itid & 1) + jc;  // 8-column chunk
                     uint32_t w[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int s0 = 8 * j + 2 * u;
                         w[u] = pack_bf16x2(s0 == r ? sBeta[r] : 0.f, s0 + 1 == r ? sBeta[r] : 0.f);
                     }
-                    st_shared_v4(sb + L::TP + r * 128 + ((j ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                    st_shared_v4(sb + L::TPS + r * 128 + ((j ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
                 }
-                return;
-            }
-            {   // diagonal 16x16 blocks: four threads per column, rows q, q+4, q+8, q+12
-                const int a = itid >> 6, jc = (itid >> 2) & 15, q = itid & 3;
-                const float* Ab = sA + (16 * a) * kLDA + 16 * a;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f}, colv[4] = {0.f, 0.f, 0.f, 0.f};
+            } else {
+                if (itid < 64) {
+                    // diagonal 16x16 blocks, one thread per column c of block a, by
+                    // forward substitution in axpy form: once T_kc is final, every
+                    // later row takes its A_ik T_kc (no exchange between threads)
+                    const int a = itid >> 4, c = itid & 15;
+                    const float* Ab = sA + (16 * a) * kLDA + 16 * a;
+                    // c0..c2: columns k, k+1, k+2 of A_aa (the loads run three steps
+                    // ahead of the substitution, which waits on nothing else)
+                    float acc[16], c0[16], c1[16], c2[16];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const float mine = (r == jc) ? 1.f : ((r > jc) ? -acc[r >> 2] : 0.f);
-                    const float t = __shfl_sync(0xffffffffu, mine, (lane & ~3) | (r & 3));
-                    if (q == (r & 3)) colv[r >> 2] = t;
+                    for (int i = 0; i < 16; ++i) {
+                        acc[i] = 0.f;
+                        c0[i] = i > 0 ? Ab[i * kLDA] : 0.f;
+                        c1[i] = i > 1 ? Ab[i * kLDA + 1] : 0.f;
+                        c2[i] = i > 2 ? Ab[i * kLDA + 2] : 0.f;
+                    }
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        if (q + 4 * i > r) acc[i] = fmaf(Ab[(q + 4 * i) * kLDA + r], t, acc[i]);
+                    for (int k = 0; k < 16; ++k) {
+                        float c3[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) c3[i] = (k + 3 < 16 && i > k + 3) ? Ab[i * kLDA + k + 3] : 0.f;
+                        const float tk = (k < c) ? 0.f : ((k == c) ? 1.f : -acc[k]);
+                        acc[k] = tk;
+#pragma unroll
+                        for (int i = k + 1; i < 16; ++i) acc[i] = fmaf(c0[i], tk, acc[i]);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            c0[i] = c1[i];
+                            c1[i] = c2[i];
+                            c2[i] = c3[i];
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        sTd[(a * 16 + i) * kLDT + c] = acc[i];
+                        store_tprime(16 * a + i, 16 * a + c, acc[i]);
+                    }
                 }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = q + 4 * i;  // row inside the block
-                    sTd[(a * 16 + r) * kLDT + jc] = colv[i];
-                    store_tprime(16 * a + r, 16 * a + jc, colv[i]);
-                }
-            }
-            nb_sync(NB_INV, 256);
-            // Blocks below the diagonal, one column chain per warp (block column
-            // bb, 8-column half nt), held in registers: for a = bb+1..3,
-            // X = sum_{k=bb}^{a-1} A_ak T_kb, then T_ab = -T_aa X, on m16n8k8 tf32
-            // MMAs. A product's accumulator fragment becomes the right-hand operand
-            // of the next product by shuffles; A and the diagonal blocks come from
-            // shared memory.
-            const int bb = iw >> 1, nt = iw & 1;
-            if (bb < 3) {
+                nb_sync(NB_INVA, 128);
+                // Blocks below the diagonal: column chains (block column bb, 8-column
+                // half nt), held in registers: for a = bb+1..3, X = sum_{k=bb}^{a-1}
+                // A_ak T_kb, then T_ab = -T_aa X, on m16n8k8 tf32 MMAs. A product's
+                // accumulator fragment becomes the right-hand operand of the next
+                // product by shuffles; A and the diagonal blocks come from shared
+                // memory. Warps 0-1 take block column 0, warps 2-3 block columns 1 and 2.
+                const int nt = iw & 1;
                 const int g = lane >> 2, t = lane & 3;
-                const int sc = 16 * bb + 8 * nt;  // first column of this warp's half
                 // accumulator (rows g | g+8, columns 2t | 2t+1) -> right operand
                 // fragments of the two 8-row k-steps (rows t | t+4, column g)
                 auto c2b = [&](const float (&c)[4], uint32_t (&bf)[2][2]) {
@@ -1147,144 +1156,126 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         bf[j][1] = to_tf32(odd ? o1 : e1);
                     }
                 };
-                uint32_t tb[3][2][2];  // right operand fragments of T_kb, k = bb..2
-                {
-                    const float* D = sTd + bb * 16 * kLDT + 8 * nt;
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        tb[0][j][0] = to_tf32(D[(8 * j + t) * kLDT + g]);
-                        tb[0][j][1] = to_tf32(D[(8 * j + t + 4) * kLDT + g]);
-                    }
-                }
-#pragma unroll
-                for (int a = 1; a < 4; ++a) {
-                    if (a <= bb) continue;
-                    float x[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int k = 0; k < 3; ++k) {
-                        if (k < bb || k >= a) continue;
+                auto chain = [&](const int bb) {
+                    const int sc = 16 * bb + 8 * nt;  // first column of this warp's half
+                    uint32_t tb[3][2][2];             // right operand fragments of T_kb, k = bb..2
+                    {
+                        const float* D = sTd + bb * 16 * kLDT + 8 * nt;
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
-                            const float* Ar = sA + (16 * a) * kLDA + 16 * k + 8 * j;
-                            const uint32_t af[4] = {to_tf32(Ar[g * kLDA + t]), to_tf32(Ar[(g + 8) * kLDA + t]),
-                                                    to_tf32(Ar[g * kLDA + t + 4]), to_tf32(Ar[(g + 8) * kLDA + t + 4])};
-                            mma_tf32_16x8x8(x, af, tb[k - bb][j]);
+                            tb[0][j][0] = to_tf32(D[(8 * j + t) * kLDT + g]);
+                            tb[0][j][1] = to_tf32(D[(8 * j + t + 4) * kLDT + g]);
                         }
                     }
-                    uint32_t xb[2][2];
-                    c2b(x, xb);
-                    float y[4] = {0.f, 0.f, 0.f, 0.f};
-                    const float* D = sTd + a * 16 * kLDT;
+                    // da = a - bb and dk = k - bb run over compile-time ranges, so the
+                    // fragment array stays in registers
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const uint32_t af[4] = {to_tf32(D[g * kLDT + 8 * j + t]), to_tf32(D[(g + 8) * kLDT + 8 * j + t]),
-                                                to_tf32(D[g * kLDT + 8 * j + t + 4]),
-                                                to_tf32(D[(g + 8) * kLDT + 8 * j + t + 4])};
-                        mma_tf32_16x8x8(y, af, xb[j]);
+                    for (int da = 1; da < 4; ++da) {
+                        const int a = bb + da;
+                        if (a > 3) break;
+                        float x[4] = {0.f, 0.f, 0.f, 0.f}, x2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int dk = 0; dk < da; ++dk) {
+                            const int k = bb + dk;
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                const float* Ar = sA + (16 * a) * kLDA + 16 * k + 8 * j;
+                                const uint32_t af[4] = {to_tf32(Ar[g * kLDA + t]), to_tf32(Ar[(g + 8) * kLDA + t]),
+                                                        to_tf32(Ar[g * kLDA + t + 4]),
+                                                        to_tf32(Ar[(g + 8) * kLDA + t + 4])};
+                                mma_tf32_16x8x8(j == 0 ? x : x2, af, tb[dk][j]);  // two independent accumulators
+                            }
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) x[e] += x2[e];
+                        uint32_t xb[2][2];
+                        c2b(x, xb);
+                        float y[4] = {0.f, 0.f, 0.f, 0.f};
+                        const float* D = sTd + a * 16 * kLDT;
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const uint32_t af[4] = {to_tf32(D[g * kLDT + 8 * j + t]), to_tf32(D[(g + 8) * kLDT + 8 * j + t]),
+                                                    to_tf32(D[g * kLDT + 8 * j + t + 4]),
+                                                    to_tf32(D[(g + 8) * kLDT + 8 * j + t + 4])};
+                            mma_tf32_16x8x8(y, af, xb[j]);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) y[e] = -y[e];
+                        const int s0 = sc + 2 * t;
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh)
+                            *reinterpret_cast<uint32_t*>(sm + L::TPS + km_off(16 * a + g + 8 * hh, s0)) =
+                                pack_bf16x2(y[2 * hh] * sBeta[s0], y[2 * hh + 1] * sBeta[s0 + 1]);
+                        if (da < 3 && a < 3) c2b(y, tb[da]);
                     }
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) y[e] = -y[e];
-                    const int s0 = sc + 2 * t;
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh)
-                        *reinterpret_cast<uint32_t*>(sm + L::TP + km_off(16 * a + g + 8 * hh, s0)) =
-                            pack_bf16x2(y[2 * hh] * sBeta[s0], y[2 * hh + 1] * sBeta[s0 + 1]);
-                    if (a < 3) c2b(y, tb[a - bb]);
+                };
+                if (iw < 2) {
+                    chain(0);
+                } else {
+                    chain(2);
+                    chain(1);
                 }
             }
-        };
-        // ---- PT (slot rows 64-127, columns 64-127) -> bf16 rows 64-127 of [T'; PT]
-        auto p6 = [&](uint32_t slot) {
-            if (quad < 2) return;
-            const int r = 32 * (quad - 2) + lane;
-            uint32_t v[32];
-            tmem_ld32(slot + 64 + 32 * hf, v);
-            tmem_ld_wait(v);
-#pragma unroll
-            for (int jc = 0; jc < 4; ++jc) {
-                uint32_t w[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]), __uint_as_float(v[8 * jc + 2 * u + 1]));
-                const int R = 64 + r;
-                st_shared_v4(sb + L::TP + R * 128 + (((4 * hf + jc) ^ (R & 7)) << 4), w[0], w[1], w[2], w[3]);
+            nb_sync(NB_INVA, 128);
+            if (itid == 0) {
+                mbar_arrive(bars + B_TPR);   // T' of chunk m staged
+                mbar_arrive(bars + B_SCRF);  // A/T scratch free
             }
-        };
-        // ---- P7: [W'; P W'] -> row operand: rows 0-63 -W' over KE, rows 64-127 QE - P W'
-        auto p7 = [&](uint32_t slot, int rb) {
-            const uint32_t rop = sb + L::ROW + rb * 32768;
-            if (quad < 2) {
-                const int r = 32 * quad + lane;
-                if (!erase) {  // additive write: delta = U, the W S term is zero
-#pragma unroll
-                    for (int jc = 0; jc < 8; ++jc)
-                        st_shared_v4(rop + hf * 16384 + r * 128 + ((jc ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
-                    return;
-                }
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t v[32];
-                    tmem_ld32(slot + 64 * hf + 32 * hh, v);
-                    tmem_ld_wait(v);
-#pragma unroll
-                    for (int jc = 0; jc < 4; ++jc) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            w[u] = pack_bf16x2(-__uint_as_float(v[8 * jc + 2 * u]), -__uint_as_float(v[8 * jc + 2 * u + 1]));
-                        st_shared_v4(rop + hf * 16384 + r * 128 + (((4 * hh + jc) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
-                    }
-                }
-            } else {
-                if (!erase) return;  // W = 0: the rows keep QE
-                const int r = 32 * (quad - 2) + lane, R = 64 + r;
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t v[32];
-                    tmem_ld32(slot + 64 * hf + 32 * hh, v);
-                    tmem_ld_wait(v);
-#pragma unroll
-                    for (int jc = 0; jc < 4; ++jc) {
-                        const uint32_t addr = rop + hf * 16384 + R * 128 + (((4 * hh + jc) ^ (R & 7)) << 4);
-                        const uint4 qv = ld_shared_v4(addr);
-                        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-                        uint32_t w[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            w[u] = pack_bf16x2(bf16_lo(qw[u]) - __uint_as_float(v[8 * jc + 2 * u]),
-                                               bf16_hi(qw[u]) - __uint_as_float(v[8 * jc + 2 * u + 1]));
-                        st_shared_v4(addr, w[0], w[1], w[2], w[3]);
-                    }
-                }
-            }
-        };
-        if (NC > 0 && itid == 0) {
+            __syncwarp();
+        }
+    } else {
+        // ============================================================ U/W warps
+        // Per chunk m: P readout, T' into [T'; PT], the PT, W and U MMAs with the
+        // readouts between them (PT -> [T'; PT], [W'; P W'] -> row operand).
+        const int utid = tid - 32 * (kInvWarp0 + 4);  // 0..127
+        int n_v = 0;
+        if (NC > 0 && utid == 0) {
             load_v(0);
             ++n_v;
             pf_v(1);
         }
-        float beta_next = load_beta(0);
         for (int m = 0; m < NC; ++m) {
             const int s = m % 3, rb = m & 1;
             const uint32_t slot = lane_addr + L::SLOT0 + 128 * s;
-            if (itid < kC) sBeta[itid] = beta_next;
-            beta_next = load_beta(m + 1);
             waitw(B_AP + s, (uint32_t)(m / 3));
-            if (m > 0 && itid == 0) {  // [T'; PT] and the v tile of the previous chunk are free
+            if (quad >= 2) {  // P (slot rows 64-127) -> bf16 K-major tile, lower incl.
+                const int r = 32 * (quad - 2) + lane;
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t v[32];
+                    tmem_ld32(slot + 32 * hh, v);
+                    tmem_ld_wait(v);
+#pragma unroll
+                    for (int jc = 0; jc < 4; ++jc) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int s2 = 32 * hh + 8 * jc + 2 * u;
+                            const float p0 = (s2 <= r) ? __uint_as_float(v[8 * jc + 2 * u]) : 0.f;
+                            const float p1 = (s2 + 1 <= r) ? __uint_as_float(v[8 * jc + 2 * u + 1]) : 0.f;
+                            w[u] = pack_bf16x2(p0, p1);
+                        }
+                        st_shared_v4(sb + L::SP + r * 128 + (((4 * hh + jc) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+            if (utid == 0 && m > 0) {  // [T'; PT] and the v tile of the previous chunk are free
                 wait1(B_UO + (m - 1) % 3, (uint32_t)((m - 1) / 3));
                 load_v(m);
                 ++n_v;
                 pf_v(m + 1);
             }
-            nb_sync(NB_INV, 256);  // beta of chunk m visible, [T'; PT] free
-            p4(slot);
-            nb_sync(NB_INV, 256);
-            p5();
+            waitw(B_TPR, (uint32_t)m);  // T' of chunk m staged (its A rows are read: W may overwrite them)
+            nb_sync(NB_INVB, 128);      // [T'; PT] free
+            for (int i = utid; i < 512; i += 128) {  // T' -> rows 0-63 of [T'; PT] (same swizzled layout)
+                const uint4 w = ld_shared_v4(sb + L::TPS + 16 * i);
+                st_shared_v4(sb + L::TP + 16 * i, w.x, w.y, w.z, w.w);
+            }
             fence_proxy_async_smem();
             tc_fence_before();
-            nb_sync(NB_INV, 256);
-            if (itid == 0) {
-                mbar_arrive(bars + B_SCRF);  // A/T scratch free
+            nb_sync(NB_INVB, 128);
+            if (utid == 0) {
+                mbar_arrive(bars + B_TPSF);  // staging tile free
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)  // PT = P T' into columns 64-127 (rows 0-63 take junk)
@@ -1292,12 +1283,28 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 mma_commit(bars + B_PT);
             }
             waitw(B_PT, (uint32_t)m);
-            p6(slot);
+            if (quad >= 2) {  // PT (slot rows 64-127, columns 64-127) -> bf16 rows 64-127 of [T'; PT]
+                const int r = 32 * (quad - 2) + lane, R = 64 + r;
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t v[32];
+                    tmem_ld32(slot + 64 + 32 * hh, v);
+                    tmem_ld_wait(v);
+#pragma unroll
+                    for (int jc = 0; jc < 4; ++jc) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]), __uint_as_float(v[8 * jc + 2 * u + 1]));
+                        st_shared_v4(sb + L::TP + R * 128 + (((4 * hh + jc) ^ (R & 7)) << 4), w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
             fence_proxy_async_smem();
             tc_fence_before();
-            nb_sync(NB_INV, 256);
+            nb_sync(NB_INVB, 128);
             if (erase) {
-                if (itid == 0) {
+                if (utid == 0) {
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // [W'; P W'] = [T'; PT] KE
@@ -1307,11 +1314,55 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
                 waitw(B_WB, (uint32_t)m);
             }
-            p7(slot, rb);
+            {   // [W'; P W'] -> row operand: rows 0-63 -W' over KE, rows 64-127 QE - P W'
+                const uint32_t rop = sb + L::ROW + rb * 32768;
+                if (quad < 2) {
+                    const int r = 32 * quad + lane;
+#pragma unroll 1
+                    for (int hh = 0; hh < 4; ++hh) {
+                        uint32_t v[32];
+                        if (erase) {
+                            tmem_ld32(slot + 32 * hh, v);
+                            tmem_ld_wait(v);
+                        }
+#pragma unroll
+                        for (int jc = 0; jc < 4; ++jc) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)  // additive write: delta = U, the W S term is zero
+                                w[u] = erase ? pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]),
+                                                           __uint_as_float(v[8 * jc + 2 * u + 1])) ^ 0x80008000u
+                                             : 0u;
+                            st_shared_v4(rop + (hh >> 1) * 16384 + r * 128 + (((4 * (hh & 1) + jc) ^ (r & 7)) << 4), w[0],
+                                         w[1], w[2], w[3]);
+                        }
+                    }
+                } else if (erase) {  // (W = 0: the rows keep QE)
+                    const int r = 32 * (quad - 2) + lane, R = 64 + r;
+#pragma unroll 1
+                    for (int hh = 0; hh < 4; ++hh) {
+                        uint32_t v[32];
+                        tmem_ld32(slot + 32 * hh, v);
+                        tmem_ld_wait(v);
+#pragma unroll
+                        for (int jc = 0; jc < 4; ++jc) {
+                            const uint32_t addr = rop + (hh >> 1) * 16384 + R * 128 + (((4 * (hh & 1) + jc) ^ (R & 7)) << 4);
+                            const uint4 qv = ld_shared_v4(addr);
+                            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                            uint32_t w[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)  // QE - P W' on bf16 pairs (P W' rounded to bf16 first)
+                                w[u] = hsub2_bf16(qw[u], pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]),
+                                                                     __uint_as_float(v[8 * jc + 2 * u + 1])));
+                            st_shared_v4(addr, w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+            }
             fence_proxy_async_smem();
             tc_fence_before();
-            nb_sync(NB_INV, 256);
-            if (itid == 0) {
+            nb_sync(NB_INVB, 128);
+            if (utid == 0) {
                 mbar_arrive(bars + B_RR + rb);  // row operand of chunk m stored
                 wait1(B_V, (uint32_t)m);
                 tc_fence_after();
@@ -1322,7 +1373,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
             __syncwarp();
         }
-        if (itid == 0) {
+        if (utid == 0) {
             drain(B_V, n_v);
             if (*s_abort) {
                 mma_commit(bars + B_FIN + 2);
