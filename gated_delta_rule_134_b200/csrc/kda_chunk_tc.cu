@@ -84,9 +84,7 @@ constexpr int kThreads = 512;
 // named barriers (0 is __syncthreads)
 constexpr int NB_TILE = 1;  // tile warps
 constexpr int NB_TOR = 2;   // tile warps, OR-vote
-constexpr int NB_INVA = 3;  // inverse warps
-constexpr int NB_INVA2 = 8; // inverse warps 0-1 (A readout)
-constexpr int NB_INVB = 9;  // U/W warps
+constexpr int NB_INV = 3;   // inverse warps
 constexpr int NB_CHLO = 4;  // chain warps 0-1
 constexpr int NB_CHB = 5;   // chain warps 2-3 -> warp 0: second half of the state operand stored
 constexpr int NB_CHHI = 6;  // chain warps 2-3
@@ -112,8 +110,7 @@ struct Layout {
     static constexpr uint32_t SP = TP + 16384;  // P, K-major 64 x 64 bf16 (rows 64-127 of [Y; P], Y = TP rows 64-127)
     static constexpr uint32_t SOP = SP + 8192;  // S half (64 channels) x DVT, bf16 MN-major, then delta
     static constexpr uint32_t OST = SOP + 64 * DVT * 2;  // 2 x [32 tok][32 ch] bf16 (64-byte swizzle): O stores
-    static constexpr uint32_t TPS = OST + 4096;          // T' staging, K-major 64 x 64 bf16
-    static constexpr uint32_t SCR = TPS + 8192;          // A fp32 [64][kLDA], T diagonal blocks [4][16][kLDT]
+    static constexpr uint32_t SCR = OST + 4096;          // A fp32 [64][kLDA], T diagonal blocks [4][16][kLDT]
     static constexpr uint32_t SA = SCR;                  //   (exact path: 16 KB staging)
     static constexpr uint32_t STD = SCR + 64 * kLDA * 4;
     static constexpr uint32_t SCR_BYTES = 64 * kLDA * 4 + 4 * 16 * kLDT * 4;
@@ -122,14 +119,15 @@ struct Layout {
     static constexpr uint32_t SOPS = SBETA + 256;   // 4 x 128 f32: operand scale per channel (by chunk mod 4)
     static constexpr uint32_t STMS = SOPS + 2048;   // 4 x 128 f32: tensor-memory scale per channel
     static constexpr uint32_t SEK = STMS + 2048;    // 128 f32: e^{G_last - G_m} of the last prepared chunk
-    static constexpr uint32_t SGL = SEK + 512;      // 128 f32: G_last of the tile warps' chunk
-    static constexpr uint32_t BARS = SGL + 512;     // mbarriers
+    static constexpr uint32_t SGM = SEK + 512;      // 128 f32: G_m of the tile warps' chunk
+    static constexpr uint32_t SGL = SGM + 512;      // 128 f32: G_last
+    static constexpr uint32_t SGML = SGL + 512;     // 128 f32: -G_m log2(e)
+    static constexpr uint32_t BARS = SGML + 512;    // mbarriers
     static constexpr uint32_t MISC = BARS + 512;    // tmem base, abort flag
     static constexpr uint32_t END = MISC + 64;
     static constexpr uint32_t SMEM_BYTES = END + 1024;   // + alignment slack
     static constexpr uint32_t SBO_V = 1024 * (DVT / 64); // K-group stride of the S / delta operands
-    static_assert(SOP % 1024 == 0 && TP % 1024 == 0 && LMAT % 1024 == 0 && OST % 1024 == 0 && TPS % 1024 == 0,
-                  "operand alignment");
+    static_assert(SOP % 1024 == 0 && TP % 1024 == 0 && LMAT % 1024 == 0 && OST % 1024 == 0, "operand alignment");
     static_assert(64 * 64 * 4 <= SCR_BYTES, "exact-path staging overflows the scratch");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     // tensor memory columns: R (fp32, lane = key channel) and three chunk slots
@@ -157,9 +155,7 @@ enum : int {
     B_SCRF = 31,  // A/T scratch of the inverse warps' chunk free
     B_EXKQ = 32,  // k/q reloaded for an exact chunk
     B_FIN = 33,   // 3: final drain of each MMA-issuing thread
-    B_TPR = 36,   // T' of the chunk staged by the inverse warps
-    B_TPSF = 37,  // staging tile copied into [T'; PT] by the U/W warps
-    NUM_BARS = 38
+    NUM_BARS = 36
 };
 
 // offset of element (row R, channel c) of a row-operand buffer (K-major, two
@@ -313,7 +309,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     float* sOpS = reinterpret_cast<float*>(sm + L::SOPS);
     float* sTmS = reinterpret_cast<float*>(sm + L::STMS);
     float* sEK = reinterpret_cast<float*>(sm + L::SEK);
+    float* sGm = reinterpret_cast<float*>(sm + L::SGM);
     float* sGl = reinterpret_cast<float*>(sm + L::SGL);
+    float* sGmL = reinterpret_cast<float*>(sm + L::SGML);
     float* sA = reinterpret_cast<float*>(sm + L::SA);
     float* sTd = reinterpret_cast<float*>(sm + L::STD);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BARS);
@@ -335,8 +333,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         tmem_alloc(s_tmem, L::TMEM_COLS);
         tmem_relinquish();
     }
-    {   // constants: [L; L] (row R: ones in columns 0..R%64) and the T' staging
-        // tile, whose blocks above the diagonal are never written again
+    {   // constants: [L; L] (row R: ones in columns 0..R%64) and the T' half of
+        // [T'; PT], whose blocks above the diagonal are never written again
         for (int i = tid; i < 128 * 8; i += kThreads) {
             const int R = i >> 3, j = i & 7, r = R & 63;
             uint32_t w[4];
@@ -346,7 +344,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 w[u] = pack_bf16x2(s <= r ? 1.f : 0.f, s + 1 <= r ? 1.f : 0.f);
             }
             st_shared_v4(sb + L::LMAT + R * 128 + ((j ^ (R & 7)) << 4), w[0], w[1], w[2], w[3]);
-            if (R < 64) st_shared_v4(sb + L::TPS + R * 128 + (j << 4), 0u, 0u, 0u, 0u);
+            if (R < 64) st_shared_v4(sb + L::TP + R * 128 + (j << 4), 0u, 0u, 0u, 0u);
         }
         for (int c = tid; c < kD; c += kThreads) sEK[c] = 1.f;
         if (v_zero)  // transition run: v = 0 stays in the v tile, which is never loaded
@@ -1035,112 +1033,104 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 mbar_wait_bounded(bars + B_FIN + 1, 0u, kDrainBudget);
             }
         }
-    } else if (warp < kInvWarp0 + 4) {
+    } else {
         // ============================================================ inverse warps
-        // Per chunk m: A readout, (I + A)^{-1} -> T' into the staging tile (the
-        // U/W warps copy it into [T'; PT] once that is free).
-        const int itid = tid - 32 * kInvWarp0;  // 0..127
-        const int iw = warp - kInvWarp0;        // 0..3
+        // Per chunk m: A/P readout, (I + A)^{-1} -> T', then the PT, W and U MMAs
+        // with the readouts between them (PT -> [T'; PT], [W'; P W'] -> row operand).
+        const int iw = warp - kInvWarp0;  // 0..7
+        const int hf = iw >> 2;           // which 32-column half of a readout this warp takes
+        const int itid = tid - 32 * kInvWarp0;
+        int n_v = 0;
         auto load_beta = [&](int m) -> float {
             const int t = m * kC + itid;
             return (itid < kC && m < NC && t < seq_len) ? __bfloat162float(beta[(tok0 + t) * H + h]) : 0.f;
         };
-        // T' (bf16) entry into the staging tile (K-major 64 x 64, 128-byte swizzle)
-        auto store_tprime = [&](int r, int s, float t) {
-            *reinterpret_cast<__nv_bfloat16*>(sm + L::TPS + km_off(r, s)) = __float2bfloat16_rn(t * sBeta[s]);
-        };
-        float beta_next = load_beta(0);
-        for (int m = 0; m < NC; ++m) {
-            const int s = m % 3;
-            const uint32_t slot = lane_addr + L::SLOT0 + 128 * s;
-            if (itid < kC) sBeta[itid] = beta_next;
-            beta_next = load_beta(m + 1);
-            waitw(B_AP + s, (uint32_t)(m / 3));
-            if (erase && quad < 2) {  // A (slot rows 0-63) -> fp32 scratch: beta_r, strictly lower
+        // ---- A (slot rows 0-63) -> fp32 scratch (beta_r, strictly lower); P (rows 64-127) -> bf16 K-major tile (lower incl.)
+        auto p4 = [&](uint32_t slot) {
+            if (quad < 2 && !erase) return;  // additive write: A is not used
+            uint32_t v[32];
+            tmem_ld32(slot + 32 * hf, v);
+            tmem_ld_wait(v);
+            if (quad < 2) {
                 const int r = 32 * quad + lane;
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t v[32];
-                    tmem_ld32(slot + 32 * hh, v);
-                    tmem_ld_wait(v);
-                    nb_sync(NB_INVA2, 64);  // (first pass: beta of chunk m visible)
-                    const float br = sBeta[r];
-                    float* dst = sA + r * kLDA + 32 * hh;
+                const float br = sBeta[r];
+                float* dst = sA + r * kLDA + 32 * hf;
 #pragma unroll
-                    for (int u = 0; u < 32; u += 4) {
-                        float4 f;
-                        f.x = (32 * hh + u + 0 < r) ? br * __uint_as_float(v[u + 0]) : 0.f;
-                        f.y = (32 * hh + u + 1 < r) ? br * __uint_as_float(v[u + 1]) : 0.f;
-                        f.z = (32 * hh + u + 2 < r) ? br * __uint_as_float(v[u + 2]) : 0.f;
-                        f.w = (32 * hh + u + 3 < r) ? br * __uint_as_float(v[u + 3]) : 0.f;
-                        *reinterpret_cast<float4*>(dst + u) = f;
-                    }
+                for (int u = 0; u < 32; u += 4) {
+                    float4 f;
+                    f.x = (32 * hf + u + 0 < r) ? br * __uint_as_float(v[u + 0]) : 0.f;
+                    f.y = (32 * hf + u + 1 < r) ? br * __uint_as_float(v[u + 1]) : 0.f;
+                    f.z = (32 * hf + u + 2 < r) ? br * __uint_as_float(v[u + 2]) : 0.f;
+                    f.w = (32 * hf + u + 3 < r) ? br * __uint_as_float(v[u + 3]) : 0.f;
+                    *reinterpret_cast<float4*>(dst + u) = f;
                 }
-            }
-            // the staging tile of the previous chunk has been copied out
-            if (m > 0) waitw(B_TPSF, (uint32_t)(m - 1));
-            nb_sync(NB_INVA, 128);  // A and beta of chunk m visible
-            if (!erase) {  // A = 0: T = I, T' = Diag(beta); thread: row itid/2, 32 columns
-                const int r = itid >> 1;
+            } else {
+                const int r = 32 * (quad - 2) + lane;
 #pragma unroll
                 for (int jc = 0; jc < 4; ++jc) {
-                    const int j = 4 * (itid & 1) + jc;  // 8-column chunk
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int s = 32 * hf + 8 * jc + 2 * u;
+                        const float p0 = (s <= r) ? __uint_as_float(v[8 * jc + 2 * u]) : 0.f;
+                        const float p1 = (s + 1 <= r) ? __uint_as_float(v[8 * jc + 2 * u + 1]) : 0.f;
+                        w[u] = pack_bf16x2(p0, p1);
+                    }
+                    st_shared_v4(sb + L::SP + r * 128 + (((4 * hf + jc) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                }
+            }
+        };
+        // ---- P5: T = (I + A)^{-1} -> T' = T Diag(beta), bf16, rows 0-63 of [T'; PT]
+        auto store_tprime = [&](int r, int s, float t) {
+            *reinterpret_cast<__nv_bfloat16*>(sm + L::TP + km_off(r, s)) = __float2bfloat16_rn(t * sBeta[s]);
+        };
+        auto p5 = [&]() {
+            if (!erase) {  // A = 0: T = I, T' = Diag(beta); thread: row itid/4, 16 columns
+                const int r = itid >> 2, j0c = 2 * (itid & 3);
+#pragma unroll
+                for (int jc = 0; jc < 2; ++jc) {
+                    const int j = j0c + jc;  // 8-column chunk
                     uint32_t w[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int s0 = 8 * j + 2 * u;
                         w[u] = pack_bf16x2(s0 == r ? sBeta[r] : 0.f, s0 + 1 == r ? sBeta[r] : 0.f);
                     }
-                    st_shared_v4(sb + L::TPS + r * 128 + ((j ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                    st_shared_v4(sb + L::TP + r * 128 + ((j ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
                 }
-            } else {
-                if (itid < 64) {
-                    // diagonal 16x16 blocks, one thread per column c of block a, by
-                    // forward substitution in axpy form: once T_kc is final, every
-                    // later row takes its A_ik T_kc (no exchange between threads)
-                    const int a = itid >> 4, c = itid & 15;
-                    const float* Ab = sA + (16 * a) * kLDA + 16 * a;
-                    // c0..c2: columns k, k+1, k+2 of A_aa (the loads run three steps
-                    // ahead of the substitution, which waits on nothing else)
-                    float acc[16], c0[16], c1[16], c2[16];
+                return;
+            }
+            {   // diagonal 16x16 blocks: four threads per column, rows q, q+4, q+8, q+12
+                const int a = itid >> 6, jc = (itid >> 2) & 15, q = itid & 3;
+                const float* Ab = sA + (16 * a) * kLDA + 16 * a;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f}, colv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        acc[i] = 0.f;
-                        c0[i] = i > 0 ? Ab[i * kLDA] : 0.f;
-                        c1[i] = i > 1 ? Ab[i * kLDA + 1] : 0.f;
-                        c2[i] = i > 2 ? Ab[i * kLDA + 2] : 0.f;
-                    }
+                for (int r = 0; r < 16; ++r) {
+                    const float mine = (r == jc) ? 1.f : ((r > jc) ? -acc[r >> 2] : 0.f);
+                    const float t = __shfl_sync(0xffffffffu, mine, (lane & ~3) | (r & 3));
+                    if (q == (r & 3)) colv[r >> 2] = t;
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        float c3[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) c3[i] = (k + 3 < 16 && i > k + 3) ? Ab[i * kLDA + k + 3] : 0.f;
-                        const float tk = (k < c) ? 0.f : ((k == c) ? 1.f : -acc[k]);
-                        acc[k] = tk;
-#pragma unroll
-                        for (int i = k + 1; i < 16; ++i) acc[i] = fmaf(c0[i], tk, acc[i]);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            c0[i] = c1[i];
-                            c1[i] = c2[i];
-                            c2[i] = c3[i];
-                        }
-                    }
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        sTd[(a * 16 + i) * kLDT + c] = acc[i];
-                        store_tprime(16 * a + i, 16 * a + c, acc[i]);
-                    }
+                    for (int i = 0; i < 4; ++i)
+                        if (q + 4 * i > r) acc[i] = fmaf(Ab[(q + 4 * i) * kLDA + r], t, acc[i]);
                 }
-                nb_sync(NB_INVA, 128);
-                // Blocks below the diagonal: column chains (block column bb, 8-column
-                // half nt), held in registers: for a = bb+1..3, X = sum_{k=bb}^{a-1}
-                // A_ak T_kb, then T_ab = -T_aa X, on m16n8k8 tf32 MMAs. A product's
-                // accumulator fragment becomes the right-hand operand of the next
-                // product by shuffles; A and the diagonal blocks come from shared
-                // memory. Warps 0-1 take block column 0, warps 2-3 block columns 1 and 2.
-                const int nt = iw & 1;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = q + 4 * i;  // row inside the block
+                    sTd[(a * 16 + r) * kLDT + jc] = colv[i];
+                    store_tprime(16 * a + r, 16 * a + jc, colv[i]);
+                }
+            }
+            nb_sync(NB_INV, 256);
+            // Blocks below the diagonal, one column chain per warp (block column
+            // bb, 8-column half nt), held in registers: for a = bb+1..3,
+            // X = sum_{k=bb}^{a-1} A_ak T_kb, then T_ab = -T_aa X, on m16n8k8 tf32
+            // MMAs. A product's accumulator fragment becomes the right-hand operand
+            // of the next product by shuffles; A and the diagonal blocks come from
+            // shared memory.
+            const int bb = iw >> 1, nt = iw & 1;
+            if (bb < 3) {
                 const int g = lane >> 2, t = lane & 3;
+                const int sc = 16 * bb + 8 * nt;  // first column of this warp's half
                 // accumulator (rows g | g+8, columns 2t | 2t+1) -> right operand
                 // fragments of the two 8-row k-steps (rows t | t+4, column g)
                 auto c2b = [&](const float (&c)[4], uint32_t (&bf)[2][2]) {
@@ -1156,126 +1146,148 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         bf[j][1] = to_tf32(odd ? o1 : e1);
                     }
                 };
-                auto chain = [&](const int bb) {
-                    const int sc = 16 * bb + 8 * nt;  // first column of this warp's half
-                    uint32_t tb[3][2][2];             // right operand fragments of T_kb, k = bb..2
-                    {
-                        const float* D = sTd + bb * 16 * kLDT + 8 * nt;
+                uint32_t tb[3][2][2];  // right operand fragments of T_kb, k = bb..2
+                {
+                    const float* D = sTd + bb * 16 * kLDT + 8 * nt;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        tb[0][j][0] = to_tf32(D[(8 * j + t) * kLDT + g]);
+                        tb[0][j][1] = to_tf32(D[(8 * j + t + 4) * kLDT + g]);
+                    }
+                }
+                // da = a - bb and dk = k - bb run over compile-time ranges, so the
+                // fragment array stays in registers
+#pragma unroll
+                for (int da = 1; da < 4; ++da) {
+                    const int a = bb + da;
+                    if (a > 3) break;
+                    float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int dk = 0; dk < da; ++dk) {
+                        const int k = bb + dk;
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
-                            tb[0][j][0] = to_tf32(D[(8 * j + t) * kLDT + g]);
-                            tb[0][j][1] = to_tf32(D[(8 * j + t + 4) * kLDT + g]);
+                            const float* Ar = sA + (16 * a) * kLDA + 16 * k + 8 * j;
+                            const uint32_t af[4] = {to_tf32(Ar[g * kLDA + t]), to_tf32(Ar[(g + 8) * kLDA + t]),
+                                                    to_tf32(Ar[g * kLDA + t + 4]), to_tf32(Ar[(g + 8) * kLDA + t + 4])};
+                            mma_tf32_16x8x8(x, af, tb[dk][j]);
                         }
                     }
-                    // da = a - bb and dk = k - bb run over compile-time ranges, so the
-                    // fragment array stays in registers
+                    uint32_t xb[2][2];
+                    c2b(x, xb);
+                    float y[4] = {0.f, 0.f, 0.f, 0.f};
+                    const float* D = sTd + a * 16 * kLDT;
 #pragma unroll
-                    for (int da = 1; da < 4; ++da) {
-                        const int a = bb + da;
-                        if (a > 3) break;
-                        float x[4] = {0.f, 0.f, 0.f, 0.f}, x2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                        for (int dk = 0; dk < da; ++dk) {
-                            const int k = bb + dk;
-#pragma unroll
-                            for (int j = 0; j < 2; ++j) {
-                                const float* Ar = sA + (16 * a) * kLDA + 16 * k + 8 * j;
-                                const uint32_t af[4] = {to_tf32(Ar[g * kLDA + t]), to_tf32(Ar[(g + 8) * kLDA + t]),
-                                                        to_tf32(Ar[g * kLDA + t + 4]),
-                                                        to_tf32(Ar[(g + 8) * kLDA + t + 4])};
-                                mma_tf32_16x8x8(j == 0 ? x : x2, af, tb[dk][j]);  // two independent accumulators
-                            }
-                        }
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) x[e] += x2[e];
-                        uint32_t xb[2][2];
-                        c2b(x, xb);
-                        float y[4] = {0.f, 0.f, 0.f, 0.f};
-                        const float* D = sTd + a * 16 * kLDT;
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const uint32_t af[4] = {to_tf32(D[g * kLDT + 8 * j + t]), to_tf32(D[(g + 8) * kLDT + 8 * j + t]),
-                                                    to_tf32(D[g * kLDT + 8 * j + t + 4]),
-                                                    to_tf32(D[(g + 8) * kLDT + 8 * j + t + 4])};
-                            mma_tf32_16x8x8(y, af, xb[j]);
-                        }
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) y[e] = -y[e];
-                        const int s0 = sc + 2 * t;
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh)
-                            *reinterpret_cast<uint32_t*>(sm + L::TPS + km_off(16 * a + g + 8 * hh, s0)) =
-                                pack_bf16x2(y[2 * hh] * sBeta[s0], y[2 * hh + 1] * sBeta[s0 + 1]);
-                        if (da < 3 && a < 3) c2b(y, tb[da]);
+                    for (int j = 0; j < 2; ++j) {
+                        const uint32_t af[4] = {to_tf32(D[g * kLDT + 8 * j + t]), to_tf32(D[(g + 8) * kLDT + 8 * j + t]),
+                                                to_tf32(D[g * kLDT + 8 * j + t + 4]),
+                                                to_tf32(D[(g + 8) * kLDT + 8 * j + t + 4])};
+                        mma_tf32_16x8x8(y, af, xb[j]);
                     }
-                };
-                if (iw < 2) {
-                    chain(0);
-                } else {
-                    chain(2);
-                    chain(1);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) y[e] = -y[e];
+                    const int s0 = sc + 2 * t;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                        *reinterpret_cast<uint32_t*>(sm + L::TP + km_off(16 * a + g + 8 * hh, s0)) =
+                            pack_bf16x2(y[2 * hh] * sBeta[s0], y[2 * hh + 1] * sBeta[s0 + 1]);
+                    if (da < 3 && a < 3) c2b(y, tb[da]);
                 }
             }
-            nb_sync(NB_INVA, 128);
-            if (itid == 0) {
-                mbar_arrive(bars + B_TPR);   // T' of chunk m staged
-                mbar_arrive(bars + B_SCRF);  // A/T scratch free
+        };
+        // ---- PT (slot rows 64-127, columns 64-127) -> bf16 rows 64-127 of [T'; PT]
+        auto p6 = [&](uint32_t slot) {
+            if (quad < 2) return;
+            const int r = 32 * (quad - 2) + lane;
+            uint32_t v[32];
+            tmem_ld32(slot + 64 + 32 * hf, v);
+            tmem_ld_wait(v);
+#pragma unroll
+            for (int jc = 0; jc < 4; ++jc) {
+                uint32_t w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]), __uint_as_float(v[8 * jc + 2 * u + 1]));
+                const int R = 64 + r;
+                st_shared_v4(sb + L::TP + R * 128 + (((4 * hf + jc) ^ (R & 7)) << 4), w[0], w[1], w[2], w[3]);
             }
-            __syncwarp();
-        }
-    } else {
-        // ============================================================ U/W warps
-        // Per chunk m: P readout, T' into [T'; PT], the PT, W and U MMAs with the
-        // readouts between them (PT -> [T'; PT], [W'; P W'] -> row operand).
-        const int utid = tid - 32 * (kInvWarp0 + 4);  // 0..127
-        int n_v = 0;
-        if (NC > 0 && utid == 0) {
-            load_v(0);
-            ++n_v;
-            pf_v(1);
-        }
-        for (int m = 0; m < NC; ++m) {
-            const int s = m % 3, rb = m & 1;
-            const uint32_t slot = lane_addr + L::SLOT0 + 128 * s;
-            waitw(B_AP + s, (uint32_t)(m / 3));
-            if (quad >= 2) {  // P (slot rows 64-127) -> bf16 K-major tile, lower incl.
-                const int r = 32 * (quad - 2) + lane;
+        };
+        // ---- P7: [W'; P W'] -> row operand: rows 0-63 -W' over KE, rows 64-127 QE - P W'
+        auto p7 = [&](uint32_t slot, int rb) {
+            const uint32_t rop = sb + L::ROW + rb * 32768;
+            if (quad < 2) {
+                const int r = 32 * quad + lane;
+                if (!erase) {  // additive write: delta = U, the W S term is zero
+#pragma unroll
+                    for (int jc = 0; jc < 8; ++jc)
+                        st_shared_v4(rop + hf * 16384 + r * 128 + ((jc ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
+                    return;
+                }
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t v[32];
-                    tmem_ld32(slot + 32 * hh, v);
+                    tmem_ld32(slot + 64 * hf + 32 * hh, v);
                     tmem_ld_wait(v);
 #pragma unroll
                     for (int jc = 0; jc < 4; ++jc) {
                         uint32_t w[4];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int s2 = 32 * hh + 8 * jc + 2 * u;
-                            const float p0 = (s2 <= r) ? __uint_as_float(v[8 * jc + 2 * u]) : 0.f;
-                            const float p1 = (s2 + 1 <= r) ? __uint_as_float(v[8 * jc + 2 * u + 1]) : 0.f;
-                            w[u] = pack_bf16x2(p0, p1);
-                        }
-                        st_shared_v4(sb + L::SP + r * 128 + (((4 * hh + jc) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                        for (int u = 0; u < 4; ++u)
+                            w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]), __uint_as_float(v[8 * jc + 2 * u + 1])) ^
+                                   0x80008000u;
+                        st_shared_v4(rop + hf * 16384 + r * 128 + (((4 * hh + jc) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                    }
+                }
+            } else {
+                if (!erase) return;  // W = 0: the rows keep QE
+                const int r = 32 * (quad - 2) + lane, R = 64 + r;
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t v[32];
+                    tmem_ld32(slot + 64 * hf + 32 * hh, v);
+                    tmem_ld_wait(v);
+#pragma unroll
+                    for (int jc = 0; jc < 4; ++jc) {
+                        const uint32_t addr = rop + hf * 16384 + R * 128 + (((4 * hh + jc) ^ (R & 7)) << 4);
+                        const uint4 qv = ld_shared_v4(addr);
+                        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                        uint32_t w[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            w[u] = hsub2_bf16(qw[u], pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]),
+                                                                 __uint_as_float(v[8 * jc + 2 * u + 1])));
+                        st_shared_v4(addr, w[0], w[1], w[2], w[3]);
                     }
                 }
             }
-            if (utid == 0 && m > 0) {  // [T'; PT] and the v tile of the previous chunk are free
+        };
+        if (NC > 0 && itid == 0) {
+            load_v(0);
+            ++n_v;
+            pf_v(1);
+        }
+        float beta_next = load_beta(0);
+        for (int m = 0; m < NC; ++m) {
+            const int s = m % 3, rb = m & 1;
+            const uint32_t slot = lane_addr + L::SLOT0 + 128 * s;
+            if (itid < kC) sBeta[itid] = beta_next;
+            beta_next = load_beta(m + 1);
+            waitw(B_AP + s, (uint32_t)(m / 3));
+            if (m > 0 && itid == 0) {  // [T'; PT] and the v tile of the previous chunk are free
                 wait1(B_UO + (m - 1) % 3, (uint32_t)((m - 1) / 3));
                 load_v(m);
                 ++n_v;
                 pf_v(m + 1);
             }
-            waitw(B_TPR, (uint32_t)m);  // T' of chunk m staged (its A rows are read: W may overwrite them)
-            nb_sync(NB_INVB, 128);      // [T'; PT] free
-            for (int i = utid; i < 512; i += 128) {  // T' -> rows 0-63 of [T'; PT] (same swizzled layout)
-                const uint4 w = ld_shared_v4(sb + L::TPS + 16 * i);
-                st_shared_v4(sb + L::TP + 16 * i, w.x, w.y, w.z, w.w);
-            }
+            nb_sync(NB_INV, 256);  // beta of chunk m visible, [T'; PT] free
+            p4(slot);
+            nb_sync(NB_INV, 256);
+            p5();
             fence_proxy_async_smem();
             tc_fence_before();
-            nb_sync(NB_INVB, 128);
-            if (utid == 0) {
-                mbar_arrive(bars + B_TPSF);  // staging tile free
+            nb_sync(NB_INV, 256);
+            if (itid == 0) {
+                mbar_arrive(bars + B_SCRF);  // A/T scratch free
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)  // PT = P T' into columns 64-127 (rows 0-63 take junk)
@@ -1283,28 +1295,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 mma_commit(bars + B_PT);
             }
             waitw(B_PT, (uint32_t)m);
-            if (quad >= 2) {  // PT (slot rows 64-127, columns 64-127) -> bf16 rows 64-127 of [T'; PT]
-                const int r = 32 * (quad - 2) + lane, R = 64 + r;
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t v[32];
-                    tmem_ld32(slot + 64 + 32 * hh, v);
-                    tmem_ld_wait(v);
-#pragma unroll
-                    for (int jc = 0; jc < 4; ++jc) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            w[u] = pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]), __uint_as_float(v[8 * jc + 2 * u + 1]));
-                        st_shared_v4(sb + L::TP + R * 128 + (((4 * hh + jc) ^ (R & 7)) << 4), w[0], w[1], w[2], w[3]);
-                    }
-                }
-            }
+            p6(slot);
             fence_proxy_async_smem();
             tc_fence_before();
-            nb_sync(NB_INVB, 128);
+            nb_sync(NB_INV, 256);
             if (erase) {
-                if (utid == 0) {
+                if (itid == 0) {
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // [W'; P W'] = [T'; PT] KE
@@ -1314,55 +1310,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
                 waitw(B_WB, (uint32_t)m);
             }
-            {   // [W'; P W'] -> row operand: rows 0-63 -W' over KE, rows 64-127 QE - P W'
-                const uint32_t rop = sb + L::ROW + rb * 32768;
-                if (quad < 2) {
-                    const int r = 32 * quad + lane;
-#pragma unroll 1
-                    for (int hh = 0; hh < 4; ++hh) {
-                        uint32_t v[32];
-                        if (erase) {
-                            tmem_ld32(slot + 32 * hh, v);
-                            tmem_ld_wait(v);
-                        }
-#pragma unroll
-                        for (int jc = 0; jc < 4; ++jc) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)  // additive write: delta = U, the W S term is zero
-                                w[u] = erase ? pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]),
-                                                           __uint_as_float(v[8 * jc + 2 * u + 1])) ^ 0x80008000u
-                                             : 0u;
-                            st_shared_v4(rop + (hh >> 1) * 16384 + r * 128 + (((4 * (hh & 1) + jc) ^ (r & 7)) << 4), w[0],
-                                         w[1], w[2], w[3]);
-                        }
-                    }
-                } else if (erase) {  // (W = 0: the rows keep QE)
-                    const int r = 32 * (quad - 2) + lane, R = 64 + r;
-#pragma unroll 1
-                    for (int hh = 0; hh < 4; ++hh) {
-                        uint32_t v[32];
-                        tmem_ld32(slot + 32 * hh, v);
-                        tmem_ld_wait(v);
-#pragma unroll
-                        for (int jc = 0; jc < 4; ++jc) {
-                            const uint32_t addr = rop + (hh >> 1) * 16384 + R * 128 + (((4 * (hh & 1) + jc) ^ (R & 7)) << 4);
-                            const uint4 qv = ld_shared_v4(addr);
-                            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-                            uint32_t w[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)  // QE - P W' on bf16 pairs (P W' rounded to bf16 first)
-                                w[u] = hsub2_bf16(qw[u], pack_bf16x2(__uint_as_float(v[8 * jc + 2 * u]),
-                                                                     __uint_as_float(v[8 * jc + 2 * u + 1])));
-                            st_shared_v4(addr, w[0], w[1], w[2], w[3]);
-                        }
-                    }
-                }
-            }
+            p7(slot, rb);
             fence_proxy_async_smem();
             tc_fence_before();
-            nb_sync(NB_INVB, 128);
-            if (utid == 0) {
+            nb_sync(NB_INV, 256);
+            if (itid == 0) {
                 mbar_arrive(bars + B_RR + rb);  // row operand of chunk m stored
                 wait1(B_V, (uint32_t)m);
                 tc_fence_after();
@@ -1373,7 +1325,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
             __syncwarp();
         }
-        if (utid == 0) {
+        if (itid == 0) {
             drain(B_V, n_v);
             if (*s_abort) {
                 mma_commit(bars + B_FIN + 2);
