@@ -11,7 +11,7 @@ import ctypes
 import os
 
 __all__ = ["load", "chunk_fwd", "chunk_fwd_varlen", "chunk_bwd", "chunk_fwd_noalloc", "noalloc_status", "decode_step",
-           "workspace_size", "workspace_status", "KDAError", "library_path", "STATUS"]
+           "workspace_size", "workspace_status", "chunk_fwd_timeout_test", "KDAError", "library_path", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libkda.so")
@@ -61,6 +61,8 @@ def load(build_if_stale: bool = True):
     lib.kda_chunk_fwd_ex.argtypes = [P] * 8 + [I] * 7 + [P, Z, I, P]
     lib.kda_chunk_fwd_ex.restype = I
     lib.kda_workspace_status.argtypes = [P, Z, P]
+    lib.kda_chunk_fwd_timeout_test.argtypes = [P] * 8 + [I] * 7 + [P, Z, ctypes.c_longlong, P]
+    lib.kda_chunk_fwd_timeout_test.restype = I
     lib.kda_workspace_status.restype = I
     lib.kda_decode_step.argtypes = [P] * 8 + [I] * 5 + [P]
     lib.kda_decode_step.restype = I
@@ -348,6 +350,37 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0=None, *, o, S_T=None, chunk: 
                                          _ptr(o), _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPE[_dtype_of(q)],
                                          _stream(stream, dev))
     _check("kda_chunk_fwd_noalloc", code)
+    return o, S_T
+
+
+def chunk_fwd_timeout_test(q, k, v, log_alpha, beta, S0=None, *, o, S_T, workspace, wait_budget_cycles: int,
+                           stream=None):
+    """kda_chunk_fwd_timeout_test: the tensor-core prefill with its first k/q
+    load withheld and every wait bounded by wait_budget_cycles SM cycles, so
+    the kernel gives up and records KDA_ERR_TIMEOUT in `workspace` (read it
+    with workspace_status). A test hook for the timeout path; o and S_T are
+    left undefined."""
+    import torch
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt, dev = q.dtype, q.device
+    _need(q, "q", (B, T, H, dk), dt, dev)
+    _need(k, "k", (B, T, H, dk), dt, dev)
+    _need(log_alpha, "log_alpha", (B, T, H, dk), dt, dev)
+    _need(v, "v", (B, T, H, dv), dt, dev)
+    _need(beta, "beta", (B, T, H), dt, dev)
+    _need(o, "o", (B, T, H, dv), dt, dev)
+    _need(S_T, "S_T", (B, H, dk, dv), torch.float32, dev)
+    if S0 is not None:
+        _need(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    ws_len = workspace.numel() * workspace.element_size()
+    with _on(dev):
+        code = lib.kda_chunk_fwd_timeout_test(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                                              _ptr(o), _ptr(S_T), B, T, H, dk, dv, 64, _DTYPE[_dtype_of(q)],
+                                              _ptr(workspace), ws_len, int(wait_budget_cycles),
+                                              _stream(stream, dev))
+    _check("kda_chunk_fwd_timeout_test", code)
     return o, S_T
 
 

@@ -140,6 +140,25 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const vo
                             workspace_bytes, KDA_ALGO_AUTO, stream);
 }
 
+kda_status_t kda_chunk_fwd_timeout_test(const void* q, const void* k, const void* v, const void* log_alpha,
+                                       const void* beta, const float* S0, void* o, float* S_T, int B, int T, int H,
+                                       int dk, int dv, int chunk, kda_dtype_t dtype, void* workspace,
+                                       size_t workspace_bytes, long long wait_budget_cycles, void* stream) {
+    if (wait_budget_cycles <= 0 || wait_budget_cycles > (1ll << 31)) return KDA_ERR_INVALID_ARG;
+    kda::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.bf16 = dtype == KDA_BF16;
+    a.erase = 1;
+    a.gate = KDA_GATE_CHANNEL;
+    a.cu_seqlens = nullptr;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+    a.test_withhold_first_load = 1;
+    a.test_wait_budget = wait_budget_cycles;
+    // Only the single-pass tensor-core kernel has the waits this exercises.
+    if (T == 0) return KDA_ERR_INVALID_ARG;
+    return run_chunk(a, dtype, KDA_ALGO_TC, stream);
+}
+
 kda_status_t kda_workspace_status(const void* workspace, size_t workspace_bytes, void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;

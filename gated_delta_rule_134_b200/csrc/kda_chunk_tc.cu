@@ -14,12 +14,12 @@
 //   O     = (q e^G) S + P delta
 //   S    <- Diag(e^{G_last}) S + (k e^{G_last - G})^T delta
 //
-// Reference-point factorisation. With G_m the gate at the chunk's middle token
-// and E_r = e^{G_r - G_m}, F_r = e^{G_m - G_r} (per channel):
-//   e^{G_r - G_s} = E_r F_s,  k e^G = (k E) e^{G_m},  k e^{G_last-G} = (k F) e^{G_last-G_m}.
+// Reference-point factorisation. G_r is counted from the chunk's entry, so
+// with E_r = e^{G_r} and F_r = e^{-G_r} (per channel):
+//   e^{G_r - G_s} = E_r F_s,  k e^G = k E,  k e^{G_last-G} = (k F) e^{G_last}.
 // Three bf16 tiles, KE = k E, QE = q E and KF = k F, feed every MMA. The
 // output is regrouped so that P never meets the state: with PT = P T',
-//   O = QE S^ + P (U - W' S^) = (QE - P W') S^ + P T' v,   S^ = e^{G_m} S, W' = T' KE,
+//   O = QE S + P (U - W' S) = (QE - P W') S + P T' v,   W' = T' KE,
 // so per chunk the state-independent MMAs are
 //   G = [L; L] g                  -> gate prefix sums (L: lower-triangular ones)
 //   [A; P] = [KE; QE] KF^T        (one M=128 MMA)
@@ -27,15 +27,15 @@
 //   [W'; P W'] = [T'; PT] KE      -> row operand [-W'; QE - P W']
 //   [U; P T' v] = [T'; PT] v      -> the chunk's accumulator
 // and the state chain needs only two:
-//   D += [-W'; QE - P W'] S^      -> rows 0-63: delta, rows 64-127: O
-//   R  = e^{G_m} S + KF^T delta   -> S_next = Diag(e^{G_last-G_m}) R
-// The tensor memory holds R, and the next chunk rescales it per channel while
-// it copies the state into the bf16 MMA operand. Each factor is a single
-// exponential, finite as long as |G_r - G_m| <= 80 and |G_m| <= 80; a vote of
-// the tile warps checks that per chunk. A chunk that fails it uses exact
-// per-pair exponentials e^{G_r - G_s} (exponent <= 0) for A and P and the
-// plain tiles k e^G, q e^G, k e^{G_last-G} (with G_m := 0); the same MMAs then
-// produce the same quantities.
+//   D += [-W'; QE - P W'] S       -> rows 0-63: delta, rows 64-127: O
+//   R  = S + KF^T delta           -> S_next = Diag(e^{G_last}) R
+// The tensor memory holds R; the per-channel factor e^{G_last} is applied
+// lazily, when the next chunk copies the state into the bf16 MMA operand (and
+// when the final state is written). Each factor is a single exponential,
+// finite as long as |G_r| <= 80; a vote of the tile warps checks that per
+// chunk. A chunk that fails it uses exact per-pair exponentials e^{G_r - G_s}
+// (exponent <= 0) for A and P and the plain tiles k e^G, q e^G,
+// k e^{G_last-G}; the same MMAs then produce the same quantities.
 //
 // Schedule. One CTA owns one (batch, head) and a DVT-wide slice of value
 // channels; its state stays in tensor memory for the whole sequence. Each
@@ -94,7 +94,7 @@ constexpr int kD = 128;   // dk = dv
 constexpr int kLDA = 68;  // fp32 row stride of the A scratch (bank spread)
 constexpr int kLDT = 20;  // fp32 row stride of the diagonal blocks of T (bank spread)
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kGuardL = 80.f * kLog2e;      // |G_r - G_m| <= 80, in log2 units
+constexpr float kGuardL = 80.f * kLog2e;      // |G_r| <= 80, in log2 units
 constexpr long long kWaitBudget = 1ll << 31;  // SM cycles (~1 s)
 constexpr long long kDrainBudget = 1ll << 24;
 
@@ -118,12 +118,10 @@ struct Layout {
     static constexpr uint32_t SBETA = SMALL;        // 64 f32: beta of the inverse warps' chunk
     static constexpr uint32_t SOPS = SBETA + 256;   // 4 x 128 f32: operand scale per channel (by chunk mod 4)
     static constexpr uint32_t STMS = SOPS + 2048;   // 4 x 128 f32: tensor-memory scale per channel
-    static constexpr uint32_t SEK = STMS + 2048;    // 128 f32: e^{G_last - G_m} of the last prepared chunk
-    static constexpr uint32_t SGM = SEK + 512;      // 128 f32: G_m of the tile warps' chunk
-    static constexpr uint32_t SGL = SGM + 512;      // 128 f32: G_last
-    static constexpr uint32_t SGML = SGL + 512;     // 128 f32: -G_m log2(e)
-    static constexpr uint32_t BARS = SGML + 512;    // mbarriers
-    static constexpr uint32_t MISC = BARS + 512;    // tmem base, abort flag
+    static constexpr uint32_t SEK = STMS + 2048;    // 128 f32: pending state factor after the last prepared chunk
+    static constexpr uint32_t SGL = SEK + 512;      // 128 f32: G_last
+    static constexpr uint32_t BARS = SGL + 512;     // mbarriers
+    static constexpr uint32_t MISC = BARS + 512;    // tmem base, abort flag, copies issued, wait budget
     static constexpr uint32_t END = MISC + 64;
     static constexpr uint32_t SMEM_BYTES = END + 1024;   // + alignment slack
     static constexpr uint32_t SBO_V = 1024 * (DVT / 64); // K-group stride of the S / delta operands
@@ -194,9 +192,6 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
 __device__ __forceinline__ void nb_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
-__device__ __forceinline__ void nb_arrive(int id, int nthreads) {
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 __device__ __forceinline__ bool nb_or(int id, int nthreads, bool pred) {
     uint32_t r;
     asm volatile(
@@ -231,6 +226,10 @@ struct SegJobs {
     float* M;    // [B*H][P-2][dk][dv]
     float* C;    // [B*H][P-2][dk][dv]
     float* Sin;  // [B*H][P-1][dk][dv]: state entering segment j at [j-1]
+    // Fault injection for the timeout test only (zero in every other launch):
+    // withhold the first k/q load, and give every wait this budget in SM cycles.
+    int withhold_first_load;
+    long long wait_budget;
 };
 
 // ERASE: 1 delta-rule family, 0 additive write. GATE: 0 per-channel log_alpha,
@@ -309,19 +308,26 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     float* sOpS = reinterpret_cast<float*>(sm + L::SOPS);
     float* sTmS = reinterpret_cast<float*>(sm + L::STMS);
     float* sEK = reinterpret_cast<float*>(sm + L::SEK);
-    float* sGm = reinterpret_cast<float*>(sm + L::SGM);
     float* sGl = reinterpret_cast<float*>(sm + L::SGL);
-    float* sGmL = reinterpret_cast<float*>(sm + L::SGML);
     float* sA = reinterpret_cast<float*>(sm + L::SA);
     float* sTd = reinterpret_cast<float*>(sm + L::STD);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BARS);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
+    // Copies issued so far, for the final drain after an abort: the last chunk
+    // whose k/q, log_alpha and v tiles were loaded (-1: none; each kind is loaded
+    // in chunk order), and the number of exact-path k/q reloads.
+    int* s_issued = reinterpret_cast<int*>(sm + L::MISC + 8);
+    // SM cycles a wait may take before it gives up (read only when a wait blocks)
+    volatile long long* s_budget = reinterpret_cast<volatile long long*>(sm + L::MISC + 40);
 
     // ---------------------------------------------------------------- setup
     if (tid == 0) {
         for (int i = 0; i < NUM_BARS; ++i) mbar_init(bars + i, (i >= B_SF && i < B_SF + 3) ? 2u : 1u);
         *s_abort = 0;
+        s_issued[0] = s_issued[1] = s_issued[2] = -1;
+        s_issued[3] = 0;
+        *s_budget = sj.wait_budget > 0 ? sj.wait_budget : kWaitBudget;
         fence_mbar_init();
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_q);
@@ -362,19 +368,20 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         *s_abort = 1;
     };
     // Bounded wait by one thread; after a timeout every later wait is skipped.
-    auto wait1 = [&](int slot, uint32_t parity) {
-        if (!*s_abort && !mbar_wait_bounded(bars + slot, parity & 1u, kWaitBudget)) fail();
+    // True when the phase completed and no thread had aborted by then (a copy
+    // issued on that condition cannot race a phase another wait skipped).
+    auto wait1 = [&](int slot, uint32_t parity) -> bool {
+        if (*s_abort) return false;
+        if (mbar_wait_bounded(bars + slot, parity & 1u, s_budget)) return !*s_abort;
+        fail();
+        return false;
     };
     // Bounded wait by a whole warp, then reconverge; MMA results readable after.
-    auto waitw = [&](int slot, uint32_t parity) {
-        wait1(slot, parity);
+    auto waitw = [&](int slot, uint32_t parity) -> bool {
+        const bool ok = wait1(slot, parity);
         __syncwarp();
         tc_fence_after();
-    };
-    // After an abort: wait (bounded) for the last phase a barrier was armed for,
-    // so no copy or MMA is still writing when the CTA exits.
-    auto drain = [&](int slot, int count) {
-        if (*s_abort && count > 0) mbar_wait_bounded(bars + slot, (uint32_t)(count - 1) & 1u, kDrainBudget);
+        return ok;
     };
 
     constexpr uint32_t ID_CS = idesc_bf16(128, 128, 0, 1);   // [L; L] x g (MN-major)
@@ -399,9 +406,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const uint64_t dV = sdesc_sw128(sb + L::RAWV, 8192, 1024);           // MN-major B
     const uint64_t dSOP = sdesc_sw128(sb + L::SOP, 1024, L::SBO_V);      // MN-major B (S, then delta)
 
-    // TMA issue helpers (one thread)
+    // TMA issue helpers (one thread). A copy that reuses a barrier is issued only
+    // after a wait that completed for real (not one skipped after an abort):
+    // arming a barrier again while its previous phase still waits for bytes
+    // would over-arrive on that phase.
     auto load_kq = [&](int m, int bar) {  // k/q tiles of chunk m into the row buffer of its parity
         uint8_t* dst = sm + L::ROW + (m & 1) * 32768;
+        if (bar == B_EXKQ) ++s_issued[3];
+        else s_issued[0] = m;
         mbar_arrive_expect_tx(bars + bar, 4 * 8192);
         for (int x = 0; x < 2; ++x) {
             tma_load_4d(dst + x * 16384, &tm_k, bars + bar, 64 * x, h, tma_t0 + m * kC, tma_b);
@@ -416,6 +428,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
     };
     auto load_g = [&](int m) {
+        s_issued[1] = m;
         mbar_arrive_expect_tx(bars + B_G + m % 3, 2 * 8192);
         for (int x = 0; x < 2; ++x)
             tma_load_4d(sm + L::COL + (m % 3) * 16384 + x * 8192, &tm_g, bars + B_G + m % 3, 64 * x, h,
@@ -430,6 +443,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             mbar_arrive(bars + B_V);
             return;
         }
+        s_issued[2] = m;
         mbar_arrive_expect_tx(bars + B_V, (DVT / 64) * 8192);
         for (int x = 0; x < DVT / 64; ++x)
             tma_load_4d(sm + L::RAWV + x * 8192, &tm_v, bars + B_V, j0 + 64 * x, h, tma_t0 + m * kC, tma_b);
@@ -501,7 +515,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         uint32_t gnext = 0;  // per-token gate row of the next chunk to place (warp 0)
         if (NC > 0) {
             if (issuer) {
-                load_kq(0, B_KQ);
+                if (!sj.withhold_first_load) load_kq(0, B_KQ);
                 if (NC > 1) load_kq(1, B_KQ + 1);
                 pf_kq(2);
                 if (GATE == 0) {
@@ -556,9 +570,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const int s = n % 3, rb = n & 1;
             const uint32_t slot = lane_addr + L::SLOT0 + 128 * s;
             if (n > 0) {
-                waitw(B_M2, (uint32_t)(n - 1));  // state update of the previous chunk done
+                const bool m2 = waitw(B_M2, (uint32_t)(n - 1));  // state update of the previous chunk done
                 if (n + 2 < NC) {  // its log_alpha/KF buffer is free: the gate tile of chunk n+2 (warp 3)
-                    if (GATE == 0 && warp == 3 && lane == 0) {
+                    if (GATE == 0 && warp == 3 && lane == 0 && m2) {
                         load_g(n + 2);
                         pf_g(n + 3);
                     }
@@ -650,9 +664,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 tmem_st_wait();
                 fence_proxy_async_smem();
                 tc_fence_before();
-                nb_arrive(NB_CHB, 96);
-                waitw(B_M1, (uint32_t)n);
-                if (warp == 2 && lane == 0 && n + 2 < NC) {  // the row buffer of this parity is free
+                // A full sync, not an arrive: warp 0 is already waiting here (it issued
+                // MMA1A before it, which the wait above needed), and after an abort, when
+                // the mbarrier waits are skipped, it keeps warps 2-3 from arriving for a
+                // later chunk before warp 0 syncs for this one (the barrier would count
+                // their arrivals into the wrong generation and warp 0 would wait forever).
+                nb_sync(NB_CHB, 96);
+                const bool m1 = waitw(B_M1, (uint32_t)n);
+                if (warp == 2 && lane == 0 && n + 2 < NC && m1) {  // the row buffer of this parity is free
                     load_kq(n + 2, B_KQ + rb);
                     pf_kq(n + 3);
                 }
@@ -706,7 +725,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 __syncwarp();
             }
         }
-        // ------------------------------------------------------------ final state S = e^{G_last - G_m} R
+        // ------------------------------------------------------------ final state S = Diag(ek) R
         if (NC > 0) waitw(B_M2, (uint32_t)(NC - 1));
         // one decision per warp: the tensor-memory loads below are warp-collective
         if (__shfl_sync(0xffffffffu, (stm && !*s_abort) ? 1 : 0, 0)) {
@@ -724,10 +743,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
         }
         if (quad >= 2 && lane == 0) bulk_wait0();  // every tensor store of O complete
-        if (issuer) {  // (chunk m's k/q load arms B_KQ + m % 2, its log_alpha load B_G + m % 3)
-            for (int x = 0; x < 2; ++x) drain(B_KQ + x, (NC - x + 1) / 2);
-            if (GATE == 0)
-                for (int x = 0; x < 3; ++x) drain(B_G + x, (NC - x + 2) / 3);
+        if (issuer) {  // after an abort: wait (bounded) for this thread's MMAs
             if (*s_abort) {
                 mma_commit(bars + B_FIN);
                 mbar_wait_bounded(bars + B_FIN, 0u, kDrainBudget);
@@ -750,7 +766,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         // the [A; P] MMA would have put them), plain tiles k e^G, q e^G, k e^{G_last-G}.
         auto exact_chunk = [&](int m, int s, int rb, int cb, int lim) {
             const uint32_t slotq = lane_addr + L::SLOT0 + 128 * s;
-            if (ttid == 0) load_kq(m, B_EXKQ);
+            if (ttid == 0 && !*s_abort) load_kq(m, B_EXKQ);
             waitw(B_EXKQ, (uint32_t)nex);
             if (m > 0) waitw(B_SCRF, (uint32_t)(m - 1));  // the inverse warps are done with the scratch
             float* stg = reinterpret_cast<float*>(sm + L::SCR);  // 16 KB: G of 64 channels, then A, then P
@@ -1026,8 +1042,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
             __syncwarp();
         }
-        if (ttid == 0) {
-            drain(B_EXKQ, nex);
+        if (ttid == 0) {  // after an abort: wait (bounded) for this thread's MMAs
             if (*s_abort) {
                 mma_commit(bars + B_FIN + 1);
                 mbar_wait_bounded(bars + B_FIN + 1, 0u, kDrainBudget);
@@ -1040,7 +1055,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const int iw = warp - kInvWarp0;  // 0..7
         const int hf = iw >> 2;           // which 32-column half of a readout this warp takes
         const int itid = tid - 32 * kInvWarp0;
-        int n_v = 0;
         auto load_beta = [&](int m) -> float {
             const int t = m * kC + itid;
             return (itid < kC && m < NC && t < seq_len) ? __bfloat162float(beta[(tok0 + t) * H + h]) : 0.f;
@@ -1263,7 +1277,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         };
         if (NC > 0 && itid == 0) {
             load_v(0);
-            ++n_v;
             pf_v(1);
         }
         float beta_next = load_beta(0);
@@ -1274,9 +1287,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             beta_next = load_beta(m + 1);
             waitw(B_AP + s, (uint32_t)(m / 3));
             if (m > 0 && itid == 0) {  // [T'; PT] and the v tile of the previous chunk are free
-                wait1(B_UO + (m - 1) % 3, (uint32_t)((m - 1) / 3));
-                load_v(m);
-                ++n_v;
+                if (wait1(B_UO + (m - 1) % 3, (uint32_t)((m - 1) / 3))) load_v(m);
                 pf_v(m + 1);
             }
             nb_sync(NB_INV, 256);  // beta of chunk m visible, [T'; PT] free
@@ -1325,8 +1336,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
             __syncwarp();
         }
-        if (itid == 0) {
-            drain(B_V, n_v);
+        if (itid == 0) {  // after an abort: wait (bounded) for this thread's MMAs
             if (*s_abort) {
                 mma_commit(bars + B_FIN + 2);
                 mbar_wait_bounded(bars + B_FIN + 2, 0u, kDrainBudget);
@@ -1336,6 +1346,26 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
+        // After an abort: wait (bounded) for the last phase armed on each copy
+        // barrier, so no tensor copy still writes shared memory when the CTA exits.
+        if (lane == 0 && *s_abort) {
+            // phases armed on each copy barrier: k/q of chunk j on B_KQ + j % 2,
+            // log_alpha on B_G + j % 3, v on B_V, exact-path reloads on B_EXKQ
+            int armed[7];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) armed[x] = s_issued[0] >= x ? (s_issued[0] - x) / 2 + 1 : 0;
+            if (sj.withhold_first_load && armed[0] > 0) --armed[0];
+#pragma unroll
+            for (int x = 0; x < 3; ++x) armed[2 + x] = s_issued[1] >= x ? (s_issued[1] - x) / 3 + 1 : 0;
+            armed[5] = s_issued[2] + 1;
+            armed[6] = s_issued[3];
+#pragma unroll
+            for (int i = 0; i < 7; ++i) {
+                const int bar = i < 5 ? B_KQ + i : (i == 5 ? B_V : B_EXKQ);
+                if (armed[i] > 0) mbar_wait_bounded(bars + bar, (uint32_t)(armed[i] - 1) & 1u, kDrainBudget);
+            }
+        }
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
     }
@@ -1494,19 +1524,22 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int scan_mode, cudaStream_t stre
     const int sms = sm_count();
     int P, L;
     scan_plan(a, scan_mode, &P, &L);
+    SegJobs one{};
+    one.withhold_first_load = a.test_withhold_first_load;
+    one.wait_budget = a.test_wait_budget;
     auto pick = [&](auto erase_c, auto gate_c) -> cudaError_t {
         constexpr int E = decltype(erase_c)::value, G = decltype(gate_c)::value;
         if (P == 0) {
             // One CTA per (batch, head) when there are enough heads to fill the
             // GPU; otherwise split the value channels in two.
             const bool wide = bh >= 96;
-            return wide ? launch_dvt<128, E, G>(a, stream, SegJobs{}, bh) : launch_dvt<64, E, G>(a, stream, SegJobs{}, bh);
+            return wide ? launch_dvt<128, E, G>(a, stream, one, bh) : launch_dvt<64, E, G>(a, stream, one, bh);
         }
         const size_t mat = (size_t)kD * kD;
         float* Mb = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + 256);
         float* Cb = Mb + (size_t)bh * (P - 2) * mat;
         float* Sin = Cb + (size_t)bh * (P - 2) * mat;
-        SegJobs sj{P, L, 1, Mb, Cb, Sin};
+        SegJobs sj{P, L, 1, Mb, Cb, Sin, one.withhold_first_load, one.wait_budget};
         cudaError_t e = launch_dvt<128, E, G>(a, stream, sj, bh * (2 * P - 3));
         if (e != cudaSuccess) return e;
         if (P > 2) {

@@ -24,6 +24,11 @@ struct ChunkArgs {
     const int* cu_seqlens;
     void* workspace;
     size_t workspace_bytes;
+    // Fault injection for the timeout test (tensor-core prefill only): withhold
+    // the first k/q load of every CTA and bound each wait by this many SM
+    // cycles, so the first wait expires. Zero in every other call.
+    int test_withhold_first_load = 0;
+    long long test_wait_budget = 0;
 };
 
 // Synchronous argument validation shared by every prefill entry point

@@ -87,6 +87,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     return true;
 }
 
+// The same, with the budget read from memory only once the first test fails
+// (keeps it out of registers across a long kernel).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, const volatile long long* budget) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const long long t0 = clock64(), b = *budget;
+    while (!mbar_try_wait_sleep(a, parity, 20000u)) {
+        if (clock64() - t0 > b) return false;
+    }
+    return true;
+}
+
 // ---------------------------------------------------------------- proxies / fences
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

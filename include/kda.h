@@ -243,6 +243,25 @@ kda_status_t kda_chunk_bwd_ex(const void *q, const void *k, const void *v, const
 kda_status_t kda_workspace_status(const void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Test hook for the timeout path above (no counterpart in the paper; not for
+ * production use). Takes the arguments of kda_chunk_fwd (KDA variant,
+ * algorithm KDA_ALGO_TC, T >= 1) plus wait_budget_cycles in [1, 2^31], and
+ * launches the tensor-core prefill with two faults injected: every CTA
+ * withholds its first k/q tile load, and every wait between warps gives up
+ * after wait_budget_cycles SM cycles instead of about one second. The first
+ * wait on that tile therefore expires; the kernel records KDA_ERR_TIMEOUT in
+ * the workspace, skips its later waits, waits (bounded) for the copies it did
+ * issue and returns. o and S_T are then undefined; kda_workspace_status
+ * reports KDA_ERR_TIMEOUT. A later normal call on the same stream and
+ * workspace is unaffected. Synchronous errors as kda_chunk_fwd_ex, plus
+ * KDA_ERR_INVALID_ARG for T = 0 or a budget out of range.
+ */
+kda_status_t kda_chunk_fwd_timeout_test(const void *q, const void *k, const void *v, const void *log_alpha,
+                                        const void *beta, const float *S0, void *o, float *S_T, int B, int T,
+                                        int H, int dk, int dv, int chunk, kda_dtype_t dtype, void *workspace,
+                                        size_t workspace_bytes, long long wait_budget_cycles, void *stream);
+
+/*
  * One recurrent decode step: kda_decode_step(q, k, v, log_alpha, beta, S -> o, S').
  *
  *   q, k, log_alpha : [N, H, dk]      dtype

@@ -100,6 +100,22 @@ def test_tc_path_rejects_shapes_it_does_not_cover():
     assert _chunk(lib, GOOD, dtype=1, dk=128, dv=128, chunk=32, algo=2) == 2
 
 
+def test_timeout_hook_rejects_bad_budget_and_shapes():
+    """The fault-injection hook checks its own arguments before any launch."""
+    lib = kda.load()
+    q, k, v, la, beta, S0, o, ST = GOOD
+
+    def hook(budget, T=64, dtype=1, dk=128):
+        return lib.kda_chunk_fwd_timeout_test(q, k, v, la, beta, S0, o, ST, 1, T, 1, dk, dk, 64, dtype, None, 0,
+                                              budget, None)
+
+    assert hook(0) == 1 and hook(-5) == 1 and hook((1 << 31) + 1) == 1   # budget out of range
+    assert hook(1 << 20, T=0) == 1                                       # nothing to withhold
+    assert hook(1 << 20, dtype=0) == 2                                   # fp32: no tensor-core kernel
+    assert hook(1 << 20, dk=64) == 2
+    assert hook(1 << 20) == 1                                            # no workspace
+
+
 def test_workspace_size_is_host_only():
     lib = kda.load()
     assert lib.kda_chunk_fwd_workspace_size(1, 16, 1, 64, 64, 64, 0, 1) == 0   # SIMT needs none
