@@ -500,7 +500,7 @@ def time_widened(args, ctx, kda, I, pf, peaks):
     if "exact_path" in args.parts:
         out["exact_path"] = _time_exact_path(args, ctx, kda, pf, steps, hbm)
     if "long_context" in args.parts:
-        out["long_context"] = _time_long_context(ctx, kda, I, hbm)
+        out["long_context"] = _time_long_context(ctx, kda, I, hbm, args.long_T)
     if "backward" in args.parts:
         out["backward"] = _time_backward(ctx, kda, pf, hbm)
     if pf.use_tc and kda.workspace_status(pf.ws, ctx.stream) != 0:
@@ -607,10 +607,12 @@ def _time_exact_path(args, ctx, kda, pf, steps, hbm):
             "ms_per_step": ms, "steps": 3, "roofline_frac": gbs / hbm, "achieved_gbs": gbs}
 
 
-def _time_long_context(ctx, kda, I, hbm):
-    """B1 H32 T131072: one pass per sequence against the segment scan."""
+def _time_long_context(ctx, kda, I, hbm, T=None):
+    """B1 H32 T131072: one pass per sequence against the segment scan. T
+    shortens the sequence for profiler captures (the same grid and segment
+    count for T >= 16384)."""
     torch = ctx.torch
-    lc = I.B1_H32_T128K
+    lc = I.B1_H32_T128K if not T else I.B1_H32_T128K.replace(T=T, name=f"{I.B1_H32_T128K.name}_profile_T{T}")
     g = torch.Generator(device=ctx.dev)
     g.manual_seed(lc.seed + 1000 * ctx.rank)
     shp = (lc.B, lc.T, lc.H)
@@ -683,6 +685,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-T", type=int, default=None,
                     help="shorter sequence for profiler captures (the printed line is then not a bench value)")
+    ap.add_argument("--long-T", type=int, default=None,
+                    help="shorter sequence for the long-context leg (profiler captures; not a bench value)")
     ap.add_argument("--parts", default="prefill,e2e,decode,widened",
                     help="comma list of prefill, e2e, decode, widened (= varlen, variants, b2_h16_t4k, exact_path, long_context, "
                          "backward) (profiling runs select one)")

@@ -50,10 +50,12 @@
 //   tile  (warps 4-7)   prefix sums out of tensor memory, KE/QE in place over
 //                       the raw k/q rows, KF over the log_alpha tile, the
 //                       overflow vote, per-channel scales; issues the [A; P]
-//                       MMA and the next chunk's prefix-sum MMA.
-//   inverse (warps 8-15) A/P readout, (I + A)^{-1} -> T', the PT, W and U
-//                       MMAs and their readouts into the row operand; issues
-//                       the v loads.
+//                       MMA, reads A (beta-scaled, fp32) and P (bf16) out of
+//                       tensor memory, then issues the next chunk's prefix-sum
+//                       MMA.
+//   inverse (warps 8-15) (I + A)^{-1} -> T', the PT, W and U MMAs and their
+//                       readouts into the row operand; issues the v loads and
+//                       stores beta a chunk ahead.
 // k/q tiles are double-buffered, the log_alpha/KF tiles triple-buffered, the
 // per-channel scales kept by chunk mod 4.
 // (I + A)^{-1}: 16x16 diagonal blocks by forward substitution (four threads per
@@ -115,8 +117,8 @@ struct Layout {
     static constexpr uint32_t STD = SCR + 64 * kLDA * 4;
     static constexpr uint32_t SCR_BYTES = 64 * kLDA * 4 + 4 * 16 * kLDT * 4;
     static constexpr uint32_t SMALL = SCR + SCR_BYTES;
-    static constexpr uint32_t SBETA = SMALL;        // 64 f32: beta of the inverse warps' chunk
-    static constexpr uint32_t SOPS = SBETA + 256;   // 4 x 128 f32: operand scale per channel (by chunk mod 4)
+    static constexpr uint32_t SBETA = SMALL;        // 2 x 64 f32: beta of the chunk (by parity)
+    static constexpr uint32_t SOPS = SBETA + 512;   // 4 x 128 f32: operand scale per channel (by chunk mod 4)
     static constexpr uint32_t STMS = SOPS + 2048;   // 4 x 128 f32: tensor-memory scale per channel
     static constexpr uint32_t SEK = STMS + 2048;    // 128 f32: pending state factor after the last prepared chunk
     static constexpr uint32_t SGL = SEK + 512;      // 128 f32: G_last
@@ -153,7 +155,8 @@ enum : int {
     B_SCRF = 31,  // A/T scratch of the inverse warps' chunk free
     B_EXKQ = 32,  // k/q reloaded for an exact chunk
     B_FIN = 33,   // 3: final drain of each MMA-issuing thread
-    NUM_BARS = 36
+    B_AR = 36,    // A (fp32 scratch) and P (bf16 tile) of the chunk read out of tensor memory
+    NUM_BARS = 37
 };
 
 // offset of element (row R, channel c) of a row-operand buffer (K-major, two
@@ -356,6 +359,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (v_zero)  // transition run: v = 0 stays in the v tile, which is never loaded
             for (int i = tid; i < (DVT / 64) * 8192 / 16; i += kThreads) st_shared_v4(sb + L::RAWV + 16 * i, 0u, 0u, 0u, 0u);
     }
+    if (tid < kC)  // beta of chunk 0 (later chunks: the inverse warps, a chunk ahead)
+        sBeta[tid] = tid < seq_len ? __bfloat162float(beta[(tok0 + tid) * H + h]) : 0.f;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -905,6 +910,59 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
             ++nex;
         };
+        // A/P of chunk m out of the slot: A (rows 0-63, scaled by beta_r, strictly
+        // lower) into the fp32 scratch, P (rows 64-127, lower incl.) into the bf16
+        // K-major tile. The scratch is free once the inverse warps finished the
+        // previous chunk's inverse, the P tile once its PT MMA completed.
+        auto readout_ap = [&](int m, int s) {
+            const uint32_t slotq = lane_addr + L::SLOT0 + 128 * s;
+            if (m > 0) waitw(quad < 2 ? B_SCRF : B_PT, (uint32_t)(m - 1));
+            waitw(B_AP + s, (uint32_t)(m / 3));
+            if (quad < 2) {
+                if (erase) {
+                    const int r = 32 * quad + lane;
+                    // (the inverse warps stored this chunk's beta before the scratch-free arrive)
+                    const float br = sBeta[(m & 1) * 64 + r];
+#pragma unroll 1
+                    for (int e8 = 0; e8 < 8; ++e8) {
+                        uint32_t v[8];
+                        tmem_ld8(slotq + 8 * e8, v);
+                        tmem_ld_wait(v);
+                        float* dst = sA + r * kLDA + 8 * e8;
+#pragma unroll
+                        for (int u = 0; u < 8; u += 4) {
+                            float4 f;
+                            f.x = (8 * e8 + u + 0 < r) ? br * __uint_as_float(v[u + 0]) : 0.f;
+                            f.y = (8 * e8 + u + 1 < r) ? br * __uint_as_float(v[u + 1]) : 0.f;
+                            f.z = (8 * e8 + u + 2 < r) ? br * __uint_as_float(v[u + 2]) : 0.f;
+                            f.w = (8 * e8 + u + 3 < r) ? br * __uint_as_float(v[u + 3]) : 0.f;
+                            *reinterpret_cast<float4*>(dst + u) = f;
+                        }
+                    }
+                }
+            } else {
+                const int r = 32 * (quad - 2) + lane;
+#pragma unroll 1
+                for (int jc = 0; jc < 8; ++jc) {
+                    uint32_t v[8];
+                    tmem_ld8(slotq + 8 * jc, v);
+                    tmem_ld_wait(v);
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int c = 8 * jc + 2 * u;
+                        const float p0 = (c <= r) ? __uint_as_float(v[2 * u]) : 0.f;
+                        const float p1 = (c + 1 <= r) ? __uint_as_float(v[2 * u + 1]) : 0.f;
+                        w[u] = pack_bf16x2(p0, p1);
+                    }
+                    st_shared_v4(sb + L::SP + r * 128 + ((jc ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            nb_sync(NB_TILE, 128);
+            if (ttid == 0) mbar_arrive(bars + B_AR);
+        };
         for (int m = 0; m < NC; ++m) {
             const int s = m % 3, rb = m & 1, cb = m % 3;
             const uint32_t slotq = lane_addr + L::SLOT0 + 128 * s;
@@ -1032,13 +1090,15 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                                     dadd(dCOLK, cb * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32), ID_AP, kk > 0);
                 }
                 mma_commit(bars + B_AP + s);
-                if (m + 1 < NC) {  // next chunk's prefix sums, once its slot is read out and its gate is in place
-                    const int s1 = (m + 1) % 3;
-                    if (m + 1 >= 3) wait1(B_SF + s1, (uint32_t)((m + 1) / 3 - 1));
-                    if (GATE != 2) wait1(B_G + s1, (uint32_t)((m + 1) / 3));
-                    tc_fence_after();
-                    cumsum_mma(m + 1);
-                }
+            }
+            __syncwarp();
+            readout_ap(m, s);
+            if (ttid == 0 && m + 1 < NC) {  // next chunk's prefix sums, once its slot is read out and its gate is in place
+                const int s1 = (m + 1) % 3;
+                if (m + 1 >= 3) wait1(B_SF + s1, (uint32_t)((m + 1) / 3 - 1));
+                if (GATE != 2) wait1(B_G + s1, (uint32_t)((m + 1) / 3));
+                tc_fence_after();
+                cumsum_mma(m + 1);
             }
             __syncwarp();
         }
@@ -1059,46 +1119,20 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const int t = m * kC + itid;
             return (itid < kC && m < NC && t < seq_len) ? __bfloat162float(beta[(tok0 + t) * H + h]) : 0.f;
         };
-        // ---- A (slot rows 0-63) -> fp32 scratch (beta_r, strictly lower); P (rows 64-127) -> bf16 K-major tile (lower incl.)
-        auto p4 = [&](uint32_t slot) {
-            if (quad < 2 && !erase) return;  // additive write: A is not used
-            uint32_t v[32];
-            tmem_ld32(slot + 32 * hf, v);
-            tmem_ld_wait(v);
-            if (quad < 2) {
-                const int r = 32 * quad + lane;
-                const float br = sBeta[r];
-                float* dst = sA + r * kLDA + 32 * hf;
-#pragma unroll
-                for (int u = 0; u < 32; u += 4) {
-                    float4 f;
-                    f.x = (32 * hf + u + 0 < r) ? br * __uint_as_float(v[u + 0]) : 0.f;
-                    f.y = (32 * hf + u + 1 < r) ? br * __uint_as_float(v[u + 1]) : 0.f;
-                    f.z = (32 * hf + u + 2 < r) ? br * __uint_as_float(v[u + 2]) : 0.f;
-                    f.w = (32 * hf + u + 3 < r) ? br * __uint_as_float(v[u + 3]) : 0.f;
-                    *reinterpret_cast<float4*>(dst + u) = f;
-                }
-            } else {
-                const int r = 32 * (quad - 2) + lane;
-#pragma unroll
-                for (int jc = 0; jc < 4; ++jc) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int s = 32 * hf + 8 * jc + 2 * u;
-                        const float p0 = (s <= r) ? __uint_as_float(v[8 * jc + 2 * u]) : 0.f;
-                        const float p1 = (s + 1 <= r) ? __uint_as_float(v[8 * jc + 2 * u + 1]) : 0.f;
-                        w[u] = pack_bf16x2(p0, p1);
-                    }
-                    st_shared_v4(sb + L::SP + r * 128 + (((4 * hf + jc) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
-                }
+        const float* sBm = sBeta;  // beta of the chunk in work (parity buffer)
+        // [T'; PT] and the v tile are free once the previous chunk's U MMA completed;
+        // then the v tile of chunk m is loaded (one thread)
+        auto tp_free = [&](int m) {
+            if (m > 0) {
+                if (wait1(B_UO + (m - 1) % 3, (uint32_t)((m - 1) / 3))) load_v(m);
+                pf_v(m + 1);
             }
         };
         // ---- P5: T = (I + A)^{-1} -> T' = T Diag(beta), bf16, rows 0-63 of [T'; PT]
         auto store_tprime = [&](int r, int s, float t) {
-            *reinterpret_cast<__nv_bfloat16*>(sm + L::TP + km_off(r, s)) = __float2bfloat16_rn(t * sBeta[s]);
+            *reinterpret_cast<__nv_bfloat16*>(sm + L::TP + km_off(r, s)) = __float2bfloat16_rn(t * sBm[s]);
         };
-        auto p5 = [&]() {
+        auto p5 = [&](int m) {
             if (!erase) {  // A = 0: T = I, T' = Diag(beta); thread: row itid/4, 16 columns
                 const int r = itid >> 2, j0c = 2 * (itid & 3);
 #pragma unroll
@@ -1108,16 +1142,18 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int s0 = 8 * j + 2 * u;
-                        w[u] = pack_bf16x2(s0 == r ? sBeta[r] : 0.f, s0 + 1 == r ? sBeta[r] : 0.f);
+                        w[u] = pack_bf16x2(s0 == r ? sBm[r] : 0.f, s0 + 1 == r ? sBm[r] : 0.f);
                     }
                     st_shared_v4(sb + L::TP + r * 128 + ((j ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
                 }
                 return;
             }
-            {   // diagonal 16x16 blocks: four threads per column, rows q, q+4, q+8, q+12
-                const int a = itid >> 6, jc = (itid >> 2) & 15, q = itid & 3;
+            // diagonal 16x16 blocks: four threads per column, rows q, q+4, q+8, q+12
+            const int a = itid >> 6, jc = (itid >> 2) & 15, q = itid & 3;
+            float colv[4] = {0.f, 0.f, 0.f, 0.f};
+            {
                 const float* Ab = sA + (16 * a) * kLDA + 16 * a;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f}, colv[4] = {0.f, 0.f, 0.f, 0.f};
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
                     const float mine = (r == jc) ? 1.f : ((r > jc) ? -acc[r >> 2] : 0.f);
@@ -1128,13 +1164,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         if (q + 4 * i > r) acc[i] = fmaf(Ab[(q + 4 * i) * kLDA + r], t, acc[i]);
                 }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = q + 4 * i;  // row inside the block
-                    sTd[(a * 16 + r) * kLDT + jc] = colv[i];
-                    store_tprime(16 * a + r, 16 * a + jc, colv[i]);
-                }
+                for (int i = 0; i < 4; ++i) sTd[(a * 16 + q + 4 * i) * kLDT + jc] = colv[i];
             }
+            // [T'; PT] is free once the previous chunk's U MMA has read it (waited
+            // here, after the diagonal blocks, which do not touch it)
+            if (itid == 0) tp_free(m);
             nb_sync(NB_INV, 256);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) store_tprime(16 * a + q + 4 * i, 16 * a + jc, colv[i]);
             // Blocks below the diagonal, one column chain per warp (block column
             // bb, 8-column half nt), held in registers: for a = bb+1..3,
             // X = sum_{k=bb}^{a-1} A_ak T_kb, then T_ab = -T_aa X, on m16n8k8 tf32
@@ -1204,7 +1241,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh)
                         *reinterpret_cast<uint32_t*>(sm + L::TP + km_off(16 * a + g + 8 * hh, s0)) =
-                            pack_bf16x2(y[2 * hh] * sBeta[s0], y[2 * hh + 1] * sBeta[s0 + 1]);
+                            pack_bf16x2(y[2 * hh] * sBm[s0], y[2 * hh + 1] * sBm[s0 + 1]);
                     if (da < 3 && a < 3) c2b(y, tb[da]);
                 }
             }
@@ -1279,21 +1316,22 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             load_v(0);
             pf_v(1);
         }
-        float beta_next = load_beta(0);
+        // beta of chunk m + 1 goes into its parity buffer at the start of chunk m:
+        // the tile warps read it for their A readout after the scratch-free
+        // arrive of chunk m (chunk 0's was stored during setup)
+        float beta_next = load_beta(1);
         for (int m = 0; m < NC; ++m) {
             const int s = m % 3, rb = m & 1;
             const uint32_t slot = lane_addr + L::SLOT0 + 128 * s;
-            if (itid < kC) sBeta[itid] = beta_next;
-            beta_next = load_beta(m + 1);
-            waitw(B_AP + s, (uint32_t)(m / 3));
-            if (m > 0 && itid == 0) {  // [T'; PT] and the v tile of the previous chunk are free
-                if (wait1(B_UO + (m - 1) % 3, (uint32_t)((m - 1) / 3))) load_v(m);
-                pf_v(m + 1);
+            sBm = sBeta + (m & 1) * 64;
+            if (itid < kC) sBeta[((m + 1) & 1) * 64 + itid] = beta_next;
+            beta_next = load_beta(m + 2);
+            waitw(B_AR, (uint32_t)m);  // A and P of chunk m in shared memory
+            if (!erase) {  // T' = Diag(beta) goes straight into [T'; PT]
+                if (itid == 0) tp_free(m);
+                nb_sync(NB_INV, 256);
             }
-            nb_sync(NB_INV, 256);  // beta of chunk m visible, [T'; PT] free
-            p4(slot);
-            nb_sync(NB_INV, 256);
-            p5();
+            p5(m);
             fence_proxy_async_smem();
             tc_fence_before();
             nb_sync(NB_INV, 256);
