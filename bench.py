@@ -586,25 +586,31 @@ def _time_b2_h16(ctx, kda, I, hbm):
 
 
 def _time_exact_path(args, ctx, kda, pf, steps, hbm):
-    """The B4 H32 T8192 shapes with a decay of -U(1.5, 3) per token and channel:
-    every full chunk then fails the overflow vote of the reference-point
-    factorisation and takes the exact per-pair path."""
+    """The B4 H32 T8192 shapes with decays too strong for the chunk-start
+    reference point (|G| > 80 within a chunk): -U(1.5, 3) per token and
+    channel (about 144 per chunk, the G_last / 2 reference takes the chunks)
+    and -U(3, 6) (about 288 per chunk, the exact per-pair path)."""
     torch = ctx.torch
     x, cfg = pf.x, pf.cfg
-    g = torch.Generator(device=ctx.dev)
-    g.manual_seed(cfg.seed + 555 + 1000 * ctx.rank)
-    la = (-(1.5 + 1.5 * torch.rand(cfg.B, cfg.T, cfg.H, cfg.dk, device=ctx.dev, generator=g))).bfloat16()
-
-    def run_e():
-        kda.chunk_fwd(x["q"], x["k"], x["v"], la, x["beta"], x["S0"], chunk=cfg.C, algo=pf.algo, o=pf.o,
-                      S_T=pf.ST, workspace=pf.ws if pf.ws_bytes else None, stream=ctx.stream)
-    ms = _time_calls(ctx, run_e, 3, 3)
     ntok = cfg.B * cfg.T
     nbytes = BYTES_PER_TOKEN_HEAD * ntok * cfg.H + pf.ST.numel() * 4
-    gbs = nbytes / (ms * 1e-3) / 1e9
-    del la
-    return {"workload": cfg.name + "_decay_U1.5_3", "value": ctx.world * ntok / (ms * 1e-3), "unit": "tokens/s",
-            "ms_per_step": ms, "steps": 3, "roofline_frac": gbs / hbm, "achieved_gbs": gbs}
+    out = {}
+    for key, lo, hi, path in (("mid_reference", 1.5, 3.0, "reference point G_last / 2"),
+                              ("exact", 3.0, 6.0, "exact per-pair exponentials")):
+        g = torch.Generator(device=ctx.dev)
+        g.manual_seed(cfg.seed + 555 + 1000 * ctx.rank)
+        la = (-(lo + (hi - lo) * torch.rand(cfg.B, cfg.T, cfg.H, cfg.dk, device=ctx.dev, generator=g))).bfloat16()
+
+        def run_e():
+            kda.chunk_fwd(x["q"], x["k"], x["v"], la, x["beta"], x["S0"], chunk=cfg.C, algo=pf.algo, o=pf.o,
+                          S_T=pf.ST, workspace=pf.ws if pf.ws_bytes else None, stream=ctx.stream)
+        ms = _time_calls(ctx, run_e, 3, 3)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        del la
+        out[key] = {"workload": f"{cfg.name}_decay_U{lo:g}_{hi:g}", "path": path,
+                    "value": ctx.world * ntok / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": 3,
+                    "roofline_frac": gbs / hbm, "achieved_gbs": gbs}
+    return out
 
 
 def _time_long_context(ctx, kda, I, hbm, T=None):

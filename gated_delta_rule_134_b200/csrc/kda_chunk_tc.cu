@@ -33,9 +33,13 @@
 // lazily, when the next chunk copies the state into the bf16 MMA operand (and
 // when the final state is written). Each factor is a single exponential,
 // finite as long as |G_r| <= 80; a vote of the tile warps checks that per
-// chunk. A chunk that fails it uses exact per-pair exponentials e^{G_r - G_s}
-// (exponent <= 0) for A and P and the plain tiles k e^G, q e^G,
-// k e^{G_last-G}; the same MMAs then produce the same quantities.
+// chunk. A chunk that fails it tries the reference point G_m = G_last / 2
+// (E = e^{G - G_m}, F = e^{G_m - G}, the state operand e^{G_m} S), which holds
+// while |G_r - G_m| <= 80, i.e. a decay of up to 160 over the chunk: the raw
+// k/q rows are reloaded and the tiles rebuilt. A chunk that fails that too
+// uses exact per-pair exponentials e^{G_r - G_s} (exponent <= 0) for A and P
+// and the plain tiles k e^G, q e^G, k e^{G_last-G}; the same MMAs then produce
+// the same quantities.
 //
 // Schedule. One CTA owns one (batch, head) and a DVT-wide slice of value
 // channels; its state stays in tensor memory for the whole sequence. Each
@@ -120,7 +124,8 @@ struct Layout {
     static constexpr uint32_t SBETA = SMALL;        // 2 x 64 f32: beta of the chunk (by parity)
     static constexpr uint32_t SOPS = SBETA + 512;   // 4 x 128 f32: operand scale per channel (by chunk mod 4)
     static constexpr uint32_t STMS = SOPS + 2048;   // 4 x 128 f32: tensor-memory scale per channel
-    static constexpr uint32_t SEK = STMS + 2048;    // 128 f32: pending state factor after the last prepared chunk
+    static constexpr uint32_t SMDS = STMS + 2048;   // 4 x 128 f32: second factor of both (middle tier, else 1)
+    static constexpr uint32_t SEK = SMDS + 2048;    // 128 f32: pending state factor after the last prepared chunk
     static constexpr uint32_t SGL = SEK + 512;      // 128 f32: G_last
     static constexpr uint32_t BARS = SGL + 512;     // mbarriers
     static constexpr uint32_t MISC = BARS + 512;    // tmem base, abort flag, copies issued, wait budget
@@ -310,6 +315,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     float* sBeta = reinterpret_cast<float*>(sm + L::SBETA);
     float* sOpS = reinterpret_cast<float*>(sm + L::SOPS);
     float* sTmS = reinterpret_cast<float*>(sm + L::STMS);
+    float* sMdS = reinterpret_cast<float*>(sm + L::SMDS);
     float* sEK = reinterpret_cast<float*>(sm + L::SEK);
     float* sGl = reinterpret_cast<float*>(sm + L::SGL);
     float* sA = reinterpret_cast<float*>(sm + L::SA);
@@ -535,15 +541,17 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
         // s1 body for one 32-column group: state rows -> bf16 operand words (times
         // the operand scale), R *= tensor-memory scale
-        auto s1_group = [&](int gq, float os, float ts, uint32_t (&pk)[16]) {
+        auto s1_group = [&](int gq, float os, float ts, float ms, uint32_t (&pk)[16]) {
             uint32_t v[32];
             tmem_ld32(lane_addr + L::S_COL + 32 * gq, v);
             tmem_ld_wait(v);
-            if (os == ts) {  // (every factored chunk) the operand is the rescaled state itself
+            if (os == ts) {  // (every factored chunk) the operand is the rescaled state itself;
+                             // two factors, so that their product may lie below the fp32 range
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     float x0, x1;
                     mul_f32x2(x0, x1, __uint_as_float(v[2 * u]), __uint_as_float(v[2 * u + 1]), ts, ts);
+                    mul_f32x2(x0, x1, x0, x1, ms, ms);
                     v[2 * u] = __float_as_uint(x0);
                     v[2 * u + 1] = __float_as_uint(x1);
                     pk[u] = pack_bf16x2(x0, x1);
@@ -588,12 +596,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
             }
             waitw(B_SC + (n & 3), (uint32_t)(n >> 2));
-            const float os = sOpS[(n & 3) * 128 + row], ts = sTmS[(n & 3) * 128 + row];
+            const float os = sOpS[(n & 3) * 128 + row], ts = sTmS[(n & 3) * 128 + row], ms = sMdS[(n & 3) * 128 + row];
             if (quad < 2) {
 #pragma unroll 1
                 for (int gq = 0; gq < DVT / 32; ++gq) {  // key channels 0-63
                     uint32_t pk[16];
-                    s1_group(gq, os, ts, pk);
+                    s1_group(gq, os, ts, ms, pk);
                     sop_store(row, gq, pk);
                 }
                 tmem_st_wait();
@@ -656,14 +664,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 constexpr int kStaged = DVT / 64;
                 uint32_t pk[kStaged][16];
 #pragma unroll
-                for (int gq = 0; gq < kStaged; ++gq) s1_group(gq, os, ts, pk[gq]);
+                for (int gq = 0; gq < kStaged; ++gq) s1_group(gq, os, ts, ms, pk[gq]);
                 waitw(B_M1A, (uint32_t)n);  // first half of the state operand consumed
 #pragma unroll
                 for (int gq = 0; gq < kStaged; ++gq) sop_store(row - 64, gq, pk[gq]);
 #pragma unroll 1
                 for (int gq = kStaged; gq < DVT / 32; ++gq) {
                     uint32_t pq[16];
-                    s1_group(gq, os, ts, pq);
+                    s1_group(gq, os, ts, ms, pq);
                     sop_store(row - 64, gq, pq);
                 }
                 tmem_st_wait();
@@ -769,8 +777,95 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         // Exact path of a chunk that fails the vote: reload the raw k/q rows, per-pair
         // exponentials for A and P (raw sums, staged and stored into the slot where
         // the [A; P] MMA would have put them), plain tiles k e^G, q e^G, k e^{G_last-G}.
+        // Middle tier for a chunk whose decay is too strong for the chunk-start
+        // reference (some |G_r| > 80): reference point G_m = G_last / 2 per channel,
+        // E = e^{G - G_m}, F = e^{G_m - G}. With a decay (G falling from 0 to G_last)
+        // every exponent is within |G_last| / 2, so it holds up to |G_last| = 160;
+        // the vote checks it. Returns false (nothing changed) when it does not
+        // hold; otherwise the raw k/q rows are reloaded and the tiles rebuilt.
+        auto mid_chunk = [&](int m, int s, int rb, int cb, int lim) -> bool {
+            const uint32_t slotq = lane_addr + L::SLOT0 + 128 * s;
+            const bool live = tok < lim;
+            float amax = 0.f;
+            if (GATE == 0) {
+#pragma unroll 1
+                for (int u8 = 0; u8 < 8; ++u8) {
+                    const int c0 = ch0 + 8 * u8;
+                    uint32_t g8[8];
+                    tmem_ld8(slotq + c0, g8);
+                    tmem_ld_wait(g8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        amax = fmaxf(amax, fabsf((__uint_as_float(g8[e]) - 0.5f * sGl[c0 + e]) * kLog2e));
+                }
+            } else {
+                uint32_t g1;
+                tmem_ld1(slotq, g1);
+                tmem_ld_wait1(g1);
+                amax = fabsf((__uint_as_float(g1) - 0.5f * sGl[0]) * kLog2e);
+            }
+            if (nb_or(NB_TOR, 128, live && !(amax <= kGuardL))) return false;
+            // reload the raw k/q rows over the tiles just written (their stores are
+            // ordered before the copy by the proxy fence and the barrier)
+            fence_proxy_async_smem();
+            nb_sync(NB_TILE, 128);
+            if (ttid == 0 && !*s_abort) load_kq(m, B_EXKQ);
+            waitw(B_EXKQ, (uint32_t)nex);
+            ++nex;
+            const uint32_t rop = sb + L::ROW + rb * 32768;
+            const uint32_t colp = sb + L::COL + cb * 16384;
+            const uint32_t km = live ? 0xFFFFFFFFu : 0u;
+            uint32_t ep1 = 0, fp1 = 0;
+            if (GATE == 1) {
+                uint32_t g1;
+                tmem_ld1(slotq, g1);
+                tmem_ld_wait1(g1);
+                const float a = (__uint_as_float(g1) - 0.5f * sGl[0]) * kLog2e;
+                ep1 = pack_bf16x2(ex2(a), ex2(a));
+                fp1 = pack_bf16x2(ex2(-a), ex2(-a));
+            }
+#pragma unroll 1
+            for (int u8 = 0; u8 < 8; ++u8) {
+                const int c0 = ch0 + 8 * u8;
+                const uint32_t ko = rop_off(tok, c0);
+                const uint32_t fo = (uint32_t)((c0 >> 6) * 8192 + tok * 128 + ((((c0 & 63) >> 3) ^ (tok & 7)) << 4));
+                const uint4 kv = ld_shared_v4(rop + ko);
+                const uint4 qv = ld_shared_v4(rop + ko + 8192);
+                const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+                const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                uint32_t ke[4], qe[4], kf[4];
+                if (GATE == 0) {
+                    uint32_t g8[8];
+                    tmem_ld8(slotq + c0, g8);
+                    tmem_ld_wait(g8);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float a0 = (__uint_as_float(g8[2 * u]) - 0.5f * sGl[c0 + 2 * u]) * kLog2e;
+                        const float a1 = (__uint_as_float(g8[2 * u + 1]) - 0.5f * sGl[c0 + 2 * u + 1]) * kLog2e;
+                        const uint32_t ep = pack_bf16x2(ex2(a0), ex2(a1));
+                        const uint32_t fp = pack_bf16x2(ex2(-a0), ex2(-a1));
+                        ke[u] = hmul2_bf16(kw[u], ep) & km;
+                        qe[u] = hmul2_bf16(qw[u], ep) & km;
+                        kf[u] = hmul2_bf16(kw[u], fp) & km;
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        ke[u] = hmul2_bf16(kw[u], ep1) & km;
+                        qe[u] = hmul2_bf16(qw[u], ep1) & km;
+                        kf[u] = hmul2_bf16(kw[u], fp1) & km;
+                    }
+                }
+                st_shared_v4(rop + ko, ke[0], ke[1], ke[2], ke[3]);
+                st_shared_v4(rop + ko + 8192, qe[0], qe[1], qe[2], qe[3]);
+                st_shared_v4(colp + fo, kf[0], kf[1], kf[2], kf[3]);
+            }
+            return true;
+        };
         auto exact_chunk = [&](int m, int s, int rb, int cb, int lim) {
             const uint32_t slotq = lane_addr + L::SLOT0 + 128 * s;
+            fence_proxy_async_smem();  // (as in the middle tier: tile stores before the copy)
+            nb_sync(NB_TILE, 128);
             if (ttid == 0 && !*s_abort) load_kq(m, B_EXKQ);
             waitw(B_EXKQ, (uint32_t)nex);
             if (m > 0) waitw(B_SCRF, (uint32_t)(m - 1));  // the inverse warps are done with the scratch
@@ -1059,7 +1154,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
             // every factor finite and normal? (NaN counts as a failure); the vote also
             // makes G_last visible to every tile thread
-            const bool exact = GATE != 2 && nb_or(NB_TOR, 128, live && !(amax <= kGuardL));
+            const bool failed = GATE != 2 && nb_or(NB_TOR, 128, live && !(amax <= kGuardL));
+            // 0: reference at the chunk start, 1: at G_last / 2, 2: exact per-pair path
+            const int tier = !failed ? 0 : (mid_chunk(m, s, rb, cb, lim) ? 1 : 2);
+            const bool exact = tier == 2;
             if (exact) exact_chunk(m, s, rb, cb, lim);
             {   // per-channel scales of this chunk. The tensor memory holds R with
                 // S = Diag(ek) R; the chain feeds S^ = Diag(os) R to MMA1 and keeps
@@ -1068,12 +1166,23 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 const float g_l = GATE == 0 ? sGl[c] : (GATE == 1 ? sGl[0] : 0.f);
                 const float ek_prev = sEK[c];
                 const int slot4 = m & 3;
-                sOpS[slot4 * 128 + c] = ek_prev;
-                if (!exact) {  // reference at the chunk start: S^ = S, KF = k e^{-G}
+                if (tier == 0) {         // reference at the chunk start: S^ = S, KF = k e^{-G}
+                    sOpS[slot4 * 128 + c] = ek_prev;
                     sTmS[slot4 * 128 + c] = ek_prev;
+                    sMdS[slot4 * 128 + c] = 1.f;
                     sEK[c] = __expf(g_l);
-                } else {       // KF = k e^{G_last - G}
+                } else if (tier == 1) {  // S^ = e^{G_m} S, KF = k e^{G_m - G}, G_m = G_last / 2
+                    // (ek_prev e^{G_m} can lie below the fp32 range while the state it
+                    // scales does not: the chain applies the two factors one after the other)
+                    const float em = __expf(0.5f * g_l);
+                    sOpS[slot4 * 128 + c] = ek_prev;
+                    sTmS[slot4 * 128 + c] = ek_prev;
+                    sMdS[slot4 * 128 + c] = em;
+                    sEK[c] = em;
+                } else {                 // exact: KF = k e^{G_last - G}
+                    sOpS[slot4 * 128 + c] = ek_prev;
                     sTmS[slot4 * 128 + c] = __expf(g_l) * ek_prev;
+                    sMdS[slot4 * 128 + c] = 1.f;
                     sEK[c] = 1.f;
                 }
             }

@@ -86,6 +86,14 @@ def test_prefill_decay_extremes(cuda_lib, algo, la):
     check_prefill(cuda_lib, small_cfg("bf16", 128, 64, 200, la=la), algo)
 
 
+@pytest.mark.parametrize("la", [(1.0, 2.0), (1.5, 3.0)])
+def test_prefill_tc_mid_reference_tier(cuda_lib, la):
+    # a decay of 64-190 per chunk: the chunk-start reference fails its guard, the
+    # G_last / 2 reference takes chunks up to 160 (stronger ones: the exact path);
+    # ragged tail, entry state
+    check_prefill(cuda_lib, small_cfg("bf16", 128, 64, 333, la=la, seed=37), "tc")
+
+
 @pytest.mark.parametrize("algo", ["simt", "tc"])
 def test_prefill_many_heads_small(cuda_lib, algo):
     # more (b, h) pairs than SMs, ragged tail
@@ -296,6 +304,12 @@ def test_prefill_variants_f32(cuda_lib, erase, gate):
 def test_prefill_variants_tc_extreme_decay(cuda_lib, erase, gate):
     # decays up to e^-6 per token: the guard sends chunks down the exact path
     check_variant(cuda_lib, small_cfg("bf16", 128, 64, 150, la=(0.5, 6.0), seed=33), "tc", erase, gate)
+
+
+@pytest.mark.parametrize("erase,gate", VARIANTS)
+def test_prefill_variants_tc_mid_reference_tier(cuda_lib, erase, gate):
+    # decays of 64-128 per chunk: every full chunk takes the G_last / 2 reference
+    check_variant(cuda_lib, small_cfg("bf16", 128, 64, 333, la=(1.0, 2.0), seed=38), "tc", erase, gate)
 
 
 @pytest.mark.parametrize("erase,gate", VARIANTS)
