@@ -691,6 +691,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-T", type=int, default=None,
                     help="shorter sequence for profiler captures (the printed line is then not a bench value)")
+    ap.add_argument("--e2e-pieces", type=int, default=4,
+                    help="pieces per sequence in the end-to-end pipeline (whole chunks each)")
     ap.add_argument("--long-T", type=int, default=None,
                     help="shorter sequence for the long-context leg (profiler captures; not a bench value)")
     ap.add_argument("--parts", default="prefill,e2e,decode,widened",
@@ -728,7 +730,7 @@ def main():
             line.update(value=whole_job_rate(ctx.world, pf.tokens_per_step, ms), ms_per_step=ms, roofline=roof,
                         clocks=clocks, gpu_launches=pf.launches_per_step * args.steps)
         if "e2e" in args.parts:
-            line["e2e"] = time_e2e(args, ctx, pf)
+            line["e2e"] = time_e2e(args, ctx, pf, args.e2e_pieces)
         if args.parts & set(WIDENED):
             line["widened"] = time_widened(args, ctx, kda, I, pf, peaks)
         del pf
