@@ -47,7 +47,8 @@
 // sums to its output, so the state-independent work of chunks m+1 and m+2
 // runs while the chain works on chunk m. Three warp groups hand work over
 // through mbarriers:
-//   chain (warps 0-3)   state -> bf16 operand, MMA1 (two halves of the key
+//   chain (warps 0-3)   state -> bf16 operand; the U MMA that starts the
+//                       chunk's accumulator, then MMA1 (two halves of the key
 //                       channels through one 16 KB operand buffer), delta ->
 //                       bf16, MMA2, O -> global; it also issues the TMA loads
 //                       of k/q and log_alpha into the buffers its MMAs free.
@@ -57,7 +58,7 @@
 //                       MMA, reads A (beta-scaled, fp32) and P (bf16) out of
 //                       tensor memory, then issues the next chunk's prefix-sum
 //                       MMA.
-//   inverse (warps 8-15) (I + A)^{-1} -> T', the PT, W and U MMAs and their
+//   inverse (warps 8-15) (I + A)^{-1} -> T', the PT and W MMAs and their
 //                       readouts into the row operand; issues the v loads and
 //                       stores beta a chunk ahead.
 // k/q tiles are double-buffered, the log_alpha/KF tiles triple-buffered, the
@@ -610,9 +611,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 nb_sync(NB_CHLO, 64);
                 if (warp == 0) {
                     if (lane == 0) {
-                        wait1(B_RR + rb, (uint32_t)(n >> 1));  // row operand of chunk n stored
-                        wait1(B_UO + s, (uint32_t)(n / 3));    // its accumulator holds [U; P T' v]
+                        wait1(B_RR + rb, (uint32_t)(n >> 1));  // row operand (and [T'; PT]) of chunk n stored
+                        wait1(B_V, (uint32_t)n);                // its v tile landed
                         tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)  // [U; P T' v] = [T'; PT] v starts the accumulator
+                            mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dTP, kk * 32), dadd(dV, kk * 2048), ID_U, kk > 0);
+                        mma_commit(bars + B_UO + s);  // [T'; PT] and the v tile read
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dROWK, rb * 32768 + kk * 32),
@@ -1219,8 +1224,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
     } else {
         // ============================================================ inverse warps
-        // Per chunk m: A/P readout, (I + A)^{-1} -> T', then the PT, W and U MMAs
-        // with the readouts between them (PT -> [T'; PT], [W'; P W'] -> row operand).
+        // Per chunk m: (I + A)^{-1} -> T', then the PT and W MMAs with the readouts
+        // after them (PT -> [T'; PT], [W'; P W'] -> row operand); the v loads.
         const int iw = warp - kInvWarp0;  // 0..7
         const int hf = iw >> 2;           // which 32-column half of a readout this warp takes
         const int itid = tid - 32 * kInvWarp0;
@@ -1229,8 +1234,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             return (itid < kC && m < NC && t < seq_len) ? __bfloat162float(beta[(tok0 + t) * H + h]) : 0.f;
         };
         const float* sBm = sBeta;  // beta of the chunk in work (parity buffer)
-        // [T'; PT] and the v tile are free once the previous chunk's U MMA completed;
-        // then the v tile of chunk m is loaded (one thread)
+        // [T'; PT] and the v tile are free once the previous chunk's U MMA (issued by
+        // the chain) completed; then the v tile of chunk m is loaded (one thread)
         auto tp_free = [&](int m) {
             if (m > 0) {
                 if (wait1(B_UO + (m - 1) % 3, (uint32_t)((m - 1) / 3))) load_v(m);
@@ -1472,15 +1477,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             fence_proxy_async_smem();
             tc_fence_before();
             nb_sync(NB_INV, 256);
-            if (itid == 0) {
-                mbar_arrive(bars + B_RR + rb);  // row operand of chunk m stored
-                wait1(B_V, (uint32_t)m);
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // [U; P T' v] = [T'; PT] v: the chunk's accumulator
-                    mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dTP, kk * 32), dadd(dV, kk * 2048), ID_U, kk > 0);
-                mma_commit(bars + B_UO + s);
-            }
+            if (itid == 0) mbar_arrive(bars + B_RR + rb);  // row operand of chunk m stored (the chain issues its U MMA)
             __syncwarp();
         }
         if (itid == 0) {  // after an abort: wait (bounded) for this thread's MMAs
