@@ -118,7 +118,11 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chu
  * Numerics: state and accumulation in fp32. With dtype KDA_F32 and the SIMT
  * algorithm every product is fp32. The tensor-core algorithm rounds MMA
  * operands (decay-scaled keys and queries, the UT inverse, W, the state copy
- * that feeds the next chunk) to bf16 and accumulates in fp32.
+ * that feeds the next chunk) to bf16 and accumulates in fp32. It factors the
+ * decay e^{G_r - G_s} of a chunk through a reference point: the chunk's start
+ * while the chunk's decay stays within 80 (in natural-log units), its middle
+ * (G_last / 2) up to 160, and exact per-pair exponentials beyond that (slower,
+ * but finite for any decay).
  * Returns KDA_OK once enqueued.
  */
 kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const void *log_alpha,
