@@ -1622,26 +1622,45 @@ int sm_count() {
 }
 
 // Segments for the chunk-parallel scan, or 0 when it does not pay.
-// Phase 1 holds B*H*(2P-3) CTAs; P is the largest count that keeps it to one
-// wave, with at least kMinSegChunks chunks per segment (forced: 2, and P >= 3).
-// L is then rounded to whole chunks and P recounted so no segment is empty.
+// Every CTA runs its chunks at about the same period, so a plan's time is its
+// depth in chunk periods: each phase takes ceil(CTAs / SMs) waves of L chunks
+// plus kFillChunks for filling and draining a CTA's pipeline (fitted to
+// measurements: B1 H32 T131072 runs P = 5 at 0.95x the time of P = 3, while
+// B2 H16 T4096, 13-chunk segments, runs P = 5 at 1.13x). Phase 1 holds
+// B*H*(2P-3) CTAs, phase 3 B*H*(P-1) units (two CTAs each when that fits one
+// wave). P runs over 3 .. NC / kMinSegChunks (forced: up to NC / 2, and P >= 3
+// whenever T has 3 chunks); L is rounded to whole chunks and P recounted so
+// no segment is empty. AUTO takes the scan only when it is shallower than one
+// pass over the whole sequence; ties go to fewer segments.
 constexpr int kMinSegChunks = 8;
+constexpr int kFillChunks = 8;
 void scan_plan(const ChunkArgs& a, int mode, int* P_out, int* L_out) {
     *P_out = 0;
     *L_out = 0;
     if (mode == 0 || a.cu_seqlens || a.T <= 0) return;
     const long bh = (long)a.B * a.H;
-    const int NC = (a.T + kC - 1) / kC;
-    if (bh <= 0) return;
-    long P = ((long)sm_count() / bh + 3) / 2;
-    P = std::min<long>(P, NC / (mode == 2 ? 2 : kMinSegChunks));
-    if (mode == 2) P = std::max<long>(P, 3);
-    if (P < 3 || NC < 3) return;
-    const int Lc = (int)((NC + P - 1) / P);
-    const int Pn = (NC + Lc - 1) / Lc;
-    if (Pn < 3) return;
-    *P_out = Pn;
-    *L_out = Lc * kC;
+    const long NC = (a.T + kC - 1) / kC;
+    if (bh <= 0 || NC < 3) return;
+    const long sms = sm_count();
+    auto waves = [&](long ctas) { return (ctas + sms - 1) / sms; };
+    const long one_pass = waves(bh) * (NC + kFillChunks);
+    const long pmax = mode == 2 ? std::max<long>(3, NC / 2) : NC / kMinSegChunks;
+    long best_P = 0, best_L = 0, best_cost = 0;
+    for (long P = 3; P <= pmax; ++P) {
+        const long Lc = (NC + P - 1) / P;
+        const long Pn = (NC + Lc - 1) / Lc;
+        if (Pn < 3 || Pn != P) continue;  // (a recounted P is visited on its own)
+        const long units3 = bh * (Pn - 1);
+        const long cost = (waves(bh * (2 * Pn - 3)) + waves(2 * units3 <= sms ? 2 * units3 : units3)) * (Lc + kFillChunks);
+        if (best_P == 0 || cost < best_cost) {
+            best_P = Pn;
+            best_L = Lc;
+            best_cost = cost;
+        }
+    }
+    if (best_P == 0 || (mode == 1 && best_cost >= one_pass)) return;
+    *P_out = (int)best_P;
+    *L_out = (int)(best_L * kC);
 }
 
 }  // namespace

@@ -199,12 +199,18 @@ def test_varlen_rejects_missing_or_misaligned_offsets():
 
 def test_scan_workspace_sizes():
     """The segment scan keeps B*H*(3P-5) fp32 [128][128] matrices after the
-    256-byte status block; it is planned only where it pays (auto) and never
-    for 128 heads (one wave of whole sequences already fills 148 SMs)."""
+    256-byte status block; it is planned only where its depth in chunk periods
+    beats one pass (auto), never for 128 heads (one wave of whole sequences
+    already fills 148 SMs). Without a GPU the planner assumes 148 SMs."""
     mat = 128 * 128 * 4
-    # 32 heads, 2048 chunks: P = 3 -> 4 matrices per head
-    assert kda.workspace_size(1, 131072, 32, 128, 128, 64, "bf16", "tc_scan") == 256 + 32 * 4 * mat
-    assert kda.workspace_size(1, 131072, 32, 128, 128, 64, "bf16", "auto") == 256 + 32 * 4 * mat
+    # 32 heads, 2048 chunks: P = 5 (phase 1 in two waves, phase 3 in one: a depth
+    # of 3 x 410 chunks against 2 x 683 for P = 3) -> 10 matrices per head
+    assert kda.workspace_size(1, 131072, 32, 128, 128, 64, "bf16", "tc_scan") == 256 + 32 * 10 * mat
+    assert kda.workspace_size(1, 131072, 32, 128, 128, 64, "bf16", "auto") == 256 + 32 * 10 * mat
+    # 16 heads x 2, 64 chunks, and 32 heads x 1, 32 chunks: short segments, where
+    # filling each CTA's pipeline weighs in: P = 3
+    assert kda.workspace_size(2, 4096, 16, 128, 128, 64, "bf16", "auto") == 256 + 32 * 4 * mat
+    assert kda.workspace_size(1, 2048, 32, 128, 128, 64, "bf16", "auto") == 256 + 32 * 4 * mat
     assert kda.workspace_size(1, 131072, 32, 128, 128, 64, "bf16", "tc") == 256
     assert kda.workspace_size(4, 8192, 32, 128, 128, 64, "bf16", "auto") == 256
     # 2 heads, 65 chunks, forced: P = 32 -> Lc = 3 chunks -> 22 segments
