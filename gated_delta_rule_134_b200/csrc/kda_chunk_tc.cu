@@ -1165,8 +1165,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const bool exact = tier == 2;
             if (exact) exact_chunk(m, s, rb, cb, lim);
             {   // per-channel scales of this chunk. The tensor memory holds R with
-                // S = Diag(ek) R; the chain feeds S^ = Diag(os) R to MMA1 and keeps
-                // Diag(ts) R + KF^T delta, whose true state is Diag(ek_new) times it.
+                // S = Diag(ek) R; the chain feeds S^ = Diag(os) Diag(ms) R to MMA1 and
+                // keeps Diag(ts) Diag(ms) R + KF^T delta (ms = 1 unless os = ts), whose
+                // true state is Diag(ek_new) times it.
                 const int c = ttid;
                 const float g_l = GATE == 0 ? sGl[c] : (GATE == 1 ? sGl[0] : 0.f);
                 const float ek_prev = sEK[c];
