@@ -47,11 +47,11 @@
 // sums to its output, so the state-independent work of chunks m+1 and m+2
 // runs while the chain works on chunk m. Three warp groups hand work over
 // through mbarriers:
-//   chain (warps 0-3)   state -> bf16 operand; the U MMA that starts the
-//                       chunk's accumulator, then MMA1 (two halves of the key
-//                       channels through one 16 KB operand buffer), delta ->
-//                       bf16, MMA2, O -> global; it also issues the TMA loads
-//                       of k/q and log_alpha into the buffers its MMAs free.
+//   chain (warps 0-3)   state -> bf16 operand (one channel row per thread);
+//                       the U MMA that starts the chunk's accumulator, then
+//                       MMA1 over all 128 key channels, delta -> bf16, MMA2,
+//                       O -> global; it also issues the TMA loads of k/q and
+//                       log_alpha into the buffers its MMAs free.
 //   tile  (warps 4-7)   prefix sums out of tensor memory, KE/QE in place over
 //                       the raw k/q rows, KF over the log_alpha tile, the
 //                       overflow vote, per-channel scales; issues the [A; P]
@@ -62,7 +62,8 @@
 //                       readouts into the row operand; issues the v loads and
 //                       stores beta a chunk ahead.
 // k/q tiles are double-buffered, the log_alpha/KF tiles triple-buffered, the
-// per-channel scales kept by chunk mod 4.
+// per-channel scales kept by chunk mod 3. The A scratch of the inverse is fp16
+// (the tf32 MMAs of the inverse read it through the same 10-bit mantissa).
 // (I + A)^{-1}: 16x16 diagonal blocks by forward substitution (four threads per
 // column), then one column chain per warp, T_ab = -T_aa sum_k A_ak T_kb, on
 // m16n8k8 tf32 MMAs; T' = T Diag(beta) is written as bf16 by the thread that
@@ -74,6 +75,8 @@
 // frees its tensor memory and returns.
 #include <algorithm>
 #include <type_traits>
+
+#include <cuda_fp16.h>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -93,12 +96,11 @@ constexpr int NB_TILE = 1;  // tile warps
 constexpr int NB_TOR = 2;   // tile warps, OR-vote
 constexpr int NB_INV = 3;   // inverse warps
 constexpr int NB_CHLO = 4;  // chain warps 0-1
-constexpr int NB_CHB = 5;   // chain warps 2-3 -> warp 0: second half of the state operand stored
 constexpr int NB_CHHI = 6;  // chain warps 2-3
 constexpr int NB_CH = 7;    // all chain warps
 constexpr int kC = 64;    // chunk
 constexpr int kD = 128;   // dk = dv
-constexpr int kLDA = 68;  // fp32 row stride of the A scratch (bank spread)
+constexpr int kLDA = 72;  // fp16 row stride of the A scratch (16-byte rows, bank spread)
 constexpr int kLDT = 20;  // fp32 row stride of the diagonal blocks of T (bank spread)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kGuardL = 80.f * kLog2e;      // |G_r| <= 80, in log2 units
@@ -115,18 +117,18 @@ struct Layout {
     static constexpr uint32_t LMAT = 131072;    // [L; L] K-major 128 x 64
     static constexpr uint32_t TP = 147456;      // [T'; PT] K-major 128 x 64
     static constexpr uint32_t SP = TP + 16384;  // P, K-major 64 x 64 bf16 (rows 64-127 of [Y; P], Y = TP rows 64-127)
-    static constexpr uint32_t SOP = SP + 8192;  // S half (64 channels) x DVT, bf16 MN-major, then delta
-    static constexpr uint32_t OST = SOP + 64 * DVT * 2;  // 2 x [32 tok][32 ch] bf16 (64-byte swizzle): O stores
-    static constexpr uint32_t SCR = OST + 4096;          // A fp32 [64][kLDA], T diagonal blocks [4][16][kLDT]
-    static constexpr uint32_t SA = SCR;                  //   (exact path: 16 KB staging)
-    static constexpr uint32_t STD = SCR + 64 * kLDA * 4;
-    static constexpr uint32_t SCR_BYTES = 64 * kLDA * 4 + 4 * 16 * kLDT * 4;
+    static constexpr uint32_t SOP = SP + 8192;  // S (128 channels) x DVT, bf16 MN-major, then delta (64 tokens)
+    static constexpr uint32_t OST = SOP + 128 * DVT * 2;  // 2 x [32 tok][32 ch] bf16 (64-byte swizzle): O stores
+    static constexpr uint32_t SCR = OST + 4096;          // A fp16 [64][kLDA], T diagonal blocks fp32 [4][16][kLDT]
+    static constexpr uint32_t SA = SCR;                  //   (exact path: 8 KB fp32 staging)
+    static constexpr uint32_t STD = SCR + 64 * kLDA * 2;
+    static constexpr uint32_t SCR_BYTES = 64 * kLDA * 2 + 4 * 16 * kLDT * 4;
     static constexpr uint32_t SMALL = SCR + SCR_BYTES;
     static constexpr uint32_t SBETA = SMALL;        // 2 x 64 f32: beta of the chunk (by parity)
-    static constexpr uint32_t SOPS = SBETA + 512;   // 4 x 128 f32: operand scale per channel (by chunk mod 4)
-    static constexpr uint32_t STMS = SOPS + 2048;   // 4 x 128 f32: tensor-memory scale per channel
-    static constexpr uint32_t SMDS = STMS + 2048;   // 4 x 128 f32: second factor of both (middle tier, else 1)
-    static constexpr uint32_t SEK = SMDS + 2048;    // 128 f32: pending state factor after the last prepared chunk
+    static constexpr uint32_t SOPS = SBETA + 512;   // 3 x 128 f32: operand scale per channel (by chunk mod 3)
+    static constexpr uint32_t STMS = SOPS + 1536;   // 3 x 128 f32: tensor-memory scale per channel
+    static constexpr uint32_t SMDS = STMS + 1536;   // 3 x 128 f32: second factor of both (middle tier, else 1)
+    static constexpr uint32_t SEK = SMDS + 1536;    // 128 f32: pending state factor after the last prepared chunk
     static constexpr uint32_t SGL = SEK + 512;      // 128 f32: G_last
     static constexpr uint32_t BARS = SGL + 512;     // mbarriers
     static constexpr uint32_t MISC = BARS + 512;    // tmem base, abort flag, copies issued, wait budget
@@ -134,7 +136,7 @@ struct Layout {
     static constexpr uint32_t SMEM_BYTES = END + 1024;   // + alignment slack
     static constexpr uint32_t SBO_V = 1024 * (DVT / 64); // K-group stride of the S / delta operands
     static_assert(SOP % 1024 == 0 && TP % 1024 == 0 && LMAT % 1024 == 0 && OST % 1024 == 0, "operand alignment");
-    static_assert(64 * 64 * 4 <= SCR_BYTES, "exact-path staging overflows the scratch");
+    static_assert(32 * 64 * 4 <= SCR_BYTES, "exact-path staging overflows the scratch");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     // tensor memory columns: R (fp32, lane = key channel) and three chunk slots
     static constexpr uint32_t S_COL = 0;
@@ -153,8 +155,8 @@ enum : int {
     B_WB = 13,    // [W'; P W'] MMA done
     B_UO = 14,    // 3: [U; P T' v] MMA of the slot's chunk done (also frees [T'; PT] and the v tile)
     B_RR = 17,    // 2: row operand [-W'; QE - P W'] of the chunk of this parity stored
-    B_SC = 19,    // 4: per-channel scales of the chunk (mod 4) stored
-    B_M1A = 23,   // MMA1, first half, done
+    B_SC = 19,    // 3 (of 4): per-channel scales of the chunk (mod 3) stored
+    B_M1A = 23,   // (unused)
     B_M1 = 24,    // MMA1 done (row operand free)
     B_M2 = 25,    // MMA2 done (KF and delta operand free, R updated)
     B_SF = 28,    // 3: the slot's chunk read out by the chain (count 2)
@@ -319,7 +321,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     float* sMdS = reinterpret_cast<float*>(sm + L::SMDS);
     float* sEK = reinterpret_cast<float*>(sm + L::SEK);
     float* sGl = reinterpret_cast<float*>(sm + L::SGL);
-    float* sA = reinterpret_cast<float*>(sm + L::SA);
+    __half* sA = reinterpret_cast<__half*>(sm + L::SA);
     float* sTd = reinterpret_cast<float*>(sm + L::STD);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BARS);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::MISC);
@@ -596,47 +598,36 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     }
                 }
             }
-            waitw(B_SC + (n & 3), (uint32_t)(n >> 2));
-            const float os = sOpS[(n & 3) * 128 + row], ts = sTmS[(n & 3) * 128 + row], ms = sMdS[(n & 3) * 128 + row];
-            if (quad < 2) {
+            waitw(B_SC + s, (uint32_t)(n / 3));
+            const float os = sOpS[s * 128 + row], ts = sTmS[s * 128 + row], ms = sMdS[s * 128 + row];
+            // the whole state (channel row `row` per thread) -> the bf16 operand of MMA1
 #pragma unroll 1
-                for (int gq = 0; gq < DVT / 32; ++gq) {  // key channels 0-63
-                    uint32_t pk[16];
-                    s1_group(gq, os, ts, ms, pk);
-                    sop_store(row, gq, pk);
-                }
-                tmem_st_wait();
-                fence_proxy_async_smem();
-                tc_fence_before();
-                nb_sync(NB_CHLO, 64);
-                if (warp == 0) {
-                    if (lane == 0) {
-                        wait1(B_RR + rb, (uint32_t)(n >> 1));  // row operand (and [T'; PT]) of chunk n stored
-                        wait1(B_V, (uint32_t)n);                // its v tile landed
-                        tc_fence_after();
+            for (int gq = 0; gq < DVT / 32; ++gq) {
+                uint32_t pk[16];
+                s1_group(gq, os, ts, ms, pk);
+                sop_store(row, gq, pk);
+            }
+            tmem_st_wait();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            nb_sync(NB_CH, 128);
+            if (issuer) {
+                wait1(B_RR + rb, (uint32_t)(n >> 1));  // row operand (and [T'; PT]) of chunk n stored
+                wait1(B_V, (uint32_t)n);                // its v tile landed
+                tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)  // [U; P T' v] = [T'; PT] v starts the accumulator
-                            mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dTP, kk * 32), dadd(dV, kk * 2048), ID_U, kk > 0);
-                        mma_commit(bars + B_UO + s);  // [T'; PT] and the v tile read
+                for (int kk = 0; kk < 4; ++kk)  // [U; P T' v] = [T'; PT] v starts the accumulator
+                    mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dTP, kk * 32), dadd(dV, kk * 2048), ID_U, kk > 0);
+                mma_commit(bars + B_UO + s);  // [T'; PT] and the v tile read
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dROWK, rb * 32768 + kk * 32),
-                                        dadd(dSOP, kk * 2 * L::SBO_V), ID_M1, 1);
-                        mma_commit(bars + B_M1A);
-                    }
-                    __syncwarp();
-                    nb_sync(NB_CHB, 96);  // key channels 64-127 stored
-                    if (lane == 0) {
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dROWK, rb * 32768 + 16384 + kk * 32),
-                                        dadd(dSOP, kk * 2 * L::SBO_V), ID_M1, 1);
-                        mma_commit(bars + B_M1);
-                    }
-                    __syncwarp();
-                }
-                waitw(B_M1, (uint32_t)n);
+                for (int kk = 0; kk < 8; ++kk)  // + [-W'; QE - P W'] S^ over all 128 key channels
+                    mma_bf16_ss(tmem + L::SLOT0 + 128 * s, dadd(dROWK, rb * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32),
+                                dadd(dSOP, kk * 2 * L::SBO_V), ID_M1, 1);
+                mma_commit(bars + B_M1);
+            }
+            __syncwarp();
+            const bool m1 = waitw(B_M1, (uint32_t)n);
+            if (quad < 2) {
                 {   // delta (slot rows 0-63) -> bf16 operand over the state operand
 #pragma unroll 1
                     for (int gq = 0; gq < DVT / 32; ++gq) {
@@ -664,31 +655,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
                 __syncwarp();
             } else {
-                // key channels 64-127: the first half of the columns staged in registers
-                // until the operand buffer is free, the rest converted after
-                constexpr int kStaged = DVT / 64;
-                uint32_t pk[kStaged][16];
-#pragma unroll
-                for (int gq = 0; gq < kStaged; ++gq) s1_group(gq, os, ts, ms, pk[gq]);
-                waitw(B_M1A, (uint32_t)n);  // first half of the state operand consumed
-#pragma unroll
-                for (int gq = 0; gq < kStaged; ++gq) sop_store(row - 64, gq, pk[gq]);
-#pragma unroll 1
-                for (int gq = kStaged; gq < DVT / 32; ++gq) {
-                    uint32_t pq[16];
-                    s1_group(gq, os, ts, ms, pq);
-                    sop_store(row - 64, gq, pq);
-                }
-                tmem_st_wait();
-                fence_proxy_async_smem();
-                tc_fence_before();
-                // A full sync, not an arrive: warp 0 is already waiting here (it issued
-                // MMA1A before it, which the wait above needed), and after an abort, when
-                // the mbarrier waits are skipped, it keeps warps 2-3 from arriving for a
-                // later chunk before warp 0 syncs for this one (the barrier would count
-                // their arrivals into the wrong generation and warp 0 would wait forever).
-                nb_sync(NB_CHB, 96);
-                const bool m1 = waitw(B_M1, (uint32_t)n);
                 if (warp == 2 && lane == 0 && n + 2 < NC && m1) {  // the row buffer of this parity is free
                     load_kq(n + 2, B_KQ + rb);
                     pf_kq(n + 3);
@@ -874,7 +840,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             if (ttid == 0 && !*s_abort) load_kq(m, B_EXKQ);
             waitw(B_EXKQ, (uint32_t)nex);
             if (m > 0) waitw(B_SCRF, (uint32_t)(m - 1));  // the inverse warps are done with the scratch
-            float* stg = reinterpret_cast<float*>(sm + L::SCR);  // 16 KB: G of 64 channels, then A, then P
+            float* stg = reinterpret_cast<float*>(sm + L::SCR);  // 8 KB: G of 32 channels, then half of A or P
             const bool live = tok < lim;
             const uint8_t* rk = sm + L::ROW + rb * 32768;
             constexpr int kPairs = kC * (kC + 1) / 2, kPer = (kPairs + 127) / 128;
@@ -891,10 +857,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 s2 = p - r * (r + 1) / 2;
             };
 #pragma unroll 1
-            for (int hc = 0; hc < 2; ++hc) {  // channels [64 hc, 64 hc + 64)
-                if ((ch0 >> 6) == hc) {       // this thread's channels: G -> fp32 [64 tok][64 ch]
+            for (int hq = 0; hq < 4; ++hq) {     // channels [32 hq, 32 hq + 32)
+                if ((ch0 >> 6) == (hq >> 1)) {  // this thread's channels: G -> fp32 [64 tok][32 ch]
 #pragma unroll 1
-                    for (int u8 = 0; u8 < 8; ++u8) {
+                    for (int u4 = 0; u4 < 4; ++u4) {
+                        const int u8 = 4 * (hq & 1) + u4;
                         uint32_t g8[8];
                         if (GATE == 0) {
                             tmem_ld8(slotq + ch0 + 8 * u8, g8);
@@ -906,7 +873,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll
                             for (int e = 0; e < 8; ++e) g8[e] = g1;
                         }
-                        float* dst = stg + tok * 64 + 8 * u8;
+                        float* dst = stg + tok * 32 + 8 * u4;
                         *reinterpret_cast<float4*>(dst) = make_float4(__uint_as_float(g8[0]), __uint_as_float(g8[1]),
                                                                       __uint_as_float(g8[2]), __uint_as_float(g8[3]));
                         *reinterpret_cast<float4*>(dst + 4) = make_float4(__uint_as_float(g8[4]), __uint_as_float(g8[5]),
@@ -923,11 +890,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         float a = av[i], pp = pv[i];
                         // rows past the sequence stay 0 (their gates may be another
                         // sequence's and overflow the exponential)
-                        for (int i2 = 0; i2 < (r < lim ? 64 : 0); ++i2) {
-                            const int c = (i2 + p) & 63, cc = 64 * hc + c;
+                        for (int i2 = 0; i2 < (r < lim ? 32 : 0); ++i2) {
+                            const int c = (i2 + p) & 31, cc = 32 * hq + c;
                             const float ks =
                                 __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(s2, cc))) *
-                                ex2((stg[r * 64 + c] - stg[s2 * 64 + c]) * kLog2e);
+                                ex2((stg[r * 32 + c] - stg[s2 * 32 + c]) * kLog2e);
                             a = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(r, cc))), ks, a);
                             pp = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rk + rop_off(64 + r, cc))),
                                       ks, pp);
@@ -978,11 +945,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     st_shared_v4(colp + fo, kf[0], kf[1], kf[2], kf[3]);
                 }
             }
-            // raw A sums, then raw P sums -> fp32 [64][64] staging -> the slot
-            // (quadrants 0/1 hold the A rows, 2/3 the P rows)
+            // raw A sums, then raw P sums -> fp32 [32][64] staging, 32 rows at a time
+            // -> the slot (quadrants 0/1 hold the A rows, 2/3 the P rows)
 #pragma unroll 1
-            for (int w = 0; w < 2; ++w) {
-                for (int i = ttid; i < 64 * 64 / 4; i += 128)
+            for (int wh = 0; wh < 4; ++wh) {
+                const int w = wh >> 1, rh = wh & 1;  // A or P; rows [32 rh, 32 rh + 32)
+                for (int i = ttid; i < 32 * 64 / 4; i += 128)
                     reinterpret_cast<float4*>(stg)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
                 nb_sync(NB_TILE, 128);
 #pragma unroll
@@ -991,12 +959,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     if (p < kPairs) {
                         int r, s2;
                         pair_rs(p, r, s2);
-                        stg[r * 64 + s2] = w == 0 ? av[i] : pv[i];
+                        if ((r >> 5) == rh) stg[(r & 31) * 64 + s2] = w == 0 ? av[i] : pv[i];
                     }
                 }
                 nb_sync(NB_TILE, 128);
-                if ((quad >> 1) == w) {
-                    const float* src = stg + (32 * (quad & 1) + lane) * 64;
+                if (quad == wh) {
+                    const float* src = stg + lane * 64;
 #pragma unroll 1
                     for (int h2 = 0; h2 < 2; ++h2) {
                         uint32_t r32[32];
@@ -1028,16 +996,16 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         uint32_t v[8];
                         tmem_ld8(slotq + 8 * e8, v);
                         tmem_ld_wait(v);
-                        float* dst = sA + r * kLDA + 8 * e8;
+                        uint32_t w[4];
 #pragma unroll
-                        for (int u = 0; u < 8; u += 4) {
-                            float4 f;
-                            f.x = (8 * e8 + u + 0 < r) ? br * __uint_as_float(v[u + 0]) : 0.f;
-                            f.y = (8 * e8 + u + 1 < r) ? br * __uint_as_float(v[u + 1]) : 0.f;
-                            f.z = (8 * e8 + u + 2 < r) ? br * __uint_as_float(v[u + 2]) : 0.f;
-                            f.w = (8 * e8 + u + 3 < r) ? br * __uint_as_float(v[u + 3]) : 0.f;
-                            *reinterpret_cast<float4*>(dst + u) = f;
+                        for (int u = 0; u < 4; ++u) {
+                            const int c = 8 * e8 + 2 * u;
+                            const float a0 = (c < r) ? br * __uint_as_float(v[2 * u]) : 0.f;
+                            const float a1 = (c + 1 < r) ? br * __uint_as_float(v[2 * u + 1]) : 0.f;
+                            const __half2 h = __floats2half2_rn(a0, a1);
+                            w[u] = *reinterpret_cast<const uint32_t*>(&h);
                         }
+                        st_shared_v4(smem_u32(sA + r * kLDA + 8 * e8), w[0], w[1], w[2], w[3]);
                     }
                 }
             } else {
@@ -1171,7 +1139,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 const int c = ttid;
                 const float g_l = GATE == 0 ? sGl[c] : (GATE == 1 ? sGl[0] : 0.f);
                 const float ek_prev = sEK[c];
-                const int slot4 = m & 3;
+                const int slot4 = m % 3;  // (the tile warps reach chunk m + 3 only after the chain read chunk m)
                 if (tier == 0) {         // reference at the chunk start: S^ = S, KF = k e^{-G}
                     sOpS[slot4 * 128 + c] = ek_prev;
                     sTmS[slot4 * 128 + c] = ek_prev;
@@ -1196,7 +1164,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             tc_fence_before();
             nb_sync(NB_TILE, 128);
             if (ttid == 0) {
-                mbar_arrive(bars + B_SC + (m & 3));
+                mbar_arrive(bars + B_SC + m % 3);
                 tc_fence_after();
                 if (!exact) {  // [A; P] = [KE; QE] KF^T over the prefix-sum columns (read)
 #pragma unroll
@@ -1267,7 +1235,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const int a = itid >> 6, jc = (itid >> 2) & 15, q = itid & 3;
             float colv[4] = {0.f, 0.f, 0.f, 0.f};
             {
-                const float* Ab = sA + (16 * a) * kLDA + 16 * a;
+                const __half* Ab = sA + (16 * a) * kLDA + 16 * a;
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
@@ -1276,7 +1244,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     if (q == (r & 3)) colv[r >> 2] = t;
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        if (q + 4 * i > r) acc[i] = fmaf(Ab[(q + 4 * i) * kLDA + r], t, acc[i]);
+                        if (q + 4 * i > r) acc[i] = fmaf(__half2float(Ab[(q + 4 * i) * kLDA + r]), t, acc[i]);
                 }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) sTd[(a * 16 + q + 4 * i) * kLDT + jc] = colv[i];
@@ -1333,9 +1301,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         const int k = bb + dk;
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
-                            const float* Ar = sA + (16 * a) * kLDA + 16 * k + 8 * j;
-                            const uint32_t af[4] = {to_tf32(Ar[g * kLDA + t]), to_tf32(Ar[(g + 8) * kLDA + t]),
-                                                    to_tf32(Ar[g * kLDA + t + 4]), to_tf32(Ar[(g + 8) * kLDA + t + 4])};
+                            const __half* Ar = sA + (16 * a) * kLDA + 16 * k + 8 * j;
+                            const uint32_t af[4] = {to_tf32(__half2float(Ar[g * kLDA + t])),
+                                                    to_tf32(__half2float(Ar[(g + 8) * kLDA + t])),
+                                                    to_tf32(__half2float(Ar[g * kLDA + t + 4])),
+                                                    to_tf32(__half2float(Ar[(g + 8) * kLDA + t + 4]))};
                             mma_tf32_16x8x8(x, af, tb[dk][j]);
                         }
                     }
